@@ -1,0 +1,386 @@
+"""Pins of the CPU oracle against what mathematics and published tables fix.
+
+No value here comes from the CUDA path.  Each test ties one oracle function to
+something independent of it: a library routine for a special case (numpy's
+binary16, scipy's Hadamard matrix, scipy's normal distribution and
+quadrature), a published table (Max 1960), a hand-derived worked example,
+an invariant, or brute force on tiny inputs.
+"""
+import math
+
+import numpy as np
+import pytest
+import scipy.integrate
+import scipy.linalg
+import scipy.special
+import scipy.stats
+import torch
+
+from conftest import read_golden
+
+RNG = np.random.default_rng(12345)
+
+
+def bf16_bits_of(x):
+    t = torch.as_tensor(np.asarray(x, np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------- scalar formats
+def test_bf16_decode_matches_torch(orc):
+    bits = RNG.integers(0, 1 << 16, size=4000).astype(np.uint16)
+    bits = bits[(bits & 0x7F80) != 0x7F80]  # finite values only
+    ref = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).double().numpy()
+    got = np.array([orc.bf16_to_double(b) for b in bits])
+    assert np.array_equal(got, ref)
+
+
+def _fp16_samples():
+    xs = list(np.concatenate([
+        RNG.standard_normal(3000) * 10.0 ** RNG.integers(-9, 6, 3000),
+        np.ldexp(RNG.random(500), -RNG.integers(14, 26, 500)),  # subnormal range
+        [0.0, -0.0, 65504.0, 65519.99, 65520.0, 70000.0, -1e9, 5.960464477539063e-08,
+         2.9802322387695312e-08, 2.98023224e-08, 1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11],
+    ]))
+    return xs
+
+
+def test_fp16_nearest_matches_numpy(orc):
+    for x in _fp16_samples():
+        got = orc.fp16_from_double(x, 0)
+        with np.errstate(over="ignore"):
+            ref = int(np.array([x], np.float64).astype(np.float16).view(np.uint16)[0])
+        assert got == ref, (x, hex(got), hex(ref))
+
+
+def test_fp16_directed_rounding_brackets(orc):
+    for x in _fp16_samples():
+        if abs(x) > 65504:
+            continue
+        dn = orc.fp16_from_double(x, -1)
+        up = orc.fp16_from_double(x, +1)
+        fdn = np.array([dn], np.uint16).view(np.float16)[0]
+        fup = np.array([up], np.uint16).view(np.float16)[0]
+        assert float(fdn) <= x <= float(fup)
+        # adjacent: nothing representable strictly between the bracket and x
+        with np.errstate(over="ignore"):
+            assert float(np.nextafter(fdn, np.float16(np.inf))) > x or float(fdn) == x
+            assert float(np.nextafter(fup, np.float16(-np.inf))) < x or float(fup) == x
+        assert orc.fp16_to_double(dn) == float(fdn)
+        assert orc.fp16_to_double(up) == float(fup)
+
+
+def test_fp16_decode_all_finite_patterns(orc):
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    f = bits.view(np.float16)
+    fin = np.isfinite(f)
+    got = np.array([orc.fp16_to_double(int(b)) for b in bits[fin][::7]])
+    assert np.array_equal(got, f[fin][::7].astype(np.float64))
+
+
+# ---------------------------------------------------------------- Hadamard
+@pytest.mark.parametrize("d", [1, 2, 4, 8, 16, 32, 64, 128])
+def test_hadamard_is_scipy_sylvester(orc, d):
+    H = orc.hadamard(d)
+    ref = scipy.linalg.hadamard(d).astype(np.float64) / math.sqrt(d)
+    assert np.array_equal(H, ref)
+    assert np.allclose(H @ H, np.eye(d), atol=1e-14)  # symmetric and involutive
+
+
+def test_hadamard_small_closed_forms(orc):
+    s = 1 / math.sqrt(2)
+    assert np.array_equal(orc.hadamard(2), np.array([[s, s], [s, -s]]))
+    H = orc.hadamard(128)
+    assert np.allclose(H[:, 0], np.full(128, 1 / math.sqrt(128)), atol=0)  # H e_0
+
+
+# ---------------------------------------------------------------- Lloyd-Max
+def test_lloyd_max_matches_max_1960(orc):
+    c, iters = orc.lloyd_max_gaussian16()
+    rows = read_golden("max1960_gaussian16.txt")
+    levels = {int(r[1]): float(r[2]) for r in rows if r[0] == "level"}
+    thr = {int(r[1]): float(r[2]) for r in rows if r[0] == "threshold"}
+    for j in range(1, 9):
+        # positive half: c[7+j]; negative half is the mirror
+        assert abs(c[7 + j] - levels[j]) <= 5.1e-4 * max(1, levels[j]), (j, c[7 + j])
+        assert abs(c[8 - j] + levels[j]) <= 5.1e-4 * max(1, levels[j])
+    mids = 0.5 * (c[:-1] + c[1:])
+    for j in range(1, 9):
+        assert abs(mids[6 + j] - thr[j]) <= 5.1e-4 * max(1, thr[j]), (j, mids[6 + j])
+    assert np.all(np.diff(c) > 0)
+    assert np.allclose(c, -c[::-1], atol=1e-14)
+
+
+def test_lloyd_max_is_a_fixed_point_by_quadrature(orc):
+    """Each level equals the conditional mean of N(0,1) on its cell, by numerical integration."""
+    c, _ = orc.lloyd_max_gaussian16()
+    b = np.concatenate([[-np.inf], 0.5 * (c[:-1] + c[1:]), [np.inf]])
+    for j in range(16):
+        mass = scipy.stats.norm.cdf(b[j + 1]) - scipy.stats.norm.cdf(b[j])
+        mom, _ = scipy.integrate.quad(lambda x: x * scipy.stats.norm.pdf(x), b[j], b[j + 1],
+                                      epsabs=1e-15, epsrel=1e-13)
+        assert abs(mom / mass - c[j]) < 1e-9, j
+
+
+def test_lloyd_max_distortion_by_quadrature(orc):
+    c, _ = orc.lloyd_max_gaussian16()
+    b = np.concatenate([[-np.inf], 0.5 * (c[:-1] + c[1:]), [np.inf]])
+    D = sum(scipy.integrate.quad(lambda x, cj=c[j]: (x - cj) ** 2 * scipy.stats.norm.pdf(x),
+                                 b[j], b[j + 1], epsabs=1e-15)[0] for j in range(16))
+    dist = float([r for r in read_golden("max1960_gaussian16.txt") if r[0] == "distortion"][0][2])
+    assert abs(D - dist) < 1e-5
+    # and the closed form for a centroid quantiser, E[X^2] - E[Q^2], agrees with the quadrature
+    P = np.diff(scipy.stats.norm.cdf(b))
+    assert abs((1.0 - np.sum(c ** 2 * P)) - D) < 1e-12
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_default_table_scaled_by_sqrt_d(orc, d):
+    c, _ = orc.lloyd_max_gaussian16()
+    t = orc.default_table(d)
+    assert t.dtype == np.float32
+    assert np.array_equal(t, (c / math.sqrt(d)).astype(np.float32))
+
+
+# ---------------------------------------------------------------- keys
+def test_key_worked_example_e0(orc):
+    g = {r[0]: r[1:] for r in read_golden("worked_examples.txt")}
+    d = 128
+    table = orc.default_table(d)
+    k = np.zeros(d, np.float32)
+    k[0] = 1.0
+    idx, n16, y = orc.encode_k(bf16_bits_of(k), table)
+    assert n16 == int(g["key_e0_norm16"][0], 16)
+    assert np.all(idx == int(g["key_e0_code"][0]))
+    assert np.allclose(y, 1 / math.sqrt(d), atol=1e-15)
+    khat = orc.decode_k(idx, n16, table)
+    assert abs(khat[0] - float(g["key_e0_khat0"][0])) < 1e-5
+    assert np.max(np.abs(khat[1:])) < 1e-12
+
+
+def test_key_zero_vector_ties_low(orc):
+    table = orc.default_table(64)
+    idx, n16, y = orc.encode_k(np.zeros(64, np.uint16), table)
+    # y = 0 is exactly the midpoint of levels 7 and 8: the tie goes to the lower index
+    assert np.all(idx == 7) and n16 == 0
+    assert np.all(orc.decode_k(idx, n16, table) == 0.0)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_key_rotation_matches_scipy_and_keeps_norm(orc, d):
+    table = orc.default_table(d)
+    Hs = scipy.linalg.hadamard(d) / math.sqrt(d)
+    for _ in range(20):
+        kb = bf16_bits_of(RNG.standard_normal(d) * RNG.lognormal(0, 1, d))
+        k = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).double().numpy()
+        idx, n16, y = orc.encode_k(kb, table)
+        assert np.allclose(y, Hs @ (k / np.linalg.norm(k)), atol=1e-14)
+        assert abs(np.linalg.norm(y) - 1.0) < 1e-14
+        assert n16 == int(np.float16(np.linalg.norm(k)).view(np.uint16))
+        # brute force: the chosen level is at least as close as every other level
+        dist = np.abs(y[:, None] - table[None, :].astype(np.float64))
+        assert np.all(dist[np.arange(d), idx] <= dist.min(axis=1))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_key_relative_mse_matches_lloyd_max_distortion(orc, d):
+    """For Gaussian keys the rotated unit coordinates are ~N(0, 1/d), so the relative
+    reconstruction error is the quantiser distortion of N(0,1) (Max 1960: 0.009497)."""
+    table = orc.default_table(d)
+    errs = []
+    for _ in range(1500):
+        kb = bf16_bits_of(RNG.standard_normal(d))
+        k = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).double().numpy()
+        idx, n16, _ = orc.encode_k(kb, table)
+        khat = orc.decode_k(idx, n16, table)
+        errs.append(np.sum((k - khat) ** 2) / np.sum(k ** 2))
+    mse = float(np.mean(errs))
+    # the coordinates are Beta- rather than exactly Gaussian-distributed; a few % slack
+    assert abs(mse - 0.009497) / 0.009497 < 0.04, mse
+
+
+# ---------------------------------------------------------------- values
+def test_value_worked_example_ramp(orc):
+    g = {r[0]: r[1:] for r in read_golden("worked_examples.txt")}
+    v = np.concatenate([np.arange(32, dtype=np.float32), np.arange(32, dtype=np.float32)])
+    q, s, z, r = orc.encode_v(bf16_bits_of(v))
+    assert int(z[0]) == int(g["value_ramp_zero16"][0], 16)
+    assert int(s[0]) == int(g["value_ramp_scale16"][0], 16)
+    assert list(q[:32]) == [int(x) for x in g["value_ramp_codes"]]
+
+
+def test_value_error_bound_and_brute_force(orc):
+    for trial in range(300):
+        scale = 10.0 ** RNG.uniform(-3, 3)
+        v = RNG.standard_t(4, 128) * scale + RNG.normal() * scale
+        vb = bf16_bits_of(v)
+        vd = torch.from_numpy(vb.view(np.int16)).view(torch.bfloat16).double().numpy()
+        q, s16, z16, r = orc.encode_v(vb)
+        vh = orc.decode_v(q, s16, z16)
+        for g in range(4):
+            sl = slice(32 * g, 32 * g + 32)
+            s = float(np.uint16(s16[g]).view(np.float16))
+            z = float(np.uint16(z16[g]).view(np.float16))
+            mn, mx = vd[sl].min(), vd[sl].max()
+            # z is the largest fp16 <= min, s the smallest fp16 >= (max - z)/15
+            assert z <= mn < float(np.nextafter(np.float16(z), np.float16(np.inf))) or z == mn
+            assert s * 15 >= mx - z
+            assert float(np.nextafter(np.float16(s), np.float16(-np.inf))) * 15 < mx - z
+            assert np.all(np.abs(vd[sl] - vh[sl]) <= s / 2 * (1 + 1e-12))
+            # brute force over the 16 grid points, ties to the even code
+            cand = np.arange(16)[None, :] * s + z
+            dist = np.abs(vd[sl][:, None] - cand)
+            best = dist.min(axis=1, keepdims=True)
+            ok = dist <= best
+            for i in range(32):
+                choices = np.nonzero(ok[i])[0]
+                want = choices[0] if len(choices) == 1 else [c for c in choices if c % 2 == 0][0]
+                assert q[32 * g + i] == want, (trial, g, i)
+            assert q[32 * g + int(np.argmin(vd[sl]))] == 0
+            assert q[32 * g + int(np.argmax(vd[sl]))] == 15
+
+
+def test_value_constant_group_is_exact(orc):
+    v = np.full(64, 3.25, np.float32)
+    q, s, z, _ = orc.encode_v(bf16_bits_of(v))
+    assert np.all(q == 0) and np.all(s == 0)
+    assert np.all(orc.decode_v(q, s, z) == 3.25)
+
+
+# ---------------------------------------------------------------- record format
+def test_record_size_and_nibble_order(orc):
+    g = {r[0]: r[1:] for r in read_golden("worked_examples.txt")}
+    assert orc.record_bytes(128) == 2336 and orc.record_bytes(64) == 1184
+    d = 128
+    K = np.zeros((1, 1, d), np.float32)
+    K[0, 0, 0] = 1.0
+    V = np.tile(np.arange(32, dtype=np.float32), 4).reshape(1, 1, d)
+    cache = np.zeros((2, 1, 2336), np.uint8)
+    rc, _, _ = orc.quantize_append(bf16_bits_of(K), bf16_bits_of(V), np.array([16 + 5], np.int32),
+                                   cache)
+    assert rc == 0
+    rec = cache[1, 0]
+    assert np.all(cache[0] == 0)
+    row = rec[5 * 64:6 * 64]
+    assert np.all(row == int(g["key_e0_byte"][0], 16))
+    assert int(rec[1024 + 10]) | (int(rec[1024 + 11]) << 8) == 0x3C00
+    vrow = rec[1056 + 5 * 64:1056 + 6 * 64]
+    want = [int(x, 16) for x in g["value_ramp_bytes"]]
+    assert list(vrow[:16]) == want and list(vrow[16:32]) == want
+    sz = rec[2080 + 5 * 16:2080 + 6 * 16]
+    assert int(sz[0]) | (int(sz[1]) << 8) == 0x4023 and int(sz[2]) | (int(sz[3]) << 8) == 0
+    # every other token row is untouched
+    mask = np.ones(2336, bool)
+    mask[5 * 64:6 * 64] = False
+    mask[1024 + 10:1024 + 12] = False
+    mask[1056 + 5 * 64:1056 + 6 * 64] = False
+    mask[2080 + 5 * 16:2080 + 6 * 16] = False
+    assert np.all(rec[mask] == 0)
+
+
+def _rand_kv(T, H, d, scale=1.0):
+    K = bf16_bits_of(RNG.standard_normal((T, H, d)) * scale)
+    V = bf16_bits_of(RNG.standard_normal((T, H, d)) * scale)
+    return K, V
+
+
+def test_append_slot_modes_and_skips_agree(orc):
+    H, d, nb = 2, 64, 6
+    K, V = _rand_kv(40, H, d)
+    rec = orc.record_bytes(d)
+    bt = np.array([[4, 1, 3], [0, 5, 2]], np.int32)
+    # 20 tokens for each of 2 sequences, logical slots; -1 skips token 7
+    logical = np.concatenate([np.arange(20), 48 + np.arange(20)]).astype(np.int32)
+    logical[7] = -1
+    phys = np.array([-1 if s < 0 else bt[s // 48, (s % 48) // 16] * 16 + s % 16 for s in logical],
+                    np.int32)
+    c1 = np.zeros((nb, H, rec), np.uint8)
+    c2 = np.zeros((nb, H, rec), np.uint8)
+    assert orc.quantize_append(K, V, logical, c1, block_table=bt)[0] == 0
+    assert orc.quantize_append(K, V, phys, c2)[0] == 0
+    assert np.array_equal(c1, c2)
+    # the skipped token's slot (block 4, offset 7) stays zero
+    assert np.all(c1[4, :, 7 * 32:8 * 32] == 0)
+
+
+def test_dequantize_invariant_to_physical_permutation(orc):
+    H, d, L = 2, 64, 70
+    K, V = _rand_kv(L, H, d)
+    rec = orc.record_bytes(d)
+    nblk = (L + 15) // 16
+    out = []
+    for perm in (np.arange(nblk), RNG.permutation(nblk)):
+        bt = perm.astype(np.int32)[None, :]
+        cache = np.zeros((nblk, H, rec), np.uint8)
+        orc.quantize_append(K, V, np.arange(L, dtype=np.int32), cache, block_table=bt)
+        out.append(orc.dequantize(cache, H, d, bt, np.array([L], np.int32), L))
+    assert np.array_equal(out[0][0], out[1][0]) and np.array_equal(out[0][1], out[1][1])
+
+
+# ---------------------------------------------------------------- attention
+def _attn_case(B=2, Hq=4, Hkv=2, d=64, L=37):
+    q = bf16_bits_of(RNG.standard_normal((B, Hq, d)))
+    Kh = RNG.standard_normal((B, L, Hkv, d))
+    Vh = RNG.standard_normal((B, L, Hkv, d))
+    return q, Kh, Vh
+
+
+def test_attention_matches_scipy_softmax(orc):
+    q, Kh, Vh = _attn_case()
+    B, Hq, d = q.shape
+    Hkv = Kh.shape[2]
+    lens = np.array([37, 11], np.int32)
+    out = orc.attention(q, Kh, Vh, lens, 0.125)
+    qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).double().numpy()
+    for b in range(B):
+        for h in range(Hq):
+            kv = h // (Hq // Hkv)
+            a = 0.125 * Kh[b, :lens[b], kv] @ qd[b, h]
+            ref = scipy.special.softmax(a) @ Vh[b, :lens[b], kv]
+            assert np.allclose(out[b, h], ref, atol=1e-13)
+
+
+def test_attention_special_cases(orc):
+    q, Kh, Vh = _attn_case(B=1, Hq=2, Hkv=1, L=9)
+    one = orc.attention(q, Kh, Vh, np.array([1], np.int32), 0.3)
+    assert np.allclose(one[0], Vh[0, 0, 0][None, :], atol=1e-15)      # one token -> its value
+    zero = orc.attention(q, Kh, Vh, np.array([9], np.int32), 0.0)
+    assert np.allclose(zero[0], Vh[0, :, 0].mean(axis=0)[None, :], atol=1e-14)  # uniform weights
+    Ks = np.repeat(Kh[:, :1], 9, axis=1)
+    same = orc.attention(q, Ks, Vh, np.array([9], np.int32), 1.0)
+    assert np.allclose(same[0], Vh[0, :, 0].mean(axis=0)[None, :], atol=1e-14)
+    Kd = np.zeros_like(Kh)
+    qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).double().numpy()
+    Kd[0, 4, 0] = 1000.0 * qd[0, 0] / np.linalg.norm(qd[0, 0])
+    dom = orc.attention(q[:, :1], Kd, Vh, np.array([9], np.int32), 1.0)
+    assert np.allclose(dom[0, 0], Vh[0, 4, 0], atol=1e-12)             # one dominant score
+    empty = orc.attention(q, Kh, Vh, np.array([0], np.int32), 1.0)
+    assert np.all(empty == 0.0)
+
+
+def test_attention_invariant_to_token_order(orc):
+    q, Kh, Vh = _attn_case(B=1, L=30)
+    p = RNG.permutation(30)
+    a = orc.attention(q, Kh, Vh, np.array([30], np.int32), 0.2)
+    b = orc.attention(q, Kh[:, p], Vh[:, p], np.array([30], np.int32), 0.2)
+    assert np.allclose(a, b, atol=1e-14)
+
+
+# ---------------------------------------------------------------- calibration
+def test_kmeans_table_lowers_mse_on_its_samples(orc):
+    d = 128
+    init = orc.default_table(d)
+    kb = bf16_bits_of(RNG.standard_t(4, (20, d)) * RNG.lognormal(0, 1, d))
+    y = orc.rotated_unit_samples(kb)
+    assert np.allclose(np.linalg.norm(y, axis=1), 1.0, atol=1e-14)
+    tab, it = orc.kmeans_table(y, init, 100)
+    assert np.all(np.diff(tab) > 0)
+
+    def mse(t):
+        t = t.astype(np.float64)
+        return np.mean(np.min((y.ravel()[:, None] - t[None, :]) ** 2, axis=1))
+
+    assert mse(tab) <= mse(init) * (1 + 1e-6)
+    # a k-means fixed point: refitting from the result changes nothing
+    tab2, it2 = orc.kmeans_table(y, tab, 100)
+    assert np.allclose(tab2, tab, atol=1e-7) and it2 <= 1
