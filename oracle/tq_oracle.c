@@ -235,11 +235,6 @@ int orc_encode_k(const uint16_t *k_bf16, int d, const float *table, uint8_t *idx
     if (!is_pow2(d) || !k_bf16 || !table || !idx || !norm16)
         return -1;
     double *k = malloc(sizeof(double) * d);
-    double *u = malloc(sizeof(double) * d);
-    double *y = malloc(sizeof(double) * d);
-    double *H = malloc(sizeof(double) * d * d);
-    orc_hadamard(d, H);
-
     double ss = 0.0;
     for (int i = 0; i < d; i++) {
         k[i] = orc_bf16_to_double(k_bf16[i]);
@@ -247,18 +242,22 @@ int orc_encode_k(const uint16_t *k_bf16, int d, const float *table, uint8_t *idx
     }
     double n = sqrt(ss);
     *norm16 = orc_fp16_from_double(n, 0);
-    for (int i = 0; i < d; i++)
-        u[i] = (n > 0.0) ? k[i] / n : 0.0;
-    hadamard_apply(d, H, u, y);
+    /* y = H_d (k / n) with H_d = S / sqrt(d), S the +-1 Sylvester matrix.
+     * The +-1 sums of bf16 values are exact in binary64, so S k is formed
+     * first and the single scale 1/(n sqrt(d)) is applied last: a coordinate
+     * that is exactly zero (or exactly on a midpoint) stays exact instead of
+     * being decided by the rounding noise of a division done beforehand. */
+    double denom = n * sqrt((double)d);
     for (int i = 0; i < d; i++) {
-        idx[i] = (uint8_t)nearest_centroid(y[i], table);
+        double acc = 0.0;
+        for (int j = 0; j < d; j++)
+            acc += (popcount_u32((unsigned)(i & j)) & 1) ? -k[j] : k[j];
+        double y = (n > 0.0) ? acc / denom : 0.0;
+        idx[i] = (uint8_t)nearest_centroid(y, table);
         if (y_out)
-            y_out[i] = y[i];
+            y_out[i] = y;
     }
     free(k);
-    free(u);
-    free(y);
-    free(H);
     return 0;
 }
 
@@ -587,24 +586,14 @@ int orc_rotated_unit_samples(const uint16_t *k_bf16, int n_vec, int d, double *o
 {
     if (!k_bf16 || !out || !is_pow2(d) || n_vec < 0)
         return -1;
-    double *H = malloc(sizeof(double) * d * d);
-    double *u = malloc(sizeof(double) * d);
-    orc_hadamard(d, H);
+    float dummy_table[16] = {0};
+    uint8_t *idx = malloc(d);
     for (int n = 0; n < n_vec; n++) {
-        double ss = 0.0;
-        for (int i = 0; i < d; i++) {
-            double v = orc_bf16_to_double(k_bf16[(size_t)n * d + i]);
-            ss += v * v;
-        }
-        double nrm = sqrt(ss);
-        for (int i = 0; i < d; i++) {
-            double v = orc_bf16_to_double(k_bf16[(size_t)n * d + i]);
-            u[i] = nrm > 0.0 ? v / nrm : 0.0;
-        }
-        hadamard_apply(d, H, u, out + (size_t)n * d);
+        uint16_t n16;
+        /* the same rotation as the key encoder; its codes are discarded */
+        orc_encode_k(k_bf16 + (size_t)n * d, d, dummy_table, idx, &n16, out + (size_t)n * d);
     }
-    free(H);
-    free(u);
+    free(idx);
     return 0;
 }
 

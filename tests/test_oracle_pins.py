@@ -158,6 +158,18 @@ def test_key_worked_example_e0(orc):
     assert np.max(np.abs(khat[1:])) < 1e-12
 
 
+def test_key_worked_example_exact_zero_ties_low(orc):
+    g = {r[0]: r[1:] for r in read_golden("worked_examples.txt")}
+    table = orc.default_table(128)
+    k = np.zeros(128, np.float32)
+    k[0] = k[1] = 1.0
+    idx, n16, y = orc.encode_k(bf16_bits_of(k), table)
+    assert n16 == int(g["key_e01_norm16"][0], 16)
+    assert np.all(idx[0::2] == int(g["key_e01_even_code"][0]))
+    assert np.all(y[1::2] == 0.0)
+    assert np.all(idx[1::2] == int(g["key_e01_odd_code"][0]))
+
+
 def test_key_zero_vector_ties_low(orc):
     table = orc.default_table(64)
     idx, n16, y = orc.encode_k(np.zeros(64, np.uint16), table)
