@@ -1,0 +1,397 @@
+"""Benchmark of the TQ4/4 hot path on B200: quantise-append + paged split-K decode.
+
+One step = one pass of the whole path over one batch of the Qwen3-8B-shaped
+layer workload (32 sequences x 8192 tokens, 32 query / 8 kv heads, d 128):
+tq_quantize_append of 32 new tokens per sequence (positions 8160..8191, so
+the cache state is the same every step) followed by tq_decode_attention of
+one query per sequence over all 8192 tokens.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl tq|reference]
+
+Rank 0 prints one JSON line.  value = quantised KV bytes the decode reads per
+step x steps / timed seconds (GB/s), over the whole step (append included),
+summed over ranks (each rank runs its own batch: weak scaling).  The cache
+(306 MB per rank) is larger than L2 (126 MB), so no L2 flush is needed.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+WORKLOAD = "qwen3_8b_layer"
+METRIC = "decode-attn quantised-KV GB/s & % of HBM peak; quantize-append tokens/s"
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def decode_bytes(w) -> int:
+    """Algorithmic bytes of one decode launch: the quantised records of every
+    valid token (record/16 per token-head), q, block tables read, output written."""
+    import bit_rotated_kv_tq_b200 as tq
+
+    rec = tq.record_bytes(w.d)
+    tokens = int(w.seq_lens.sum())
+    nblk = int(((w.seq_lens + 15) // 16).sum())
+    return tokens * w.Hkv * rec // 16 + w.B * w.Hq * w.d * 2 + nblk * 4 + w.B * w.Hq * w.d * 4
+
+
+def decode_kv_bytes(w) -> int:
+    import bit_rotated_kv_tq_b200 as tq
+
+    return int(w.seq_lens.sum()) * w.Hkv * tq.record_bytes(w.d) // 16
+
+
+def append_bytes(w, T) -> int:
+    import bit_rotated_kv_tq_b200 as tq
+
+    return T * w.Hkv * (2 * w.d * 2 + tq.record_bytes(w.d) // 16) + T * 4
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def smi_id(local: int) -> str:
+    """The nvidia-smi id (PCI bus id when torch exposes it) of local CUDA device `local`."""
+    props = torch.cuda.get_device_properties(local)
+    bus = getattr(props, "pci_bus_id", None)
+    if bus is not None and getattr(props, "pci_domain_id", None) is not None:
+        return f"{props.pci_domain_id:08x}:{bus:02x}:{getattr(props, 'pci_device_id', 0):02x}.0"
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+def dist_setup(n_gpus):
+    if n_gpus <= 1 or "RANK" not in os.environ:
+        return 0, 1, 0
+    import datetime
+
+    import torch.distributed as dist
+
+    local = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                            device_id=torch.device("cuda", local))
+    return dist.get_rank(), dist.get_world_size(), local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_sample(w, n_seqs: int):
+    """Prepare the oracle's cache for the first n_seqs sequences (untimed)."""
+    import oracle
+    from workloads import bf16_bits
+
+    oracle.build()
+    L = int(w.seq_lens[0])
+    nblk = (L + 15) // 16
+    cache = np.zeros((n_seqs * nblk, w.Hkv, oracle.record_bytes(w.d)), np.uint8)
+    bt = np.arange(n_seqs * nblk, dtype=np.int32).reshape(n_seqs, nblk)
+    kv = [w.kv(b) for b in range(n_seqs)]
+    Ks = np.concatenate([bf16_bits(k) for k, _ in kv])
+    Vs = np.concatenate([bf16_bits(v) for _, v in kv])
+    slots = np.concatenate([np.arange(L, dtype=np.int32) + b * nblk * 16 for b in range(n_seqs)])
+    rc, _, _ = oracle.quantize_append(Ks, Vs, slots, cache, block_table=bt)
+    assert rc == 0
+    app = [w.kv(b, L - w.append_tokens, L) for b in range(n_seqs)]
+    aK = np.concatenate([bf16_bits(k) for k, _ in app])
+    aV = np.concatenate([bf16_bits(v) for _, v in app])
+    aS = np.concatenate([np.arange(L - w.append_tokens, L, dtype=np.int32) + b * nblk * 16
+                         for b in range(n_seqs)])
+    q = bf16_bits(w.q()[:n_seqs])
+    return dict(cache=cache, bt=bt, lens=np.full(n_seqs, L, np.int32), L=L, aK=aK, aV=aV, aS=aS, q=q)
+
+
+def oracle_step(w, s):
+    """One oracle pass over the sample: append its new tokens, then decode."""
+    import oracle
+
+    oracle.quantize_append(s["aK"], s["aV"], s["aS"], s["cache"], block_table=s["bt"])
+    Kh, Vh = oracle.dequantize(s["cache"], w.Hkv, w.d, s["bt"], s["lens"], s["L"])
+    return oracle.attention(s["q"], Kh, Vh, s["lens"], w.scale)
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on a bounded sample."""
+    if rank != 0:
+        return
+    w = W.make(WORKLOAD)
+    n_seqs = 1
+    s = oracle_sample(w, n_seqs)
+    for _ in range(args.warmup):
+        oracle_step(w, s)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, s)
+    dt = time.perf_counter() - t0
+    kv_bytes = n_seqs * s["L"] * w.Hkv * (18 * w.d + 32) // 16
+    value = kv_bytes * args.steps / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": cfg(w, "oracle sample"),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{n_seqs} of {w.B} sequences (all 8 kv heads, 8192 tokens, "
+                                   f"32-token append) per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cfg(w, l2):
+    return {"workload": f"{w.name}: {w.B} seqs x {int(w.seq_lens[0])} tokens, {w.Hq} q / {w.Hkv} kv heads, "
+                        f"d {w.d}, block 16, shuffled block tables, {w.append_tokens}-token append per seq",
+            "global_batch": w.B, "seq_len": int(w.seq_lens[0]), "l2": l2}
+
+
+# ---------------------------------------------------------------- GPU arm
+def run_tq(args, rank, world, local):
+    import bit_rotated_kv_tq_b200 as tq
+
+    tq.load()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = W.make(WORKLOAD)
+    cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    lens = torch.from_numpy(w.seq_lens).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for K, V, slots in w.population():
+        tq.quantize_append(K.to(dev), V.to(dev), slots.to(dev), cache, block_table=bt, status=status)
+    aK, aV, aS = w.append_batch()
+    aK, aV, aS = aK.to(dev), aV.to(dev), aS.to(dev)
+    q = w.q().to(dev)
+    max_len = int(w.seq_lens.max())
+    S = tq.default_splits(w.B, w.Hkv, max_len)
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, tq.workspace_bytes(w.B, w.Hq, w.d, S)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    T = aK.shape[0]
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        tq.quantize_append(aK, aV, aS, cache, block_table=bt, status=status, stream=stream)
+        if ev:
+            ev[1].record(stream)
+        tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws, num_splits=S,
+                            status=status, stream=stream)
+        if ev:
+            ev[2].record(stream)
+
+    torch.cuda.synchronize(dev)
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(smi_id(local)) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = start.elapsed_time(end)
+    app_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = max_over_ranks(total_ms, world)
+    dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
+    app_avg = max_over_ranks(sum(app_ms) / len(app_ms), world)
+
+    # end to end through the same public calls with host buffers
+    h_q = w.q().pin_memory()
+    h_K, h_V, h_S = aK.cpu().pin_memory(), aV.cpu().pin_memory(), aS.cpu().pin_memory()
+    h_out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32).pin_memory()
+    d_q, d_K, d_V, d_S = torch.empty_like(q), torch.empty_like(aK), torch.empty_like(aV), torch.empty_like(aS)
+
+    def e2e_step():
+        d_q.copy_(h_q, non_blocking=True)
+        d_K.copy_(h_K, non_blocking=True)
+        d_V.copy_(h_V, non_blocking=True)
+        d_S.copy_(h_S, non_blocking=True)
+        tq.quantize_append(d_K, d_V, d_S, cache, block_table=bt, status=status, stream=stream)
+        tq.decode_attention(d_q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws, num_splits=S,
+                            status=status, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+        stream.synchronize()
+
+    for _ in range(3):
+        e2e_step()
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    e2e_s = max_over_ranks(time.perf_counter() - t0, world)
+    h2d = h_q.numel() * 2 + h_K.numel() * 2 + h_V.numel() * 2 + h_S.numel() * 4
+    d2h = h_out.numel() * 4
+
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+
+    kv = decode_kv_bytes(w)
+    value = world * kv * args.steps / (total_ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+    dec_bytes = decode_bytes(w)
+    achieved = dec_bytes / (dec_avg / 1e3) / 1e9
+    clocks = clk.summary()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s = oracle_sample(w, 1)
+        oracle_step(w, s)
+        n_rep = 3
+        t0 = time.perf_counter()
+        for _ in range(n_rep):
+            oracle_step(w, s)
+        dt = (time.perf_counter() - t0) / n_rep
+        cpu = {"value": s["L"] * w.Hkv * tq.record_bytes(w.d) // 16 / dt / 1e9, "unit": "GB/s", "cores": 1,
+               "kind": "oracle",
+               "sample": f"1 of {w.B} sequences (8 kv heads x {s['L']} tokens + {w.append_tokens}-token append), "
+                         f"{n_rep} passes, {dt:.2f} s each"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": cfg(w, "inputs larger than L2: 306 MB cache per rank vs 126 MB L2, no flush"),
+            "decode_gbs": kv / (dec_avg / 1e3) / 1e9,
+            "decode_hbm_frac": kv / (dec_avg / 1e3) / 1e9 / peak,
+            "decode_ms": dec_avg, "append_ms": app_avg,
+            "append_tokens_per_s": T / (app_avg / 1e3),
+            "append_hbm_frac": append_bytes(w, T) / (app_avg / 1e3) / 1e9 / peak,
+            "num_splits": S,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "kernel": "tq_decode_attention (split kernel + combine)",
+                         "peak_source": f"{peak_kind} hbm_gbs"},
+            "e2e": {"value": world * kv * args.steps / e2e_s / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * (2 + (1 if S > 1 else 0)),
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", 0))
+        world = int(os.environ.get("WORLD_SIZE", args.gpus))
+        run_reference(args, rank, world)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_tq(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,215 @@
+"""Python binding of the TQ4/4 C-ABI library (include/tq.h) for B200.
+
+Argument marshalling only: every step of the append / decode / dequantise
+path runs in the CUDA kernels of ``libtq_b200.so``.  PyTorch supplies device
+memory and the current stream.  There is no fallback: if the shared library
+is missing, every call raises.
+
+Method: "TurboQuant 在 AMD GPU 上把長上下文延遲壓下來" (TQ4/4: Walsh-Hadamard-
+rotated keys with a 16-entry table, uniform 4-bit values) and
+"UltraQuant：4-bit KV 快取加速長代理" (Lloyd-Max or re-fitted centroid table).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
+
+BLOCK = 16
+VALUE_GROUP = 32
+
+TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_ALIGNMENT, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(6)
+STATUS_BAD_SLOT, STATUS_BAD_BLOCK, STATUS_RANGE, STATUS_BAD_LEN = 1, 2, 4, 8
+
+
+class TQError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"tq error {code}: {msg}")
+        self.code = code
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("data", ctypes.c_void_p)]
+
+
+_lib = None
+_P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+def load(path: str | None = None):
+    """Load the shared library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: run `python bit_rotated_kv_tq_b200/build.py`")
+    L = ctypes.CDLL(p)
+    L.tq_record_bytes.restype = _Z
+    L.tq_record_bytes.argtypes = [_I]
+    L.tq_cache_bytes.restype = _Z
+    L.tq_cache_bytes.argtypes = [_I, _I, _I]
+    L.tq_lloyd_max_table.argtypes = [_I, _P]
+    L.tq_fit_k_table.argtypes = [_P, _I, _I, _P, _I, _P]
+    L.tq_quantize_append.argtypes = [_P, _P, _P, _I, _I, _P, _I, ctypes.POINTER(_Cache), _P, _P, _P]
+    L.tq_decode_default_splits.argtypes = [_I, _I, _I]
+    L.tq_decode_workspace_bytes.restype = _Z
+    L.tq_decode_workspace_bytes.argtypes = [_I, _I, _I, _I]
+    L.tq_decode_attention.argtypes = [_P, ctypes.POINTER(_Cache), _P, _P, _I, _P, _I, _I, _I, _F,
+                                      _P, _P, _Z, _I, _P, _P]
+    L.tq_dequantize.argtypes = [ctypes.POINTER(_Cache), _P, _P, _I, _P, _I, _I, _P, _P, _P, _P]
+    L.tq_last_error.restype = ctypes.c_char_p
+    L.tq_last_error.argtypes = []
+    _lib = L
+    return L
+
+
+def _check(rc: int):
+    if rc != TQ_OK:
+        raise TQError(rc, load().tq_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dtype, name):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+# ------------------------------------------------------------------ sizes, tables
+def record_bytes(head_dim: int) -> int:
+    return int(load().tq_record_bytes(head_dim))
+
+
+def lloyd_max_table(head_dim: int) -> np.ndarray:
+    out = np.zeros(16, np.float32)
+    _check(load().tq_lloyd_max_table(head_dim, out.ctypes.data_as(_P)))
+    return out
+
+
+def fit_k_table(keys: torch.Tensor, init: np.ndarray, max_iter: int = 100):
+    """keys: bf16 [n][d] (host); returns (fp32[16] table, iterations)."""
+    k = keys.detach().to("cpu").contiguous()
+    if k.dtype != torch.bfloat16 or k.dim() != 2:
+        raise ValueError("keys must be a 2-D bf16 tensor")
+    bits = k.view(torch.int16).numpy().view(np.uint16)
+    init = np.ascontiguousarray(init, np.float32)
+    out = np.zeros(16, np.float32)
+    rc = load().tq_fit_k_table(bits.ctypes.data_as(_P), k.shape[0], k.shape[1],
+                               init.ctypes.data_as(_P), max_iter, out.ctypes.data_as(_P))
+    if rc < 0:
+        _check(-rc)
+    return out, rc
+
+
+# ------------------------------------------------------------------ cache
+class Cache:
+    """A paged TQ4/4 cache: uint8 [num_blocks][num_kv_heads][record] in device memory."""
+
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, device="cuda", data=None):
+        nbytes = int(load().tq_cache_bytes(num_blocks, num_kv_heads, head_dim))
+        if nbytes == 0:
+            raise TQError(TQ_ERR_UNSUPPORTED, f"cache shape ({num_blocks}, {num_kv_heads}, {head_dim})")
+        rec = record_bytes(head_dim)
+        if data is None:
+            data = torch.zeros((num_blocks, num_kv_heads, rec), dtype=torch.uint8, device=device)
+        if tuple(data.shape) != (num_blocks, num_kv_heads, rec) or data.dtype != torch.uint8:
+            raise ValueError("cache data has the wrong shape or dtype")
+        self.data = data
+        self.num_blocks, self.num_kv_heads, self.head_dim = num_blocks, num_kv_heads, head_dim
+        self._c = _Cache(num_blocks, num_kv_heads, head_dim, 0, data.data_ptr())
+
+    @property
+    def c(self):
+        self._c.data = self.data.data_ptr()
+        return ctypes.byref(self._c)
+
+
+# ------------------------------------------------------------------ hot calls
+def quantize_append(K, V, slot_mapping, cache: Cache, block_table=None, k_tables=None,
+                    status=None, stream=None):
+    """Quantise K, V (bf16 [T][H_kv][d], CUDA) into `cache` at `slot_mapping` (int32 [T]).
+
+    With block_table (int32 [num_seqs][max_blocks]) the slots are logical:
+    seq * max_blocks * 16 + position.
+    """
+    _dev(K, torch.bfloat16, "K")
+    _dev(V, torch.bfloat16, "V")
+    _dev(slot_mapping, torch.int32, "slot_mapping")
+    _dev(block_table, torch.int32, "block_table")
+    _dev(k_tables, torch.float32, "k_tables")
+    _dev(status, torch.int32, "status")
+    T = K.shape[0]
+    ns, mb = (0, 0) if block_table is None else (block_table.shape[0], block_table.shape[1])
+    _check(load().tq_quantize_append(_ptr(K), _ptr(V), _ptr(block_table), ns, mb, _ptr(slot_mapping),
+                                     T, cache.c, _ptr(k_tables), _ptr(status), _stream(stream)))
+
+
+def default_splits(B: int, H_kv: int, max_seq_len: int) -> int:
+    return int(load().tq_decode_default_splits(B, H_kv, max_seq_len))
+
+
+def workspace_bytes(B: int, H_q: int, head_dim: int, num_splits: int) -> int:
+    return int(load().tq_decode_workspace_bytes(B, H_q, head_dim, num_splits))
+
+
+def decode_attention(q, cache: Cache, block_tables, seq_lens, max_seq_len: int, scale: float,
+                     out=None, workspace=None, num_splits: int = 0, k_tables=None, status=None,
+                     stream=None):
+    """Split-K decode attention over the compressed cache; returns fp32 [B][H_q][d]."""
+    _dev(q, torch.bfloat16, "q")
+    _dev(block_tables, torch.int32, "block_tables")
+    _dev(seq_lens, torch.int32, "seq_lens")
+    _dev(k_tables, torch.float32, "k_tables")
+    _dev(status, torch.int32, "status")
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _dev(out, torch.float32, "out")
+    S = num_splits or default_splits(B, cache.num_kv_heads, max_seq_len)
+    if workspace is None:
+        nb = workspace_bytes(B, Hq, d, S)
+        workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=q.device)
+    _check(load().tq_decode_attention(_ptr(q), cache.c, _ptr(k_tables), _ptr(block_tables),
+                                      block_tables.shape[1], _ptr(seq_lens), B, Hq, int(max_seq_len),
+                                      float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                      int(num_splits), _ptr(status), _stream(stream)))
+    return out
+
+
+def dequantize(cache: Cache, block_tables, seq_lens, max_len: int, k_tables=None, status=None,
+               stream=None):
+    """(K_hat, V_hat) fp32 [B][max_len][H_kv][d] in the original domain (checks only)."""
+    _dev(block_tables, torch.int32, "block_tables")
+    _dev(seq_lens, torch.int32, "seq_lens")
+    _dev(k_tables, torch.float32, "k_tables")
+    _dev(status, torch.int32, "status")
+    B = block_tables.shape[0]
+    shape = (B, max_len, cache.num_kv_heads, cache.head_dim)
+    Kh = torch.empty(shape, dtype=torch.float32, device=block_tables.device)
+    Vh = torch.empty(shape, dtype=torch.float32, device=block_tables.device)
+    _check(load().tq_dequantize(cache.c, _ptr(k_tables), _ptr(block_tables), block_tables.shape[1],
+                                _ptr(seq_lens), B, max_len, _ptr(Kh), _ptr(Vh), _ptr(status),
+                                _stream(stream)))
+    return Kh, Vh

@@ -1,0 +1,68 @@
+// tq_common.cuh -- record layout and small device helpers shared by the
+// TQ4/4 kernels (append, decode, combine, dequantise).
+//
+// Record of one (physical block, kv head), 16 tokens, head_dim D:
+//   [0, 8D)         key codes    [16][D/2] bytes, element 2j in the low nibble of byte j
+//   [8D, 8D+32)     key norms    [16] fp16
+//   [8D+32, 16D+32) value codes  [16][D/2] bytes
+//   [16D+32, 18D+32) value groups [16][D/32] x (fp16 scale, fp16 zero)
+// The cache is [num_blocks][H_kv][record]; every field starts 16-byte aligned.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/tq.h"
+
+namespace tq {
+
+constexpr int kBlock = 16;  // tokens per cache block
+constexpr int kGroup = 32;  // value elements per scale/zero group
+constexpr unsigned kFull = 0xffffffffu;
+
+template <int D>
+struct Rec {
+    static constexpr int kCodeRow = D / 2;                 // bytes of one token's codes
+    static constexpr int kKCodes = 0;
+    static constexpr int kKNorm = kBlock * kCodeRow;        // 8D
+    static constexpr int kVCodes = kKNorm + 2 * kBlock;     // 8D + 32
+    static constexpr int kVGroups = kVCodes + kBlock * kCodeRow;  // 16D + 32
+    static constexpr int kGroups = D / kGroup;
+    static constexpr int kBytes = kVGroups + kBlock * kGroups * 4;  // 18D + 32
+    static_assert(kKNorm % 16 == 0 && kVCodes % 16 == 0 && kVGroups % 16 == 0 &&
+                      kBytes % 16 == 0,
+                  "record fields must stay 16-byte aligned");
+};
+
+// bf16 pair (packed in a uint32, element 0 in the low half) -> two floats, exact
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
+    return __half2float(__ushort_as_half(h));
+}
+
+// streaming 16-byte read-only load (inputs are read once)
+__device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ void flag_status(int32_t* status, int bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// Correctly rounded double -> fp16 toward +infinity, for x >= 0.
+__device__ __forceinline__ uint16_t double_to_half_up_nonneg(double x) {
+    __half h = __double2half(x);  // round to nearest even
+    uint16_t b = __half_as_ushort(h);
+    if ((double)__half2float(h) < x) b = (uint16_t)(b + 1);  // next representable above
+    return b;
+}
+
+}  // namespace tq

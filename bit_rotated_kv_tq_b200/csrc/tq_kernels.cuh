@@ -1,0 +1,60 @@
+// tq_kernels.cuh -- argument blocks and launchers of the TQ4/4 kernels
+// (internal to the library; the public interface is include/tq.h).
+#pragma once
+
+#include "tq_common.cuh"
+
+namespace tq {
+
+struct AppendArgs {
+    const uint16_t* K;          // bf16 [T][Hkv][D]
+    const uint16_t* V;          // bf16 [T][Hkv][D]
+    const int32_t* block_table; // [num_seqs][max_blocks] or null
+    int num_seqs, max_blocks;
+    const int32_t* slots;       // [T]
+    int T;
+    unsigned char* cache;
+    int num_blocks, Hkv;
+    const float* k_tables;      // [Hkv][16] or null
+    float default_table[16];
+    int32_t* status;
+};
+
+struct DecodeArgs {
+    const uint16_t* q;           // bf16 [B][Hq][D]
+    const unsigned char* cache;  // [num_blocks][Hkv][record]
+    int num_blocks, Hkv, Hq, B;
+    const float* k_tables;       // [Hkv][16] or null
+    float default_table[16];
+    const int32_t* block_tables; // [B][max_blocks]
+    int max_blocks;
+    const int32_t* seq_lens;     // [B]
+    float scale_log2;            // scale * log2(e)
+    float* out;                  // [B][Hq][D]
+    float* ws_o;                 // [B][Hq][S][D] partial outputs (unnormalised)
+    float2* ws_ml;               // [B][Hq][S] (running max in log2 units, sum)
+    int num_splits;
+    int blocks_per_split;
+    int32_t* status;
+};
+
+struct DequantArgs {
+    const unsigned char* cache;
+    int num_blocks, Hkv;
+    const float* k_tables;
+    float default_table[16];
+    const int32_t* block_tables;
+    int max_blocks;
+    const int32_t* seq_lens;
+    int B, max_len;
+    float* K_hat;  // [B][max_len][Hkv][D]
+    float* V_hat;
+    int32_t* status;
+};
+
+size_t append_smem_bytes(int Hkv);
+cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, int head_dim, cudaStream_t stream);
+cudaError_t launch_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);
+
+}  // namespace tq

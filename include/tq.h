@@ -1,0 +1,162 @@
+/*
+ * tq.h -- C ABI of the TQ4/4 KV-cache library for NVIDIA B200 (sm_100a).
+ *
+ * TQ4/4 keeps 4-bit keys and 4-bit values ("TurboQuant 在 AMD GPU 上把長上下文
+ * 延遲壓下來", summary table and section 2):
+ *   key   : rotated by the normalised Walsh-Hadamard transform over head_dim
+ *           (section 4 of that page), stored as an fp16 L2 norm plus a 4-bit
+ *           index per element into a 16-entry centroid table (the Lloyd-Max
+ *           table, or one re-fitted on ~20 rotated vectors: "UltraQuant：4-bit
+ *           KV 快取加速長代理", section 「方法怎麼做，白話講」);
+ *   value : asymmetric uniform 4-bit codes with one fp16 scale and one fp16
+ *           zero point per group of 32 elements (section 2: "standard
+ *           uniform quantization").
+ * Both live in a paged cache of 16-token blocks.
+ *
+ * Conventions for every call below:
+ *   - Pointers marked (device) are CUDA device pointers owned by the caller;
+ *     the library never allocates, frees or synchronises inside a hot call.
+ *     Pointers marked (host) are ordinary host memory.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); work is
+ *     enqueued asynchronously on it.
+ *   - Return value: TQ_OK, or a TQ_ERR_* code after which nothing was
+ *     enqueued; tq_last_error() then gives a message (per calling thread).
+ *   - `status` (device, may be NULL) is one int32 that kernels OR TQ_STATUS_*
+ *     bits into when they meet bad data they cannot check on the host (a
+ *     block id out of range, ...).  The caller zeroes it and reads it back
+ *     whenever it likes.  Kernels never trap; a flagged element is skipped.
+ *   - bf16/fp16 arrays are raw 16-bit IEEE patterns; all arrays are dense,
+ *     row-major, with the shapes given.
+ *
+ * Cache record: one per (physical block, kv head), 16 tokens, 16-byte
+ * aligned fields, little-endian, element 2j in the low nibble of byte j:
+ *   [0,      8d)        key codes    [16][d/2] bytes
+ *   [8d,     8d+32)     key norms    [16] fp16
+ *   [8d+32,  16d+32)    value codes  [16][d/2] bytes
+ *   [16d+32, 18d+32)    value groups [16][d/32] x (fp16 scale, fp16 zero)
+ * = 2336 bytes at d = 128, 1184 bytes at d = 64.  The cache is
+ * [num_blocks][num_kv_heads][record].
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#define TQ_BLOCK_TOKENS 16
+#define TQ_VALUE_GROUP 32
+
+enum {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1, /* null pointer, negative size, inconsistent shape */
+    TQ_ERR_UNSUPPORTED = 2, /* head_dim not 64/128, H_q % H_kv != 0, too many splits */
+    TQ_ERR_ALIGNMENT = 3,   /* a pointer misses its required alignment */
+    TQ_ERR_CUDA = 4,        /* a CUDA runtime call failed (message has the CUDA error) */
+    TQ_ERR_WORKSPACE = 5    /* workspace pointer NULL or smaller than required */
+};
+
+/* device status bits */
+enum {
+    TQ_STATUS_BAD_SLOT = 1,  /* append: slot or logical slot outside the cache / table */
+    TQ_STATUS_BAD_BLOCK = 2, /* a block-table entry outside [0, num_blocks) */
+    TQ_STATUS_RANGE = 4,     /* a key norm or value scale/zero overflowed fp16 */
+    TQ_STATUS_BAD_LEN = 8    /* seq_len < 0 or > max_blocks * 16 (treated as 0) */
+};
+
+typedef struct {
+    int32_t num_blocks;   /* physical 16-token blocks */
+    int32_t num_kv_heads; /* H_kv */
+    int32_t head_dim;     /* d: 64 or 128 */
+    int32_t reserved;     /* must be 0 */
+    void* data;           /* (device) [num_blocks][num_kv_heads][record], 16-byte aligned */
+} tq_cache_t;
+
+/* Bytes of one (block, kv head) record (2336 at d=128, 1184 at d=64); 0 if d unsupported. */
+TQ_API size_t tq_record_bytes(int head_dim);
+/* Bytes of a whole cache; 0 on an unsupported shape. */
+TQ_API size_t tq_cache_bytes(int num_blocks, int num_kv_heads, int head_dim);
+
+/* (host) Default key table for head_dim d: the 16-level Lloyd-Max quantiser of
+ * N(0,1) scaled by 1/sqrt(d) (the rotated unit vector has coordinates of
+ * variance 1/d), rounded to fp32, ascending.  "UltraQuant：4-bit KV 快取加速
+ * 長代理", 「方法怎麼做，白話講」: the theoretical Lloyd-Max centroid table. */
+TQ_API int tq_lloyd_max_table(int head_dim, float out16[16]);
+
+/* (host) Re-fit a 16-entry key table on n calibration key vectors (bf16
+ * [n][head_dim], host): rotate each unit-normalised vector, then run 1-D
+ * k-means (Lloyd) from init16 for at most max_iter rounds; empty cells keep
+ * their level; the result is sorted and rounded to fp32.  Same page and
+ * section: centroids re-fitted on about 20 rotated vectors.  Returns the
+ * iteration count (>= 0) or -TQ_ERR_*. */
+TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim, const float init16[16],
+                   int max_iter, float out16[16]);
+
+/* Quantise T new tokens and write them into the cache (the TQ4/4 write path).
+ *   K, V        (device) bf16 [T][H_kv][d], 16-byte aligned
+ *   block_table (device, may be NULL) int32 [num_seqs][max_blocks]
+ *   slot_mapping(device) int32 [T]:
+ *       block_table == NULL: physical slot = block * 16 + offset;
+ *       block_table != NULL: logical slot = seq * (max_blocks * 16) + position,
+ *                            mapped to block_table[seq][position / 16];
+ *       -1 skips the token.
+ *   k_tables    (device, may be NULL) fp32 [H_kv][16] strictly ascending
+ *               per-head key tables; NULL = tq_lloyd_max_table(d) for all heads.
+ * Slots outside the cache set TQ_STATUS_BAD_SLOT / _BAD_BLOCK and are skipped.
+ * Two tokens mapped to one slot race (last writer wins, per field). */
+TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block_table, int num_seqs,
+                       int max_blocks, const int32_t* slot_mapping, int T,
+                       const tq_cache_t* cache, const float* k_tables, int32_t* status,
+                       void* stream);
+
+/* Number of context splits tq_decode_attention uses when num_splits == 0. */
+TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len);
+/* Workspace bytes for tq_decode_attention with this many splits (fp32 partial
+ * outputs and softmax statistics per (sequence, query head, split)). */
+TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_splits);
+
+/* Decode attention over the compressed cache, one query per sequence:
+ *   out[b][h] = sum_t softmax_t(scale * <q[b][h], k_hat_t>) * v_hat_t,
+ * t < seq_lens[b], with the keys/values the cache holds for kv head
+ * h / (H_q / H_kv).  The query is rotated by the same Hadamard transform
+ * once, so scores are computed in the rotated domain against the stored
+ * centroids; K and V are dequantised in registers and never written out.
+ *   q            (device) bf16 [B][H_q][d]
+ *   block_tables (device) int32 [B][max_blocks]
+ *   seq_lens     (device) int32 [B], each in [0, max_blocks*16]
+ *   max_seq_len  (host)   upper bound of seq_lens (sizes the split grid); a
+ *                         longer seq_len sets TQ_STATUS_BAD_LEN and is cut
+ *   out          (device) fp32 [B][H_q][d]; a sequence of length 0 gets 0
+ *   workspace    (device) >= tq_decode_workspace_bytes(...), 16-byte aligned
+ *   num_splits   0 = tq_decode_default_splits(...), else 1..1024
+ * Splits of one sequence are merged by a log-sum-exp combine kernel. */
+TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const float* k_tables,
+                        const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                        int B, int H_q, int max_seq_len, float scale, float* out,
+                        void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
+                        void* stream);
+
+/* Dequantise every valid token (checks only): K_hat and V_hat (device) fp32
+ * [B][max_len][H_kv][d] in the original (unrotated) domain,
+ * k_hat = fp16 norm * H * C[idx],  v_hat = code * scale + zero;
+ * rows at or past seq_lens[b] are written as 0. */
+TQ_API int tq_dequantize(const tq_cache_t* cache, const float* k_tables, const int32_t* block_tables,
+                  int max_blocks, const int32_t* seq_lens, int B, int max_len, float* K_hat,
+                  float* V_hat, int32_t* status, void* stream);
+
+/* Message of the last failing call on this thread ("" if none). */
+TQ_API const char* tq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

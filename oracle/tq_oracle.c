@@ -200,6 +200,21 @@ int orc_hadamard(int d, double *H)
     return 0;
 }
 
+/* The dense normalised matrix of the most recent d, built once by orc_hadamard
+ * (the oracle is single-threaded; rebuilding it for every vector only costs time). */
+static const double *hadamard_cached(int d)
+{
+    static double *H = NULL;
+    static int Hd = 0;
+    if (Hd != d) {
+        free(H);
+        H = malloc(sizeof(double) * d * d);
+        orc_hadamard(d, H);
+        Hd = d;
+    }
+    return H;
+}
+
 /* y = H x with the dense matrix (deliberately not a fast transform) */
 static void hadamard_apply(int d, const double *H, const double *x, double *y)
 {
@@ -248,10 +263,11 @@ int orc_encode_k(const uint16_t *k_bf16, int d, const float *table, uint8_t *idx
      * that is exactly zero (or exactly on a midpoint) stays exact instead of
      * being decided by the rounding noise of a division done beforehand. */
     double denom = n * sqrt((double)d);
+    const double *Hs = hadamard_cached(d); /* only its signs are used here */
     for (int i = 0; i < d; i++) {
         double acc = 0.0;
         for (int j = 0; j < d; j++)
-            acc += (popcount_u32((unsigned)(i & j)) & 1) ? -k[j] : k[j];
+            acc += (Hs[(size_t)i * d + j] < 0.0) ? -k[j] : k[j];
         double y = (n > 0.0) ? acc / denom : 0.0;
         idx[i] = (uint8_t)nearest_centroid(y, table);
         if (y_out)
@@ -266,8 +282,7 @@ int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const float *table,
     if (!is_pow2(d) || !idx || !table || !k_hat)
         return -1;
     double *c = malloc(sizeof(double) * d);
-    double *H = malloc(sizeof(double) * d * d);
-    orc_hadamard(d, H);
+    const double *H = hadamard_cached(d);
     double n = orc_fp16_to_double(norm16);
     for (int i = 0; i < d; i++)
         c[i] = (double)table[idx[i] & 15];
@@ -276,7 +291,6 @@ int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const float *table,
     for (int i = 0; i < d; i++)
         k_hat[i] *= n;
     free(c);
-    free(H);
     return 0;
 }
 

@@ -1,0 +1,106 @@
+"""Test-side helpers: read the documented TQ4/4 record layout and compare the
+GPU path with the oracle under the parity rule.
+
+Parity rule (the TQ4/4 statement of what must match):
+  - packed codes bit-exact, except elements whose oracle decision input lies
+    within 1e-6 of a decision threshold (a centroid midpoint for keys, a .5
+    rounding point of (v - z)/s for values); such mismatches are counted and
+    must be at most 1e-5 of all elements;
+  - fp16 norms, scales and zero points exact, except a norm within 1e-6
+    (relative) of an fp16 rounding midpoint (counted the same way);
+  - attention within max-abs 2e-3 and rel-L2 1e-3 of the oracle's fp64
+    attention over its own dequantised K/V.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+CODE_TOL = 1e-6
+COUNT_TOL = 1e-5
+ATTN_MAX_ABS = 2e-3
+ATTN_REL_L2 = 1e-3
+
+
+def layout(d):
+    row = d // 2
+    kn = 16 * row
+    vc = kn + 32
+    vg = vc + 16 * row
+    return row, kn, vc, vg, vg + 16 * (d // 32) * 4
+
+
+def unpack_record(rec: np.ndarray, d: int):
+    """rec uint8 [record] -> kidx [16][d], knorm uint16 [16], vq [16][d], vs, vz uint16 [16][d/32]."""
+    row, kn, vc, vg, total = layout(d)
+    assert rec.shape[-1] == total
+    kc = rec[..., :kn].reshape(rec.shape[:-1] + (16, row))
+    kidx = np.stack([kc & 15, kc >> 4], axis=-1).reshape(rec.shape[:-1] + (16, d))
+    knorm = rec[..., kn:kn + 32].copy().view(np.uint16).reshape(rec.shape[:-1] + (16,))
+    vcb = rec[..., vc:vc + 16 * row].reshape(rec.shape[:-1] + (16, row))
+    vq = np.stack([vcb & 15, vcb >> 4], axis=-1).reshape(rec.shape[:-1] + (16, d))
+    sz = rec[..., vg:total].copy().view(np.uint16).reshape(rec.shape[:-1] + (16, d // 32, 2))
+    return kidx, knorm, vq, sz[..., 0], sz[..., 1]
+
+
+def key_boundary_distance(ky: np.ndarray, table: np.ndarray) -> np.ndarray:
+    """Distance of each rotated unit coordinate to the nearest fp64 midpoint of the table."""
+    t = table.astype(np.float64)
+    mids = 0.5 * (t[:-1] + t[1:])
+    return np.min(np.abs(ky[..., None] - mids), axis=-1)
+
+
+def value_boundary_distance(vr: np.ndarray) -> np.ndarray:
+    return np.abs(vr - (np.floor(vr) + 0.5))
+
+
+def fp16_midpoint_rel_distance(n: np.ndarray) -> np.ndarray:
+    """Relative distance of a positive norm to the nearest fp16 rounding midpoint."""
+    n = np.asarray(n, np.float64)
+    h = n.astype(np.float16).astype(np.float64)
+    up = np.nextafter(n.astype(np.float16), np.float16(np.inf)).astype(np.float64)
+    dn = np.nextafter(n.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
+    mids = np.stack([(h + up) / 2, (h + dn) / 2], axis=-1)
+    return np.min(np.abs(mids - n[..., None]), axis=-1) / np.maximum(n, 1e-300)
+
+
+class CodeReport:
+    def __init__(self):
+        self.elements = 0
+        self.mismatch = 0
+        self.far_mismatch = 0
+        self.notes = []
+
+    def add(self, got, want, dist, what):
+        got = np.asarray(got)
+        want = np.asarray(want)
+        bad = got != want
+        self.elements += got.size
+        n = int(bad.sum())
+        self.mismatch += n
+        if n:
+            far = bad & (np.broadcast_to(dist, got.shape) >= CODE_TOL)
+            nf = int(far.sum())
+            self.far_mismatch += nf
+            self.notes.append(f"{what}: {n} mismatches ({nf} not near a threshold)")
+
+    def check(self):
+        assert self.far_mismatch == 0, "; ".join(self.notes)
+        assert self.mismatch <= COUNT_TOL * max(1, self.elements), \
+            f"{self.mismatch} near-threshold mismatches of {self.elements}: " + "; ".join(self.notes)
+        return self.mismatch
+
+
+def attn_errors(got: np.ndarray, want: np.ndarray):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    max_abs = float(np.max(np.abs(got - want))) if got.size else 0.0
+    den = float(np.linalg.norm(want))
+    rel = float(np.linalg.norm(got - want) / den) if den > 0 else float(np.linalg.norm(got - want))
+    return max_abs, rel
+
+
+def check_attention(got, want, what=""):
+    max_abs, rel = attn_errors(got, want)
+    assert max_abs <= ATTN_MAX_ABS and rel <= ATTN_REL_L2, \
+        f"{what}: max-abs {max_abs:.3e} (<= {ATTN_MAX_ABS}), rel-L2 {rel:.3e} (<= {ATTN_REL_L2})"
+    return max_abs, rel

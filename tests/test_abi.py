@@ -1,0 +1,124 @@
+"""Host-side checks of the C-ABI library: it loads, exports every symbol that
+include/tq.h declares, and its host-only routines (tables, sizes, argument
+validation) behave as documented.  No call here launches GPU work."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import bit_rotated_kv_tq_b200 as tq
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "tq.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_rotated_kv_tq_b200 import build
+
+    build.build()
+    return tq.load()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"TQ_API\s+[\w\s\*]+?\b(tq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_symbols()
+    for want in ("tq_quantize_append", "tq_decode_attention", "tq_dequantize", "tq_last_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+        assert isinstance(getattr(lib, name), ctypes._CFuncPtr)
+
+
+def test_record_and_cache_sizes(lib, orc):
+    for d in (64, 128):
+        assert tq.record_bytes(d) == orc.record_bytes(d)
+        assert lib.tq_cache_bytes(10, 3, d) == 30 * orc.record_bytes(d)
+    assert tq.record_bytes(96) == 0 and lib.tq_cache_bytes(0, 1, 64) == 0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_default_table_equals_oracle(lib, orc, d):
+    assert np.array_equal(tq.lloyd_max_table(d), orc.default_table(d))
+
+
+def test_default_table_other_power_of_two(lib, orc):
+    assert np.array_equal(tq.lloyd_max_table(256), orc.default_table(256))
+    with pytest.raises(tq.TQError):
+        tq.lloyd_max_table(96)
+
+
+def test_fit_k_table_equals_oracle(lib, orc):
+    rng = np.random.default_rng(7)
+    for d in (64, 128):
+        keys = torch.from_numpy((rng.standard_t(4, (20, d)) * rng.lognormal(0, 1, d)).astype(np.float32))
+        keys = keys.to(torch.bfloat16)
+        init = orc.default_table(d)
+        got, it = tq.fit_k_table(keys, init, 100)
+        bits = keys.view(torch.int16).numpy().view(np.uint16)
+        want, it2 = orc.kmeans_table(orc.rotated_unit_samples(bits), init, 100)
+        assert np.array_equal(got, want) and it == it2
+
+
+def _cache_struct(num_blocks=4, heads=2, d=128, data=0x1000):
+    return tq._Cache(num_blocks, heads, d, 0, data)
+
+
+def test_argument_validation_without_launch(lib):
+    """Every case is rejected by host validation before anything is enqueued."""
+    P = ctypes.c_void_p
+    c = _cache_struct(d=96)
+    rc = lib.tq_quantize_append(P(16), P(16), None, 0, 0, P(16), 4, ctypes.byref(c), None, None, None)
+    assert rc == tq.TQ_ERR_UNSUPPORTED and b"head_dim" in lib.tq_last_error()
+    c = _cache_struct(data=0)
+    rc = lib.tq_quantize_append(P(16), P(16), None, 0, 0, P(16), 4, ctypes.byref(c), None, None, None)
+    assert rc == tq.TQ_ERR_INVALID_ARG
+    c = _cache_struct(data=0x1008)
+    rc = lib.tq_quantize_append(P(16), P(16), None, 0, 0, P(16), 4, ctypes.byref(c), None, None, None)
+    assert rc == tq.TQ_ERR_ALIGNMENT
+    c = _cache_struct()
+    rc = lib.tq_quantize_append(P(24), P(16), None, 0, 0, P(16), 4, ctypes.byref(c), None, None, None)
+    assert rc == tq.TQ_ERR_ALIGNMENT
+    rc = lib.tq_quantize_append(None, P(16), None, 0, 0, P(16), 4, ctypes.byref(c), None, None, None)
+    assert rc == tq.TQ_ERR_INVALID_ARG
+    rc = lib.tq_quantize_append(None, None, None, 0, 0, None, 0, ctypes.byref(c), None, None, None)
+    assert rc == tq.TQ_OK  # T == 0 is a no-op
+    # decode: GQA group 3 unsupported; workspace too small; bad split count
+    c = _cache_struct(heads=2)
+    args = dict(q=P(16), k=None, bt=P(16), mb=4, sl=P(16), B=1, Hq=6, L=64, scale=0.1, out=P(16),
+                ws=None, wsb=0, S=0)
+
+    def dec(**kw):
+        a = {**args, **kw}
+        return lib.tq_decode_attention(a["q"], ctypes.byref(c), a["k"], a["bt"], a["mb"], a["sl"], a["B"],
+                                       a["Hq"], a["L"], ctypes.c_float(a["scale"]), a["out"], a["ws"],
+                                       a["wsb"], a["S"], None, None)
+
+    assert dec() == tq.TQ_ERR_UNSUPPORTED
+    assert dec(Hq=4, S=4) == tq.TQ_ERR_WORKSPACE
+    assert dec(Hq=4, S=2000) == tq.TQ_ERR_UNSUPPORTED
+    assert dec(Hq=4, L=65) == tq.TQ_ERR_INVALID_ARG  # max_seq_len beyond max_blocks * 16
+    assert dec(Hq=4, scale=float("nan")) == tq.TQ_ERR_INVALID_ARG
+    assert dec(Hq=4, B=0) == tq.TQ_OK
+    assert lib.tq_decode_workspace_bytes(2, 8, 128, 4) == 2 * 8 * 4 * (128 * 4 + 8)
+    assert lib.tq_decode_workspace_bytes(2, 8, 128, 1) == 0
+    # dequantize: misaligned output
+    rc = lib.tq_dequantize(ctypes.byref(c), None, P(16), 4, P(16), 1, 8, P(20), P(16), None, None)
+    assert rc == tq.TQ_ERR_ALIGNMENT
+
+
+def test_binding_refuses_host_tensors(lib):
+    c = tq.Cache.__new__(tq.Cache)
+    K = torch.zeros((1, 2, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        tq.quantize_append(K, K, torch.zeros(1, dtype=torch.int32), c)

@@ -38,6 +38,8 @@ import numpy as np
 import torch
 
 BLOCK = 16
+CHUNK = 4096          # tokens per random stream chunk
+PREFIX_KEY = 1 << 20  # stream key of a shared prefix
 
 # stream tags: np.random.default_rng([seed, TAG, ...])
 _K, _V, _KSCALE, _VSCALE, _OUTLIER, _SPIKE, _Q, _TABLE, _SUFFIX, _CALIB, _PHYS = range(11)
@@ -60,7 +62,6 @@ class Workload:
     chunk: int = 0                 # prefill chunk length (prefill_small_head)
     calibrate: bool = False
     extra: dict = field(default_factory=dict)
-    _prefix_cache: dict = field(default_factory=dict, repr=False)
 
     @property
     def G(self) -> int:
@@ -90,11 +91,11 @@ class Workload:
                 m[h, rng.choice(self.d, size=4, replace=False)] = 20.0
         return m
 
-    def _draw(self, tag: int, key: int, n_tokens: int) -> np.ndarray:
-        """[n_tokens][Hkv][d] float32 for stream (tag, key)."""
-        rng = np.random.default_rng([self.seed, tag, key])
-        shape = (n_tokens, self.Hkv, self.d)
-        n = int(np.prod(shape))
+    def _chunk(self, tag: int, key: int, c: int) -> np.ndarray:
+        """Chunk c (tokens [c*CHUNK, (c+1)*CHUNK)) of stream (tag, key): float32 [CHUNK][Hkv][d]."""
+        rng = np.random.default_rng([self.seed, tag, key, c])
+        shape = (CHUNK, self.Hkv, self.d)
+        n = CHUNK * self.Hkv * self.d
         z = rng.standard_normal(n, dtype=np.float32)
         if self.dist == "student_t":
             # t(4) = Z / sqrt(W/4), W ~ chi-square(4) = 2 (E1 + E2), E ~ Exp(1)
@@ -105,28 +106,38 @@ class Workload:
             z /= w
         z = z.reshape(shape)
         if self.dist == "normal_spike":
-            srng = np.random.default_rng([self.seed, _SPIKE, tag, key])
-            spikes = srng.random(n_tokens) < 0.02
+            spikes = rng.random(CHUNK) < 0.02  # 2% of tokens, whole token vector x10
             z[spikes] *= 10.0
         return z
 
+    def _draw(self, tag: int, key: int, start: int, stop: int) -> np.ndarray:
+        """Tokens [start, stop) of stream (tag, key), float32 [stop-start][Hkv][d]."""
+        if stop <= start:
+            return np.zeros((0, self.Hkv, self.d), np.float32)
+        c0, c1 = start // CHUNK, (stop - 1) // CHUNK
+        if c1 - c0 >= 4:  # long ranges: draw the chunks in parallel
+            with ThreadPoolExecutor(min(32, os.cpu_count() or 1)) as ex:
+                parts = list(ex.map(lambda c: self._chunk(tag, key, c), range(c0, c1 + 1)))
+        else:
+            parts = [self._chunk(tag, key, c) for c in range(c0, c1 + 1)]
+        full = parts[0] if len(parts) == 1 else np.concatenate(parts, axis=0)
+        return full[start - c0 * CHUNK: stop - c0 * CHUNK]
+
     def _segment(self, tag: int, b: int, start: int, stop: int) -> np.ndarray:
-        """Tokens [start, stop) of sequence b before per-channel scaling (float32)."""
-        if self.shared_prefix and start < self.shared_prefix:
-            # the shared prefix is one stream (its own key) seen by every sequence
-            if tag not in self._prefix_cache:
-                self._prefix_cache[tag] = self._draw(tag, 0x7FFFFFFF, self.shared_prefix)
-            pre = self._prefix_cache[tag]
-            parts = [pre[start:min(stop, self.shared_prefix)]]
-            if stop > self.shared_prefix:
-                suf = self._draw(tag, b, int(self.seq_lens[b]) - self.shared_prefix)
-                parts.append(suf[: stop - self.shared_prefix])
-            return np.concatenate(parts, axis=0)
-        if self.shared_prefix:
-            suf = self._draw(tag, b, int(self.seq_lens[b]) - self.shared_prefix)
-            return suf[start - self.shared_prefix: stop - self.shared_prefix]
-        full = self._draw(tag, b, int(self.seq_lens[b]))
-        return full[start:stop]
+        """Tokens [start, stop) of sequence b before per-channel scaling (float32).
+
+        With a shared prefix, positions below it come from one prefix stream
+        (the same for every sequence) and the rest from the sequence's own stream.
+        """
+        P = self.shared_prefix
+        if not P:
+            return self._draw(tag, b, start, stop)
+        parts = []
+        if start < P:
+            parts.append(self._draw(tag, PREFIX_KEY, start, min(stop, P)))
+        if stop > P:
+            parts.append(self._draw(tag, b, max(start, P) - P, stop - P))
+        return parts[0] if len(parts) == 1 else np.concatenate(parts, axis=0)
 
     def kv(self, b: int, start: int = 0, stop: int | None = None):
         """(K, V) bf16 tensors [stop-start][Hkv][d] for tokens [start, stop) of sequence b."""
@@ -152,12 +163,13 @@ class Workload:
         return K[torch.from_numpy(pos)].permute(1, 0, 2).contiguous()
 
     # ------------------------------------------------------------ population
-    def population(self, max_tokens: int = 1 << 18):
+    def population(self, max_tokens: int = 1 << 17):
         """Yield (K, V, logical_slots) batches that write every token of every sequence once.
 
-        A logical slot is seq * (max_blocks * 16) + position (tokens of the
-        shared prefix's full blocks are written through sequence 0 only).
-        Batches are built with a thread pool; each holds at most max_tokens tokens.
+        A logical slot is seq * (max_blocks * 16) + position; tokens of the
+        shared prefix's full blocks are written through sequence 0 only.
+        Pieces of at most CHUNK tokens are drawn in a thread pool and grouped
+        into batches of at most max_tokens tokens.
         """
         cap = self.max_blocks * BLOCK
         shared_full = (self.shared_prefix // BLOCK) * BLOCK
@@ -165,10 +177,12 @@ class Workload:
         for b in range(self.B):
             start = 0 if (b == 0 or not shared_full) else shared_full
             L = int(self.seq_lens[b])
-            for s in range(start, L, max_tokens):
-                pieces.append((b, s, min(L, s + max_tokens)))
-        batch, size = [], 0
-        groups = []
+            s = start
+            while s < L:
+                e = min(L, (s // CHUNK + 1) * CHUNK)
+                pieces.append((b, s, e))
+                s = e
+        groups, batch, size = [], [], 0
         for p in pieces:
             n = p[2] - p[1]
             if batch and size + n > max_tokens:
@@ -185,8 +199,7 @@ class Workload:
             slots = torch.arange(s, e, dtype=torch.int32) + b * cap
             return K, V, slots
 
-        workers = min(32, os.cpu_count() or 1)
-        with ThreadPoolExecutor(workers) as ex:
+        with ThreadPoolExecutor(min(32, os.cpu_count() or 1)) as ex:
             for g in groups:
                 parts = list(ex.map(make, g))
                 yield (torch.cat([p[0] for p in parts]), torch.cat([p[1] for p in parts]),
