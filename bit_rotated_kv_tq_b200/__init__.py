@@ -103,24 +103,28 @@ def record_bytes(head_dim: int) -> int:
 
 
 def lloyd_max_table(head_dim: int) -> np.ndarray:
-    out = np.zeros(16, np.float32)
+    """The default fp16 key table (numpy float16 [16])."""
+    out = np.zeros(16, np.uint16)
     _check(load().tq_lloyd_max_table(head_dim, out.ctypes.data_as(_P)))
-    return out
+    return out.view(np.float16)
 
 
 def fit_k_table(keys: torch.Tensor, init: np.ndarray, max_iter: int = 100):
-    """keys: bf16 [n][d] (host); returns (fp32[16] table, iterations)."""
+    """keys: bf16 [n][d] (host), init: float16 [16]; returns (float16 [16] table, iterations)."""
     k = keys.detach().to("cpu").contiguous()
     if k.dtype != torch.bfloat16 or k.dim() != 2:
         raise ValueError("keys must be a 2-D bf16 tensor")
     bits = k.view(torch.int16).numpy().view(np.uint16)
-    init = np.ascontiguousarray(init, np.float32)
-    out = np.zeros(16, np.float32)
+    init = np.ascontiguousarray(init)
+    if init.dtype != np.float16:
+        raise ValueError("init must be a float16 table")
+    init = init.view(np.uint16)
+    out = np.zeros(16, np.uint16)
     rc = load().tq_fit_k_table(bits.ctypes.data_as(_P), k.shape[0], k.shape[1],
                                init.ctypes.data_as(_P), max_iter, out.ctypes.data_as(_P))
     if rc < 0:
         _check(-rc)
-    return out, rc
+    return out.view(np.float16), rc
 
 
 # ------------------------------------------------------------------ cache
@@ -158,7 +162,7 @@ def quantize_append(K, V, slot_mapping, cache: Cache, block_table=None, k_tables
     _dev(V, torch.bfloat16, "V")
     _dev(slot_mapping, torch.int32, "slot_mapping")
     _dev(block_table, torch.int32, "block_table")
-    _dev(k_tables, torch.float32, "k_tables")
+    _dev(k_tables, torch.float16, "k_tables")
     _dev(status, torch.int32, "status")
     T = K.shape[0]
     ns, mb = (0, 0) if block_table is None else (block_table.shape[0], block_table.shape[1])
@@ -181,7 +185,7 @@ def decode_attention(q, cache: Cache, block_tables, seq_lens, max_seq_len: int, 
     _dev(q, torch.bfloat16, "q")
     _dev(block_tables, torch.int32, "block_tables")
     _dev(seq_lens, torch.int32, "seq_lens")
-    _dev(k_tables, torch.float32, "k_tables")
+    _dev(k_tables, torch.float16, "k_tables")
     _dev(status, torch.int32, "status")
     B, Hq, d = q.shape
     if out is None:
@@ -203,7 +207,7 @@ def dequantize(cache: Cache, block_tables, seq_lens, max_len: int, k_tables=None
     """(K_hat, V_hat) fp32 [B][max_len][H_kv][d] in the original domain (checks only)."""
     _dev(block_tables, torch.int32, "block_tables")
     _dev(seq_lens, torch.int32, "seq_lens")
-    _dev(k_tables, torch.float32, "k_tables")
+    _dev(k_tables, torch.float16, "k_tables")
     _dev(status, torch.int32, "status")
     B = block_tables.shape[0]
     shape = (B, max_len, cache.num_kv_heads, cache.head_dim)

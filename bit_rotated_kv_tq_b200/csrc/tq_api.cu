@@ -82,23 +82,27 @@ void lloyd_max_half(double c[8]) {
     }
 }
 
+uint16_t to_half_bits(double x) { return __half_as_ushort(__double2half(x)); }
+
+void scaled_table(int d, uint16_t out[16]) {
+    double c[8];
+    lloyd_max_half(c);
+    const double s = 1.0 / sqrt((double)d);
+    for (int j = 0; j < 8; j++) {
+        out[8 + j] = to_half_bits(c[j] * s);
+        out[7 - j] = to_half_bits(-c[j] * s);
+    }
+}
+
 struct DefaultTables {
     std::once_flag once[2];
-    float t[2][16];
+    uint16_t t[2][16];
 };
 DefaultTables g_tables;
 
-const float* default_table(int d) {
+const uint16_t* default_table(int d) {
     const int k = d == 128 ? 1 : 0;
-    std::call_once(g_tables.once[k], [&] {
-        double c[8];
-        lloyd_max_half(c);
-        const double s = 1.0 / sqrt((double)d);
-        for (int j = 0; j < 8; j++) {
-            g_tables.t[k][8 + j] = (float)(c[j] * s);
-            g_tables.t[k][7 - j] = (float)(-c[j] * s);
-        }
-    });
+    std::call_once(g_tables.once[k], [&] { scaled_table(d, g_tables.t[k]); });
     return g_tables.t[k];
 }
 
@@ -136,26 +140,19 @@ TQ_API size_t tq_cache_bytes(int num_blocks, int num_kv_heads, int head_dim) {
     return (size_t)num_blocks * (size_t)num_kv_heads * tq_record_bytes(head_dim);
 }
 
-TQ_API int tq_lloyd_max_table(int head_dim, float out16[16]) {
+TQ_API int tq_lloyd_max_table(int head_dim, uint16_t out16[16]) {
     if (!out16) return fail(TQ_ERR_INVALID_ARG, "tq_lloyd_max_table: out16 is NULL");
     if (head_dim <= 0 || (head_dim & (head_dim - 1)))
         return fail(TQ_ERR_UNSUPPORTED, "tq_lloyd_max_table: head_dim %d", head_dim);
-    if (supported_d(head_dim)) {
-        memcpy(out16, default_table(head_dim), 16 * sizeof(float));
-    } else {
-        double c[8];
-        lloyd_max_half(c);
-        const double s = 1.0 / sqrt((double)head_dim);
-        for (int j = 0; j < 8; j++) {
-            out16[8 + j] = (float)(c[j] * s);
-            out16[7 - j] = (float)(-c[j] * s);
-        }
-    }
+    if (supported_d(head_dim))
+        memcpy(out16, default_table(head_dim), 16 * sizeof(uint16_t));
+    else
+        scaled_table(head_dim, out16);
     return ok();
 }
 
-TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim, const float init16[16],
-                   int max_iter, float out16[16]) {
+TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim,
+                          const uint16_t init16[16], int max_iter, uint16_t out16[16]) {
     if (!keys_bf16 || !init16 || !out16 || n < 0 || max_iter < 0)
         return -fail(TQ_ERR_INVALID_ARG, "tq_fit_k_table: bad argument");
     if (head_dim <= 0 || (head_dim & (head_dim - 1)) || head_dim > 4096)
@@ -185,7 +182,7 @@ TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim, const 
         for (int i = 0; i < d; i++) ys[(size_t)v * d + i] = nrm > 0.0 ? buf[i] / den : 0.0;
     }
     double c[16];
-    for (int j = 0; j < 16; j++) c[j] = init16[j];
+    for (int j = 0; j < 16; j++) c[j] = (double)__half2float(__ushort_as_half(init16[j]));
     const size_t N = ys.size();
     std::vector<int> cell(N, -1);
     int it = 0;
@@ -217,14 +214,14 @@ TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim, const 
             if (cnt[j]) c[j] = sum[j] / cnt[j];
     }
     std::sort(c, c + 16);
-    for (int j = 0; j < 16; j++) out16[j] = (float)c[j];
+    for (int j = 0; j < 16; j++) out16[j] = to_half_bits(c[j]);
     ok();
     return it;
 }
 
 TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block_table, int num_seqs,
                        int max_blocks, const int32_t* slot_mapping, int T,
-                       const tq_cache_t* cache, const float* k_tables, int32_t* status,
+                       const tq_cache_t* cache, const uint16_t* k_tables, int32_t* status,
                        void* stream) {
     int err;
     if (!check_cache(cache, &err)) return err;
@@ -240,7 +237,7 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
         return fail(TQ_ERR_ALIGNMENT, "tq_quantize_append: K and V must be 16-byte aligned");
     if (!aligned(slot_mapping, 4) || (block_table && !aligned(block_table, 4)) ||
         (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
-        return fail(TQ_ERR_ALIGNMENT, "tq_quantize_append: int32/fp32 arrays must be 4-byte aligned");
+        return fail(TQ_ERR_ALIGNMENT, "tq_quantize_append: int32 arrays and tables must be 4-byte aligned");
     tq::AppendArgs a;
     a.K = static_cast<const uint16_t*>(K);
     a.V = static_cast<const uint16_t*>(V);
@@ -278,7 +275,7 @@ TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_sp
     return rows * head_dim * sizeof(float) + rows * sizeof(float2);
 }
 
-TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const float* k_tables,
+TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
                         const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
                         int B, int H_q, int max_seq_len, float scale, float* out,
                         void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
@@ -344,7 +341,7 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const flo
     return ok();
 }
 
-TQ_API int tq_dequantize(const tq_cache_t* cache, const float* k_tables, const int32_t* block_tables,
+TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, const int32_t* block_tables,
                   int max_blocks, const int32_t* seq_lens, int B, int max_len, float* K_hat,
                   float* V_hat, int32_t* status, void* stream) {
     int err;

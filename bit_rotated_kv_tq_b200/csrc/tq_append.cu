@@ -52,12 +52,12 @@ struct BinEntry {
 };
 
 // Build the per-head bin tables in shared memory (called by the whole CTA).
-__device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const float* k_tables,
-                           const float* default_table) {
+__device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t* k_tables,
+                           const uint16_t* default_table) {
     for (int h = threadIdx.x; h < Hkv; h += blockDim.x) {
         HeadBins& b = hb[h];
-        const float* src = k_tables ? k_tables + 16 * h : default_table;
-        for (int k = 0; k < 16; k++) b.c[k] = src[k];
+        const uint16_t* src = k_tables ? k_tables + 16 * h : default_table;
+        for (int k = 0; k < 16; k++) b.c[k] = half_bits_to_float(src[k]);
         for (int k = 0; k < 15; k++) b.mid[k] = 0.5f * (b.c[k] + b.c[k + 1]);
         b.mid[15] = __int_as_float(0x7f800000);
         float range = b.mid[14] - b.mid[0];

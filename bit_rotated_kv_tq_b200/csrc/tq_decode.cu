@@ -86,8 +86,8 @@ __global__ void __launch_bounds__(128) decode_split_kernel(DecodeArgs a) {
     const int je = min(jb + a.blocks_per_split, nblk);
 
     if (threadIdx.x < 16)
-        ctab[threadIdx.x] = a.k_tables ? a.k_tables[kv * 16 + threadIdx.x]
-                                       : a.default_table[threadIdx.x];
+        ctab[threadIdx.x] = half_bits_to_float(a.k_tables ? a.k_tables[kv * 16 + threadIdx.x]
+                                                          : a.default_table[threadIdx.x]);
     rotate_queries<D, G>(a, b, kv, qs);
     __syncthreads();
 

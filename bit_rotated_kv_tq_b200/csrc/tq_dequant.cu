@@ -14,7 +14,7 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
     using R = Rec<D>;
     __shared__ float ctab[64][16];
     for (int i = threadIdx.x; i < a.Hkv * 16 && i < 64 * 16; i += blockDim.x)
-        ctab[i / 16][i % 16] = a.k_tables ? a.k_tables[i] : a.default_table[i % 16];
+        ctab[i / 16][i % 16] = half_bits_to_float(a.k_tables ? a.k_tables[i] : a.default_table[i % 16]);
     __syncthreads();
 
     const int lane = threadIdx.x & 31, sub = lane % LPV, grp = lane / LPV;

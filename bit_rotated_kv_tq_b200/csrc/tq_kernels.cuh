@@ -15,8 +15,8 @@ struct AppendArgs {
     int T;
     unsigned char* cache;
     int num_blocks, Hkv;
-    const float* k_tables;      // [Hkv][16] or null
-    float default_table[16];
+    const uint16_t* k_tables;   // fp16 [Hkv][16] or null
+    uint16_t default_table[16]; // fp16
     int32_t* status;
 };
 
@@ -24,8 +24,8 @@ struct DecodeArgs {
     const uint16_t* q;           // bf16 [B][Hq][D]
     const unsigned char* cache;  // [num_blocks][Hkv][record]
     int num_blocks, Hkv, Hq, B;
-    const float* k_tables;       // [Hkv][16] or null
-    float default_table[16];
+    const uint16_t* k_tables;    // fp16 [Hkv][16] or null
+    uint16_t default_table[16];  // fp16
     const int32_t* block_tables; // [B][max_blocks]
     int max_blocks;
     const int32_t* seq_lens;     // [B]
@@ -41,8 +41,8 @@ struct DecodeArgs {
 struct DequantArgs {
     const unsigned char* cache;
     int num_blocks, Hkv;
-    const float* k_tables;
-    float default_table[16];
+    const uint16_t* k_tables;   // fp16 [Hkv][16] or null
+    uint16_t default_table[16];
     const int32_t* block_tables;
     int max_blocks;
     const int32_t* seq_lens;

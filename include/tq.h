@@ -86,20 +86,23 @@ TQ_API size_t tq_record_bytes(int head_dim);
 /* Bytes of a whole cache; 0 on an unsupported shape. */
 TQ_API size_t tq_cache_bytes(int num_blocks, int num_kv_heads, int head_dim);
 
-/* (host) Default key table for head_dim d: the 16-level Lloyd-Max quantiser of
+/* Key tables are 16 fp16 values (raw bit patterns), strictly ascending, so that
+ * every centroid is an exact fp16 tensor-core operand.
+ *
+ * (host) Default key table for head_dim d: the 16-level Lloyd-Max quantiser of
  * N(0,1) scaled by 1/sqrt(d) (the rotated unit vector has coordinates of
- * variance 1/d), rounded to fp32, ascending.  "UltraQuant：4-bit KV 快取加速
- * 長代理", 「方法怎麼做，白話講」: the theoretical Lloyd-Max centroid table. */
-TQ_API int tq_lloyd_max_table(int head_dim, float out16[16]);
+ * variance 1/d), rounded to nearest fp16, ascending.  "UltraQuant：4-bit KV
+ * 快取加速長代理", 「方法怎麼做，白話講」: the theoretical Lloyd-Max table. */
+TQ_API int tq_lloyd_max_table(int head_dim, uint16_t out16[16]);
 
 /* (host) Re-fit a 16-entry key table on n calibration key vectors (bf16
  * [n][head_dim], host): rotate each unit-normalised vector, then run 1-D
  * k-means (Lloyd) from init16 for at most max_iter rounds; empty cells keep
- * their level; the result is sorted and rounded to fp32.  Same page and
+ * their level; the result is sorted and rounded to fp16.  Same page and
  * section: centroids re-fitted on about 20 rotated vectors.  Returns the
  * iteration count (>= 0) or -TQ_ERR_*. */
-TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim, const float init16[16],
-                   int max_iter, float out16[16]);
+TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim,
+                          const uint16_t init16[16], int max_iter, uint16_t out16[16]);
 
 /* Quantise T new tokens and write them into the cache (the TQ4/4 write path).
  *   K, V        (device) bf16 [T][H_kv][d], 16-byte aligned
@@ -109,13 +112,13 @@ TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim, const 
  *       block_table != NULL: logical slot = seq * (max_blocks * 16) + position,
  *                            mapped to block_table[seq][position / 16];
  *       -1 skips the token.
- *   k_tables    (device, may be NULL) fp32 [H_kv][16] strictly ascending
+ *   k_tables    (device, may be NULL) fp16 [H_kv][16] strictly ascending
  *               per-head key tables; NULL = tq_lloyd_max_table(d) for all heads.
  * Slots outside the cache set TQ_STATUS_BAD_SLOT / _BAD_BLOCK and are skipped.
  * Two tokens mapped to one slot race (last writer wins, per field). */
 TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block_table, int num_seqs,
                        int max_blocks, const int32_t* slot_mapping, int T,
-                       const tq_cache_t* cache, const float* k_tables, int32_t* status,
+                       const tq_cache_t* cache, const uint16_t* k_tables, int32_t* status,
                        void* stream);
 
 /* Number of context splits tq_decode_attention uses when num_splits == 0. */
@@ -139,7 +142,7 @@ TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_sp
  *   workspace    (device) >= tq_decode_workspace_bytes(...), 16-byte aligned
  *   num_splits   0 = tq_decode_default_splits(...), else 1..1024
  * Splits of one sequence are merged by a log-sum-exp combine kernel. */
-TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const float* k_tables,
+TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
                         const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
                         int B, int H_q, int max_seq_len, float scale, float* out,
                         void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
@@ -149,7 +152,7 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const flo
  * [B][max_len][H_kv][d] in the original (unrotated) domain,
  * k_hat = fp16 norm * H * C[idx],  v_hat = code * scale + zero;
  * rows at or past seq_lens[b] are written as 0. */
-TQ_API int tq_dequantize(const tq_cache_t* cache, const float* k_tables, const int32_t* block_tables,
+TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, const int32_t* block_tables,
                   int max_blocks, const int32_t* seq_lens, int B, int max_len, float* K_hat,
                   float* V_hat, int32_t* status, void* stream);
 

@@ -89,6 +89,14 @@ def _c(a, dtype):
     return np.ascontiguousarray(a, dtype=dtype)
 
 
+def _h(table):
+    """fp16 table(s) as contiguous uint16 bit patterns."""
+    t = np.ascontiguousarray(table)
+    if t.dtype != np.float16:
+        raise TypeError("key tables are fp16 arrays")
+    return t.view(np.uint16)
+
+
 def _check(rc, what):
     if rc < 0:
         raise ValueError(f"oracle {what} failed with code {rc}")
@@ -118,9 +126,10 @@ def lloyd_max_gaussian16(tol: float = 1e-15, max_iter: int = 10_000_000):
 
 
 def default_table(d: int) -> np.ndarray:
-    out = np.zeros(16, np.float32)
+    """fp16 [16] default key table (as a numpy float16 array)."""
+    out = np.zeros(16, np.uint16)
     _check(lib().orc_default_table(d, _ptr(out)), "default_table")
-    return out
+    return out.view(np.float16)
 
 
 def hadamard(d: int) -> np.ndarray:
@@ -137,7 +146,7 @@ def encode_k(k_bits: np.ndarray, table: np.ndarray):
     idx = np.zeros(d, np.uint8)
     n16 = np.zeros(1, np.uint16)
     y = np.zeros(d, np.float64)
-    _check(lib().orc_encode_k(_ptr(k), d, _ptr(_c(table, np.float32)), _ptr(idx), _ptr(n16), _ptr(y)),
+    _check(lib().orc_encode_k(_ptr(k), d, _ptr(_h(table)), _ptr(idx), _ptr(n16), _ptr(y)),
            "encode_k")
     return idx, int(n16[0]), y
 
@@ -146,7 +155,7 @@ def decode_k(idx: np.ndarray, norm16: int, table: np.ndarray) -> np.ndarray:
     idx = _c(idx, np.uint8)
     d = idx.shape[-1]
     out = np.zeros(d, np.float64)
-    _check(lib().orc_decode_k(_ptr(idx), int(norm16), d, _ptr(_c(table, np.float32)), _ptr(out)),
+    _check(lib().orc_decode_k(_ptr(idx), int(norm16), d, _ptr(_h(table)), _ptr(out)),
            "decode_k")
     return out
 
@@ -200,7 +209,7 @@ def quantize_append(K_bits, V_bits, slots, cache, tables=None, block_table=None,
     sl = _c(slots, np.int32)
     assert cache.dtype == np.uint8 and cache.flags.c_contiguous
     num_blocks = cache.shape[0]
-    tb = None if tables is None else _c(tables, np.float32)
+    tb = None if tables is None else _h(tables)
     bt = None if block_table is None else _c(block_table, np.int32)
     num_seqs = 0 if bt is None else bt.shape[0]
     max_blocks = 0 if bt is None else bt.shape[1]
@@ -217,7 +226,7 @@ def dequantize(cache, Hkv, d, block_tables, seq_lens, max_len, tables=None):
     B, max_blocks = bt.shape
     Kh = np.zeros((B, max_len, Hkv, d), np.float64)
     Vh = np.zeros((B, max_len, Hkv, d), np.float64)
-    tb = None if tables is None else _c(tables, np.float32)
+    tb = None if tables is None else _h(tables)
     rc = lib().orc_dequantize(_ptr(cache), cache.shape[0], Hkv, d, _ptr(tb), _ptr(bt), max_blocks,
                               _ptr(sl), B, max_len, _ptr(Kh), _ptr(Vh))
     _check(rc, "dequantize")
@@ -244,8 +253,9 @@ def rotated_unit_samples(k_bits) -> np.ndarray:
 
 
 def kmeans_table(samples, init, max_iter: int = 100):
+    """Re-fit a 16-entry fp16 table on scalar samples; returns (float16 [16], iterations)."""
     s = _c(samples, np.float64).ravel()
-    out = np.zeros(16, np.float32)
-    it = _check(lib().orc_kmeans_table(_ptr(s), s.size, _ptr(_c(init, np.float32)), max_iter, _ptr(out)),
+    out = np.zeros(16, np.uint16)
+    it = _check(lib().orc_kmeans_table(_ptr(s), s.size, _ptr(_h(init)), max_iter, _ptr(out)),
                 "kmeans_table")
-    return out, it
+    return out.view(np.float16), it

@@ -159,17 +159,18 @@ int orc_lloyd_max_gaussian16(double c[16], double tol, int max_iter, int *iters_
     return (it >= max_iter) ? -1 : 0;
 }
 
-int orc_default_table(int d, float out[16])
+int orc_default_table(int d, uint16_t out[16])
 {
     if (d <= 0)
         return -1;
     double c[16];
     if (orc_lloyd_max_gaussian16(c, 1e-15, 10000000, NULL) != 0)
         return -2;
-    /* the rotated unit vector has coordinates of variance 1/d */
+    /* the rotated unit vector has coordinates of variance 1/d; the table is
+     * stored as fp16 (round to nearest) */
     double sigma = 1.0 / sqrt((double)d);
     for (int j = 0; j < 16; j++)
-        out[j] = orc_fp32_from_double(c[j] * sigma);
+        out[j] = orc_fp16_from_double(c[j] * sigma, 0);
     return 0;
 }
 
@@ -230,12 +231,12 @@ static void hadamard_apply(int d, const double *H, const double *x, double *y)
 /* keys                                                                 */
 /* ------------------------------------------------------------------ */
 
-static int nearest_centroid(double y, const float *table)
+static int nearest_centroid(double y, const uint16_t *table)
 {
     int best = 0;
-    double bd = fabs(y - (double)table[0]);
+    double bd = fabs(y - orc_fp16_to_double(table[0]));
     for (int c = 1; c < 16; c++) {
-        double dc = fabs(y - (double)table[c]);
+        double dc = fabs(y - orc_fp16_to_double(table[c]));
         if (dc < bd) { /* strict: a tie keeps the lower index */
             bd = dc;
             best = c;
@@ -244,7 +245,7 @@ static int nearest_centroid(double y, const float *table)
     return best;
 }
 
-int orc_encode_k(const uint16_t *k_bf16, int d, const float *table, uint8_t *idx,
+int orc_encode_k(const uint16_t *k_bf16, int d, const uint16_t *table, uint8_t *idx,
                  uint16_t *norm16, double *y_out)
 {
     if (!is_pow2(d) || !k_bf16 || !table || !idx || !norm16)
@@ -277,7 +278,7 @@ int orc_encode_k(const uint16_t *k_bf16, int d, const float *table, uint8_t *idx
     return 0;
 }
 
-int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const float *table, double *k_hat)
+int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const uint16_t *table, double *k_hat)
 {
     if (!is_pow2(d) || !idx || !table || !k_hat)
         return -1;
@@ -285,7 +286,7 @@ int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const float *table,
     const double *H = hadamard_cached(d);
     double n = orc_fp16_to_double(norm16);
     for (int i = 0; i < d; i++)
-        c[i] = (double)table[idx[i] & 15];
+        c[i] = orc_fp16_to_double(table[idx[i] & 15]);
     /* H is symmetric and H*H = I, so H also undoes the rotation */
     hadamard_apply(d, H, c, k_hat);
     for (int i = 0; i < d; i++)
@@ -428,19 +429,19 @@ int orc_unpack_token(const uint8_t *record, int d, int offset, uint8_t *kidx, ui
 /* paged cache                                                          */
 /* ------------------------------------------------------------------ */
 
-static const float *head_table(const float *tables, const float *deflt, int h)
+static const uint16_t *head_table(const uint16_t *tables, const uint16_t *deflt, int h)
 {
     return tables ? tables + 16 * h : deflt;
 }
 
 int orc_quantize_append(const uint16_t *K, const uint16_t *V, int T, int Hkv, int d,
                         const int32_t *block_table, int num_seqs, int max_blocks,
-                        const int32_t *slots, const float *tables, uint8_t *cache,
+                        const int32_t *slots, const uint16_t *tables, uint8_t *cache,
                         int num_blocks, double *ky, double *vr)
 {
     if (T < 0 || Hkv <= 0 || !is_pow2(d) || d % ORC_VGROUP || !slots || !cache)
         return -1;
-    float deflt[16];
+    uint16_t deflt[16];
     if (!tables && orc_default_table(d, deflt) != 0)
         return -2;
     size_t rec = orc_record_bytes(d);
@@ -489,14 +490,14 @@ int orc_quantize_append(const uint16_t *K, const uint16_t *V, int T, int Hkv, in
     return rc;
 }
 
-int orc_dequantize(const uint8_t *cache, int num_blocks, int Hkv, int d, const float *tables,
+int orc_dequantize(const uint8_t *cache, int num_blocks, int Hkv, int d, const uint16_t *tables,
                    const int32_t *block_tables, int max_blocks, const int32_t *seq_lens, int B,
                    int max_len, double *Khat, double *Vhat)
 {
     if (!cache || !block_tables || !seq_lens || !Khat || !Vhat || !is_pow2(d) ||
         d % ORC_VGROUP)
         return -1;
-    float deflt[16];
+    uint16_t deflt[16];
     if (!tables && orc_default_table(d, deflt) != 0)
         return -2;
     size_t rec = orc_record_bytes(d);
@@ -600,7 +601,7 @@ int orc_rotated_unit_samples(const uint16_t *k_bf16, int n_vec, int d, double *o
 {
     if (!k_bf16 || !out || !is_pow2(d) || n_vec < 0)
         return -1;
-    float dummy_table[16] = {0};
+    uint16_t dummy_table[16] = {0};
     uint8_t *idx = malloc(d);
     for (int n = 0; n < n_vec; n++) {
         uint16_t n16;
@@ -617,13 +618,13 @@ static int cmp_double(const void *a, const void *b)
     return (x > y) - (x < y);
 }
 
-int orc_kmeans_table(const double *samples, int n, const float *init, int max_iter, float out[16])
+int orc_kmeans_table(const double *samples, int n, const uint16_t *init, int max_iter, uint16_t out[16])
 {
     if (!samples || !init || !out || n < 0 || max_iter < 0)
         return -1;
     double c[16];
     for (int j = 0; j < 16; j++)
-        c[j] = (double)init[j];
+        c[j] = orc_fp16_to_double(init[j]);
     int *assign = malloc(sizeof(int) * (n > 0 ? n : 1));
     for (int i = 0; i < n; i++)
         assign[i] = -1;
@@ -661,7 +662,7 @@ int orc_kmeans_table(const double *samples, int n, const float *init, int max_it
     }
     qsort(c, 16, sizeof(double), cmp_double);
     for (int j = 0; j < 16; j++)
-        out[j] = orc_fp32_from_double(c[j]);
+        out[j] = orc_fp16_from_double(c[j], 0);
     free(assign);
     return it;
 }

@@ -46,18 +46,19 @@ float orc_fp32_from_double(double x); /* round to nearest even */
 
 /* Lloyd-Max 16-level quantiser of the standard normal N(0,1). */
 int orc_lloyd_max_gaussian16(double c[16], double tol, int max_iter, int *iters_used);
-/* Default key table for head_dim d: fp32(c_j / sqrt(d)), ascending. */
-int orc_default_table(int d, float out[16]);
+/* Default key table for head_dim d: fp16(c_j / sqrt(d)) bit patterns, ascending.
+ * Every key table is 16 fp16 values (bit patterns), strictly ascending. */
+int orc_default_table(int d, uint16_t out[16]);
 
 /* Dense normalised Sylvester Hadamard matrix, H[i*d+j] = (-1)^popcount(i&j)/sqrt(d). */
 int orc_hadamard(int d, double *H);
 
 /* Key encode: n = ||k||, u = k/n, y = H u, idx_i = argmin_c |y_i - C[c]| (ties: lower c).
  * y_out (may be NULL) receives the rotated unit coordinates. */
-int orc_encode_k(const uint16_t *k_bf16, int d, const float *table, uint8_t *idx,
+int orc_encode_k(const uint16_t *k_bf16, int d, const uint16_t *table, uint8_t *idx,
                  uint16_t *norm16, double *y_out);
 /* Key decode to the original domain: k_hat = fp16(n) * H * C[idx]. */
-int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const float *table, double *k_hat);
+int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const uint16_t *table, double *k_hat);
 
 /* Value encode per group of 32: z = fp16 down(min), s = fp16 up((max - z)/15),
  * q = clamp(round_half_even((v - z)/s), 0, 15) (q = 0 when s = 0).
@@ -79,16 +80,16 @@ int orc_unpack_token(const uint8_t *record, int d, int offset, uint8_t *kidx, ui
  *   block_table == NULL: slots[t] is a physical slot (block*16 + offset), -1 skips.
  *   block_table != NULL ([num_seqs][max_blocks]): slots[t] is a logical slot
  *     seq*(max_blocks*16) + position, mapped through the table; -1 skips.
- * tables: NULL = default table for every head, else [Hkv][16] fp32.
+ * tables: NULL = default table for every head, else [Hkv][16] fp16 bits.
  * ky/vr (may be NULL): [T][Hkv][d] rotated unit key coordinates and (v-z)/s. */
 int orc_quantize_append(const uint16_t *K, const uint16_t *V, int T, int Hkv, int d,
                         const int32_t *block_table, int num_seqs, int max_blocks,
-                        const int32_t *slots, const float *tables, uint8_t *cache,
+                        const int32_t *slots, const uint16_t *tables, uint8_t *cache,
                         int num_blocks, double *ky, double *vr);
 
 /* Gather + dequantise every valid token of every sequence into
  * Khat, Vhat fp64 [B][max_len][Hkv][d] (original domain); rows past seq_len are 0. */
-int orc_dequantize(const uint8_t *cache, int num_blocks, int Hkv, int d, const float *tables,
+int orc_dequantize(const uint8_t *cache, int num_blocks, int Hkv, int d, const uint16_t *tables,
                    const int32_t *block_tables, int max_blocks, const int32_t *seq_lens, int B,
                    int max_len, double *Khat, double *Vhat);
 
@@ -100,8 +101,8 @@ int orc_attention(const uint16_t *q, int B, int Hq, int Hkv, int d, const double
 
 /* 1-D k-means (Lloyd) refit of a 16-entry table on n scalar samples, starting
  * from init; empty clusters keep their centroid; the result is sorted and
- * rounded to fp32.  Returns the number of iterations run (>= 0). */
-int orc_kmeans_table(const double *samples, int n, const float *init, int max_iter, float out[16]);
+ * rounded to fp16.  Returns the number of iterations run (>= 0). */
+int orc_kmeans_table(const double *samples, int n, const uint16_t *init, int max_iter, uint16_t out[16]);
 /* The calibration samples of one head: unit-normalised, rotated key vectors. */
 int orc_rotated_unit_samples(const uint16_t *k_bf16, int n_vec, int d, double *out);
 

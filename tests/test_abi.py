@@ -64,6 +64,7 @@ def test_fit_k_table_equals_oracle(lib, orc):
         keys = torch.from_numpy((rng.standard_t(4, (20, d)) * rng.lognormal(0, 1, d)).astype(np.float32))
         keys = keys.to(torch.bfloat16)
         init = orc.default_table(d)
+        assert init.dtype == np.float16
         got, it = tq.fit_k_table(keys, init, 100)
         bits = keys.view(torch.int16).numpy().view(np.uint16)
         want, it2 = orc.kmeans_table(orc.rotated_unit_samples(bits), init, 100)

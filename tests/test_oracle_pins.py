@@ -138,8 +138,8 @@ def test_lloyd_max_distortion_by_quadrature(orc):
 def test_default_table_scaled_by_sqrt_d(orc, d):
     c, _ = orc.lloyd_max_gaussian16()
     t = orc.default_table(d)
-    assert t.dtype == np.float32
-    assert np.array_equal(t, (c / math.sqrt(d)).astype(np.float32))
+    assert t.dtype == np.float16
+    assert np.array_equal(t, (c / math.sqrt(d)).astype(np.float16))
 
 
 # ---------------------------------------------------------------- keys
@@ -153,8 +153,9 @@ def test_key_worked_example_e0(orc):
     assert n16 == int(g["key_e0_norm16"][0], 16)
     assert np.all(idx == int(g["key_e0_code"][0]))
     assert np.allclose(y, 1 / math.sqrt(d), atol=1e-15)
+    assert int(table.view(np.uint16)[11]) == int(g["key_e0_table11"][0], 16)
     khat = orc.decode_k(idx, n16, table)
-    assert abs(khat[0] - float(g["key_e0_khat0"][0])) < 1e-5
+    assert abs(khat[0] - float(g["key_e0_khat0"][0])) < 1e-6
     assert np.max(np.abs(khat[1:])) < 1e-12
 
 
@@ -392,7 +393,23 @@ def test_kmeans_table_lowers_mse_on_its_samples(orc):
         t = t.astype(np.float64)
         return np.mean(np.min((y.ravel()[:, None] - t[None, :]) ** 2, axis=1))
 
-    assert mse(tab) <= mse(init) * (1 + 1e-6)
-    # a k-means fixed point: refitting from the result changes nothing
-    tab2, it2 = orc.kmeans_table(y, tab, 100)
-    assert np.allclose(tab2, tab, atol=1e-7) and it2 <= 1
+    assert mse(tab) <= mse(init) * (1 + 1e-3)  # Lloyd steps never raise the MSE (fp16 rounding aside)
+
+
+def test_kmeans_on_gaussian_samples_reaches_lloyd_max_distortion(orc):
+    """On many samples of N(0, 1/d), k-means from the Lloyd-Max table converges to a
+    table whose distortion is no worse than Lloyd-Max's on those samples and not
+    meaningfully better than the population optimum (Max 1960: 0.009497 sigma^2)."""
+    d = 64
+    init = orc.default_table(d)
+    rng = np.random.default_rng(99)
+    y = rng.standard_normal(400_000) / math.sqrt(d)
+    tab, it = orc.kmeans_table(y, init, 1000)
+    assert it < 1000 and np.all(np.diff(tab.astype(np.float64)) > 0)
+
+    def mse(t):
+        t = t.astype(np.float64)
+        return np.mean(np.min((y[:, None] - t[None, :]) ** 2, axis=1)) * d
+
+    assert mse(tab) <= mse(init) * (1 + 1e-4)
+    assert 0.0095 * 0.98 <= mse(tab) <= 0.0095 * 1.02

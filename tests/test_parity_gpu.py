@@ -63,7 +63,8 @@ class OracleSeq:
         Kb = bf16_bits(K[:, h:h + 1].contiguous())
         Vb = bf16_bits(V[:, h:h + 1].contiguous())
         nblk = (L + 15) // 16
-        self.table = np.ascontiguousarray(table, np.float32)
+        self.table = np.ascontiguousarray(table)
+        assert self.table.dtype == np.float16
         self.cache = np.zeros((nblk, 1, orc.record_bytes(w.d)), np.uint8)
         rc, self.ky, self.vr = orc.quantize_append(Kb, Vb, np.arange(L, dtype=np.int32), self.cache,
                                                    tables=self.table[None], want_aux=True)
@@ -178,7 +179,7 @@ def test_dense_custom_table_exact_count_path(tq, orc):
     base = orc.default_table(w.d).astype(np.float64)
     t = base.copy()
     t[7], t[8], t[9] = -1e-4, 0.0, 1e-4  # midpoints 7 and 8 fall in one bin
-    t = t.astype(np.float32)
+    t = t.astype(np.float16)
     assert np.all(np.diff(t) > 0)
     tables = np.tile(t, (w.Hkv, 1))
     g = GpuState(tq, w, tables)
