@@ -261,9 +261,10 @@ TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len) {
     if (B <= 0 || H_kv <= 0 || max_seq_len <= 0) return 1;
     const int nblk = (max_seq_len + tq::kBlock - 1) / tq::kBlock;
     const long long pairs = (long long)B * H_kv;
-    // aim for ~16 CTAs per SM, with at least 16 blocks (256 tokens) per split
-    long long s = (16LL * device_sms() + pairs - 1) / pairs;
-    s = std::min<long long>(s, std::max(1, nblk / 16));
+    // The split kernel runs two 8-warp CTAs per SM.  Aim for about four waves
+    // of CTAs over the GPU, keeping at least 32 blocks (4 per warp) per split.
+    long long s = (8LL * device_sms() + pairs - 1) / pairs;
+    s = std::min<long long>(s, std::max(1, nblk / 32));
     s = std::max<long long>(1, std::min<long long>(s, 1024));
     const int bps = (int)((nblk + s - 1) / s);
     return (nblk + bps - 1) / bps;

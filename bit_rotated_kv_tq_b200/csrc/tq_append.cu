@@ -308,7 +308,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
             unsigned char* rec =
                 a.cache + ((size_t)blk * a.Hkv + h) * (size_t)R::kBytes;
             *reinterpret_cast<uint32_t*>(rec + R::kKCodes + off * R::kCodeRow + sub * 4) = kw;
-            *reinterpret_cast<uint32_t*>(rec + R::kVCodes + off * R::kCodeRow + sub * 4) = vw;
+            unsigned char* vrow = rec + R::kVCodes + off * R::kCodeRow;
+#pragma unroll
+            for (int i = 0; i < 4; i++) vrow[R::vpos(sub * 4 + i)] = (unsigned char)(vw >> (8 * i));
             if (sub == 0) *reinterpret_cast<uint16_t*>(rec + R::kKNorm + off * 2) = n16;
             if ((sub & 3) == 0) {
                 const uint16_t z16 = __half_as_ushort(zh);

@@ -4,7 +4,9 @@
 // Record of one (physical block, kv head), 16 tokens, head_dim D:
 //   [0, 8D)         key codes    [16][D/2] bytes, element 2j in the low nibble of byte j
 //   [8D, 8D+32)     key norms    [16] fp16
-//   [8D+32, 16D+32) value codes  [16][D/2] bytes
+//   [8D+32, 16D+32) value codes  [16][D/2] bytes, same nibble order; value byte j is
+//                   stored at row offset (j % 8) * (D/16) + j / 8 so that the bytes one
+//                   lane feeds to the tensor cores (j = 8m + g, m = 0..D/16-1) are contiguous
 //   [16D+32, 18D+32) value groups [16][D/32] x (fp16 scale, fp16 zero)
 // The cache is [num_blocks][H_kv][record]; every field starts 16-byte aligned.
 #pragma once
@@ -30,6 +32,8 @@ struct Rec {
     static constexpr int kVCodes = kKNorm + 2 * kBlock;     // 8D + 32
     static constexpr int kVGroups = kVCodes + kBlock * kCodeRow;  // 16D + 32
     static constexpr int kGroups = D / kGroup;
+    static constexpr int kVStride = D / 16;  // value byte j -> row offset (j % 8) * kVStride + j / 8
+    static __host__ __device__ constexpr int vpos(int j) { return (j % 8) * kVStride + j / 8; }
     static constexpr int kBytes = kVGroups + kBlock * kGroups * 4;  // 18D + 32
     static_assert(kKNorm % 16 == 0 && kVCodes % 16 == 0 && kVGroups % 16 == 0 &&
                       kBytes % 16 == 0,

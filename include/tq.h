@@ -29,10 +29,12 @@
  *     row-major, with the shapes given.
  *
  * Cache record: one per (physical block, kv head), 16 tokens, 16-byte
- * aligned fields, little-endian, element 2j in the low nibble of byte j:
- *   [0,      8d)        key codes    [16][d/2] bytes
+ * aligned fields, little-endian; code byte j holds element 2j in its low
+ * nibble and element 2j+1 in its high nibble:
+ *   [0,      8d)        key codes    [16][d/2] bytes, byte j at row offset j
  *   [8d,     8d+32)     key norms    [16] fp16
- *   [8d+32,  16d+32)    value codes  [16][d/2] bytes
+ *   [8d+32,  16d+32)    value codes  [16][d/2] bytes, byte j at row offset
+ *                       (j mod 8)*(d/16) + j/8 (the tensor-core fragment order)
  *   [16d+32, 18d+32)    value groups [16][d/32] x (fp16 scale, fp16 zero)
  * = 2336 bytes at d = 128, 1184 bytes at d = 64.  The cache is
  * [num_blocks][num_kv_heads][record].
@@ -70,7 +72,9 @@ enum {
     TQ_STATUS_BAD_SLOT = 1,  /* append: slot or logical slot outside the cache / table */
     TQ_STATUS_BAD_BLOCK = 2, /* a block-table entry outside [0, num_blocks) */
     TQ_STATUS_RANGE = 4,     /* a key norm or value scale/zero overflowed fp16 */
-    TQ_STATUS_BAD_LEN = 8    /* seq_len < 0 or > max_blocks * 16 (treated as 0) */
+    TQ_STATUS_BAD_LEN = 8,   /* seq_len < 0 or > max_blocks * 16 (treated as 0) */
+    TQ_STATUS_TIMEOUT = 16   /* a kernel gave up waiting (~1 s) for its own copy: the
+                                call's output is incomplete; never expected */
 };
 
 typedef struct {

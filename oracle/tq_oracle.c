@@ -361,8 +361,10 @@ int orc_decode_v(const uint8_t *q, const uint16_t *scale16, const uint16_t *zero
 /*                       as (fp16 scale, fp16 zero) pairs               */
 /*   total 16d + 32 + 64*(d/32) bytes (2336 at d=128, 1184 at d=64)    */
 /*                                                                      */
-/* In a code row, byte j holds element 2j in its low nibble and element */
-/* 2j+1 in its high nibble.  Multi-byte fields are little-endian.       */
+/* Code byte j of a row holds element 2j in its low nibble and element  */
+/* 2j+1 in its high nibble.  Key byte j sits at row offset j; value     */
+/* byte j sits at row offset (j mod 8) * (d/16) + floor(j / 8).         */
+/* Multi-byte fields are little-endian.                                 */
 /* ------------------------------------------------------------------ */
 
 size_t orc_record_bytes(int d)
@@ -374,6 +376,8 @@ size_t orc_record_bytes(int d)
 static size_t off_knorm(int d) { return (size_t)ORC_BLOCK * d / 2; }
 static size_t off_vcodes(int d) { return off_knorm(d) + ORC_BLOCK * 2; }
 static size_t off_vsz(int d) { return off_vcodes(d) + (size_t)ORC_BLOCK * d / 2; }
+/* row offset of value code byte j (interleaved order, see above) */
+static size_t vpos(int d, int j) { return (size_t)(j % 8) * (d / 16) + (size_t)(j / 8); }
 
 static void put_u16(uint8_t *p, uint16_t v)
 {
@@ -392,7 +396,7 @@ int orc_pack_token(uint8_t *record, int d, int offset, const uint8_t *kidx, uint
     uint8_t *vc = record + off_vcodes(d) + (size_t)offset * (d / 2);
     for (int j = 0; j < d / 2; j++) {
         kc[j] = (uint8_t)((kidx[2 * j] & 15) | ((kidx[2 * j + 1] & 15) << 4));
-        vc[j] = (uint8_t)((vq[2 * j] & 15) | ((vq[2 * j + 1] & 15) << 4));
+        vc[vpos(d, j)] = (uint8_t)((vq[2 * j] & 15) | ((vq[2 * j + 1] & 15) << 4));
     }
     put_u16(record + off_knorm(d) + 2 * offset, knorm);
     uint8_t *sz = record + off_vsz(d) + (size_t)offset * (d / ORC_VGROUP) * 4;
@@ -413,8 +417,8 @@ int orc_unpack_token(const uint8_t *record, int d, int offset, uint8_t *kidx, ui
     for (int j = 0; j < d / 2; j++) {
         kidx[2 * j] = kc[j] & 15;
         kidx[2 * j + 1] = kc[j] >> 4;
-        vq[2 * j] = vc[j] & 15;
-        vq[2 * j + 1] = vc[j] >> 4;
+        vq[2 * j] = vc[vpos(d, j)] & 15;
+        vq[2 * j + 1] = vc[vpos(d, j)] >> 4;
     }
     *knorm = get_u16(record + off_knorm(d) + 2 * offset);
     const uint8_t *sz = record + off_vsz(d) + (size_t)offset * (d / ORC_VGROUP) * 4;

@@ -29,6 +29,12 @@ def layout(d):
     return row, kn, vc, vg, vg + 16 * (d // 32) * 4
 
 
+def value_positions(d):
+    """Row offset of value code byte j: (j mod 8) * (d/16) + j // 8 (interleaved order)."""
+    j = np.arange(d // 2)
+    return (j % 8) * (d // 16) + j // 8
+
+
 def unpack_record(rec: np.ndarray, d: int):
     """rec uint8 [record] -> kidx [16][d], knorm uint16 [16], vq [16][d], vs, vz uint16 [16][d/32]."""
     row, kn, vc, vg, total = layout(d)
@@ -37,6 +43,7 @@ def unpack_record(rec: np.ndarray, d: int):
     kidx = np.stack([kc & 15, kc >> 4], axis=-1).reshape(rec.shape[:-1] + (16, d))
     knorm = rec[..., kn:kn + 32].copy().view(np.uint16).reshape(rec.shape[:-1] + (16,))
     vcb = rec[..., vc:vc + 16 * row].reshape(rec.shape[:-1] + (16, row))
+    vcb = vcb[..., value_positions(d)]  # back to natural byte order
     vq = np.stack([vcb & 15, vcb >> 4], axis=-1).reshape(rec.shape[:-1] + (16, d))
     sz = rec[..., vg:total].copy().view(np.uint16).reshape(rec.shape[:-1] + (16, d // 32, 2))
     return kidx, knorm, vq, sz[..., 0], sz[..., 1]

@@ -278,8 +278,12 @@ def test_record_size_and_nibble_order(orc):
     assert np.all(row == int(g["key_e0_byte"][0], 16))
     assert int(rec[1024 + 10]) | (int(rec[1024 + 11]) << 8) == 0x3C00
     vrow = rec[1056 + 5 * 64:1056 + 6 * 64]
+    assert list(vrow) == [int(x, 16) for x in g["value_ramp_stored_d128"]]
+    # undoing the interleave gives the natural code bytes of the worked example
+    j = np.arange(64)
+    natural = vrow[(j % 8) * 8 + j // 8]
     want = [int(x, 16) for x in g["value_ramp_bytes"]]
-    assert list(vrow[:16]) == want and list(vrow[16:32]) == want
+    assert list(natural[:16]) == want and list(natural[16:32]) == want
     sz = rec[2080 + 5 * 16:2080 + 6 * 16]
     assert int(sz[0]) | (int(sz[1]) << 8) == 0x4023 and int(sz[2]) | (int(sz[3]) << 8) == 0
     # every other token row is untouched

@@ -161,6 +161,10 @@ def test_dequantize_matches_oracle(tq, orc):
     ("prefill_small_head", dict(B=3, ctx=1500), 0),   # d = 64, GQA 8
     ("long_context", dict(B=1, ctx=4100), 64),        # many splits, one partly empty
     ("tiny", dict(B=2, ctx=17), 2),                   # one full block plus one token
+    ("qwen3_8b_layer", dict(B=2, ctx=300, Hq=8), 3),  # GQA 1
+    ("qwen3_8b_layer", dict(B=2, ctx=300, Hq=16), 0), # GQA 2
+    ("qwen3_8b_layer", dict(B=2, ctx=300, Hq=64), 2), # GQA 8 at d = 128
+    ("prefill_small_head", dict(B=2, ctx=200, Hq=8), 1),  # GQA 4 at d = 64
 ])
 def test_reduced_configs(tq, orc, name, over, S):
     w = W.make(name, **over)

@@ -251,6 +251,8 @@ def make(name: str, **over) -> Workload:
     B = over.pop("B", B)
     ctx = over.pop("ctx", ctx)
     seed = over.pop("seed", seed)
+    Hq = over.pop("Hq", Hq)
+    Hkv = over.pop("Hkv", Hkv)
     extra = {}
     if name == "agentic":
         prefix = over.pop("prefix", 25000)
