@@ -150,13 +150,20 @@ def dist_setup(n_gpus):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The maximum of x over all ranks (device timings are compared this way)."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, steps: int, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: every rank processed units_per_rank per step."""
+    return world * units_per_rank * steps / max_seconds
 
 
 def barrier(world):
@@ -325,7 +332,7 @@ def run_tq(args, rank, world, local):
     assert int(status.item()) == 0, f"device status {int(status.item())}"
 
     kv = decode_kv_bytes(w)
-    value = world * kv * args.steps / (total_ms / 1e3) / 1e9
+    value = weak_scaling_value(kv, args.steps, world, total_ms / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     dec_bytes = decode_bytes(w)
     achieved = dec_bytes / (dec_avg / 1e3) / 1e9
@@ -361,7 +368,7 @@ def run_tq(args, rank, world, local):
                          "frac": achieved / peak, "traffic": None,
                          "kernel": "tq_decode_attention (split kernel + combine)",
                          "peak_source": f"{peak_kind} hbm_gbs"},
-            "e2e": {"value": world * kv * args.steps / e2e_s / 1e9, "unit": "GB/s",
+            "e2e": {"value": weak_scaling_value(kv, args.steps, world, e2e_s) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": args.steps * (2 + (1 if S > 1 else 0)),
             "clocks": clocks,

@@ -1,0 +1,64 @@
+"""Host-side logic of the N > 1 bench path on world-size-2 gloo ranks (CPU).
+
+Each rank runs an independent replica of the batch (weak scaling, no data-path
+collective); the only cross-rank steps are a barrier and the max over ranks of
+the device timings.  These run here without a GPU.
+"""
+import os
+import socket
+import subprocess
+import sys
+
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from conftest import ROOT
+
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = [0.010, 0.013][rank]  # rank 1 is the slow one
+        bench.barrier(world)
+        m = bench.max_over_ranks(mine, world)
+        v = bench.weak_scaling_value(306.2e6, 20, world, m)
+        q.put((rank, m, v))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_value_on_gloo():
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for rank, m, v in res:
+        assert m == 0.013  # every rank sees the slowest rank's time
+        assert abs(v - 2 * 306.2e6 * 20 / 0.013) < 1e-3 * v
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun, ranks other than 0 exit 0 without work or output."""
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "0"], env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0 and r.stdout.strip() == ""
