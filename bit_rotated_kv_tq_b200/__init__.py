@@ -65,6 +65,10 @@ def load(path: str | None = None):
     L.tq_decode_attention.argtypes = [_P, ctypes.POINTER(_Cache), _P, _P, _I, _P, _I, _I, _I, _F,
                                       _P, _P, _Z, _I, _P, _P]
     L.tq_dequantize.argtypes = [ctypes.POINTER(_Cache), _P, _P, _I, _P, _I, _I, _P, _P, _P, _P]
+    L.tq_decode_attention_static.argtypes = [_P, ctypes.POINTER(_Cache), _P, _P, _I, _P, _I, _I, _I, _F,
+                                             _P, _I, _P, _P]
+    L.tq_decode_static_scratch_bytes.restype = _Z
+    L.tq_decode_static_scratch_bytes.argtypes = []
     L.tq_last_error.restype = ctypes.c_char_p
     L.tq_last_error.argtypes = []
     _lib = L
@@ -199,6 +203,26 @@ def decode_attention(q, cache: Cache, block_tables, seq_lens, max_seq_len: int, 
                                       block_tables.shape[1], _ptr(seq_lens), B, Hq, int(max_seq_len),
                                       float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                       int(num_splits), _ptr(status), _stream(stream)))
+    return out
+
+
+def decode_attention_static(q, cache: Cache, block_tables, seq_lens, max_seq_len: int, scale: float,
+                            out=None, num_splits: int = 0, k_tables=None, status=None, stream=None):
+    """decode_attention for callers that cannot allocate: no workspace argument; the split
+    partials use the library's fixed device array (see tq_decode_attention_static)."""
+    _dev(q, torch.bfloat16, "q")
+    _dev(block_tables, torch.int32, "block_tables")
+    _dev(seq_lens, torch.int32, "seq_lens")
+    _dev(k_tables, torch.float16, "k_tables")
+    _dev(status, torch.int32, "status")
+    B, Hq, d = q.shape
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _dev(out, torch.float32, "out")
+    _check(load().tq_decode_attention_static(_ptr(q), cache.c, _ptr(k_tables), _ptr(block_tables),
+                                             block_tables.shape[1], _ptr(seq_lens), B, Hq,
+                                             int(max_seq_len), float(scale), _ptr(out), int(num_splits),
+                                             _ptr(status), _stream(stream)))
     return out
 
 

@@ -128,6 +128,11 @@ bool check_cache(const tq_cache_t* c, int* err) {
 
 }  // namespace
 
+namespace tq {
+// Record a failure for tq_last_error() from another translation unit.
+int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace tq
+
 extern "C" {
 
 TQ_API size_t tq_record_bytes(int head_dim) {

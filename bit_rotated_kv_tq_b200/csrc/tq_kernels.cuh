@@ -53,6 +53,7 @@ struct DequantArgs {
 };
 
 size_t append_smem_bytes(int Hkv);
+int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int head_dim, cudaStream_t stream);
 cudaError_t launch_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);

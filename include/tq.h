@@ -152,6 +152,33 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
                         void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
                         void* stream);
 
+/* Decode attention without a caller workspace.  No page describes this call;
+ * it exists for callers that cannot allocate device memory at all -- an
+ * operator or plugin hosted by another runtime usually receives only the
+ * tensors of the call while the host runtime owns (and pools) every other
+ * byte of device memory, so it has no way to hand over a workspace.
+ * Same arguments, result and checks as tq_decode_attention minus workspace /
+ * ws_bytes; the split partials go to a fixed array compiled into the library
+ * (tq_decode_static_scratch_bytes() bytes, 8 MiB, present on every GPU that
+ * loads the library until the process exits).  The call allocates and frees
+ * nothing.  A split plan whose partials exceed the array
+ * (tq_decode_workspace_bytes(B, H_q, d, splits) > 8 MiB) is rejected with
+ * TQ_ERR_WORKSPACE before anything is enqueued; pass fewer splits (1 needs
+ * none) or use tq_decode_attention.
+ * The first call on a device looks the array's address up
+ * (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  All calls share the one array and it keeps the last
+ * call's contents (nothing in it needs to start at zero): calls that overlap
+ * on the GPU -- on different streams, or from different threads -- race on
+ * it and must be ordered by the caller. */
+TQ_API int tq_decode_attention_static(const void* q, const tq_cache_t* cache,
+                                      const uint16_t* k_tables, const int32_t* block_tables,
+                                      int max_blocks, const int32_t* seq_lens, int B, int H_q,
+                                      int max_seq_len, float scale, float* out, int num_splits,
+                                      int32_t* status, void* stream);
+/* Size in bytes of the fixed array tq_decode_attention_static uses. */
+TQ_API size_t tq_decode_static_scratch_bytes(void);
+
 /* Dequantise every valid token (checks only): K_hat and V_hat (device) fp32
  * [B][max_len][H_kv][d] in the original (unrotated) domain,
  * k_hat = fp16 norm * H * C[idx],  v_hat = code * scale + zero;
