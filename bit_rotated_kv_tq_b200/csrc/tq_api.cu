@@ -232,6 +232,8 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
     if (!check_cache(cache, &err)) return err;
     if (T < 0) return fail(TQ_ERR_INVALID_ARG, "tq_quantize_append: T < 0");
     if (T == 0) return ok();
+    if ((long long)T * cache->num_kv_heads >= 0x7fffffffLL)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_quantize_append: T * H_kv must stay below 2^31");
     if (!K || !V || !slot_mapping)
         return fail(TQ_ERR_INVALID_ARG, "tq_quantize_append: K, V and slot_mapping are required");
     if (block_table && (num_seqs <= 0 || max_blocks <= 0))

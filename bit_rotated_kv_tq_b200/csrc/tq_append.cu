@@ -12,16 +12,20 @@
 //
 // Work split: one vector (token, kv head) is spread over D/8 lanes holding 8
 // elements each, so a warp handles 2 (D=128) or 4 (D=64) vectors per pass;
-// loads are 16-byte per lane and fully coalesced.  The rotation is an in-
-// register butterfly over 3 index bits plus xor-shuffles over the rest.
+// loads are 16-byte per lane and fully coalesced.  The grid is persistent
+// (one wave of resident CTAs) and every warp loads its next pass before it
+// computes the current one, so the global-load latency overlaps the math.
+// The rotation is an in-register butterfly over 3 index bits plus
+// xor-shuffles over the lane bits (a sign-FMA per element and stage).
 //
 // Exactness: the fast path runs in fp32.  Every decision it takes (fp16
-// rounding of the norm, the nearest centroid, the rounding of (v - z)/s) is
-// re-taken in fp64 from the bf16 inputs whenever the fp32 input lies inside
-// the fp32 error bound of the decision threshold.  The fp64 recomputation
-// forms the +-1 Hadamard sums exactly and divides once by n*sqrt(D), which is
-// the definition evaluated with exact sums, so the stored codes are those of
-// the exact-arithmetic definition except within ~1e-15 of a threshold.
+// rounding of the norm, the nearest centroid, the rounding of (v - z)/s and
+// the fp16 rounding up of the scale) is re-taken in fp64 from the bf16
+// inputs whenever the fp32 input lies inside the fp32 error bound of the
+// decision threshold.  The fp64 recomputation forms the +-1 Hadamard sums
+// exactly and divides once by n*sqrt(D), which is the definition evaluated
+// with exact sums, so the stored codes are those of the exact-arithmetic
+// definition except within ~1e-15 of a threshold.
 #include "tq_kernels.cuh"
 
 namespace tq {
@@ -38,15 +42,17 @@ constexpr float kNormMargin = 1.5e-6f;
 // (fp32 error <= 3 ulp of 15, i.e. 2.7e-6).
 constexpr float kValueMargin = 1.0f / 4096.0f;
 
-constexpr int kBins = 128;  // uniform bins over the midpoint range, per head
+// Uniform bins over y in [-1, 1] (a unit vector's coordinates), width 1/64:
+// bin = (int)(64 y + 64) in [0, 128].
+constexpr int kBins = 129;
+constexpr float kBinScale = 64.0f;
 
 struct HeadBins {
-    float c[16];    // the head's table
-    float mid[16];  // fp32 midpoints m_0..m_14; mid[15] = +inf
-    float lo, inv_w, w;
-    int dense;      // 1: some bin holds more than one midpoint -> exact count path
+    float c[16];  // the head's table
+    int dense;    // 1: some bin holds more than one midpoint -> exact count path
+    int pad;      // keeps the BinEntry array that follows 8-byte aligned
 };
-struct BinEntry {
+struct __align__(8) BinEntry {
     float mid;  // the one midpoint inside the bin (with margins), or +inf
     int k_lo;   // number of midpoints strictly below the bin
 };
@@ -55,29 +61,22 @@ struct BinEntry {
 __device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t* k_tables,
                            const uint16_t* default_table) {
     for (int h = threadIdx.x; h < Hkv; h += blockDim.x) {
-        HeadBins& b = hb[h];
         const uint16_t* src = k_tables ? k_tables + 16 * h : default_table;
-        for (int k = 0; k < 16; k++) b.c[k] = half_bits_to_float(src[k]);
-        for (int k = 0; k < 15; k++) b.mid[k] = 0.5f * (b.c[k] + b.c[k + 1]);
-        b.mid[15] = __int_as_float(0x7f800000);
-        float range = b.mid[14] - b.mid[0];
-        float w = (range > 0.f ? range : 1e-3f) / (kBins - 4);
-        b.w = w;
-        b.inv_w = 1.0f / w;
-        b.lo = b.mid[0] - 2.0f * w;
-        b.dense = 0;
+        for (int k = 0; k < 16; k++) hb[h].c[k] = half_bits_to_float(src[k]);
+        hb[h].dense = 0;
     }
     __syncthreads();
     const float delta = 2.0f * kKeyMargin;
+    const float w = 1.0f / kBinScale;
     for (int e = threadIdx.x; e < Hkv * kBins; e += blockDim.x) {
-        int h = e / kBins, bin = e % kBins;
-        const HeadBins& b = hb[h];
-        float ext_lo = b.lo + bin * b.w - delta;
-        float ext_hi = b.lo + (bin + 1) * b.w + delta;
+        const int h = e / kBins, bin = e % kBins;
+        const float* c = hb[h].c;
+        const float ext_lo = -1.0f + bin * w - delta;
+        const float ext_hi = -1.0f + (bin + 1) * w + delta;
         int below = 0, inside = 0;
         float m_in = __int_as_float(0x7f800000);
         for (int k = 0; k < 15; k++) {
-            float m = b.mid[k];
+            const float m = 0.5f * (c[k] + c[k + 1]);  // exact: fp16 values
             if (m < ext_lo) below++;
             else if (m <= ext_hi) { inside++; m_in = m; }
         }
@@ -88,73 +87,107 @@ __device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t
     __syncthreads();
 }
 
+// n / d for n < 2^32 with M = (2^64 - 1) / d + 1 (exact: the error term of
+// n * M / 2^64 stays below 2^-32 < 1/d); d == 1 is flagged by M == 0.
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, uint64_t M) {
+    return M ? (uint32_t)__umul64hi((uint64_t)n, M) : n;
+}
+
+// fp32 neighbours of 1/15: the value rounded up and rounded down.
+__device__ __forceinline__ float inv15_up() { return __uint_as_float(0x3d888889u); }
+__device__ __forceinline__ float inv15_dn() { return __uint_as_float(0x3d888888u); }
+
+// One warp pass's inputs (prefetched one pass ahead).
+struct Pass {
+    uint4 k, v;  // this lane's 8 bf16 keys / values
+    int slot;    // slot_mapping entry of the token (-1: skip)
+    int pb;      // physical block read from the block table (when one is given)
+    uint32_t vec;
+    bool in;
+};
+
 template <int D>
-__global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+__device__ __forceinline__ void load_pass(const AppendArgs& a, uint32_t p, uint32_t npass,
+                                          uint32_t total, int grp, int sub, Pass& L) {
+    constexpr int VPW = 32 / (D / 8);
+    L.vec = p * VPW + grp;
+    L.in = p < npass && L.vec < total;
+    L.slot = -1;
+    L.pb = -1;
+    L.k = make_uint4(0, 0, 0, 0);
+    L.v = make_uint4(0, 0, 0, 0);
+    if (L.in) {
+        const uint32_t t = fast_div(L.vec, a.div_hkv);
+        L.slot = __ldg(a.slots + t);
+        const size_t eoff = (size_t)L.vec * D + sub * 8;  // vec = t * Hkv + h
+        L.k = ld_stream_u4(a.K + eoff);
+        L.v = ld_stream_u4(a.V + eoff);
+    }
+}
+
+// With a block table, fetch the physical block of the pass's slot (issued one
+// pass before it is used).
+__device__ __forceinline__ void fetch_block(const AppendArgs& a, Pass& L) {
+    if (a.block_table && L.in && L.slot >= 0) {
+        const uint32_t s = (uint32_t)L.slot;
+        const uint32_t seq = fast_div(s, a.div_cap);
+        const uint32_t pos = s - seq * (uint32_t)(a.max_blocks * kBlock);
+        L.pb = seq < (uint32_t)a.num_seqs
+                   ? __ldg(a.block_table + (size_t)seq * a.max_blocks + pos / kBlock)
+                   : -2;  // -2: the logical slot is outside the table
+    }
+}
+
+// f32x2 helpers (B200 packed fp32 pipe)
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+    return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a - b, one rounding
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// 1.5 * 2^23: x + kRound rounds x (0 <= x < 2^22) to the nearest integer,
+// ties to even, and leaves that integer in the low mantissa bits.
+constexpr float kRound = 12582912.0f;
+
+template <int D>
+__global__ void __launch_bounds__(256, 2) append_kernel(AppendArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     HeadBins* hb = reinterpret_cast<HeadBins*>(smem);
     BinEntry* bins = reinterpret_cast<BinEntry*>(hb + a.Hkv);
     build_bins(hb, bins, a.Hkv, a.k_tables, a.default_table);
 
-    constexpr int LPV = D / 8;      // lanes per vector
-    constexpr int VPW = 32 / LPV;   // vectors per warp pass
+    constexpr int LPV = D / 8;     // lanes per vector
+    constexpr int VPW = 32 / LPV;  // vectors per warp pass
     using R = Rec<D>;
     const int lane = threadIdx.x & 31;
     const int sub = lane % LPV;
     const int grp = lane / LPV;
-    const long long total = (long long)a.T * a.Hkv;
-    const long long warps = (long long)gridDim.x * (blockDim.x / 32);
-    const long long warp_id = (long long)blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    const uint32_t total = (uint32_t)a.T * (uint32_t)a.Hkv;
+    const uint32_t npass = (total + VPW - 1) / VPW;
+    const uint32_t nwarps = gridDim.x * (blockDim.x / 32);
+    const uint32_t cap = (uint32_t)(a.max_blocks * kBlock);
 
-    for (long long base = warp_id * VPW; base < total; base += warps * VPW) {
-        const long long vec = base + grp;
-        int t = 0, h = 0, blk = -1, off = 0;
-        if (vec < total) {
-            t = (int)(vec / a.Hkv);
-            h = (int)(vec - (long long)t * a.Hkv);
-            int s = a.slots[t];
-            if (s >= 0) {
-                if (a.block_table) {
-                    long long cap = (long long)a.max_blocks * kBlock;
-                    long long seq = s / cap, pos = s - seq * cap;
-                    if (seq < a.num_seqs) {
-                        int pb = a.block_table[seq * a.max_blocks + pos / kBlock];
-                        if (pb >= 0 && pb < a.num_blocks) {
-                            blk = pb;
-                            off = (int)(pos % kBlock);
-                        } else if (sub == 0) {
-                            flag_status(a.status, TQ_STATUS_BAD_BLOCK);
-                        }
-                    } else if (sub == 0) {
-                        flag_status(a.status, TQ_STATUS_BAD_SLOT);
-                    }
-                } else {
-                    if (s / kBlock < a.num_blocks) {
-                        blk = s / kBlock;
-                        off = s % kBlock;
-                    } else if (sub == 0) {
-                        flag_status(a.status, TQ_STATUS_BAD_SLOT);
-                    }
-                }
-            }
-        }
-        const bool work = blk >= 0;
-        // every lane takes part in the shuffles; lanes without work carry zeros
-        uint4 kraw = make_uint4(0, 0, 0, 0), vraw = make_uint4(0, 0, 0, 0);
-        if (work) {
-            const size_t eoff = ((size_t)t * a.Hkv + h) * D + sub * 8;
-            kraw = ld_stream_u4(a.K + eoff);
-            vraw = ld_stream_u4(a.V + eoff);
-        }
-        float k[8];
-        k[0] = bf16_lo(kraw.x); k[1] = bf16_hi(kraw.x);
-        k[2] = bf16_lo(kraw.y); k[3] = bf16_hi(kraw.y);
-        k[4] = bf16_lo(kraw.z); k[5] = bf16_hi(kraw.z);
-        k[6] = bf16_lo(kraw.w); k[7] = bf16_hi(kraw.w);
+    Pass cur, nxt;
+    uint32_t pass = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    load_pass<D>(a, pass, npass, total, grp, sub, cur);
+    fetch_block(a, cur);
 
-        // ---- key: norm
-        float ss = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; e++) ss = fmaf(k[e], k[e], ss);
+    for (; pass < npass; pass += nwarps) {
+        load_pass<D>(a, pass + nwarps, npass, total, grp, sub, nxt);
+        const uint32_t t = fast_div(cur.vec, a.div_hkv);
+        const int h = cur.in ? (int)(cur.vec - t * (uint32_t)a.Hkv) : 0;
+
+        // ---- key: norm (elements 2i, 2i+1 in P[i])
+        float2 P[4];
+        P[0] = make_float2(bf16_lo(cur.k.x), bf16_hi(cur.k.x));
+        P[1] = make_float2(bf16_lo(cur.k.y), bf16_hi(cur.k.y));
+        P[2] = make_float2(bf16_lo(cur.k.z), bf16_hi(cur.k.z));
+        P[3] = make_float2(bf16_lo(cur.k.w), bf16_hi(cur.k.w));
+        float2 q2 = mul2(P[0], P[0]);
+        q2 = __ffma2_rn(P[1], P[1], q2);
+        q2 = __ffma2_rn(P[2], P[2], q2);
+        q2 = __ffma2_rn(P[3], P[3], q2);
+        float ss = q2.x + q2.y;
 #pragma unroll
         for (int m = 1; m < LPV; m <<= 1) ss += __shfl_xor_sync(kFull, ss, m);
         const float n = sqrtf(ss);
@@ -165,27 +198,26 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
         // fp32 error bound: take the fp64 path
         near |= !(ss >= 1e-30f && ss <= 1e30f) && ss != 0.f;
 
-        // ---- key: unnormalised Hadamard butterfly (3 in-lane bits, log2(LPV) lane bits)
-        float S[8];
+        // ---- key: unnormalised Hadamard butterfly.  Index bit 0 lies inside a
+        // pair, bits 1-2 across pairs (packed adds), the rest across lanes.
+        float2 Q[4];
 #pragma unroll
-        for (int e = 0; e < 8; e++) S[e] = k[e];
-#pragma unroll
-        for (int b = 1; b < 8; b <<= 1) {
-#pragma unroll
-            for (int e = 0; e < 8; e++)
-                if (!(e & b)) {
-                    float x = S[e], y = S[e | b];
-                    S[e] = x + y;
-                    S[e | b] = x - y;
-                }
+        for (int i = 0; i < 4; i++) Q[i] = make_float2(P[i].x + P[i].y, P[i].x - P[i].y);
+        {
+            const float2 a0 = add2(Q[0], Q[1]), a1 = sub2(Q[0], Q[1]);
+            const float2 a2 = add2(Q[2], Q[3]), a3 = sub2(Q[2], Q[3]);
+            Q[0] = add2(a0, a2); Q[2] = sub2(a0, a2);
+            Q[1] = add2(a1, a3); Q[3] = sub2(a1, a3);
         }
 #pragma unroll
         for (int m = 1; m < LPV; m <<= 1) {
-            const bool upper = sub & m;
+            const float sg = (sub & m) ? -1.f : 1.f;  // upper half: partner - own
+            const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-            for (int e = 0; e < 8; e++) {
-                float p = __shfl_xor_sync(kFull, S[e], m);
-                S[e] = upper ? p - S[e] : S[e] + p;
+            for (int i = 0; i < 4; i++) {
+                const float2 pr = make_float2(__shfl_xor_sync(kFull, Q[i].x, m),
+                                              __shfl_xor_sync(kFull, Q[i].y, m));
+                Q[i] = __ffma2_rn(sg2, Q[i], pr);
             }
         }
         const float inv = ss > 0.f ? rsqrtf(ss * (float)D) : 0.f;
@@ -194,40 +226,60 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
         const HeadBins& B = hb[h];
         const BinEntry* hbins = bins + h * kBins;
         uint32_t kw = 0;
-        if (!B.dense) {
+        float y[8];
+        {
+            const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
-            for (int e = 0; e < 8; e++) {
-                float y = S[e] * inv;
-                float pos = fminf(fmaxf((y - B.lo) * B.inv_w, 0.f), (float)(kBins - 1));
-                BinEntry be = hbins[(int)pos];
-                int idx = be.k_lo + (y > be.mid ? 1 : 0);
-                near |= fabsf(y - be.mid) < kKeyMargin;
-                kw |= (uint32_t)idx << (4 * e);
+            for (int i = 0; i < 4; i++) {
+                const float2 yy = mul2(Q[i], inv2);
+                y[2 * i] = yy.x;
+                y[2 * i + 1] = yy.y;
             }
+        }
+        if (!B.dense) {
+            uint32_t nib[8];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const float2 ps = __ffma2_rn(make_float2(y[2 * i], y[2 * i + 1]),
+                                            make_float2(kBinScale, kBinScale),
+                                            make_float2(kBinScale, kBinScale));
+                const int b0 = max(min((int)ps.x, kBins - 1), 0);
+                const int b1 = max(min((int)ps.y, kBins - 1), 0);
+                const BinEntry e0 = hbins[b0], e1 = hbins[b1];
+                const float d0 = y[2 * i] - e0.mid, d1 = y[2 * i + 1] - e1.mid;
+                nib[2 * i] = (uint32_t)(e0.k_lo + (d0 > 0.f ? 1 : 0));
+                nib[2 * i + 1] = (uint32_t)(e1.k_lo + (d1 > 0.f ? 1 : 0));
+                near |= fmaxf(fabsf(d0), fabsf(d1)) < kKeyMargin;
+            }
+            // bytes (nib[2j] | nib[2j+1] << 4), j = 0..3, into one word
+            const uint32_t b01 = __byte_perm(nib[0] | (nib[1] << 4), nib[2] | (nib[3] << 4), 0x0040);
+            const uint32_t b23 = __byte_perm(nib[4] | (nib[5] << 4), nib[6] | (nib[7] << 4), 0x0040);
+            kw = __byte_perm(b01, b23, 0x5410);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; e++) {
-                float y = S[e] * inv;
                 int idx = 0;
                 for (int j = 0; j < 15; j++) {
-                    idx += y > B.mid[j] ? 1 : 0;
-                    near |= fabsf(y - B.mid[j]) < kKeyMargin;
+                    const float dm = y[e] - 0.5f * (B.c[j] + B.c[j + 1]);
+                    idx += dm > 0.f ? 1 : 0;
+                    near |= fabsf(dm) < kKeyMargin;
                 }
                 kw |= (uint32_t)idx << (4 * e);
             }
         }
-        near = near && work;
+        near = near && cur.in && cur.slot >= 0;
 
         // ---- key: fp64 recomputation when any decision of the warp is close
         if (__any_sync(kFull, near)) {
-            double kd[8], Sd[8];
+            double Sd[8];
             double ssd = 0.0;
 #pragma unroll
-            for (int e = 0; e < 8; e++) {
-                kd[e] = (double)k[e];
-                ssd = fma(kd[e], kd[e], ssd);
-                Sd[e] = kd[e];
+            for (int i = 0; i < 4; i++) {
+                Sd[2 * i] = (double)P[i].x;
+                Sd[2 * i + 1] = (double)P[i].y;
             }
+#pragma unroll
+            for (int e = 0; e < 8; e++) ssd = fma(Sd[e], Sd[e], ssd);
 #pragma unroll
             for (int m = 1; m < LPV; m <<= 1) ssd += __shfl_xor_sync(kFull, ssd, m);
             const double nd = sqrt(ssd);
@@ -236,9 +288,9 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
 #pragma unroll
                 for (int e = 0; e < 8; e++)
                     if (!(e & b)) {
-                        double x = Sd[e], y = Sd[e | b];
-                        Sd[e] = x + y;
-                        Sd[e | b] = x - y;
+                        const double x = Sd[e], yv = Sd[e | b];
+                        Sd[e] = x + yv;
+                        Sd[e | b] = x - yv;
                     }
             }
 #pragma unroll
@@ -246,37 +298,35 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
                 const bool upper = sub & m;
 #pragma unroll
                 for (int e = 0; e < 8; e++) {
-                    double p = __shfl_xor_sync(kFull, Sd[e], m);
+                    const double p = __shfl_xor_sync(kFull, Sd[e], m);
                     Sd[e] = upper ? p - Sd[e] : Sd[e] + p;
                 }
             }
-            if (work) {
+            if (cur.in) {
                 n16 = __half_as_ushort(__double2half(nd));
                 const double denom = nd * sqrt((double)D);
                 kw = 0;
 #pragma unroll
                 for (int e = 0; e < 8; e++) {
-                    double y = nd > 0.0 ? Sd[e] / denom : 0.0;
+                    const double yd = nd > 0.0 ? Sd[e] / denom : 0.0;
                     int idx = 0;
                     for (int j = 0; j < 15; j++)
-                        idx += y > 0.5 * ((double)B.c[j] + (double)B.c[j + 1]) ? 1 : 0;
+                        idx += yd > 0.5 * ((double)B.c[j] + (double)B.c[j + 1]) ? 1 : 0;
                     kw |= (uint32_t)idx << (4 * e);
                 }
             }
         }
 
         // ---- values: group of 32 = 4 lanes
-        float v[8];
-        v[0] = bf16_lo(vraw.x); v[1] = bf16_hi(vraw.x);
-        v[2] = bf16_lo(vraw.y); v[3] = bf16_hi(vraw.y);
-        v[4] = bf16_lo(vraw.z); v[5] = bf16_hi(vraw.z);
-        v[6] = bf16_lo(vraw.w); v[7] = bf16_hi(vraw.w);
-        float mn = v[0], mx = v[0];
-#pragma unroll
-        for (int e = 1; e < 8; e++) {
-            mn = fminf(mn, v[e]);
-            mx = fmaxf(mx, v[e]);
-        }
+        float2 V2[4];
+        V2[0] = make_float2(bf16_lo(cur.v.x), bf16_hi(cur.v.x));
+        V2[1] = make_float2(bf16_lo(cur.v.y), bf16_hi(cur.v.y));
+        V2[2] = make_float2(bf16_lo(cur.v.z), bf16_hi(cur.v.z));
+        V2[3] = make_float2(bf16_lo(cur.v.w), bf16_hi(cur.v.w));
+        float mn = fminf(fminf(fminf(V2[0].x, V2[0].y), fminf(V2[1].x, V2[1].y)),
+                         fminf(fminf(V2[2].x, V2[2].y), fminf(V2[3].x, V2[3].y)));
+        float mx = fmaxf(fmaxf(fmaxf(V2[0].x, V2[0].y), fmaxf(V2[1].x, V2[1].y)),
+                         fmaxf(fmaxf(V2[2].x, V2[2].y), fmaxf(V2[3].x, V2[3].y)));
 #pragma unroll
         for (int m = 1; m < 4; m <<= 1) {
             mn = fminf(mn, __shfl_xor_sync(kFull, mn, m));
@@ -284,29 +334,69 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
         }
         const __half zh = __float2half_rd(mn);  // exact: mn is a bf16 value
         const float zf = __half2float(zh);
-        const uint16_t s16 = double_to_half_up_nonneg(((double)mx - (double)zf) / 15.0);
+        // s = fp16 rounded up from (mx - z)/15: bracket the quotient in fp32 with
+        // directed roundings; if both ends round up to the same fp16 value it is
+        // the answer, otherwise (an fp16 value inside the bracket) use fp64.
+        uint16_t s16;
+        {
+            const float hi = __fmul_ru(__fsub_ru(mx, zf), inv15_up());
+            const float lo = __fmul_rd(__fsub_rd(mx, zf), inv15_dn());
+            const uint16_t s_hi = __half_as_ushort(__float2half_ru(hi));
+            const uint16_t s_lo = __half_as_ushort(__float2half_ru(lo));
+            s16 = s_hi;
+            if (s_hi != s_lo) s16 = double_to_half_up_nonneg(((double)mx - (double)zf) / 15.0);
+        }
         const float sf = half_bits_to_float(s16);
         uint32_t vw = 0;
         if (sf > 0.f) {
-            const float inv_s = 1.0f / sf;
+            const float inv_s = __frcp_rn(sf);
+            const float2 z2 = make_float2(zf, zf), is2 = make_float2(inv_s, inv_s);
+            const float2 rnd = make_float2(kRound, kRound);
+            uint32_t qb[8];
+            bool tie = false;
 #pragma unroll
-            for (int e = 0; e < 8; e++) {
-                float r = (v[e] - zf) * inv_s;
-                unsigned q;
-                if (fabsf(r - floorf(r) - 0.5f) < kValueMargin) {
-                    // near a .5 rounding point: exact quotient in fp64
-                    double rd = ((double)v[e] - (double)zf) / (double)sf;
-                    q = (unsigned)rint(rd);
-                } else {
-                    q = __float2uint_rn(r);
-                }
-                vw |= (q > 15u ? 15u : q) << (4 * e);
+            for (int i = 0; i < 4; i++) {
+                const float2 r = mul2(sub2(V2[i], z2), is2);  // (v - z) / s, in [0, 15]
+                const float2 tr = add2(r, rnd);               // round half to even
+                const float2 d = sub2(r, sub2(tr, rnd));      // r - round(r)
+                tie |= fmaxf(fabsf(d.x), fabsf(d.y)) > 0.5f - kValueMargin;
+                qb[2 * i] = __float_as_uint(tr.x);            // low byte = code
+                qb[2 * i + 1] = __float_as_uint(tr.y);
             }
+            if (tie) {  // a .5 point within the fp32 error: exact quotients in fp64
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    qb[2 * i] = (uint32_t)rint(((double)V2[i].x - (double)zf) / (double)sf);
+                    qb[2 * i + 1] = (uint32_t)rint(((double)V2[i].y - (double)zf) / (double)sf);
+                }
+            }
+            const uint32_t even = __byte_perm(__byte_perm(qb[0], qb[2], 0x0040),
+                                              __byte_perm(qb[4], qb[6], 0x0040), 0x5410);
+            const uint32_t odd = __byte_perm(__byte_perm(qb[1], qb[3], 0x0040),
+                                             __byte_perm(qb[5], qb[7], 0x0040), 0x5410);
+            vw = ((even & 0x0f0f0f0fu) | ((odd & 0x0f0f0f0fu) << 4));
         }
 
-        if (work) {
-            unsigned char* rec =
-                a.cache + ((size_t)blk * a.Hkv + h) * (size_t)R::kBytes;
+        // ---- where this vector goes (the block-table read was issued a pass ago)
+        int blk = -1, off = 0;
+        if (cur.in && cur.slot >= 0) {
+            if (a.block_table) {
+                if (cur.pb >= 0 && cur.pb < a.num_blocks) {
+                    blk = cur.pb;
+                    off = (int)(((uint32_t)cur.slot - fast_div((uint32_t)cur.slot, a.div_cap) * cap) %
+                                kBlock);
+                } else if (sub == 0) {
+                    flag_status(a.status, cur.pb == -2 ? TQ_STATUS_BAD_SLOT : TQ_STATUS_BAD_BLOCK);
+                }
+            } else if (cur.slot / kBlock < a.num_blocks) {
+                blk = cur.slot / kBlock;
+                off = cur.slot % kBlock;
+            } else if (sub == 0) {
+                flag_status(a.status, TQ_STATUS_BAD_SLOT);
+            }
+        }
+        if (blk >= 0) {
+            unsigned char* rec = a.cache + ((size_t)blk * a.Hkv + h) * (size_t)R::kBytes;
             *reinterpret_cast<uint32_t*>(rec + R::kKCodes + off * R::kCodeRow + sub * 4) = kw;
             unsigned char* vrow = rec + R::kVCodes + off * R::kCodeRow;
 #pragma unroll
@@ -314,14 +404,16 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
             if (sub == 0) *reinterpret_cast<uint16_t*>(rec + R::kKNorm + off * 2) = n16;
             if ((sub & 3) == 0) {
                 const uint16_t z16 = __half_as_ushort(zh);
-                *reinterpret_cast<uint32_t*>(rec + R::kVGroups +
-                                             (off * R::kGroups + sub / 4) * 4) =
+                *reinterpret_cast<uint32_t*>(rec + R::kVGroups + (off * R::kGroups + sub / 4) * 4) =
                     (uint32_t)s16 | ((uint32_t)z16 << 16);
-                bool bad = !isfinite(sf) || !isfinite(zf) ||
-                           (sub == 0 && !isfinite(half_bits_to_float(n16)));
+                const bool bad = !isfinite(sf) || !isfinite(zf) ||
+                                 (sub == 0 && !isfinite(half_bits_to_float(n16)));
                 if (bad) flag_status(a.status, TQ_STATUS_RANGE);
             }
         }
+
+        fetch_block(a, nxt);  // its slot has arrived by now
+        cur = nxt;
     }
 }
 
@@ -329,21 +421,41 @@ size_t append_smem_bytes(int Hkv) {
     return (size_t)Hkv * sizeof(HeadBins) + (size_t)Hkv * kBins * sizeof(BinEntry);
 }
 
-cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream) {
+// (2^64 - 1) / d + 1: the multiplier of fast_div (0 for d == 1).
+static uint64_t div_magic(uint32_t d) { return d <= 1 ? 0 : ~0ull / d + 1; }
+
+template <int D>
+static int resident_ctas(int num_sms, size_t smem) {
+    static int per_sm[2] = {0, 0};  // by (smem size class); set once per process
+    const int key = smem > 16384 ? 1 : 0;
+    if (!per_sm[key]) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_kernel<D>, 256, smem) !=
+                cudaSuccess || n <= 0)
+            n = 1;
+        per_sm[key] = n;
+    }
+    return per_sm[key] * num_sms;
+}
+
+cudaError_t launch_append(const AppendArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
+    AppendArgs a = args;
+    a.div_hkv = div_magic((uint32_t)a.Hkv);
+    a.div_cap = div_magic((uint32_t)(a.max_blocks > 0 ? a.max_blocks * kBlock : 1));
     const int threads = 256;
     const long long vectors = (long long)a.T * a.Hkv;
     const int vpw = 32 / (head_dim / 8);
-    long long warps_needed = (vectors + vpw - 1) / vpw;
+    const long long warps_needed = (vectors + vpw - 1) / vpw;
     long long blocks = (warps_needed + threads / 32 - 1) / (threads / 32);
-    const long long cap = (long long)num_sms * 8;  // grid-stride beyond 8 CTAs per SM
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
     const size_t smem = append_smem_bytes(a.Hkv);
-    if (head_dim == 128) {
+    const long long cap = head_dim == 128 ? resident_ctas<128>(num_sms, smem)
+                                          : resident_ctas<64>(num_sms, smem);
+    if (blocks > cap) blocks = cap;  // one wave; warps loop over the passes
+    if (blocks < 1) blocks = 1;
+    if (head_dim == 128)
         append_kernel<128><<<(unsigned)blocks, threads, smem, stream>>>(a);
-    } else {
+    else
         append_kernel<64><<<(unsigned)blocks, threads, smem, stream>>>(a);
-    }
     return cudaGetLastError();
 }
 

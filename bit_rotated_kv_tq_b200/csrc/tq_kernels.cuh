@@ -18,6 +18,7 @@ struct AppendArgs {
     const uint16_t* k_tables;   // fp16 [Hkv][16] or null
     uint16_t default_table[16]; // fp16
     int32_t* status;
+    uint64_t div_hkv, div_cap;  // fast-division multipliers (set by the launcher)
 };
 
 struct DecodeArgs {
