@@ -19,9 +19,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -69,60 +67,83 @@ def append_bytes(w, T) -> int:
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples while the timed region runs."""
+    """SM clock and clock-event reasons, polled through NVML every ~1 ms by a
+    thread while the timed region runs (read-only; no setting is changed).
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    mark_start()/mark_end() bracket the timed region on the host clock; the
+    summary uses the samples inside it, or the nearest ones when the region is
+    shorter than a polling period."""
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
-        self.proc = None
-        self.path = None
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, bus_id: str):
+        self.bus_id = bus_id
+        self.samples = []  # (host time, sm MHz, reason bits)
+        self.t0 = self.t1 = None
+        self.err = None
 
     def __enter__(self):
+        import threading
+
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
-            os.close(fd)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(self.bus_id)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: report it, do not fail the bench
+            self.err = f"nvml unavailable: {type(e).__name__}"
+            return self
+        self.stop = False
+
+        def poll():
+            while not self.stop:
+                try:
+                    mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                    rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                    self.samples.append((time.perf_counter(), mhz, rs))
+                except Exception:
+                    pass
+                time.sleep(0.001)
+
+        self.th = threading.Thread(target=poll, daemon=True)
+        self.th.start()
+        time.sleep(0.02)  # a few samples before the region starts
         return self
 
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        if self.err is None:
+            time.sleep(0.005)
+            self.stop = True
+            self.th.join(timeout=2)
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        if self.err is not None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no samples"]}
+        inside = [s for s in self.samples if self.t0 <= s[0] <= self.t1]
+        if not inside:  # region shorter than a polling period: the samples around it
+            inside = sorted(self.samples, key=lambda s: min(abs(s[0] - self.t0), abs(s[0] - self.t1)))[:2]
+        bits = 0
+        for s in inside:
+            bits |= s[2]
+        reasons = [name for name, const in self.REASONS if bits & getattr(self.nv, const, 0)]
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside)}
 
 
 def smi_id(local: int) -> str:
-    """The nvidia-smi id (PCI bus id when torch exposes it) of local CUDA device `local`."""
+    """The NVML / nvidia-smi id (PCI bus id when torch exposes it) of local CUDA device `local`."""
     props = torch.cuda.get_device_properties(local)
     bus = getattr(props, "pci_bus_id", None)
     if bus is not None and getattr(props, "pci_domain_id", None) is not None:
@@ -236,6 +257,30 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def profiled_traffic(w):
+    """DRAM bytes (read + write) per launch of the decode split kernel, from the
+    committed ncu summary, or None when the kernel source has changed since it was
+    taken or the workload is not the one the figure was scaled to."""
+    import hashlib
+
+    prof = os.path.join(ROOT, "profiles", "decode_split_kernel_qwen3_8b_layer.md")
+    src = os.path.join(ROOT, "bit_rotated_kv_tq_b200", "csrc", "tq_decode.cu")
+    if not (os.path.exists(prof) and os.path.exists(src)):
+        return None
+    fields = {}
+    with open(prof) as f:
+        for ln in f:
+            if ":" in ln and not ln.startswith(("|", " ", "#")):
+                k, v = ln.split(":", 1)
+                fields[k.strip()] = v.strip()
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    key = f"traffic_bytes_per_launch_b{w.B}"
+    if fields.get("source_sha256") != sha or key not in fields or int(w.seq_lens[0]) != 8192:
+        return None
+    return int(fields[key])
+
+
 def cfg(w, l2):
     return {"workload": f"{w.name}: {w.B} seqs x {int(w.seq_lens[0])} tokens, {w.Hq} q / {w.Hkv} kv heads, "
                         f"d {w.d}, block 16, shuffled block tables, {w.append_tokens}-token append per seq",
@@ -249,7 +294,7 @@ def run_tq(args, rank, world, local):
     tq.load()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    w = W.make(WORKLOAD)
+    w = W.make(WORKLOAD, B=args.batch) if args.batch else W.make(WORKLOAD)
     cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
     bt = torch.from_numpy(w.block_tables).to(dev)
     lens = torch.from_numpy(w.seq_lens).to(dev)
@@ -288,11 +333,13 @@ def run_tq(args, rank, world, local):
     barrier(world)
     torch.cuda.synchronize(dev)
     with ClockSampler(smi_id(local)) as clk:
+        clk.mark_start()
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         end.record(stream)
         torch.cuda.synchronize(dev)
+        clk.mark_end()
     barrier(world)
     total_ms = start.elapsed_time(end)
     app_ms = [e[0].elapsed_time(e[1]) for e in evs]
@@ -357,7 +404,7 @@ def run_tq(args, rank, world, local):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": cfg(w, "inputs larger than L2: 306 MB cache per rank vs 126 MB L2, no flush"),
+            "config": cfg(w, f"inputs larger than L2: {kv / 1e6:.0f} MB cache read per rank vs 126 MB L2, no flush"),
             "decode_gbs": kv / (dec_avg / 1e3) / 1e9,
             "decode_hbm_frac": kv / (dec_avg / 1e3) / 1e9 / peak,
             "decode_ms": dec_avg, "append_ms": app_avg,
@@ -365,7 +412,7 @@ def run_tq(args, rank, world, local):
             "append_hbm_frac": append_bytes(w, T) / (app_avg / 1e3) / 1e9 / peak,
             "num_splits": S,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None,
+                         "frac": achieved / peak, "traffic": profiled_traffic(w),
                          "kernel": "tq_decode_attention (split kernel + combine)",
                          "peak_source": f"{peak_kind} hbm_gbs"},
             "e2e": {"value": weak_scaling_value(kv, args.steps, world, e2e_s) / 1e9, "unit": "GB/s",
@@ -384,6 +431,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="sequences per rank (default: the workload's 32); smaller values make the "
+                         "profiling case, not a bench line")
     args = ap.parse_args()
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", 0))
