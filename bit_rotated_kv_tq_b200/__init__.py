@@ -24,7 +24,8 @@ BLOCK = 16
 VALUE_GROUP = 32
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_ALIGNMENT, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(6)
-STATUS_BAD_SLOT, STATUS_BAD_BLOCK, STATUS_RANGE, STATUS_BAD_LEN, STATUS_TIMEOUT = 1, 2, 4, 8, 16
+STATUS_BAD_SLOT, STATUS_BAD_BLOCK, STATUS_RANGE, STATUS_BAD_LEN, STATUS_TIMEOUT, STATUS_INTERNAL = \
+    1, 2, 4, 8, 16, 32
 
 
 class TQError(RuntimeError):

@@ -267,14 +267,27 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
 TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len) {
     if (B <= 0 || H_kv <= 0 || max_seq_len <= 0) return 1;
     const int nblk = (max_seq_len + tq::kBlock - 1) / tq::kBlock;
-    const long long pairs = (long long)B * H_kv;
-    // The split kernel runs two 8-warp CTAs per SM.  Aim for about four waves
-    // of CTAs over the GPU, keeping at least 32 blocks (4 per warp) per split.
-    long long s = (8LL * device_sms() + pairs - 1) / pairs;
-    s = std::min<long long>(s, std::max(1, nblk / 32));
-    s = std::max<long long>(1, std::min<long long>(s, 1024));
-    const int bps = (int)((nblk + s - 1) / s);
-    return (nblk + bps - 1) / bps;
+    const long long items = (long long)B * H_kv;  // one group of up to four query heads each
+    const long long halves = 2LL * device_sms();
+    // The split kernel is persistent: two halves of 8 warps per SM, each taking
+    // (item, split) units in turn.  Estimated time, in units of one record per
+    // warp: rounds of units x (records per warp per unit + per-unit overhead),
+    // plus the combine pass when there is more than one split.
+    constexpr double kUnitOverhead = 0.75, kCombine = 2.5;
+    int best_s = 1;
+    double best = 1e300;
+    for (int s = 1; s <= 64 && s <= nblk; s++) {
+        const int bps = (nblk + s - 1) / s;
+        const int S = (nblk + bps - 1) / bps;
+        if (S != s) continue;  // the same plan as a smaller s
+        const long long rounds = (items * S + halves - 1) / halves;
+        const double cost = (double)rounds * ((bps + 7) / 8 + kUnitOverhead) + (S > 1 ? kCombine : 0.0);
+        if (cost < best) {
+            best = cost;
+            best_s = S;
+        }
+    }
+    return best_s;
 }
 
 TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_splits) {
@@ -315,6 +328,9 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
     const int nblk = (max_seq_len + tq::kBlock - 1) / tq::kBlock;
     int bps = nblk > 0 ? (nblk + S_req - 1) / S_req : 1;
     int S = nblk > 0 ? (nblk + bps - 1) / bps : 1;
+    const long long units = (long long)B * Hkv * ((G + 3) / 4) * S;
+    if (units > 0x7fffffffLL)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * splits too large");
     if (S > 1) {
         const size_t need = tq_decode_workspace_bytes(B, H_q, d, S);
         if (!workspace || ws_bytes < need)
@@ -344,7 +360,7 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
                                                  (size_t)B * H_q * S * d)
                     : nullptr;
     a.status = status;
-    cudaError_t e = tq::launch_decode(a, d, (cudaStream_t)stream);
+    cudaError_t e = tq::launch_decode(a, d, device_sms(), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");
     return ok();
 }

@@ -398,14 +398,15 @@ __global__ void __launch_bounds__(256, 2) append_kernel(AppendArgs a) {
         if (blk >= 0) {
             unsigned char* rec = a.cache + ((size_t)blk * a.Hkv + h) * (size_t)R::kBytes;
             *reinterpret_cast<uint32_t*>(rec + R::kKCodes + off * R::kCodeRow + sub * 4) = kw;
-            unsigned char* vrow = rec + R::kVCodes + off * R::kCodeRow;
+            // bytes j = 4 sub + i share m = sub / 2 and spread over r = 4 (sub % 2) + i
+            unsigned char* vdst = rec + R::kVCodes + R::vcode_pos(off, 4 * sub);
 #pragma unroll
-            for (int i = 0; i < 4; i++) vrow[R::vpos(sub * 4 + i)] = (unsigned char)(vw >> (8 * i));
+            for (int i = 0; i < 4; i++) vdst[i * R::kPairChunk] = (unsigned char)(vw >> (8 * i));
             if (sub == 0) *reinterpret_cast<uint16_t*>(rec + R::kKNorm + off * 2) = n16;
             if ((sub & 3) == 0) {
-                const uint16_t z16 = __half_as_ushort(zh);
-                *reinterpret_cast<uint32_t*>(rec + R::kVGroups + (off * R::kGroups + sub / 4) * 4) =
-                    (uint32_t)s16 | ((uint32_t)z16 << 16);
+                const int gp = R::group_pos(off, sub / 4);
+                *reinterpret_cast<uint16_t*>(rec + R::kVScale + gp) = s16;
+                *reinterpret_cast<uint16_t*>(rec + R::kVZero + gp) = __half_as_ushort(zh);
                 const bool bad = !isfinite(sf) || !isfinite(zf) ||
                                  (sub == 0 && !isfinite(half_bits_to_float(n16)));
                 if (bad) flag_status(a.status, TQ_STATUS_RANGE);

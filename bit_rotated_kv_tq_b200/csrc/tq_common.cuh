@@ -2,12 +2,14 @@
 // TQ4/4 kernels (append, decode, combine, dequantise).
 //
 // Record of one (physical block, kv head), 16 tokens, head_dim D:
-//   [0, 8D)         key codes    [16][D/2] bytes, element 2j in the low nibble of byte j
-//   [8D, 8D+32)     key norms    [16] fp16
-//   [8D+32, 16D+32) value codes  [16][D/2] bytes, same nibble order; value byte j is
-//                   stored at row offset (j % 8) * (D/16) + j / 8 so that the bytes one
-//                   lane feeds to the tensor cores (j = 8m + g, m = 0..D/16-1) are contiguous
-//   [16D+32, 18D+32) value groups [16][D/32] x (fp16 scale, fp16 zero)
+//   [0, 8D)           key codes    [16][D/2] bytes, element 2j in the low nibble of byte j
+//   [8D, 8D+32)       key norms    [16] fp16
+//   [8D+32, 16D+32)   value codes  8D bytes, same nibble order, placed for the decode
+//                     fragments: byte j = 8m + r of token t sits at
+//                     (8 (t/2) + r) (D/8) + 4 (m/2) + 2 (t%2) + (m%2)
+//   [16D+32, 17D+32)  value scales fp16, the one of token t, group G at byte
+//                     2 (4 (c (D/32) + G) + u), c = (t%8)/2, u = 2 (t/8) + t%2
+//   [17D+32, 18D+32)  value zeros  fp16, same placement
 // The cache is [num_blocks][H_kv][record]; every field starts 16-byte aligned.
 #pragma once
 
@@ -26,17 +28,27 @@ constexpr unsigned kFull = 0xffffffffu;
 
 template <int D>
 struct Rec {
-    static constexpr int kCodeRow = D / 2;                 // bytes of one token's codes
+    static constexpr int kCodeRow = D / 2;                        // bytes of one token's codes
     static constexpr int kKCodes = 0;
-    static constexpr int kKNorm = kBlock * kCodeRow;        // 8D
-    static constexpr int kVCodes = kKNorm + 2 * kBlock;     // 8D + 32
-    static constexpr int kVGroups = kVCodes + kBlock * kCodeRow;  // 16D + 32
+    static constexpr int kKNorm = kBlock * kCodeRow;               // 8D
+    static constexpr int kVCodes = kKNorm + 2 * kBlock;            // 8D + 32
+    static constexpr int kVScale = kVCodes + kBlock * kCodeRow;    // 16D + 32
+    static constexpr int kVZero = kVScale + D;                     // 17D + 32
     static constexpr int kGroups = D / kGroup;
-    static constexpr int kVStride = D / 16;  // value byte j -> row offset (j % 8) * kVStride + j / 8
-    static __host__ __device__ constexpr int vpos(int j) { return (j % 8) * kVStride + j / 8; }
-    static constexpr int kBytes = kVGroups + kBlock * kGroups * 4;  // 18D + 32
-    static_assert(kKNorm % 16 == 0 && kVCodes % 16 == 0 && kVGroups % 16 == 0 &&
-                      kBytes % 16 == 0,
+    static constexpr int kBytes = kVZero + D;                      // 18D + 32
+    static constexpr int kPairChunk = D / 8;  // value bytes of one (token pair, r) chunk
+    // value byte j of token t, relative to kVCodes
+    static __host__ __device__ constexpr int vcode_pos(int t, int j) {
+        return (8 * (t >> 1) + (j & 7)) * kPairChunk + 4 * ((j >> 3) >> 1) + 2 * (t & 1) +
+               ((j >> 3) & 1);
+    }
+    // scale (zero) of token t, group G, relative to kVScale (kVZero)
+    static __host__ __device__ constexpr int group_pos(int t, int G) {
+        return 2 * (4 * (((t & 7) >> 1) * kGroups + G) + 2 * (t >> 3) + (t & 1));
+    }
+    static_assert(D % 32 == 0, "head_dim must be a multiple of 32");
+    static_assert(kKNorm % 16 == 0 && kVCodes % 16 == 0 && kVScale % 16 == 0 &&
+                      kVZero % 16 == 0 && kBytes % 16 == 0,
                   "record fields must stay 16-byte aligned");
 };
 

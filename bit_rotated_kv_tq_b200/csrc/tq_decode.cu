@@ -7,22 +7,30 @@
 // Values: v_hat = code * s + z per group of 32, so
 //   o = sum_t p_t v_hat_t = sum_t (p_t s_t,g) code_t + sum_t p_t z_t,g.
 //
-// Work: one CTA per (split, kv head, sequence); 8 warps take the split's
-// 16-token blocks round-robin.  Each warp streams its blocks' records (2336
-// bytes at d=128, 1184 at d=64) through a private ring of shared-memory
-// stages with bulk asynchronous copies (cp.async.bulk + mbarrier).  Per block
-// every product runs on the tensor cores (mma.sync m16n8k16, fp32 accumulate):
-//   q.K  A = 16 tokens x 16 dims of fp16 centroids, fetched two at a time
-//        from a 256-entry byte -> (C[lo], C[hi]) table held once per lane
-//        (conflict-free); B = q~ as fp16 high and low parts in adjacent
-//        columns of the same head, so scores carry q~ to ~22 bits;
-//   p.V  A = 16 dims x 16 tokens of value codes made exact fp16 integers by
-//        a mask-and-bias nibble trick; B = p_t s_t,g as exact fp16 two-part
-//        products (an fma two-product of the fp16 halves of p and the fp16
-//        scale);
-//   p.z  A = the fp16 zero points (exact), B = p as fp16 high and low parts.
+// Work.  An item is (sequence, kv head, group of four query heads); a unit is
+// (item, split of the context).  The grid is persistent: one CTA of 16 warps
+// per SM, made of two independent halves of 8 warps, each half walking its
+// own list of units.  Within a unit the 8 warps take the split's 16-token
+// blocks round-robin.  Each warp streams its records through a private ring
+// of shared-memory stages with bulk asynchronous copies (cp.async.bulk +
+// mbarrier); the ring runs across unit boundaries, so the next unit's first
+// records are in flight while a unit's partial results are merged.
+//
+// Per record every product runs on the tensor cores (mma.sync m16n8k16, fp32
+// accumulate), with exact fp16 operands only:
+//   q.K  A = q~ (rows: head r/2 mod 4, high fp16 part in rows 0-7, low part in
+//        rows 8-15), B = centroids of 8 tokens from a byte -> (C[lo], C[hi])
+//        table with one copy per lane; one prmt forms each table address.
+//        Lane (g, c) ends with the full scores of head g/2 at tokens 2c, 2c+1,
+//        2c+8, 2c+9: exactly the operand it feeds to p.V, so no transpose.
+//   p.V  A = value codes as fp16 subnormals (the nibble masked in place is
+//        n 2^-24, or n 2^-20 for a high nibble: exact, no bias to remove);
+//        B = p_t s_t,g as an exact two-part fp16 product, the high part in
+//        column 2h and the low part in column 2h+1 of head h.
+//   p.z  A = fp16 zero points (rows 0-7) and ones (rows 8-15), B = p as fp16
+//        parts: gives sum_t p_t z_t,g and the softmax denominator.
 // Softmax runs online in base 2 (scale * log2 e is folded into q~) and the
-// accumulators are rescaled only when a running maximum moves.  Each split
+// accumulators are rescaled only when a running maximum moves.  Each unit
 // leaves an unnormalised partial (o, m, l) that the combine kernel merges; a
 // single split writes the output directly.
 #include "tq_kernels.cuh"
@@ -30,12 +38,53 @@
 namespace tq {
 namespace {
 
-constexpr int kNW = 8;      // warps per CTA
-constexpr int kStages = 3;  // records in flight per warp
-constexpr int kLutWords = 256 * 32;
+constexpr int kNW = 8;                   // warps per half (per unit)
+constexpr int kHalves = 2;               // independent halves per CTA
+constexpr int kWarps = kNW * kHalves;    // 16 warps, 512 threads
+constexpr int kStages = 3;               // records in flight per warp
+constexpr int kSlots = kWarps * kStages;
+constexpr int kHeads = 4;                // query heads per item
+constexpr uint32_t kLutBytes = 1u << 16; // 256 byte values x (2 halves x 32 lanes x 4 B)
+constexpr uint32_t kOnes = 0x3C003C00u;  // fp16 (1, 1)
 
+// ------------------------------------------------------------------ PTX helpers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.b32 [%0], %1;" ::"r"(a), "r"(v));
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(v));
+}
+__device__ __forceinline__ void stsf(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v));
+}
+__device__ __forceinline__ float ldsf(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+// barrier among the 256 threads of one half (ids 1, 2; 0 is __syncthreads)
+__device__ __forceinline__ void half_sync(int half) {
+    asm volatile("bar.sync %0, 256;" ::"r"(1 + half) : "memory");
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -87,6 +136,15 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// the same with a zero accumulator in
+__device__ __forceinline__ void mma16816_z(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                           uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.f));
+}
+
 // 2^x for x <= 0 (softmax weights); the hardware approximation is accurate to
 // ~2 ulp and flushes results below 2^-126 to zero.
 __device__ __forceinline__ float ex2(float x) {
@@ -98,130 +156,245 @@ __device__ __forceinline__ float ex2(float x) {
 __device__ __forceinline__ uint32_t h2u(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 u2h(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
-// fp16 pair (x0 in the low half) and its rounding remainder as a second pair
-__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    const __half2 h = __floats2half2_rn(x0, x1);
+// The two fp16 operand parts of p for this lane's column: a high-part lane
+// (sel = 0) gets u = 0, w = fp16(p); a low-part lane (sel = 1) gets
+// u = fp16(p), w = fp16(p - u).  p0 goes to the low half of each pair.
+__device__ __forceinline__ void split_uw(float p0, float p1, float sel, uint32_t mask, uint32_t& u,
+                                         uint32_t& w) {
+    const __half2 h = __floats2half2_rn(p0, p1);
     const float2 f = __half22float2(h);
-    hi = h2u(h);
-    lo = h2u(__floats2half2_rn(x0 - f.x, x1 - f.y));
+    w = h2u(__floats2half2_rn(fmaf(-sel, f.x, p0), fmaf(-sel, f.y, p1)));
+    u = h2u(h) & mask;
 }
 
-// (ph + pl) * s as a high part and a low part, all fp16 pairs:
-//   hi = fl(ph * s); r = ph * s - hi is exact (fma two-product);
-//   lo = fl(r + pl * s).  hi + lo equals p * s to ~2^-21 relative.
-__device__ __forceinline__ void scaled_pair(uint32_t ph, uint32_t pl, uint32_t s, uint32_t& hi,
-                                            uint32_t& lo) {
-    const __half2 h = __hmul2(u2h(ph), u2h(s));
-    const __half2 r = __hfma2(u2h(ph), u2h(s), __hneg2(h));
-    hi = h2u(h);
-    lo = h2u(__hfma2(u2h(pl), u2h(s), r));
+// This lane's part of p * s: fl(w s + (u s - fl(u s))).  With u = 0 it is
+// fl(p_hi s); with (u, w) = (p_hi, p_lo) it is the remainder of p_hi s (exact
+// by the fma two-product) plus p_lo s, so the two columns sum to p s within
+// ~2^-21 relative.
+__device__ __forceinline__ uint32_t ps_part(uint32_t u, uint32_t w, uint32_t s) {
+    const __half2 x = __hmul2(u2h(u), u2h(s));
+    const __half2 r = __hfma2(u2h(u), u2h(s), __hneg2(x));
+    return h2u(__hfma2(u2h(w), u2h(s), r));
 }
 
-// X holds the code bytes of two tokens in bytes 0 and 2.  Low nibbles ->
-// exact fp16 pair (n0, n1); high nibbles -> exact fp16 pair (n0', n1').
-// 0x6400 | n is the fp16 value 1024 + n; 0x6400 | (n << 4) is 1024 + 16 n.
-__device__ __forceinline__ void value_pair(uint32_t X, uint32_t& lo_nib, uint32_t& hi_nib) {
-    const uint32_t a = (X & 0x000F000Fu) | 0x64006400u;
-    const uint32_t b = (X & 0x00F000F0u) | 0x64006400u;
-    lo_nib = h2u(__hsub2(u2h(a), u2h(0x64006400u)));                    // - 1024
-    hi_nib = h2u(__hfma2(u2h(b), u2h(0x2C002C00u), u2h(0xD400D400u)));  // / 16 - 64
+// ------------------------------------------------------------------ shared memory plan
+// Shared-window addresses for a dynamic region that starts at s0.  The table
+// must sit on a 64 KB boundary so that one prmt can splice a code byte into
+// the address; whole warp rings fill the space below it first.
+template <int D>
+struct Plan {
+    static constexpr uint32_t kRec = Rec<D>::kBytes;
+    static constexpr uint32_t kRing = kStages * kRec;  // one warp's stages, contiguous
+    static constexpr uint32_t kMergeHalf = kNW * (kHeads * D + 2 * kHeads) * 4;
+    uint32_t lut, low, hi, merge, qh, ql, ids, bars, end;
+    __host__ __device__ explicit Plan(uint32_t s0) {
+        lut = (s0 + kLutBytes - 1) & ~(kLutBytes - 1);
+        const uint32_t n = (lut - s0) / kRing;
+        low = n < (uint32_t)kWarps ? n : (uint32_t)kWarps;
+        hi = lut + kLutBytes;
+        merge = hi + (kWarps - low) * kRing;
+        qh = merge + kHalves * kMergeHalf;
+        ql = qh + kHalves * kHeads * D * 2;
+        ids = ql + kHalves * kHeads * D * 2;
+        bars = ids + kSlots * 4;
+        end = bars + kSlots * 8;
+    }
+    // first stage of warp w's ring
+    __host__ __device__ uint32_t ring(uint32_t s0, int w) const {
+        return (uint32_t)w < low ? s0 + w * kRing : hi + (w - low) * kRing;
+    }
+};
+
+// Bytes to request so that the plan fits wherever the dynamic region starts
+// (the start depends on the reserved shared memory of the device).
+template <int D>
+uint32_t plan_bytes() {
+    uint32_t worst = 0;
+    for (uint32_t s0 = 0; s0 <= 8192; s0 += 16) {
+        const Plan<D> p(s0);
+        if (p.end - s0 > worst) worst = p.end - s0;
+    }
+    return worst;
 }
 
-// Table addresses (word indices (byte << 5) | lane) of the two low bytes of x.
-__device__ __forceinline__ void lut_idx2(uint32_t x, uint32_t lane2, uint32_t& i0, uint32_t& i1) {
-    const uint32_t t = __byte_perm(x, 0u, 0x4140u) * 32u + lane2;  // (b0, b1) in 16-bit halves
-    i0 = t & 0xffffu;
-    i1 = t >> 16;
-}
+// ------------------------------------------------------------------ units
+// What one warp needs to know about a unit: the item's coordinates, the
+// sequence length, and this warp's share of the split's blocks.
+struct Unit {
+    int u;                  // unit index (>= units: past the end)
+    int b, kv, quad, split;
+    int L;                  // tokens of the sequence (clamped)
+    int nk;                 // records of this warp in the unit
+    const int32_t* bt;      // block-table entry of this warp's first record
+    const unsigned char* src;  // record of block 0 for this kv head
+};
 
-template <int D, int GP>
-__global__ void __launch_bounds__(kNW * 32, 2) decode_split_kernel(DecodeArgs a) {
-    constexpr int KS = D / 16;   // k-steps of q.K
-    constexpr int MT = D / 16;   // m-tiles of p.V
-    constexpr int NG = D / 32;   // value groups
-    constexpr int BPL = D / 8;   // key-code bytes per lane per token
-    constexpr int VPL = D / 16;  // value-code bytes per lane per token
-    constexpr int NT = GP / 4;   // n-tiles: 4 heads x (hi, lo) per tile
-    constexpr int KW = BPL / 4;  // key-code words per lane per token
-    constexpr int VW = VPL / 4;  // value-code words per lane per token
-    constexpr int REC = Rec<D>::kBytes;
-    using R = Rec<D>;
-
-    __shared__ uint32_t lut[kLutWords];
-    __shared__ float ctab[16];
-    extern __shared__ __align__(128) unsigned char dsm[];
-    constexpr size_t kRing = (size_t)kNW * kStages * REC;
-    constexpr size_t kMerge = (size_t)kNW * GP * D * 4 + 2 * kNW * GP * 4;
-    unsigned char* ring = dsm;
-    uint64_t* mbar = reinterpret_cast<uint64_t*>(dsm + (kRing > kMerge ? kRing : kMerge));
-    float* qs = reinterpret_cast<float*>(mbar + kNW * kStages);  // [GP][D]
-    float* ps = qs + GP * D;                                      // [NW][16][GP]
-    float* pc = ps + kNW * 16 * GP;                               // [NW][GP]
-    float* zs = pc + kNW * GP;                                    // [NW][NG][GP]
-
-    const int split = blockIdx.x, kv = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int g = lane >> 2, c = lane & 3;
-    const int G = a.Hq / a.Hkv;
-
-    int L = a.seq_lens[b];
+template <int D>
+__device__ __forceinline__ void unit_at(Unit& s, int u, const DecodeArgs& a, int warp,
+                                        bool report) {
+    s.u = u;
+    s.nk = 0;
+    if (u >= a.units) return;
+    const int item = u % a.items;
+    s.split = u / a.items;
+    s.quad = item % a.quads;
+    const int bk = item / a.quads;
+    s.kv = bk % a.Hkv;
+    s.b = bk / a.Hkv;
+    int L = a.seq_lens[s.b];
+    const bool first = report && s.kv == 0 && s.quad == 0 && s.split == 0;
     if (L < 0 || L > a.max_blocks * kBlock) {
-        if (tid == 0 && split == 0 && kv == 0) flag_status(a.status, TQ_STATUS_BAD_LEN);
+        if (first) flag_status(a.status, TQ_STATUS_BAD_LEN);
         L = 0;
     }
     if (L > a.num_splits * a.blocks_per_split * kBlock) {
-        if (tid == 0 && split == 0 && kv == 0) flag_status(a.status, TQ_STATUS_BAD_LEN);
+        if (first) flag_status(a.status, TQ_STATUS_BAD_LEN);
         L = a.num_splits * a.blocks_per_split * kBlock;
     }
+    s.L = L;
     const int nblk = (L + kBlock - 1) / kBlock;
-    const int jb = split * a.blocks_per_split;
-    const int je = min(jb + a.blocks_per_split, nblk);
-    const int nk = je - jb - warp > 0 ? (je - jb - warp + kNW - 1) / kNW : 0;
+    const int jb = s.split * a.blocks_per_split;
+    const int left = min(jb + a.blocks_per_split, nblk) - jb - warp;
+    s.nk = left > 0 ? (left + kNW - 1) / kNW : 0;
+    s.bt = a.block_tables + (size_t)s.b * a.max_blocks + jb + warp;
+    s.src = a.cache + (size_t)s.kv * Rec<D>::kBytes;
+}
 
-    // ---- per-warp copy ring
-    const uint32_t bar0 = smem_u32(mbar + warp * kStages);
-    const uint32_t ring0 = smem_u32(ring + (size_t)warp * kStages * REC);
+// N consecutive 32-bit words (N = 2 or 4) of shared memory
+template <int N>
+__device__ __forceinline__ void ldw(uint32_t a, uint32_t (&w)[N]) {
+    static_assert(N == 2 || N == 4, "8- or 16-byte loads");
+    if constexpr (N == 4) {
+        const uint4 v = lds128(a);
+        w[0] = v.x;
+        w[1] = v.y;
+        w[2] = v.z;
+        w[3] = v.w;
+    } else {
+        const uint2 v = lds64(a);
+        w[0] = v.x;
+        w[1] = v.y;
+    }
+}
+
+// ------------------------------------------------------------------ split kernel
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
+    constexpr int KS = D / 16;   // k-steps of q.K = m-tiles of p.V
+    constexpr int NG = D / 32;   // value groups
+    constexpr int KB = D / 8;    // key bytes of a lane per token = bytes of a value chunk
+    constexpr int KW = KB / 4;   // words of those (= NG)
+    constexpr int EPL = D / 32;  // query elements per lane in the rotation
+    constexpr uint32_t REC = Rec<D>::kBytes;
+    using R = Rec<D>;
+    extern __shared__ __align__(128) unsigned char dsm[];
+
+    const int tid = threadIdx.x, lane = tid & 31, wa = tid >> 5;
+    const int half = wa / kNW, warp = wa % kNW;
+    const int ht = tid - half * kNW * 32;  // thread index within the half
+    const int g = lane >> 2, c = lane & 3;
+    const uint32_t s0 = smem_u32(dsm);
+    const Plan<D> P(s0);
+    if (P.end - s0 > a.smem_bytes) {  // cannot happen with the launcher's size; never touch memory
+        if (tid == 0 && blockIdx.x == 0) flag_status(a.status, TQ_STATUS_INTERNAL);
+        return;
+    }
+    const int G = a.Hq / a.Hkv;
+    const int stride = kHalves * gridDim.x;  // units per round over all halves
+    const int v = kHalves * blockIdx.x + half;
+
+    // ---- this warp's ring: slots, barriers, and the block id of each stage
+    const uint32_t bar0 = P.bars + wa * kStages * 8;
+    const uint32_t idw = P.ids + wa * kStages * 4;
+    const uint32_t ringw = P.ring(s0, wa);
     if (lane == 0) {
+#pragma unroll
         for (int s = 0; s < kStages; s++) mbar_init(bar0 + 8 * s, 1);
         fence_mbar_init();
     }
     __syncwarp();
-    const int32_t* bt_row = a.block_tables + (size_t)b * a.max_blocks;
-    auto load_id = [&](int k) { return k < nk ? bt_row[jb + warp + kNW * k] : -1; };
-    int idA = load_id(lane), idB = load_id(32 + lane), kA = 0;
-    auto get_id = [&](int k) {
-        const int r = k - kA;
-        const int x = __shfl_sync(kFull, idA, r & 31);
-        const int y = __shfl_sync(kFull, idB, r & 31);
-        return r < 32 ? x : y;
-    };
-    const unsigned char* cache_kv = a.cache + (size_t)kv * REC;
-    auto issue = [&](int k, int id) {  // lane 0 only
-        const uint32_t bar = bar0 + 8 * (k % kStages);
-        if (id >= 0 && id < a.num_blocks) {
-            fence_proxy_async();
-            mbar_expect_tx(bar, REC);
-            bulk_g2s(ring0 + (k % kStages) * REC, cache_kv + (size_t)id * a.Hkv * REC, REC, bar);
-        } else {
-            mbar_arrive(bar);
-        }
-    };
-    for (int k = 0; k < kStages && k < nk; k++) {
-        const int id = get_id(k);
-        if (lane == 0) issue(k, id);
-    }
 
-    // ---- centroid table of this head
-    const uint16_t* tab = a.k_tables ? a.k_tables + kv * 16 : a.default_table;
-    if (tid < 16) ctab[tid] = half_bits_to_float(tab[tid]);
-    // ---- rotate the queries of this kv head (heads >= G stay zero)
-    {
-        constexpr int EPL = D / 32;
-        const float sc = a.scale_log2 * rsqrtf((float)D);
-        for (int h = warp; h < GP; h += kNW) {
+    // ---- issue cursor: the next record of this warp's stream (all its units, in order)
+    Unit is;
+    unit_at<D>(is, v, a, warp, false);
+    while (is.u < a.units && is.nk == 0) unit_at<D>(is, is.u + stride, a, warp, false);
+    int irem = is.nk, istage = 0;
+    const int32_t* ibt = is.bt;
+    int nid = is.u < a.units ? *ibt : -1;
+    // Copy the record of block nid into stage istage (one elected lane, no branch),
+    // note its id for the consumer, and move the cursor on.
+    auto issue = [&]() {
+        if (is.u >= a.units) return;
+        const uint32_t bar = bar0 + 8 * istage;
+        const uint32_t valid = (uint32_t)(nid >= 0 && nid < a.num_blocks);
+        const uint32_t me = (uint32_t)(lane == 0);
+        const unsigned char* src = is.src + (size_t)(valid ? nid : 0) * a.Hkv * REC;
+        asm volatile(
+            "{\n .reg .pred pc, pa, pm;\n"
+            " setp.ne.u32 pm, %0, 0;\n"
+            " setp.ne.and.u32 pc, %1, 0, pm;\n"
+            " setp.eq.and.u32 pa, %1, 0, pm;\n"
+            " @pc fence.proxy.async.shared::cta;\n"
+            " @pc mbarrier.arrive.expect_tx.shared::cta.b64 _, [%2], %3;\n"
+            " @pc cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%4], [%5], %3, [%2];\n"
+            " @pa mbarrier.arrive.shared::cta.b64 _, [%2];\n"
+            " @pm st.shared.b32 [%6], %7;\n"
+            "}\n" ::"r"(me), "r"(valid), "r"(bar), "r"(REC), "r"(ringw + istage * REC), "l"(src),
+            "r"(idw + 4 * istage), "r"(nid)
+            : "memory");
+        istage = istage == kStages - 1 ? 0 : istage + 1;
+        if (--irem == 0) {
+            do unit_at<D>(is, is.u + stride, a, warp, false);
+            while (is.u < a.units && is.nk == 0);
+            irem = is.nk;
+            ibt = is.bt;
+        } else {
+            ibt += kNW;
+        }
+        nid = is.u < a.units ? *ibt : -1;
+    };
+#pragma unroll 1
+    for (int k = 0; k < kStages; k++) issue();
+    __syncwarp();
+
+    // ---- per-lane constants of the consumer
+    const uint32_t lanebase = P.lut | ((uint32_t)half << 7) | ((uint32_t)lane << 2);
+    const float lo_sel = (float)(g & 1);  // this lane feeds the low part of its head
+    const uint32_t lo_mask = (g & 1) ? 0xffffffffu : 0u;
+    const uint32_t qsrc_h = P.qh + (uint32_t)((half * kHeads + (g >> 1)) * D * 2);
+    const uint32_t qsrc_l = P.ql + (uint32_t)((half * kHeads + (g >> 1)) * D * 2);
+    const uint32_t mb = P.merge + half * Plan<D>::kMergeHalf;  // [warp][head][D] o, then m, l
+    const uint32_t mb_m = mb + kNW * kHeads * D * 4, mb_l = mb_m + kNW * kHeads * 4;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool aborted = false;
+    const uint16_t* lut_tab = nullptr;  // table held by this half's side of the LUT
+
+#pragma unroll 1
+    for (int u = v; u < a.units; u += stride) {
+        Unit cu;
+        unit_at<D>(cu, u, a, warp, warp == 0 && lane == 0);
+        const int h0 = cu.kv * G + cu.quad * kHeads;  // first query head of the item
+        const int nh = min(kHeads, G - cu.quad * kHeads);
+
+        // ---- the centroid-pair table of this kv head, on this half's side of
+        // each 256-byte row: word (row, lane) = (C[row & 15], C[row >> 4])
+        const uint16_t* tab = a.k_tables ? a.k_tables + cu.kv * 16 : nullptr;
+        if (u == v || tab != lut_tab) {
+            lut_tab = tab;
+#pragma unroll 1
+            for (int it = 0; it < 8; it++) {
+                const int row = 32 * warp + 4 * it + (lane >> 3);
+                const uint32_t lo = tab ? tab[row & 15] : a.default_table[row & 15];
+                const uint32_t hi = tab ? tab[row >> 4] : a.default_table[row >> 4];
+                sts128(P.lut + row * 256 + half * 128 + (lane & 7) * 16, lo | (hi << 16));
+            }
+        }
+        // ---- rotate this item's queries: q~ = H q * scale log2(e) / sqrt(D), as fp16 parts
+        if (warp < kHeads) {
             float x[EPL];
-            if (h < G) {
-                const uint16_t* src = a.q + ((size_t)b * a.Hq + kv * G + h) * D + lane * EPL;
+            if (warp < nh) {
+                const uint16_t* src = a.q + ((size_t)cu.b * a.Hq + h0 + warp) * D + lane * EPL;
 #pragma unroll
                 for (int e = 0; e < EPL; e++) x[e] = __uint_as_float((uint32_t)src[e] << 16);
             } else {
@@ -233,9 +406,9 @@ __global__ void __launch_bounds__(kNW * 32, 2) decode_split_kernel(DecodeArgs a)
 #pragma unroll
                 for (int e = 0; e < EPL; e++)
                     if (!(e & m)) {
-                        const float u = x[e], v = x[e | m];
-                        x[e] = u + v;
-                        x[e | m] = u - v;
+                        const float p = x[e], q = x[e | m];
+                        x[e] = p + q;
+                        x[e | m] = p - q;
                     }
 #pragma unroll
             for (int m = 1; m < 32; m <<= 1) {
@@ -246,318 +419,216 @@ __global__ void __launch_bounds__(kNW * 32, 2) decode_split_kernel(DecodeArgs a)
                     x[e] = upper ? p - x[e] : x[e] + p;
                 }
             }
+            const float sc = a.scale_log2 * rsqrtf((float)D);
+            const uint32_t dh = P.qh + (uint32_t)(((half * kHeads + warp) * D + lane * EPL) * 2);
+            const uint32_t dl = P.ql + (uint32_t)(((half * kHeads + warp) * D + lane * EPL) * 2);
 #pragma unroll
-            for (int e = 0; e < EPL; e++) qs[h * D + lane * EPL + e] = x[e] * sc;
+            for (int e = 0; e < EPL; e += 2) {
+                const float y0 = x[e] * sc, y1 = x[e + 1] * sc;
+                const __half2 hp = __floats2half2_rn(y0, y1);
+                const float2 hf = __half22float2(hp);
+                sts32(dh + 2 * e, h2u(hp));
+                sts32(dl + 2 * e, h2u(__floats2half2_rn(y0 - hf.x, y1 - hf.y)));
+            }
         }
-    }
-    __syncthreads();
-    // ---- centroid pair table, one copy per lane: lut[(byte << 5) | lane]
-    for (int e = tid; e < kLutWords; e += kNW * 32) {
-        const int v = e >> 5;
-        lut[e] = h2u(__floats2half2_rn(ctab[v & 15], ctab[v >> 4]));
-    }
+        half_sync(half);
 
-    // ---- query fragments (B of q.K).  Column n of tile t is head 4t + n/2,
-    // its high fp16 part for even n and its low part for odd n; this lane
-    // supplies column g.
-    const bool hi_role = (g & 1) == 0;
-    uint32_t bq[NT][KS][2];
+        // ---- q.K A fragments: rows g (high part) and g + 8 (low part) of head
+        // g/2; k = 2c, 2c+1 | 2c+8, 2c+9 of step ks are the dims of key bytes
+        // j = c*KB + 2ks and j + 1 (a fixed permutation of the dims)
+        uint32_t qa[KS][4];
 #pragma unroll
-    for (int t = 0; t < NT; t++) {
-        const int h = 4 * t + (g >> 1);
-#pragma unroll
-        for (int ks = 0; ks < KS; ks++)
-#pragma unroll
-            for (int r = 0; r < 2; r++) {
-                const int j = c * BPL + 2 * ks + r;  // key-code byte -> dims 2j, 2j+1
-                uint32_t hi, lo;
-                split_pair(qs[h * D + 2 * j], qs[h * D + 2 * j + 1], hi, lo);
-                bq[t][ks][r] = hi_role ? hi : lo;
-            }
-    }
-    __syncthreads();  // lut complete
-
-    // ---- per-lane state.  Score / output layout: lane (g, c) holds head
-    // 4t + c of tile t, tokens g and g + 8 (dims 2(8m + g), +1 of m-tile m).
-    float mrun[NT], lrun[NT];
-    float O[MT][NT][4];
-    float Z[NT][4];  // p.z accumulator: rows = value groups (g < NG), head 4t + c
-#pragma unroll
-    for (int t = 0; t < NT; t++) {
-        mrun[t] = -INFINITY;
-        lrun[t] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; i++) Z[t][i] = 0.f;
-#pragma unroll
-        for (int m = 0; m < MT; m++)
-#pragma unroll
-            for (int i = 0; i < 4; i++) O[m][t][i] = 0.f;
-    }
-    float* wps = ps + warp * 16 * GP;
-    float* wpc = pc + warp * GP;
-    const uint32_t lane2 = (uint32_t)lane | ((uint32_t)lane << 16);
-    const int ph_head = g >> 1;  // this lane's B-fragment head within each tile
-    bool aborted = false;
-    int stage = 0;
-    uint32_t phase = 0;
-
-    for (int k = 0; k < nk; k++) {
-        if (k - kA == 32) {  // next batch of block ids
-            idA = idB;
-            kA += 32;
-            idB = load_id(kA + 32 + lane);
+        for (int ks = 0; ks < KS; ks++) {
+            const uint32_t j = c * KB + 2 * ks;
+            const uint2 hv = lds64(qsrc_h + 4 * j), lv = lds64(qsrc_l + 4 * j);
+            qa[ks][0] = hv.x;
+            qa[ks][1] = lv.x;
+            qa[ks][2] = hv.y;
+            qa[ks][3] = lv.y;
         }
-        const int id = get_id(k);
-        const bool ok = mbar_wait(bar0 + 8 * stage, phase);
-        if (!__all_sync(kFull, ok)) {
-            if (lane == 0) flag_status(a.status, TQ_STATUS_TIMEOUT);
-            aborted = true;
-            break;
+
+        // ---- this warp's records of the unit
+        float O[KS][4];  // p.V: rows = dims (16m + 2g, 16m + 2g + 1), cols = head c (hi, lo)
+        float Z[4];      // p.z: rows g = zero sums of group g, rows g + 8 = sum of p
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            Z[i] = 0.f;
+#pragma unroll
+            for (int m = 0; m < KS; m++) O[m][i] = 0.f;
         }
-        if (id < 0 || id >= a.num_blocks) {
-            if (lane == 0) flag_status(a.status, TQ_STATUS_BAD_BLOCK);
-        } else {
-            const unsigned char* rec = ring + (size_t)(warp * kStages + stage) * REC;
-            const int nvalid = min(kBlock, L - (jb + warp + kNW * k) * kBlock);
+        float mrun = -INFINITY;  // running maximum of head g/2
+        const int nk = aborted ? 0 : cu.nk;
+        // tokens in this warp's last record of the unit (< 16 only at the end of the sequence)
+        const int last_valid = cu.L - (cu.split * a.blocks_per_split + warp + kNW * (nk - 1)) * kBlock;
+#pragma unroll 1
+        for (int k = 0; k < nk; k++) {
+            const uint32_t rec = ringw + stage * REC;
+            const bool ok = mbar_wait(bar0 + 8 * stage, phase);
+            if (!__all_sync(kFull, ok)) {
+                if (lane == 0) flag_status(a.status, TQ_STATUS_TIMEOUT);
+                aborted = true;
+                break;
+            }
+            const int id = (int)lds32(idw + 4 * stage);
+            if (id >= 0 && id < a.num_blocks) {
+                const bool partial = k == nk - 1 && last_valid < kBlock;
 
-            // -------- q.K: tokens g and g+8, this lane's BPL key-code bytes
-            uint32_t kw0[KW], kw1[KW];
-            {
-                const unsigned char* krow0 = rec + R::kKCodes + g * (D / 2) + c * BPL;
-                const unsigned char* krow1 = krow0 + 8 * (D / 2);
+                // -------- q.K: B = centroids of tokens g (tile 0) and g + 8 (tile 1)
+                uint32_t kw0[KW], kw1[KW];
+                ldw<KW>(rec + g * (D / 2) + c * KB, kw0);
+                ldw<KW>(rec + (g + 8) * (D / 2) + c * KB, kw1);
+                float s0[4], s1[4];
 #pragma unroll
-                for (int w = 0; w < KW; w += 2) {
-                    const uint2 u0 = *reinterpret_cast<const uint2*>(krow0 + 4 * w);
-                    const uint2 u1 = *reinterpret_cast<const uint2*>(krow1 + 4 * w);
-                    kw0[w] = u0.x;
-                    kw0[w + 1] = u0.y;
-                    kw1[w] = u1.x;
-                    kw1[w + 1] = u1.y;
+                for (int ks = 0; ks < KS; ks++) {
+                    // table address: the code byte spliced into byte 1 of lanebase
+                    const uint32_t sa = (ks & 1) ? 0x7624u : 0x7604u;
+                    const uint32_t sb = (ks & 1) ? 0x7634u : 0x7614u;
+                    const uint32_t w0 = kw0[ks >> 1], w1 = kw1[ks >> 1];
+                    const uint32_t b00 = lds32(__byte_perm(w0, lanebase, sa));
+                    const uint32_t b01 = lds32(__byte_perm(w0, lanebase, sb));
+                    const uint32_t b10 = lds32(__byte_perm(w1, lanebase, sa));
+                    const uint32_t b11 = lds32(__byte_perm(w1, lanebase, sb));
+                    if (ks == 0) {
+                        mma16816_z(s0, qa[0][0], qa[0][1], qa[0][2], qa[0][3], b00, b01);
+                        mma16816_z(s1, qa[0][0], qa[0][1], qa[0][2], qa[0][3], b10, b11);
+                    } else {
+                        mma16816(s0, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
+                        mma16816(s1, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
+                    }
                 }
-            }
-            float acc[NT][4];
-#pragma unroll
-            for (int t = 0; t < NT; t++)
-#pragma unroll
-                for (int i = 0; i < 4; i++) acc[t][i] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < KS; ks++) {
-                const int wi = ks >> 1, sh = (ks & 1) * 16;  // bytes 2ks, 2ks+1 of the chunk
-                uint32_t i0, i2, i1, i3;
-                lut_idx2(kw0[wi] >> sh, lane2, i0, i2);
-                lut_idx2(kw1[wi] >> sh, lane2, i1, i3);
-                const uint32_t a0 = lut[i0], a1 = lut[i1], a2 = lut[i2], a3 = lut[i3];
-#pragma unroll
-                for (int t = 0; t < NT; t++) mma16816(acc[t], a0, a1, a2, a3, bq[t][ks][0], bq[t][ks][1]);
-            }
-            const float n_a =
-                half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec + R::kKNorm + 2 * g));
-            const float n_b = half_bits_to_float(
-                *reinterpret_cast<const uint16_t*>(rec + R::kKNorm + 2 * (g + 8)));
-            float sa[NT], sb[NT];  // scores of tokens g, g+8 for head 4t + c
-#pragma unroll
-            for (int t = 0; t < NT; t++) {
-                sa[t] = (acc[t][0] + acc[t][1]) * n_a;
-                sb[t] = (acc[t][2] + acc[t][3]) * n_b;
-            }
-            const bool partial = nvalid < kBlock;  // the last block of a sequence
-            if (partial) {
-#pragma unroll
-                for (int t = 0; t < NT; t++) {
-                    sa[t] = g < nvalid ? sa[t] : -INFINITY;
-                    sb[t] = g + 8 < nvalid ? sb[t] : -INFINITY;
+                // scores of head g/2 at tokens 2c, 2c+1, 2c+8, 2c+9 (base 2)
+                const float2 na = __half22float2(u2h(lds32(rec + R::kKNorm + 4 * c)));
+                const float2 nb = __half22float2(u2h(lds32(rec + R::kKNorm + 16 + 4 * c)));
+                float x0 = (s0[0] + s0[2]) * na.x, x1 = (s0[1] + s0[3]) * na.y;
+                float x2 = (s1[0] + s1[2]) * nb.x, x3 = (s1[1] + s1[3]) * nb.y;
+                uint32_t mA = 0xffffffffu, mB = 0xffffffffu;  // valid tokens (fp16 lanes)
+                if (partial) {  // the last block of the sequence
+                    const int t = 2 * c, nvalid = last_valid;
+                    x0 = t < nvalid ? x0 : -INFINITY;
+                    x1 = t + 1 < nvalid ? x1 : -INFINITY;
+                    x2 = t + 8 < nvalid ? x2 : -INFINITY;
+                    x3 = t + 9 < nvalid ? x3 : -INFINITY;
+                    mA = (t < nvalid ? 0xffffu : 0u) | (t + 1 < nvalid ? 0xffff0000u : 0u);
+                    mB = (t + 8 < nvalid ? 0xffffu : 0u) | (t + 9 < nvalid ? 0xffff0000u : 0u);
                 }
-            }
 
-            // -------- online softmax
-            bool grew = false;
-            float corr[NT];
+                // -------- online softmax
+                float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+                const float mn = fmaxf(mrun, mx);
+                if (__any_sync(kFull, mn > mrun)) {
+                    const float corr = __shfl_sync(kFull, ex2(mrun - mn), 8 * c);  // head c
 #pragma unroll
-            for (int t = 0; t < NT; t++) {
-                float x = fmaxf(sa[t], sb[t]);
+                    for (int i = 0; i < 4; i++) {
+                        Z[i] *= corr;
 #pragma unroll
-                for (int m = 4; m < 32; m <<= 1) x = fmaxf(x, __shfl_xor_sync(kFull, x, m));
-                const float mn = fmaxf(mrun[t], x);
-                grew |= mn > mrun[t];
-                corr[t] = ex2(mrun[t] - mn);
-                mrun[t] = mn;
-                sa[t] = ex2(sa[t] - mn);
-                sb[t] = ex2(sb[t] - mn);
-                lrun[t] = fmaf(lrun[t], corr[t], sa[t] + sb[t]);
-            }
-            if (__any_sync(kFull, grew)) {
-#pragma unroll
-                for (int t = 0; t < NT; t++) {
-#pragma unroll
-                    for (int i = 0; i < 4; i++) Z[t][i] *= corr[t];
-#pragma unroll
-                    for (int m = 0; m < MT; m++)
-#pragma unroll
-                        for (int i = 0; i < 4; i++) O[m][t][i] *= corr[t];
+                        for (int m = 0; m < KS; m++) O[m][i] *= corr;
+                    }
                 }
-            }
+                mrun = mn;
+                uint32_t u01, w01, u89, w89;
+                split_uw(ex2(x0 - mn), ex2(x1 - mn), lo_sel, lo_mask, u01, w01);
+                split_uw(ex2(x2 - mn), ex2(x3 - mn), lo_sel, lo_mask, u89, w89);
+
+                // -------- p.z and sum p
+                uint2 zz = lds64(rec + R::kVZero + (c * NG + (g & (NG - 1))) * 8);
+                uint32_t sw[2 * NG];
 #pragma unroll
-            for (int t = 0; t < NT; t++) {
-                wps[g * GP + 4 * t + c] = sa[t];
-                wps[(g + 8) * GP + 4 * t + c] = sb[t];
+                for (int i = 0; i < 2 * NG; i += 4) {
+                    uint32_t t4[4];
+                    ldw<4>(rec + R::kVScale + c * NG * 8 + 4 * i, t4);
+#pragma unroll
+                    for (int e = 0; e < 4; e++) sw[i + e] = t4[e];
+                }
+                if (partial) {  // stale fields of unwritten tokens must not reach the products
+                    zz.x &= mA;
+                    zz.y &= mB;
+#pragma unroll
+                    for (int G_ = 0; G_ < NG; G_++) {
+                        sw[2 * G_] &= mA;
+                        sw[2 * G_ + 1] &= mB;
+                    }
+                }
+                mma16816(Z, zz.x, kOnes, zz.y, kOnes, w01, w89);
+
+                // -------- p.V: word G of a chunk holds m-tiles 2G (bytes 0, 2) and
+                // 2G + 1 (bytes 1, 3) of tokens 2c, 2c+1 (va) and 2c+8, 2c+9 (vb)
+                uint32_t va[KW], vb[KW];
+                ldw<KW>(rec + R::kVCodes + (c * 8 + g) * KB, va);
+                ldw<KW>(rec + R::kVCodes + ((c + 4) * 8 + g) * KB, vb);
+#pragma unroll
+                for (int G_ = 0; G_ < NG; G_++) {
+                    const uint32_t b0 = ps_part(u01, w01, sw[2 * G_]);
+                    const uint32_t b1 = ps_part(u89, w89, sw[2 * G_ + 1]);
+                    const uint32_t A0 = va[G_], B0 = vb[G_], A1 = A0 >> 8, B1 = B0 >> 8;
+                    mma16816(O[2 * G_], A0 & 0x000F000Fu, A0 & 0x00F000F0u, B0 & 0x000F000Fu,
+                             B0 & 0x00F000F0u, b0, b1);
+                    mma16816(O[2 * G_ + 1], A1 & 0x000F000Fu, A1 & 0x00F000F0u, B1 & 0x000F000Fu,
+                             B1 & 0x00F000F0u, b0, b1);
+                }
+            } else if (lane == 0) {
+                flag_status(a.status, TQ_STATUS_BAD_BLOCK);
             }
             __syncwarp();
+            issue();  // the record after the ring's last: into the slot just read
+            if (++stage == kStages) {
+                stage = 0;
+                phase ^= 1u;
+            }
+        }
 
-            // -------- B fragments of p (this lane: column g -> head 4t + g/2,
-            // tokens 2c, 2c+1 and 2c+8, 2c+9), fp16 high and low parts
-            const int t0 = 2 * c, t2 = 2 * c + 8;
-            uint32_t bph[NT][2], bpl[NT][2];
+        // ---- this warp's share -> merge buffer (o with the zero-point term, m, l of head c)
+        {
+            float zs[NG];
 #pragma unroll
-            for (int t = 0; t < NT; t++) {
-                const int h = 4 * t + ph_head;
-                split_pair(wps[t0 * GP + h], wps[(t0 + 1) * GP + h], bph[t][0], bpl[t][0]);
-                split_pair(wps[t2 * GP + h], wps[(t2 + 1) * GP + h], bph[t][1], bpl[t][1]);
+            for (int G_ = 0; G_ < NG; G_++) zs[G_] = __shfl_sync(kFull, Z[0] + Z[1], 4 * G_ + c);
+            const uint32_t ro = mb + (uint32_t)((warp * kHeads + c) * D * 4);
+#pragma unroll
+            for (int m = 0; m < KS; m++) {
+                stsf(ro + (16 * m + 2 * g) * 4, fmaf(O[m][0] + O[m][1], 0x1p24f, zs[m >> 1]));
+                stsf(ro + (16 * m + 2 * g + 1) * 4, fmaf(O[m][2] + O[m][3], 0x1p20f, zs[m >> 1]));
             }
-            // value groups (s, z) of tokens t0, t0+1, t2, t2+1; masked for a partial block
-            const unsigned char* vg = rec + R::kVGroups;
-            uint32_t sz[4][NG];
-#pragma unroll
-            for (int w = 0; w < NG; w += 2) {
-#pragma unroll
-                for (int u = 0; u < 4; u++) {
-                    const int tok = (u < 2 ? t0 : t2) + (u & 1);
-                    const uint2 q2 = *reinterpret_cast<const uint2*>(vg + tok * NG * 4 + 4 * w);
-                    sz[u][w] = q2.x;
-                    sz[u][w + 1] = q2.y;
-                }
-            }
-            if (partial) {
-#pragma unroll
-                for (int u = 0; u < 4; u++) {
-                    const bool v = (u < 2 ? t0 : t2) + (u & 1) < nvalid;
-#pragma unroll
-                    for (int w = 0; w < NG; w++) sz[u][w] = v ? sz[u][w] : 0u;
-                }
-            }
-            // -------- p.z: A rows = value groups (row g < NG), tokens as columns
-            {
-                uint32_t za0 = 0u, za2 = 0u;
-#pragma unroll
-                for (int w = 0; w < NG; w++)
-                    if (g == w) {
-                        za0 = __byte_perm(sz[0][w], sz[1][w], 0x7632u);  // (z_t0, z_t0+1)
-                        za2 = __byte_perm(sz[2][w], sz[3][w], 0x7632u);
-                    }
-#pragma unroll
-                for (int t = 0; t < NT; t++) {
-                    mma16816(Z[t], za0, 0u, za2, 0u, hi_role ? bph[t][0] : bpl[t][0],
-                             hi_role ? bph[t][1] : bpl[t][1]);
-                }
-            }
-            // -------- p.V
-            const unsigned char* vrow = rec + R::kVCodes + g * VPL;
-            uint32_t cw[4][VW];
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const int tok = (u < 2 ? t0 : t2) + (u & 1);
-#pragma unroll
-                for (int w = 0; w < VW; w++)
-                    cw[u][w] = *reinterpret_cast<const uint32_t*>(vrow + tok * (D / 2) + 4 * w);
-            }
-#pragma unroll
-            for (int G_ = 0; G_ < NG; G_++) {
-                const uint32_t s01 = __byte_perm(sz[0][G_], sz[1][G_], 0x5410u);  // (s_t0, s_t0+1)
-                const uint32_t s23 = __byte_perm(sz[2][G_], sz[3][G_], 0x5410u);
-                uint32_t b0[NT], b1[NT];
-#pragma unroll
-                for (int t = 0; t < NT; t++) {
-                    uint32_t h0, l0, h1, l1;
-                    scaled_pair(bph[t][0], bpl[t][0], s01, h0, l0);
-                    scaled_pair(bph[t][1], bpl[t][1], s23, h1, l1);
-                    b0[t] = hi_role ? h0 : l0;
-                    b1[t] = hi_role ? h1 : l1;
-                }
-#pragma unroll
-                for (int mm = 0; mm < 2; mm++) {
-                    const int m = 2 * G_ + mm;
-                    const int wi = m >> 2;
-                    const uint32_t sel = (uint32_t)(m & 3) | ((uint32_t)(4 + (m & 3)) << 8);
-                    uint32_t a0, a1, a2, a3;
-                    value_pair(__byte_perm(cw[0][wi], cw[1][wi], sel), a0, a1);
-                    value_pair(__byte_perm(cw[2][wi], cw[3][wi], sel), a2, a3);
-#pragma unroll
-                    for (int t = 0; t < NT; t++) mma16816(O[m][t], a0, a1, a2, a3, b0[t], b1[t]);
-                }
+            const float mh = __shfl_sync(kFull, mrun, 8 * c);
+            if (g == 0) {
+                stsf(mb_m + (warp * kHeads + c) * 4, mh);
+                stsf(mb_l + (warp * kHeads + c) * 4, Z[2] + Z[3]);
             }
         }
-        __syncwarp();
-        const int kn = k + kStages;
-        if (kn < nk) {
-            const int idn = get_id(kn);
-            if (lane == 0) issue(kn, idn);
-        }
-        if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1u;
+        half_sync(half);
+
+        // ---- merge the 8 warps and write the unit's partial (or the output)
+#pragma unroll 1
+        for (int idx = ht; idx < nh * D; idx += kNW * 32) {
+            const int h = idx / D, i = idx % D;
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < kNW; w++) M = fmaxf(M, ldsf(mb_m + (w * kHeads + h) * 4));
+            float o = 0.f, l = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < kNW; w++) {
+                    const float f = ex2(ldsf(mb_m + (w * kHeads + h) * 4) - M);
+                    o = fmaf(f, ldsf(mb + ((w * kHeads + h) * D + i) * 4), o);
+                    l = fmaf(f, ldsf(mb_l + (w * kHeads + h) * 4), l);
+                }
+            }
+            const size_t row = (size_t)cu.b * a.Hq + h0 + h;
+            if (a.num_splits == 1) {
+                a.out[row * D + i] = l > 0.f ? o / l : 0.f;
+            } else {
+                const size_t pr = row * a.num_splits + cu.split;
+                a.ws_o[pr * D + i] = o;
+                if (i == 0) a.ws_ml[pr] = make_float2(M, l);
+            }
         }
     }
+
     if (aborted) {  // give copies still in flight a bounded chance to land
+#pragma unroll 1
         for (int s = 0; s < kStages; s++) {
             mbar_wait(bar0 + 8 * s, 0);
             mbar_wait(bar0 + 8 * s, 1);
-        }
-    }
-
-    // ---- finish this warp: l over tokens; z terms to shared memory
-#pragma unroll
-    for (int t = 0; t < NT; t++) {
-#pragma unroll
-        for (int m = 4; m < 32; m <<= 1) lrun[t] += __shfl_xor_sync(kFull, lrun[t], m);
-    }
-    float* wzs = zs + warp * NG * GP;
-    if (g < NG) {
-#pragma unroll
-        for (int t = 0; t < NT; t++) wzs[g * GP + 4 * t + c] = Z[t][0] + Z[t][1];
-    }
-    __syncthreads();  // every warp is done with its ring; zs is written
-
-    float* red_o = reinterpret_cast<float*>(ring);  // [NW][GP][D]
-    float* red_m = red_o + kNW * GP * D;            // [NW][GP]
-    float* red_l = red_m + kNW * GP;                // [NW][GP]
-#pragma unroll
-    for (int t = 0; t < NT; t++) {
-        const int h = 4 * t + c;
-        if (g == 0) {
-            red_m[warp * GP + h] = mrun[t];
-            red_l[warp * GP + h] = lrun[t];
-        }
-#pragma unroll
-        for (int m = 0; m < MT; m++) {
-            const int dA = 2 * (8 * m + g);
-            const float z = wzs[(m >> 1) * GP + h];
-            red_o[(warp * GP + h) * D + dA] = O[m][t][0] + O[m][t][1] + z;
-            red_o[(warp * GP + h) * D + dA + 1] = O[m][t][2] + O[m][t][3] + z;
-        }
-    }
-    __syncthreads();
-
-    // ---- merge the warps and write the split's partial (or the output)
-    for (int idx = tid; idx < G * D; idx += kNW * 32) {
-        const int h = idx / D, i = idx % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kNW; w++) M = fmaxf(M, red_m[w * GP + h]);
-        float o = 0.f, l = 0.f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w = 0; w < kNW; w++) {
-                const float f = ex2(red_m[w * GP + h] - M);
-                o = fmaf(f, red_o[(w * GP + h) * D + i], o);
-                l = fmaf(f, red_l[w * GP + h], l);
-            }
-        }
-        const int hh = kv * G + h;
-        if (a.num_splits == 1) {
-            a.out[((size_t)b * a.Hq + hh) * D + i] = l > 0.f ? o / l : 0.f;
-        } else {
-            const size_t row = ((size_t)b * a.Hq + hh) * a.num_splits + split;
-            a.ws_o[row * D + i] = o;
-            if (i == 0) a.ws_ml[row] = make_float2(M, l);
         }
     }
 }
@@ -582,36 +653,42 @@ __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
     a.out[(size_t)bh * D + i] = l > 0.f ? o / l : 0.f;
 }
 
-template <int D, int GP>
-constexpr size_t decode_smem_bytes() {
-    constexpr size_t ring = (size_t)kNW * kStages * Rec<D>::kBytes;
-    constexpr size_t merge = (size_t)kNW * GP * D * 4 + 2 * kNW * GP * 4;
-    return (ring > merge ? ring : merge) + kNW * kStages * 8 + GP * D * 4 + kNW * 16 * GP * 4 +
-           kNW * GP * 4 + kNW * GP * (D / 32) * 4;
-}
-
-template <int D, int GP>
-cudaError_t launch_dg(const DecodeArgs& a, cudaStream_t stream) {
-    constexpr size_t smem = decode_smem_bytes<D, GP>();
-    static bool configured = false;  // per instantiation; setting it twice is harmless
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int D>
+cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
+    static uint32_t smem = 0;
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (!smem) smem = plan_bytes<D>();
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
         if (e != cudaSuccess) return e;
-        configured = true;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
     }
-    dim3 grid(a.num_splits, a.Hkv, a.B);
-    decode_split_kernel<D, GP><<<grid, kNW * 32, smem, stream>>>(a);
+    a.smem_bytes = smem;
+    const int halves = (a.units + kHalves - 1) / kHalves;
+    const int grid = halves < num_sms ? halves : num_sms;
+    decode_split_kernel<D><<<grid, kWarps * 32, smem, stream>>>(a);
     if (a.num_splits > 1) combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeArgs& a, int head_dim, cudaStream_t stream) {
+uint32_t decode_smem_bytes(int head_dim) {
+    return head_dim == 128 ? plan_bytes<128>() : plan_bytes<64>();
+}
+
+cudaError_t launch_decode(const DecodeArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
+    DecodeArgs a = args;
     const int G = a.Hq / a.Hkv;
-    if (head_dim == 128) return G <= 4 ? launch_dg<128, 4>(a, stream) : launch_dg<128, 8>(a, stream);
-    return G <= 4 ? launch_dg<64, 4>(a, stream) : launch_dg<64, 8>(a, stream);
+    a.quads = (G + kHeads - 1) / kHeads;
+    a.items = a.B * a.Hkv * a.quads;
+    a.units = a.items * a.num_splits;
+    if (num_sms < 1) num_sms = 1;
+    return head_dim == 128 ? launch_d<128>(a, num_sms, stream) : launch_d<64>(a, num_sms, stream);
 }
 
 }  // namespace tq

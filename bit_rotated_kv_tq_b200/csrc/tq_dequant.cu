@@ -52,14 +52,13 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
         uint32_t kw = 0, vw = 0;
         if (rec) {
             kw = *reinterpret_cast<const uint32_t*>(rec + R::kKCodes + off * R::kCodeRow + sub * 4);
-            const unsigned char* vrow = rec + R::kVCodes + off * R::kCodeRow;
+            const unsigned char* vsrc = rec + R::kVCodes + R::vcode_pos(off, 4 * sub);
 #pragma unroll
-            for (int i = 0; i < 4; i++) vw |= (uint32_t)vrow[R::vpos(sub * 4 + i)] << (8 * i);
+            for (int i = 0; i < 4; i++) vw |= (uint32_t)vsrc[i * R::kPairChunk] << (8 * i);
             nrm = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec + R::kKNorm + off * 2));
-            const uint32_t sz = *reinterpret_cast<const uint32_t*>(
-                rec + R::kVGroups + (off * R::kGroups + sub / 4) * 4);
-            s = half_bits_to_float((uint16_t)(sz & 0xffff));
-            z = half_bits_to_float((uint16_t)(sz >> 16));
+            const int gp = R::group_pos(off, sub / 4);
+            s = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec + R::kVScale + gp));
+            z = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec + R::kVZero + gp));
         }
         const float* C = ctab[h < 64 ? h : 0];
 #pragma unroll

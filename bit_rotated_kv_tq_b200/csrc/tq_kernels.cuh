@@ -37,6 +37,11 @@ struct DecodeArgs {
     int num_splits;
     int blocks_per_split;
     int32_t* status;
+    // set by the launcher
+    int quads;            // groups of four query heads per kv head
+    int items;            // B * Hkv * quads
+    int units;            // items * num_splits
+    uint32_t smem_bytes;  // dynamic shared memory of the split kernel
 };
 
 struct DequantArgs {
@@ -56,7 +61,8 @@ struct DequantArgs {
 size_t append_smem_bytes(int Hkv);
 int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, int head_dim, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, int head_dim, int num_sms, cudaStream_t stream);
+uint32_t decode_smem_bytes(int head_dim);  // dynamic shared memory of the split kernel
 cudaError_t launch_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 
 }  // namespace tq

@@ -33,9 +33,13 @@
  * nibble and element 2j+1 in its high nibble:
  *   [0,      8d)        key codes    [16][d/2] bytes, byte j at row offset j
  *   [8d,     8d+32)     key norms    [16] fp16
- *   [8d+32,  16d+32)    value codes  [16][d/2] bytes, byte j at row offset
- *                       (j mod 8)*(d/16) + j/8 (the tensor-core fragment order)
- *   [16d+32, 18d+32)    value groups [16][d/32] x (fp16 scale, fp16 zero)
+ *   [8d+32,  16d+32)    value codes, 8d bytes: byte j = 8m + r of token t at
+ *                       (8 (t/2) + r) (d/8) + 4 (m/2) + 2 (t%2) + (m%2)
+ *   [16d+32, 17d+32)    value scales fp16: token t, group G at byte
+ *                       2 (4 (c (d/32) + G) + u), c = (t%8)/2, u = 2 (t/8) + t%2
+ *   [17d+32, 18d+32)    value zeros fp16, same placement
+ * (the value placement puts each decode thread's tensor-core operands in
+ * contiguous 8- or 16-byte runs)
  * = 2336 bytes at d = 128, 1184 bytes at d = 64.  The cache is
  * [num_blocks][num_kv_heads][record].
  */
@@ -73,8 +77,10 @@ enum {
     TQ_STATUS_BAD_BLOCK = 2, /* a block-table entry outside [0, num_blocks) */
     TQ_STATUS_RANGE = 4,     /* a key norm or value scale/zero overflowed fp16 */
     TQ_STATUS_BAD_LEN = 8,   /* seq_len < 0 or > max_blocks * 16 (treated as 0) */
-    TQ_STATUS_TIMEOUT = 16   /* a kernel gave up waiting (~1 s) for its own copy: the
+    TQ_STATUS_TIMEOUT = 16,  /* a kernel gave up waiting (~1 s) for its own copy: the
                                 call's output is incomplete; never expected */
+    TQ_STATUS_INTERNAL = 32  /* the decode kernel's shared-memory plan did not fit its
+                                allocation: nothing was computed; never expected */
 };
 
 typedef struct {

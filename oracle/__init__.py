@@ -184,6 +184,15 @@ def record_bytes(d: int) -> int:
     return int(lib().orc_record_bytes(d))
 
 
+def pack_token(record: np.ndarray, d: int, offset: int, kidx, knorm: int, vq, vscale, vzero):
+    """Write one token's fields into a record (uint8 numpy array, modified in place)."""
+    if record.dtype != np.uint8 or not record.flags.c_contiguous:
+        raise ValueError("record must be a contiguous uint8 array")
+    _check(lib().orc_pack_token(_ptr(record), d, offset, _ptr(_c(kidx, np.uint8)), int(knorm),
+                                _ptr(_c(vq, np.uint8)), _ptr(_c(vscale, np.uint16)),
+                                _ptr(_c(vzero, np.uint16))), "pack_token")
+
+
 def unpack_token(record: np.ndarray, d: int, offset: int):
     rec = _c(record, np.uint8)
     kidx = np.zeros(d, np.uint8)

@@ -356,28 +356,48 @@ int orc_decode_v(const uint8_t *q, const uint16_t *scale16, const uint16_t *zero
 /*                                                                      */
 /*   offset 0            key codes   [16 tokens][d/2 bytes]             */
 /*   offset 8d           key norms   [16 tokens] fp16                   */
-/*   offset 8d+32        value codes [16 tokens][d/2 bytes]             */
-/*   offset 16d+32       value scale/zero [16 tokens][d/32 groups]      */
-/*                       as (fp16 scale, fp16 zero) pairs               */
-/*   total 16d + 32 + 64*(d/32) bytes (2336 at d=128, 1184 at d=64)    */
+/*   offset 8d+32        value codes, 8d bytes (placement below)        */
+/*   offset 16d+32       value scales, d bytes: fp16 per (token, group) */
+/*   offset 17d+32       value zeros,  d bytes: same placement          */
+/*   total 18d + 32 bytes (2336 at d=128, 1184 at d=64)                 */
 /*                                                                      */
-/* Code byte j of a row holds element 2j in its low nibble and element  */
-/* 2j+1 in its high nibble.  Key byte j sits at row offset j; value     */
-/* byte j sits at row offset (j mod 8) * (d/16) + floor(j / 8).         */
-/* Multi-byte fields are little-endian.                                 */
+/* Code byte j of a token holds element 2j in its low nibble and        */
+/* element 2j+1 in its high nibble.  Key byte j of token t sits at      */
+/* t*(d/2) + j.  Multi-byte fields are little-endian.                   */
+/*                                                                      */
+/* The pages fix the contents of an entry but not the byte order; the   */
+/* placement of the value fields is chosen so that a decode thread      */
+/* finds its operands contiguous:                                       */
+/*   value byte j of token t, with pair p = t/2, e = t%2, m = j/8,      */
+/*   r = j%8, sits at (8p + r)*(d/8) + 4*(m/2) + 2e + (m%2);            */
+/*   the scale (and zero) of token t, group G, with c = (t%8)/2 and     */
+/*   u = 2*(t/8) + t%2, sits at 2*(4*(c*(d/32) + G) + u) within its     */
+/*   area.                                                              */
 /* ------------------------------------------------------------------ */
 
 size_t orc_record_bytes(int d)
 {
-    return (size_t)ORC_BLOCK * (size_t)d / 2 * 2 + ORC_BLOCK * 2 +
-           (size_t)ORC_BLOCK * (size_t)(d / ORC_VGROUP) * 4;
+    return (size_t)ORC_BLOCK * (size_t)d / 2 * 2 + ORC_BLOCK * 2 + (size_t)2 * d;
 }
 
 static size_t off_knorm(int d) { return (size_t)ORC_BLOCK * d / 2; }
 static size_t off_vcodes(int d) { return off_knorm(d) + ORC_BLOCK * 2; }
-static size_t off_vsz(int d) { return off_vcodes(d) + (size_t)ORC_BLOCK * d / 2; }
-/* row offset of value code byte j (interleaved order, see above) */
-static size_t vpos(int d, int j) { return (size_t)(j % 8) * (d / 16) + (size_t)(j / 8); }
+static size_t off_vscale(int d) { return off_vcodes(d) + (size_t)ORC_BLOCK * d / 2; }
+static size_t off_vzero(int d) { return off_vscale(d) + (size_t)d; }
+
+/* offset of value code byte j of token t within the value-code area */
+static size_t vcode_pos(int d, int t, int j)
+{
+    int p = t / 2, e = t % 2, m = j / 8, r = j % 8;
+    return (size_t)(8 * p + r) * (d / 8) + 4 * (m / 2) + 2 * e + (m % 2);
+}
+
+/* offset of the scale (or zero) of token t, group G within its area */
+static size_t group_pos(int d, int t, int G)
+{
+    int c = (t % 8) / 2, u = 2 * (t / 8) + t % 2;
+    return (size_t)2 * (4 * (c * (d / ORC_VGROUP) + G) + u);
+}
 
 static void put_u16(uint8_t *p, uint16_t v)
 {
@@ -390,19 +410,18 @@ static uint16_t get_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)
 int orc_pack_token(uint8_t *record, int d, int offset, const uint8_t *kidx, uint16_t knorm,
                    const uint8_t *vq, const uint16_t *vscale, const uint16_t *vzero)
 {
-    if (!record || offset < 0 || offset >= ORC_BLOCK || d % ORC_VGROUP)
+    if (!record || offset < 0 || offset >= ORC_BLOCK || d <= 0 || d % ORC_VGROUP)
         return -1;
     uint8_t *kc = record + (size_t)offset * (d / 2);
-    uint8_t *vc = record + off_vcodes(d) + (size_t)offset * (d / 2);
+    uint8_t *vc = record + off_vcodes(d);
     for (int j = 0; j < d / 2; j++) {
         kc[j] = (uint8_t)((kidx[2 * j] & 15) | ((kidx[2 * j + 1] & 15) << 4));
-        vc[vpos(d, j)] = (uint8_t)((vq[2 * j] & 15) | ((vq[2 * j + 1] & 15) << 4));
+        vc[vcode_pos(d, offset, j)] = (uint8_t)((vq[2 * j] & 15) | ((vq[2 * j + 1] & 15) << 4));
     }
     put_u16(record + off_knorm(d) + 2 * offset, knorm);
-    uint8_t *sz = record + off_vsz(d) + (size_t)offset * (d / ORC_VGROUP) * 4;
     for (int g = 0; g < d / ORC_VGROUP; g++) {
-        put_u16(sz + 4 * g, vscale[g]);
-        put_u16(sz + 4 * g + 2, vzero[g]);
+        put_u16(record + off_vscale(d) + group_pos(d, offset, g), vscale[g]);
+        put_u16(record + off_vzero(d) + group_pos(d, offset, g), vzero[g]);
     }
     return 0;
 }
@@ -410,21 +429,21 @@ int orc_pack_token(uint8_t *record, int d, int offset, const uint8_t *kidx, uint
 int orc_unpack_token(const uint8_t *record, int d, int offset, uint8_t *kidx, uint16_t *knorm,
                      uint8_t *vq, uint16_t *vscale, uint16_t *vzero)
 {
-    if (!record || offset < 0 || offset >= ORC_BLOCK || d % ORC_VGROUP)
+    if (!record || offset < 0 || offset >= ORC_BLOCK || d <= 0 || d % ORC_VGROUP)
         return -1;
     const uint8_t *kc = record + (size_t)offset * (d / 2);
-    const uint8_t *vc = record + off_vcodes(d) + (size_t)offset * (d / 2);
+    const uint8_t *vc = record + off_vcodes(d);
     for (int j = 0; j < d / 2; j++) {
+        uint8_t vb = vc[vcode_pos(d, offset, j)];
         kidx[2 * j] = kc[j] & 15;
         kidx[2 * j + 1] = kc[j] >> 4;
-        vq[2 * j] = vc[vpos(d, j)] & 15;
-        vq[2 * j + 1] = vc[vpos(d, j)] >> 4;
+        vq[2 * j] = vb & 15;
+        vq[2 * j + 1] = vb >> 4;
     }
     *knorm = get_u16(record + off_knorm(d) + 2 * offset);
-    const uint8_t *sz = record + off_vsz(d) + (size_t)offset * (d / ORC_VGROUP) * 4;
     for (int g = 0; g < d / ORC_VGROUP; g++) {
-        vscale[g] = get_u16(sz + 4 * g);
-        vzero[g] = get_u16(sz + 4 * g + 2);
+        vscale[g] = get_u16(record + off_vscale(d) + group_pos(d, offset, g));
+        vzero[g] = get_u16(record + off_vzero(d) + group_pos(d, offset, g));
     }
     return 0;
 }

@@ -25,28 +25,43 @@ def layout(d):
     row = d // 2
     kn = 16 * row
     vc = kn + 32
-    vg = vc + 16 * row
-    return row, kn, vc, vg, vg + 16 * (d // 32) * 4
+    vs = vc + 16 * row
+    return row, kn, vc, vs, vs + d, vs + 2 * d
 
 
-def value_positions(d):
-    """Row offset of value code byte j: (j mod 8) * (d/16) + j // 8 (interleaved order)."""
-    j = np.arange(d // 2)
-    return (j % 8) * (d // 16) + j // 8
+def value_code_positions(d):
+    """[16][d/2] offsets of value byte j of token t in the value-code area:
+    (8 (t // 2) + j % 8) (d/8) + 4 ((j // 8) // 2) + 2 (t % 2) + (j // 8) % 2."""
+    t = np.arange(16)[:, None]
+    j = np.arange(d // 2)[None, :]
+    m, r = j // 8, j % 8
+    return (8 * (t // 2) + r) * (d // 8) + 4 * (m // 2) + 2 * (t % 2) + m % 2
+
+
+def group_positions(d):
+    """[16][d/32] byte offsets of the scale (zero) of token t, group G in its area:
+    2 (4 (c (d/32) + G) + u) with c = (t % 8) // 2, u = 2 (t // 8) + t % 2."""
+    t = np.arange(16)[:, None]
+    G = np.arange(d // 32)[None, :]
+    c, u = (t % 8) // 2, 2 * (t // 8) + t % 2
+    return 2 * (4 * (c * (d // 32) + G) + u)
 
 
 def unpack_record(rec: np.ndarray, d: int):
     """rec uint8 [record] -> kidx [16][d], knorm uint16 [16], vq [16][d], vs, vz uint16 [16][d/32]."""
-    row, kn, vc, vg, total = layout(d)
+    row, kn, vc, vs, vz, total = layout(d)
     assert rec.shape[-1] == total
     kc = rec[..., :kn].reshape(rec.shape[:-1] + (16, row))
     kidx = np.stack([kc & 15, kc >> 4], axis=-1).reshape(rec.shape[:-1] + (16, d))
     knorm = rec[..., kn:kn + 32].copy().view(np.uint16).reshape(rec.shape[:-1] + (16,))
-    vcb = rec[..., vc:vc + 16 * row].reshape(rec.shape[:-1] + (16, row))
-    vcb = vcb[..., value_positions(d)]  # back to natural byte order
+    vcb = rec[..., vc:vs][..., value_code_positions(d)]  # natural [16][d/2] byte order
     vq = np.stack([vcb & 15, vcb >> 4], axis=-1).reshape(rec.shape[:-1] + (16, d))
-    sz = rec[..., vg:total].copy().view(np.uint16).reshape(rec.shape[:-1] + (16, d // 32, 2))
-    return kidx, knorm, vq, sz[..., 0], sz[..., 1]
+    gp = group_positions(d)
+
+    def u16(area):
+        return area[..., gp].astype(np.uint16) | (area[..., gp + 1].astype(np.uint16) << 8)
+
+    return kidx, knorm, vq, u16(rec[..., vs:vz]), u16(rec[..., vz:total])
 
 
 def key_boundary_distance(ky: np.ndarray, table: np.ndarray) -> np.ndarray:

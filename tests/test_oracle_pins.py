@@ -277,21 +277,31 @@ def test_record_size_and_nibble_order(orc):
     row = rec[5 * 64:6 * 64]
     assert np.all(row == int(g["key_e0_byte"][0], 16))
     assert int(rec[1024 + 10]) | (int(rec[1024 + 11]) << 8) == 0x3C00
-    vrow = rec[1056 + 5 * 64:1056 + 6 * 64]
-    assert list(vrow) == [int(x, 16) for x in g["value_ramp_stored_d128"]]
-    # undoing the interleave gives the natural code bytes of the worked example
-    j = np.arange(64)
-    natural = vrow[(j % 8) * 8 + j // 8]
+    vc = rec[1056:1056 + 1024]
+    chunk19 = [int(x, 16) for x in g["value_ramp_chunk19_d128"]]
+    assert list(vc[19 * 16:20 * 16]) == chunk19
+    odd_pos = [2, 3, 6, 7, 10, 11, 14, 15]
+    for r in range(8):  # chunk 16 + r: 0x11*r at m-even, 0x11*(r+8) at m-odd positions
+        ch = vc[(16 + r) * 16:(17 + r) * 16]
+        assert list(ch[odd_pos]) == [0x11 * r, 0x11 * (r + 8)] * 4
+        assert not np.any(np.delete(ch, odd_pos))
+    # reading the bytes back in natural order gives the worked example's code bytes
+    natural = [vc[(16 + j % 8) * 16 + 4 * (j // 16) + 2 + (j // 8) % 2] for j in range(64)]
     want = [int(x, 16) for x in g["value_ramp_bytes"]]
-    assert list(natural[:16]) == want and list(natural[16:32]) == want
-    sz = rec[2080 + 5 * 16:2080 + 6 * 16]
-    assert int(sz[0]) | (int(sz[1]) << 8) == 0x4023 and int(sz[2]) | (int(sz[3]) << 8) == 0
-    # every other token row is untouched
+    assert natural[:16] == want and natural[16:32] == want
+    offs = [int(x) for x in g["value_ramp_group_offsets_d128"]]
+    scale_area, zero_area = rec[2080:2208], rec[2208:2336]
+    for o in offs:
+        assert int(scale_area[o]) | (int(scale_area[o + 1]) << 8) == int(g["value_ramp_scale16"][0], 16)
+        assert int(zero_area[o]) | (int(zero_area[o + 1]) << 8) == int(g["value_ramp_zero16"][0], 16)
+    # every other byte is untouched
     mask = np.ones(2336, bool)
     mask[5 * 64:6 * 64] = False
     mask[1024 + 10:1024 + 12] = False
-    mask[1056 + 5 * 64:1056 + 6 * 64] = False
-    mask[2080 + 5 * 16:2080 + 6 * 16] = False
+    for r in range(8):
+        mask[1056 + (16 + r) * 16:1056 + (17 + r) * 16] = False
+    for o in offs:
+        mask[2080 + o:2080 + o + 2] = False
     assert np.all(rec[mask] == 0)
 
 
@@ -417,3 +427,38 @@ def test_kmeans_on_gaussian_samples_reaches_lloyd_max_distortion(orc):
 
     assert mse(tab) <= mse(init) * (1 + 1e-4)
     assert 0.0095 * 0.98 <= mse(tab) <= 0.0095 * 1.02
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_record_placement_round_trip(orc, d):
+    """The oracle's placement of every field and the test-side reader (written
+    separately from the documented formulas) agree on a record with every token,
+    code, norm, scale and zero distinct enough to expose a swapped index."""
+    from parity_util import unpack_record
+
+    rec = orc.record_bytes(d)
+    assert rec == 18 * d + 32
+    r = np.random.default_rng(7)
+    kidx = r.integers(0, 16, (16, d)).astype(np.uint8)
+    vq = r.integers(0, 16, (16, d)).astype(np.uint8)
+    kn = r.integers(0, 0x7bff, 16).astype(np.uint16)
+    vs = r.integers(0, 0x7bff, (16, d // 32)).astype(np.uint16)
+    vz = r.integers(0, 0xfbff, (16, d // 32)).astype(np.uint16)
+    record = np.zeros(rec, np.uint8)
+    for t in range(16):
+        orc.pack_token(record, d, t, kidx[t], kn[t], vq[t], vs[t], vz[t])
+    # every byte of the record is written by exactly one field of one token
+    counts = np.zeros(rec, np.int64)
+    for t in range(16):
+        probe = np.zeros(rec, np.uint8)
+        orc.pack_token(probe, d, t, np.full(d, 15, np.uint8), 0xffff, np.full(d, 15, np.uint8),
+                       np.full(d // 32, 0xffff, np.uint16), np.full(d // 32, 0xffff, np.uint16))
+        counts += probe == 0xff
+    assert np.all(counts == 1)
+    gk, gn, gv, gs, gz = unpack_record(record, d)
+    assert np.array_equal(gk, kidx) and np.array_equal(gn, kn) and np.array_equal(gv, vq)
+    assert np.array_equal(gs, vs) and np.array_equal(gz, vz)
+    for t in range(16):
+        k2, n2, v2, s2, z2 = orc.unpack_token(record, d, t)
+        assert np.array_equal(k2, kidx[t]) and n2 == kn[t] and np.array_equal(v2, vq[t])
+        assert np.array_equal(s2, vs[t]) and np.array_equal(z2, vz[t])
