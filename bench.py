@@ -411,6 +411,7 @@ def run_tq(args, rank, world, local):
             "append_tokens_per_s": T / (app_avg / 1e3),
             "append_hbm_frac": append_bytes(w, T) / (app_avg / 1e3) / 1e9 / peak,
             "num_splits": S,
+            "partition": "even cut of (item, block) space over the grid" if S == 0 else f"{S} splits per item",
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": profiled_traffic(w),
                          "kernel": "tq_decode_attention (split kernel + combine)",

@@ -265,35 +265,19 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
 }
 
 TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len) {
-    if (B <= 0 || H_kv <= 0 || max_seq_len <= 0) return 1;
-    const int nblk = (max_seq_len + tq::kBlock - 1) / tq::kBlock;
-    const long long items = (long long)B * H_kv;  // one group of up to four query heads each
-    const long long halves = 2LL * device_sms();
-    // The split kernel is persistent: two halves of 8 warps per SM, each taking
-    // (item, split) units in turn.  Estimated time, in units of one record per
-    // warp: rounds of units x (records per warp per unit + per-unit overhead),
-    // plus the combine pass when there is more than one split.
-    constexpr double kUnitOverhead = 0.75, kCombine = 2.5;
-    int best_s = 1;
-    double best = 1e300;
-    for (int s = 1; s <= 64 && s <= nblk; s++) {
-        const int bps = (nblk + s - 1) / s;
-        const int S = (nblk + bps - 1) / bps;
-        if (S != s) continue;  // the same plan as a smaller s
-        const long long rounds = (items * S + halves - 1) / halves;
-        const double cost = (double)rounds * ((bps + 7) / 8 + kUnitOverhead) + (S > 1 ? kCombine : 0.0);
-        if (cost < best) {
-            best = cost;
-            best_s = S;
-        }
-    }
-    return best_s;
+    (void)B;
+    (void)H_kv;
+    (void)max_seq_len;
+    return 0;  // the library cuts the work evenly over the whole GPU
 }
 
 TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_splits) {
-    if (B <= 0 || H_q <= 0 || !supported_d(head_dim) || num_splits <= 1) return 0;
-    const size_t rows = (size_t)B * H_q * num_splits;
-    return rows * head_dim * sizeof(float) + rows * sizeof(float2);
+    if (B <= 0 || H_q <= 0 || !supported_d(head_dim) || num_splits == 1 || num_splits < 0) return 0;
+    // ranges: at most two per SM half-pair with the even cut, else at most
+    // items * S + 1 with items <= B * H_q
+    const long long ranges =
+        num_splits == 0 ? 2LL * device_sms() : (long long)B * H_q * num_splits + 1;
+    return (size_t)ranges * 2 * 4 * ((size_t)head_dim * sizeof(float) + sizeof(float2));
 }
 
 TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
@@ -324,21 +308,6 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
         (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
         return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: q/out/tables must be 4-byte aligned");
     const int d = cache->head_dim;
-    const int S_req = num_splits ? num_splits : tq_decode_default_splits(B, Hkv, max_seq_len);
-    const int nblk = (max_seq_len + tq::kBlock - 1) / tq::kBlock;
-    int bps = nblk > 0 ? (nblk + S_req - 1) / S_req : 1;
-    int S = nblk > 0 ? (nblk + bps - 1) / bps : 1;
-    const long long units = (long long)B * Hkv * ((G + 3) / 4) * S;
-    if (units > 0x7fffffffLL)
-        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * splits too large");
-    if (S > 1) {
-        const size_t need = tq_decode_workspace_bytes(B, H_q, d, S);
-        if (!workspace || ws_bytes < need)
-            return fail(TQ_ERR_WORKSPACE, "tq_decode_attention: workspace %zu bytes < %zu needed",
-                        workspace ? ws_bytes : (size_t)0, need);
-        if (!aligned(workspace, 16))
-            return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: workspace must be 16-byte aligned");
-    }
     tq::DecodeArgs a;
     a.q = static_cast<const uint16_t*>(q);
     a.cache = static_cast<const unsigned char*>(cache->data);
@@ -353,12 +322,22 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
     a.seq_lens = seq_lens;
     a.scale_log2 = scale * 1.44269504088896340736f;
     a.out = out;
-    a.num_splits = S;
-    a.blocks_per_split = bps;
+    a.num_splits = num_splits;
+    a.max_seq_len = max_seq_len;
+    if (!tq::decode_plan(a, device_sms()))
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * num_splits too large");
+    const size_t need = tq::decode_workspace_for(a, d);
+    if (need) {
+        if (!workspace || ws_bytes < need)
+            return fail(TQ_ERR_WORKSPACE, "tq_decode_attention: workspace %zu bytes < %zu needed",
+                        workspace ? ws_bytes : (size_t)0, need);
+        if (!aligned(workspace, 16))
+            return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: workspace must be 16-byte aligned");
+    }
     a.ws_o = static_cast<float*>(workspace);
-    a.ws_ml = S > 1 ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
-                                                 (size_t)B * H_q * S * d)
-                    : nullptr;
+    a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
+                                               (size_t)a.nranges * 2 * 4 * d)
+                   : nullptr;
     a.status = status;
     cudaError_t e = tq::launch_decode(a, d, device_sms(), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");

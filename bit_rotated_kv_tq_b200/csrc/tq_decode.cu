@@ -217,47 +217,77 @@ uint32_t plan_bytes() {
     return worst;
 }
 
-// ------------------------------------------------------------------ units
-// What one warp needs to know about a unit: the item's coordinates, the
-// sequence length, and this warp's share of the split's blocks.
-struct Unit {
-    int u;                  // unit index (>= units: past the end)
-    int b, kv, quad, split;
+// ------------------------------------------------------------------ segments
+// The work is the virtual record space items x nmax (nmax = blocks of the
+// longest sequence), cut into ranges of R consecutive records; half h takes
+// ranges h, h + H, ...  A segment is the part of one item inside one range.
+// An item that lies wholly inside a range is finished there ("direct"); the
+// others leave one partial per range, in slot 0 if the item is the range's
+// first, else slot 1 (only the range's last item can be split besides the first).
+struct Seg {
+    int r;                  // range (>= nranges: past the end)
+    int i, i_first, i_last; // item, and the first and last items of the range
+    int b, kv, quad;
     int L;                  // tokens of the sequence (clamped)
-    int nk;                 // records of this warp in the unit
+    int jb;                 // first block of the segment
+    int nk;                 // records of this warp in the segment
+    bool direct;
     const int32_t* bt;      // block-table entry of this warp's first record
     const unsigned char* src;  // record of block 0 for this kv head
 };
 
 template <int D>
-__device__ __forceinline__ void unit_at(Unit& s, int u, const DecodeArgs& a, int warp,
-                                        bool report) {
-    s.u = u;
-    s.nk = 0;
-    if (u >= a.units) return;
-    const int item = u % a.items;
-    s.split = u / a.items;
-    s.quad = item % a.quads;
-    const int bk = item / a.quads;
+__device__ __forceinline__ void seg_item(Seg& s, const DecodeArgs& a, int warp, bool report) {
+    const long long base = (long long)s.i * a.nmax;
+    const long long p0 = (long long)s.r * a.R;
+    const long long p1 = min(p0 + a.R, (long long)a.items * a.nmax);
+    const int lo = (int)(max(p0, base) - base), hi = (int)(min(p1, base + a.nmax) - base);
+    s.direct = lo == 0 && hi == a.nmax;
+    s.quad = s.i % a.quads;
+    const int bk = s.i / a.quads;
     s.kv = bk % a.Hkv;
     s.b = bk / a.Hkv;
     int L = a.seq_lens[s.b];
-    const bool first = report && s.kv == 0 && s.quad == 0 && s.split == 0;
+    const bool first = report && s.kv == 0 && s.quad == 0 && lo == 0;
     if (L < 0 || L > a.max_blocks * kBlock) {
         if (first) flag_status(a.status, TQ_STATUS_BAD_LEN);
         L = 0;
     }
-    if (L > a.num_splits * a.blocks_per_split * kBlock) {
+    if (L > a.nmax * kBlock) {
         if (first) flag_status(a.status, TQ_STATUS_BAD_LEN);
-        L = a.num_splits * a.blocks_per_split * kBlock;
+        L = a.nmax * kBlock;
     }
     s.L = L;
     const int nblk = (L + kBlock - 1) / kBlock;
-    const int jb = s.split * a.blocks_per_split;
-    const int left = min(jb + a.blocks_per_split, nblk) - jb - warp;
+    s.jb = lo;
+    const int left = min(hi, nblk) - lo - warp;
     s.nk = left > 0 ? (left + kNW - 1) / kNW : 0;
-    s.bt = a.block_tables + (size_t)s.b * a.max_blocks + jb + warp;
+    s.bt = a.block_tables + (size_t)s.b * a.max_blocks + lo + warp;
     s.src = a.cache + (size_t)s.kv * Rec<D>::kBytes;
+}
+
+// first segment of range r (or past the end)
+template <int D>
+__device__ __forceinline__ void seg_range(Seg& s, int r, const DecodeArgs& a, int warp, bool report) {
+    s.r = r;
+    s.nk = 0;
+    if (r >= a.nranges) return;
+    const long long p0 = (long long)r * a.R;
+    const long long p1 = min(p0 + a.R, (long long)a.items * a.nmax);
+    s.i = s.i_first = (int)(p0 / a.nmax);
+    s.i_last = (int)((p1 - 1) / a.nmax);
+    seg_item<D>(s, a, warp, report);
+}
+
+template <int D>
+__device__ __forceinline__ void seg_next(Seg& s, int stride, const DecodeArgs& a, int warp,
+                                         bool report) {
+    if (s.i < s.i_last) {
+        s.i++;
+        seg_item<D>(s, a, warp, report);
+    } else {
+        seg_range<D>(s, s.r + stride, a, warp, report);
+    }
 }
 
 // N consecutive 32-bit words (N = 2 or 4) of shared memory
@@ -300,7 +330,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
         return;
     }
     const int G = a.Hq / a.Hkv;
-    const int stride = kHalves * gridDim.x;  // units per round over all halves
+    const int stride = kHalves * gridDim.x;  // ranges per round over all halves
     const int v = kHalves * blockIdx.x + half;
 
     // ---- this warp's ring: slots, barriers, and the block id of each stage
@@ -314,17 +344,17 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     }
     __syncwarp();
 
-    // ---- issue cursor: the next record of this warp's stream (all its units, in order)
-    Unit is;
-    unit_at<D>(is, v, a, warp, false);
-    while (is.u < a.units && is.nk == 0) unit_at<D>(is, is.u + stride, a, warp, false);
+    // ---- issue cursor: the next record of this warp's stream (all its segments, in order)
+    Seg is;
+    seg_range<D>(is, v, a, warp, false);
+    while (is.r < a.nranges && is.nk == 0) seg_next<D>(is, stride, a, warp, false);
     int irem = is.nk, istage = 0;
     const int32_t* ibt = is.bt;
-    int nid = is.u < a.units ? *ibt : -1;
+    int nid = is.r < a.nranges ? *ibt : -1;
     // Copy the record of block nid into stage istage (one elected lane, no branch),
     // note its id for the consumer, and move the cursor on.
     auto issue = [&]() {
-        if (is.u >= a.units) return;
+        if (is.r >= a.nranges) return;
         const uint32_t bar = bar0 + 8 * istage;
         const uint32_t valid = (uint32_t)(nid >= 0 && nid < a.num_blocks);
         const uint32_t me = (uint32_t)(lane == 0);
@@ -344,14 +374,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             : "memory");
         istage = istage == kStages - 1 ? 0 : istage + 1;
         if (--irem == 0) {
-            do unit_at<D>(is, is.u + stride, a, warp, false);
-            while (is.u < a.units && is.nk == 0);
+            do seg_next<D>(is, stride, a, warp, false);
+            while (is.r < a.nranges && is.nk == 0);
             irem = is.nk;
             ibt = is.bt;
         } else {
             ibt += kNW;
         }
-        nid = is.u < a.units ? *ibt : -1;
+        nid = is.r < a.nranges ? *ibt : -1;
     };
 #pragma unroll 1
     for (int k = 0; k < kStages; k++) issue();
@@ -370,17 +400,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     bool aborted = false;
     const uint16_t* lut_tab = nullptr;  // table held by this half's side of the LUT
 
+    Seg cu;
+    seg_range<D>(cu, v, a, warp, warp == 0 && lane == 0);
+    bool first_seg = true;
 #pragma unroll 1
-    for (int u = v; u < a.units; u += stride) {
-        Unit cu;
-        unit_at<D>(cu, u, a, warp, warp == 0 && lane == 0);
+    for (; cu.r < a.nranges; seg_next<D>(cu, stride, a, warp, warp == 0 && lane == 0)) {
         const int h0 = cu.kv * G + cu.quad * kHeads;  // first query head of the item
         const int nh = min(kHeads, G - cu.quad * kHeads);
 
         // ---- the centroid-pair table of this kv head, on this half's side of
         // each 256-byte row: word (row, lane) = (C[row & 15], C[row >> 4])
         const uint16_t* tab = a.k_tables ? a.k_tables + cu.kv * 16 : nullptr;
-        if (u == v || tab != lut_tab) {
+        if (first_seg || tab != lut_tab) {
+            first_seg = false;
             lut_tab = tab;
 #pragma unroll 1
             for (int it = 0; it < 8; it++) {
@@ -459,7 +491,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
         float mrun = -INFINITY;  // running maximum of head g/2
         const int nk = aborted ? 0 : cu.nk;
         // tokens in this warp's last record of the unit (< 16 only at the end of the sequence)
-        const int last_valid = cu.L - (cu.split * a.blocks_per_split + warp + kNW * (nk - 1)) * kBlock;
+        const int last_valid = cu.L - (cu.jb + warp + kNW * (nk - 1)) * kBlock;
 #pragma unroll 1
         for (int k = 0; k < nk; k++) {
             const uint32_t rec = ringw + stage * REC;
@@ -613,11 +645,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                     l = fmaf(f, ldsf(mb_l + (w * kHeads + h) * 4), l);
                 }
             }
-            const size_t row = (size_t)cu.b * a.Hq + h0 + h;
-            if (a.num_splits == 1) {
-                a.out[row * D + i] = l > 0.f ? o / l : 0.f;
+            if (cu.direct) {
+                a.out[((size_t)cu.b * a.Hq + h0 + h) * D + i] = l > 0.f ? o / l : 0.f;
             } else {
-                const size_t pr = row * a.num_splits + cu.split;
+                const size_t pr = ((size_t)cu.r * 2 + (cu.i == cu.i_first ? 0 : 1)) * kHeads + h;
                 a.ws_o[pr * D + i] = o;
                 if (i == 0) a.ws_ml[pr] = make_float2(M, l);
             }
@@ -633,20 +664,33 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     }
 }
 
-// out[b][h] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s, M = max_s m_s.
+// Items cut by range boundaries: out[b][h] = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r
+// over the ranges r that hold part of the item, M = max_r m_r.  Whole items
+// were written by the split kernel and are skipped.
 template <int D>
 __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
     const int bh = blockIdx.x;
     const int i = threadIdx.x;
-    const size_t row0 = (size_t)bh * a.num_splits;
+    const int G = a.Hq / a.Hkv;
+    const int b = bh / a.Hq, hh = bh % a.Hq;
+    const int kv = hh / G, quad = (hh % G) / kHeads, h = (hh % G) % kHeads;
+    const int item = (b * a.Hkv + kv) * a.quads + quad;
+    const long long base = (long long)item * a.nmax;
+    const int rA = (int)(base / a.R), rB = (int)((base + a.nmax - 1) / a.R);
+    if (rA == rB) return;  // whole inside one range: already written
+    auto part = [&](int r) {
+        const int slot = (long long)r * a.R / a.nmax == item ? 0 : 1;
+        return ((size_t)r * 2 + slot) * kHeads + h;
+    };
     float M = -INFINITY;
-    for (int s = 0; s < a.num_splits; s++) M = fmaxf(M, a.ws_ml[row0 + s].x);
+    for (int r = rA; r <= rB; r++) M = fmaxf(M, a.ws_ml[part(r)].x);
     float o = 0.f, l = 0.f;
     if (M != -INFINITY) {
-        for (int s = 0; s < a.num_splits; s++) {
-            const float2 ml = a.ws_ml[row0 + s];
+        for (int r = rA; r <= rB; r++) {
+            const size_t pr = part(r);
+            const float2 ml = a.ws_ml[pr];
             const float f = ex2(ml.x - M);
-            o = fmaf(f, a.ws_o[(row0 + s) * D + i], o);
+            o = fmaf(f, a.ws_o[pr * D + i], o);
             l = fmaf(f, ml.y, l);
         }
     }
@@ -668,10 +712,10 @@ cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
     a.smem_bytes = smem;
-    const int halves = (a.units + kHalves - 1) / kHalves;
+    const int halves = (a.nranges + kHalves - 1) / kHalves;
     const int grid = halves < num_sms ? halves : num_sms;
     decode_split_kernel<D><<<grid, kWarps * 32, smem, stream>>>(a);
-    if (a.num_splits > 1) combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a);
+    if (decode_needs_combine(a)) combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -681,13 +725,38 @@ uint32_t decode_smem_bytes(int head_dim) {
     return head_dim == 128 ? plan_bytes<128>() : plan_bytes<64>();
 }
 
-cudaError_t launch_decode(const DecodeArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
-    DecodeArgs a = args;
+// Ranges: with num_splits = 0 the virtual records are cut evenly over every
+// half of a full grid; with num_splits = S each range is ceil(nmax / S) records
+// (S = 1: one range per item, nothing to combine).
+bool decode_plan(DecodeArgs& a, int num_sms) {
     const int G = a.Hq / a.Hkv;
     a.quads = (G + kHeads - 1) / kHeads;
     a.items = a.B * a.Hkv * a.quads;
-    a.units = a.items * a.num_splits;
+    a.nmax = a.max_seq_len > 0 ? (a.max_seq_len + kBlock - 1) / kBlock : 1;
+    const long long V = (long long)a.items * a.nmax;
+    if (a.num_splits > 0) {
+        a.R = (a.nmax + a.num_splits - 1) / a.num_splits;
+    } else {
+        const long long H = (long long)kHalves * num_sms;
+        a.R = (V + H - 1) / H;
+    }
+    if (a.R < 1) a.R = 1;
+    const long long nr = (V + a.R - 1) / a.R;
+    a.nranges = nr > 0x7fffffffLL ? 0 : (int)nr;
+    return a.nranges > 0;
+}
+
+bool decode_needs_combine(const DecodeArgs& a) { return a.nranges > 1 && a.R % a.nmax != 0; }
+
+size_t decode_workspace_for(const DecodeArgs& a, int head_dim) {
+    if (!decode_needs_combine(a)) return 0;
+    return (size_t)a.nranges * 2 * kHeads * (head_dim * sizeof(float) + sizeof(float2));
+}
+
+cudaError_t launch_decode(const DecodeArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
+    DecodeArgs a = args;
     if (num_sms < 1) num_sms = 1;
+    if (!decode_plan(a, num_sms)) return cudaErrorInvalidValue;
     return head_dim == 128 ? launch_d<128>(a, num_sms, stream) : launch_d<64>(a, num_sms, stream);
 }
 

@@ -60,18 +60,14 @@ TQ_API int tq_decode_attention_static(const void* q, const tq_cache_t* cache,
         return tq_decode_attention(q, cache, k_tables, block_tables, max_blocks, seq_lens, B, H_q,
                                    max_seq_len, scale, out, nullptr, 0, num_splits, status, stream);
     }
-    const int S_req = num_splits ? num_splits
-                                 : tq_decode_default_splits(B, cache->num_kv_heads, max_seq_len);
-    const int nblk = (max_seq_len + tq::kBlock - 1) / tq::kBlock;
-    const int bps = nblk > 0 ? (nblk + S_req - 1) / S_req : 1;
-    const int S = nblk > 0 ? (nblk + bps - 1) / bps : 1;
-    const size_t need = tq_decode_workspace_bytes(B, H_q, cache->head_dim, S);
+    const size_t need = tq_decode_workspace_bytes(B, H_q, cache->head_dim, num_splits);
     if (need > kScratchBytes) {
         char msg[256];
         snprintf(msg, sizeof msg,
-                 "tq_decode_attention_static: %d splits need %zu bytes of partials, more than the "
-                 "library's fixed %zu-byte scratch; pass fewer splits or use tq_decode_attention",
-                 S, need, kScratchBytes);
+                 "tq_decode_attention_static: num_splits %d may need %zu bytes of partials, more "
+                 "than the library's fixed %zu-byte scratch; pass 0 or fewer splits, or use "
+                 "tq_decode_attention",
+                 num_splits, need, kScratchBytes);
         return tq::set_last_error(TQ_ERR_WORKSPACE, msg);
     }
     cudaError_t e = cudaSuccess;
@@ -82,9 +78,9 @@ TQ_API int tq_decode_attention_static(const void* q, const tq_cache_t* cache,
                  cudaGetErrorString(e));
         return tq::set_last_error(TQ_ERR_CUDA, msg);
     }
-    // Every partial slot is written by its split before the combine reads it,
-    // so nothing in the scratch has to start at zero.  The split plan here and
-    // in tq_decode_attention come from the same num_splits, so they agree.
+    // Every partial slot is written by the split kernel before the combine reads
+    // it, so nothing in the scratch has to start at zero; the bound above covers
+    // the plan tq_decode_attention makes from the same num_splits.
     return tq_decode_attention(q, cache, k_tables, block_tables, max_blocks, seq_lens, B, H_q,
                                max_seq_len, scale, out, ws, kScratchBytes, num_splits, status,
                                stream);

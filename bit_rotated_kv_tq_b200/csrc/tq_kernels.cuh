@@ -32,15 +32,17 @@ struct DecodeArgs {
     const int32_t* seq_lens;     // [B]
     float scale_log2;            // scale * log2(e)
     float* out;                  // [B][Hq][D]
-    float* ws_o;                 // [B][Hq][S][D] partial outputs (unnormalised)
-    float2* ws_ml;               // [B][Hq][S] (running max in log2 units, sum)
-    int num_splits;
-    int blocks_per_split;
+    float* ws_o;                 // [ranges][2][4][D] partial outputs (unnormalised)
+    float2* ws_ml;               // [ranges][2][4] (running max in log2 units, sum)
+    int num_splits;              // 0: even cut over the grid; S: ranges of nmax/S blocks
+    int max_seq_len;
     int32_t* status;
-    // set by the launcher
+    // set by decode_plan
     int quads;            // groups of four query heads per kv head
     int items;            // B * Hkv * quads
-    int units;            // items * num_splits
+    int nmax;             // blocks of the longest sequence (>= 1)
+    long long R;          // records per range of the virtual space items x nmax
+    int nranges;
     uint32_t smem_bytes;  // dynamic shared memory of the split kernel
 };
 
@@ -63,6 +65,9 @@ int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 uint32_t decode_smem_bytes(int head_dim);  // dynamic shared memory of the split kernel
+bool decode_plan(DecodeArgs& a, int num_sms);            // ranges; false: too many
+bool decode_needs_combine(const DecodeArgs& a);          // some item is cut by a range
+size_t decode_workspace_for(const DecodeArgs& a, int head_dim);  // partials, bytes
 cudaError_t launch_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 
 }  // namespace tq

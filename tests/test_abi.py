@@ -111,7 +111,9 @@ def test_argument_validation_without_launch(lib):
     assert dec(Hq=4, L=65) == tq.TQ_ERR_INVALID_ARG  # max_seq_len beyond max_blocks * 16
     assert dec(Hq=4, scale=float("nan")) == tq.TQ_ERR_INVALID_ARG
     assert dec(Hq=4, B=0) == tq.TQ_OK
-    assert lib.tq_decode_workspace_bytes(2, 8, 128, 4) == 2 * 8 * 4 * (128 * 4 + 8)
+    # explicit splits: at most B * H_q * S + 1 ranges, two partial slots of four heads each
+    assert lib.tq_decode_workspace_bytes(2, 8, 128, 4) == (2 * 8 * 4 + 1) * 2 * 4 * (128 * 4 + 8)
+    assert lib.tq_decode_workspace_bytes(2, 8, 64, 3) == (2 * 8 * 3 + 1) * 2 * 4 * (64 * 4 + 8)
     assert lib.tq_decode_workspace_bytes(2, 8, 128, 1) == 0
     # dequantize: misaligned output
     rc = lib.tq_dequantize(ctypes.byref(c), None, P(16), 4, P(16), 1, 8, P(20), P(16), None, None)
