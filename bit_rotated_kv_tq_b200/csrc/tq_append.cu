@@ -87,11 +87,6 @@ __device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t
     __syncthreads();
 }
 
-// n / d for n < 2^32 with M = (2^64 - 1) / d + 1 (exact: the error term of
-// n * M / 2^64 stays below 2^-32 < 1/d); d == 1 is flagged by M == 0.
-__device__ __forceinline__ uint32_t fast_div(uint32_t n, uint64_t M) {
-    return M ? (uint32_t)__umul64hi((uint64_t)n, M) : n;
-}
 
 // fp32 neighbours of 1/15: the value rounded up and rounded down.
 __device__ __forceinline__ float inv15_up() { return __uint_as_float(0x3d888889u); }
@@ -422,8 +417,6 @@ size_t append_smem_bytes(int Hkv) {
     return (size_t)Hkv * sizeof(HeadBins) + (size_t)Hkv * kBins * sizeof(BinEntry);
 }
 
-// (2^64 - 1) / d + 1: the multiplier of fast_div (0 for d == 1).
-static uint64_t div_magic(uint32_t d) { return d <= 1 ? 0 : ~0ull / d + 1; }
 
 template <int D>
 static int resident_ctas(int num_sms, size_t smem) {

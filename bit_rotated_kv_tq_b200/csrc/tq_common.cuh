@@ -69,6 +69,14 @@ __device__ __forceinline__ uint4 ld_stream_u4(const void* p) {
     return r;
 }
 
+// n / d for n < 2^32 with M = (2^64 - 1) / d + 1 (exact: the error term of
+// n * M / 2^64 stays below 2^-32 < 1/d); d == 1 is flagged by M == 0.
+__device__ __forceinline__ uint32_t fast_div(uint32_t n, uint64_t M) {
+    return M ? (uint32_t)__umul64hi((uint64_t)n, M) : n;
+}
+// the multiplier of fast_div for divisor d (0 for d == 1)
+inline uint64_t div_magic(uint32_t d) { return d <= 1 ? 0 : ~0ull / d + 1; }
+
 __device__ __forceinline__ void flag_status(int32_t* status, int bits) {
     if (status) atomicOr(status, bits);
 }

@@ -238,15 +238,15 @@ struct Seg {
 
 template <int D>
 __device__ __forceinline__ void seg_item(Seg& s, const DecodeArgs& a, int warp, bool report) {
-    const long long base = (long long)s.i * a.nmax;
-    const long long p0 = (long long)s.r * a.R;
-    const long long p1 = min(p0 + a.R, (long long)a.items * a.nmax);
-    const int lo = (int)(max(p0, base) - base), hi = (int)(min(p1, base + a.nmax) - base);
+    const int base = s.i * a.nmax;
+    const int p0 = s.r * a.R;
+    const int p1 = min(p0 + a.R, a.vrec);
+    const int lo = max(p0, base) - base, hi = min(p1, base + a.nmax) - base;
     s.direct = lo == 0 && hi == a.nmax;
-    s.quad = s.i % a.quads;
-    const int bk = s.i / a.quads;
-    s.kv = bk % a.Hkv;
-    s.b = bk / a.Hkv;
+    const int bk = (int)fast_div((uint32_t)s.i, a.div_quads);
+    s.quad = s.i - bk * a.quads;
+    s.b = (int)fast_div((uint32_t)bk, a.div_hkv);
+    s.kv = bk - s.b * a.Hkv;
     int L = a.seq_lens[s.b];
     const bool first = report && s.kv == 0 && s.quad == 0 && lo == 0;
     if (L < 0 || L > a.max_blocks * kBlock) {
@@ -272,10 +272,10 @@ __device__ __forceinline__ void seg_range(Seg& s, int r, const DecodeArgs& a, in
     s.r = r;
     s.nk = 0;
     if (r >= a.nranges) return;
-    const long long p0 = (long long)r * a.R;
-    const long long p1 = min(p0 + a.R, (long long)a.items * a.nmax);
-    s.i = s.i_first = (int)(p0 / a.nmax);
-    s.i_last = (int)((p1 - 1) / a.nmax);
+    const int p0 = r * a.R;
+    const int p1 = min(p0 + a.R, a.vrec);
+    s.i = s.i_first = (int)fast_div((uint32_t)p0, a.div_nmax);
+    s.i_last = (int)fast_div((uint32_t)(p1 - 1), a.div_nmax);
     seg_item<D>(s, a, warp, report);
 }
 
@@ -675,11 +675,11 @@ __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
     const int b = bh / a.Hq, hh = bh % a.Hq;
     const int kv = hh / G, quad = (hh % G) / kHeads, h = (hh % G) % kHeads;
     const int item = (b * a.Hkv + kv) * a.quads + quad;
-    const long long base = (long long)item * a.nmax;
-    const int rA = (int)(base / a.R), rB = (int)((base + a.nmax - 1) / a.R);
+    const int base = item * a.nmax;
+    const int rA = base / a.R, rB = (base + a.nmax - 1) / a.R;
     if (rA == rB) return;  // whole inside one range: already written
     auto part = [&](int r) {
-        const int slot = (long long)r * a.R / a.nmax == item ? 0 : 1;
+        const int slot = r * a.R / a.nmax == item ? 0 : 1;
         return ((size_t)r * 2 + slot) * kHeads + h;
     };
     float M = -INFINITY;
@@ -734,16 +734,22 @@ bool decode_plan(DecodeArgs& a, int num_sms) {
     a.items = a.B * a.Hkv * a.quads;
     a.nmax = a.max_seq_len > 0 ? (a.max_seq_len + kBlock - 1) / kBlock : 1;
     const long long V = (long long)a.items * a.nmax;
+    if (V >= (1LL << 30)) return false;
+    long long R;
     if (a.num_splits > 0) {
-        a.R = (a.nmax + a.num_splits - 1) / a.num_splits;
+        R = (a.nmax + a.num_splits - 1) / a.num_splits;
     } else {
         const long long H = (long long)kHalves * num_sms;
-        a.R = (V + H - 1) / H;
+        R = (V + H - 1) / H;
     }
-    if (a.R < 1) a.R = 1;
-    const long long nr = (V + a.R - 1) / a.R;
-    a.nranges = nr > 0x7fffffffLL ? 0 : (int)nr;
-    return a.nranges > 0;
+    if (R < 1) R = 1;
+    a.vrec = (int)V;
+    a.R = (int)R;
+    a.nranges = (int)((V + R - 1) / R);
+    a.div_nmax = div_magic((uint32_t)a.nmax);
+    a.div_hkv = div_magic((uint32_t)a.Hkv);
+    a.div_quads = div_magic((uint32_t)a.quads);
+    return true;
 }
 
 bool decode_needs_combine(const DecodeArgs& a) { return a.nranges > 1 && a.R % a.nmax != 0; }

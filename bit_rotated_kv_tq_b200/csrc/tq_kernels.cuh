@@ -41,8 +41,10 @@ struct DecodeArgs {
     int quads;            // groups of four query heads per kv head
     int items;            // B * Hkv * quads
     int nmax;             // blocks of the longest sequence (>= 1)
-    long long R;          // records per range of the virtual space items x nmax
+    int vrec;             // virtual records items x nmax (< 2^30)
+    int R;                // records per range
     int nranges;
+    uint64_t div_nmax, div_hkv, div_quads;  // fast_div multipliers
     uint32_t smem_bytes;  // dynamic shared memory of the split kernel
 };
 
