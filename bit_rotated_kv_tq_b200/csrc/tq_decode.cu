@@ -18,11 +18,11 @@
 //
 // Per record every product runs on the tensor cores (mma.sync m16n8k16, fp32
 // accumulate), with exact fp16 operands only:
-//   q.K  A = q~ (rows: head r/2 mod 4, high fp16 part in rows 0-7, low part in
-//        rows 8-15), B = centroids of 8 tokens from a byte -> (C[lo], C[hi])
-//        table with one copy per lane; one prmt forms each table address.
-//        Lane (g, c) ends with the full scores of head g/2 at tokens 2c, 2c+1,
-//        2c+8, 2c+9: exactly the operand it feeds to p.V, so no transpose.
+//   q.K  A = centroids of the 16 tokens from a byte -> (C[lo], C[hi]) table
+//        with one copy per lane (one prmt forms each table address), B = q~
+//        with head h's high fp16 part in column 2h and its low part in 2h+1,
+//        so the scores carry q~ to ~22 bits.  Four shuffles move each head's
+//        weights into the layout p.V takes them in.
 //   p.V  A = value codes as fp16 subnormals (the nibble masked in place is
 //        n 2^-24, or n 2^-20 for a high nibble: exact, no bias to remove);
 //        B = p_t s_t,g as an exact two-part fp16 product, the high part in
@@ -391,8 +391,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     const uint32_t lanebase = P.lut | ((uint32_t)half << 7) | ((uint32_t)lane << 2);
     const float lo_sel = (float)(g & 1);  // this lane feeds the low part of its head
     const uint32_t lo_mask = (g & 1) ? 0xffffffffu : 0u;
-    const uint32_t qsrc_h = P.qh + (uint32_t)((half * kHeads + (g >> 1)) * D * 2);
-    const uint32_t qsrc_l = P.ql + (uint32_t)((half * kHeads + (g >> 1)) * D * 2);
+    const uint32_t qsrc = ((g & 1) ? P.ql : P.qh) + (uint32_t)((half * kHeads + (g >> 1)) * D * 2);
     const uint32_t mb = P.merge + half * Plan<D>::kMergeHalf;  // [warp][head][D] o, then m, l
     const uint32_t mb_m = mb + kNW * kHeads * D * 4, mb_l = mb_m + kNW * kHeads * 4;
     int stage = 0;
@@ -465,18 +464,15 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
         }
         half_sync(half);
 
-        // ---- q.K A fragments: rows g (high part) and g + 8 (low part) of head
-        // g/2; k = 2c, 2c+1 | 2c+8, 2c+9 of step ks are the dims of key bytes
-        // j = c*KB + 2ks and j + 1 (a fixed permutation of the dims)
-        uint32_t qa[KS][4];
+        // ---- q.K B fragments: column g is head g/2, its high fp16 part for even
+        // g and its low part for odd g; k = 2c, 2c+1 | 2c+8, 2c+9 of step ks are
+        // the dims of key bytes j = c*KB + 2ks and j + 1 (a fixed permutation)
+        uint32_t qb[KS][2];
 #pragma unroll
         for (int ks = 0; ks < KS; ks++) {
-            const uint32_t j = c * KB + 2 * ks;
-            const uint2 hv = lds64(qsrc_h + 4 * j), lv = lds64(qsrc_l + 4 * j);
-            qa[ks][0] = hv.x;
-            qa[ks][1] = lv.x;
-            qa[ks][2] = hv.y;
-            qa[ks][3] = lv.y;
+            const uint2 v2 = lds64(qsrc + 4 * (c * KB + 2 * ks));
+            qb[ks][0] = v2.x;
+            qb[ks][1] = v2.y;
         }
 
         // ---- this warp's records of the unit
@@ -488,7 +484,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
 #pragma unroll
             for (int m = 0; m < KS; m++) O[m][i] = 0.f;
         }
-        float mrun = -INFINITY;  // running maximum of head g/2
+        float mrun = -INFINITY;  // running maximum of head c
         const int nk = aborted ? 0 : cu.nk;
         // tokens in this warp's last record of the unit (< 16 only at the end of the sequence)
         const int last_valid = cu.L - (cu.jb + warp + kNW * (nk - 1)) * kBlock;
@@ -505,52 +501,50 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             if (id >= 0 && id < a.num_blocks) {
                 const bool partial = k == nk - 1 && last_valid < kBlock;
 
-                // -------- q.K: B = centroids of tokens g (tile 0) and g + 8 (tile 1)
+                // -------- q.K: A = centroids of tokens g (rows 0-7) and g + 8 (rows 8-15)
                 uint32_t kw0[KW], kw1[KW];
                 ldw<KW>(rec + g * (D / 2) + c * KB, kw0);
                 ldw<KW>(rec + (g + 8) * (D / 2) + c * KB, kw1);
-                float s0[4], s1[4];
+                float sc[4];
 #pragma unroll
                 for (int ks = 0; ks < KS; ks++) {
                     // table address: the code byte spliced into byte 1 of lanebase
                     const uint32_t sa = (ks & 1) ? 0x7624u : 0x7604u;
                     const uint32_t sb = (ks & 1) ? 0x7634u : 0x7614u;
                     const uint32_t w0 = kw0[ks >> 1], w1 = kw1[ks >> 1];
-                    const uint32_t b00 = lds32(__byte_perm(w0, lanebase, sa));
-                    const uint32_t b01 = lds32(__byte_perm(w0, lanebase, sb));
-                    const uint32_t b10 = lds32(__byte_perm(w1, lanebase, sa));
-                    const uint32_t b11 = lds32(__byte_perm(w1, lanebase, sb));
-                    if (ks == 0) {
-                        mma16816_z(s0, qa[0][0], qa[0][1], qa[0][2], qa[0][3], b00, b01);
-                        mma16816_z(s1, qa[0][0], qa[0][1], qa[0][2], qa[0][3], b10, b11);
-                    } else {
-                        mma16816(s0, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b00, b01);
-                        mma16816(s1, qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b10, b11);
-                    }
+                    const uint32_t a0 = lds32(__byte_perm(w0, lanebase, sa));
+                    const uint32_t a2 = lds32(__byte_perm(w0, lanebase, sb));
+                    const uint32_t a1 = lds32(__byte_perm(w1, lanebase, sa));
+                    const uint32_t a3 = lds32(__byte_perm(w1, lanebase, sb));
+                    if (ks == 0)
+                        mma16816_z(sc, a0, a1, a2, a3, qb[0][0], qb[0][1]);
+                    else
+                        mma16816(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
                 }
-                // scores of head g/2 at tokens 2c, 2c+1, 2c+8, 2c+9 (base 2)
-                const float2 na = __half22float2(u2h(lds32(rec + R::kKNorm + 4 * c)));
-                const float2 nb = __half22float2(u2h(lds32(rec + R::kKNorm + 16 + 4 * c)));
-                float x0 = (s0[0] + s0[2]) * na.x, x1 = (s0[1] + s0[3]) * na.y;
-                float x2 = (s1[0] + s1[2]) * nb.x, x3 = (s1[1] + s1[3]) * nb.y;
+                // scores of head c at tokens g and g + 8 (base 2): columns 2c, 2c+1
+                // hold the high and low parts of the query
+                const uint32_t nw = lds32(rec + R::kKNorm + 4 * (g >> 1));
+                const uint32_t nw8 = lds32(rec + R::kKNorm + 16 + 4 * (g >> 1));
+                const float na = __half2float(__ushort_as_half((uint16_t)((g & 1) ? nw >> 16 : nw)));
+                const float nb = __half2float(__ushort_as_half((uint16_t)((g & 1) ? nw8 >> 16 : nw8)));
+                float xa = (sc[0] + sc[1]) * na, xb = (sc[2] + sc[3]) * nb;
                 uint32_t mA = 0xffffffffu, mB = 0xffffffffu;  // valid tokens (fp16 lanes)
                 if (partial) {  // the last block of the sequence
                     const int t = 2 * c, nvalid = last_valid;
-                    x0 = t < nvalid ? x0 : -INFINITY;
-                    x1 = t + 1 < nvalid ? x1 : -INFINITY;
-                    x2 = t + 8 < nvalid ? x2 : -INFINITY;
-                    x3 = t + 9 < nvalid ? x3 : -INFINITY;
+                    xa = g < nvalid ? xa : -INFINITY;
+                    xb = g + 8 < nvalid ? xb : -INFINITY;
                     mA = (t < nvalid ? 0xffffu : 0u) | (t + 1 < nvalid ? 0xffff0000u : 0u);
                     mB = (t + 8 < nvalid ? 0xffffu : 0u) | (t + 9 < nvalid ? 0xffff0000u : 0u);
                 }
 
-                // -------- online softmax
-                float mx = fmaxf(fmaxf(x0, x1), fmaxf(x2, x3));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+                // -------- online softmax (head c: lanes with the same c)
+                float mx = fmaxf(xa, xb);
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
                 const float mn = fmaxf(mrun, mx);
                 if (__any_sync(kFull, mn > mrun)) {
-                    const float corr = __shfl_sync(kFull, ex2(mrun - mn), 8 * c);  // head c
+                    const float corr = ex2(mrun - mn);
 #pragma unroll
                     for (int i = 0; i < 4; i++) {
                         Z[i] *= corr;
@@ -559,9 +553,15 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                     }
                 }
                 mrun = mn;
+                const float pa = ex2(xa - mn), pb = ex2(xb - mn);
+                // to the p.V operand: head g/2 at tokens 2c, 2c+1, 2c+8, 2c+9 lives in
+                // lanes (2c, g/2) and (2c+1, g/2), as their tokens g and g + 8
+                const int s_even = 8 * c + (g >> 1), s_odd = s_even + 4;
+                const float p0 = __shfl_sync(kFull, pa, s_even), p1 = __shfl_sync(kFull, pa, s_odd);
+                const float p2 = __shfl_sync(kFull, pb, s_even), p3 = __shfl_sync(kFull, pb, s_odd);
                 uint32_t u01, w01, u89, w89;
-                split_uw(ex2(x0 - mn), ex2(x1 - mn), lo_sel, lo_mask, u01, w01);
-                split_uw(ex2(x2 - mn), ex2(x3 - mn), lo_sel, lo_mask, u89, w89);
+                split_uw(p0, p1, lo_sel, lo_mask, u01, w01);
+                split_uw(p2, p3, lo_sel, lo_mask, u89, w89);
 
                 // -------- p.z and sum p
                 uint2 zz = lds64(rec + R::kVZero + (c * NG + (g & (NG - 1))) * 8);
@@ -621,7 +621,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 stsf(ro + (16 * m + 2 * g) * 4, fmaf(O[m][0] + O[m][1], 0x1p24f, zs[m >> 1]));
                 stsf(ro + (16 * m + 2 * g + 1) * 4, fmaf(O[m][2] + O[m][3], 0x1p20f, zs[m >> 1]));
             }
-            const float mh = __shfl_sync(kFull, mrun, 8 * c);
+            const float mh = mrun;  // head c
             if (g == 0) {
                 stsf(mb_m + (warp * kHeads + c) * 4, mh);
                 stsf(mb_l + (warp * kHeads + c) * 4, Z[2] + Z[3]);
