@@ -114,6 +114,21 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase) {
         if (clock64() - t0 > (1LL << 31)) return false;
     return true;
 }
+// The same for a whole warp, kept out of line: the common case (the phase has
+// completed) is one try_wait and one vote at the call site.
+__device__ __noinline__ bool mbar_wait_warp_slow(uint32_t bar, uint32_t phase) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, phase));
+}
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t phase) {
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, phase))) return true;
+    return mbar_wait_warp_slow(bar, phase);
+}
+// OR bits into the status word from lane 0 only, without a branch
+__device__ __forceinline__ void flag_lane0(int32_t* status, int bits, int lane) {
+    const uint32_t p = (uint32_t)(lane == 0 && status != nullptr);
+    asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %0, 0;\n @p red.global.or.b32 [%1], %2;\n}\n"
+                 ::"r"(p), "l"(status), "r"(bits) : "memory");
+}
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
                                          uint32_t bar) {
     asm volatile(
@@ -344,6 +359,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     }
     __syncwarp();
 
+    const long long rec_stride = (long long)a.Hkv * REC;  // bytes between blocks of one kv head
     // ---- issue cursor: the next record of this warp's stream (all its segments, in order)
     Seg is;
     seg_range<D>(is, v, a, warp, false);
@@ -356,9 +372,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     auto issue = [&]() {
         if (is.r >= a.nranges) return;
         const uint32_t bar = bar0 + 8 * istage;
-        const uint32_t valid = (uint32_t)(nid >= 0 && nid < a.num_blocks);
+        const uint32_t valid = (uint32_t)((uint32_t)nid < (uint32_t)a.num_blocks);
         const uint32_t me = (uint32_t)(lane == 0);
-        const unsigned char* src = is.src + (size_t)(valid ? nid : 0) * a.Hkv * REC;
+        const unsigned char* src = is.src + (long long)nid * rec_stride;  // used only if valid
         asm volatile(
             "{\n .reg .pred pc, pa, pm;\n"
             " setp.ne.u32 pm, %0, 0;\n"
@@ -491,14 +507,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
 #pragma unroll 1
         for (int k = 0; k < nk; k++) {
             const uint32_t rec = ringw + stage * REC;
-            const bool ok = mbar_wait(bar0 + 8 * stage, phase);
-            if (!__all_sync(kFull, ok)) {
-                if (lane == 0) flag_status(a.status, TQ_STATUS_TIMEOUT);
+            if (!mbar_wait_warp(bar0 + 8 * stage, phase)) {
+                flag_lane0(a.status, TQ_STATUS_TIMEOUT, lane);
                 aborted = true;
                 break;
             }
             const int id = (int)lds32(idw + 4 * stage);
-            if (id >= 0 && id < a.num_blocks) {
+            if (__all_sync(kFull, (uint32_t)id < (uint32_t)a.num_blocks)) {
                 const bool partial = k == nk - 1 && last_valid < kBlock;
 
                 // -------- q.K: A = centroids of tokens g (rows 0-7) and g + 8 (rows 8-15)
@@ -599,8 +614,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                     mma16816(O[2 * G_ + 1], A1 & 0x000F000Fu, A1 & 0x00F000F0u, B1 & 0x000F000Fu,
                              B1 & 0x00F000F0u, b0, b1);
                 }
-            } else if (lane == 0) {
-                flag_status(a.status, TQ_STATUS_BAD_BLOCK);
+            } else {
+                flag_lane0(a.status, TQ_STATUS_BAD_BLOCK, lane);
             }
             __syncwarp();
             issue();  // the record after the ring's last: into the slot just read
