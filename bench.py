@@ -281,6 +281,20 @@ def profiled_traffic(w):
     return int(fields[key])
 
 
+def combine_runs(w, S, dev) -> bool:
+    """Whether tq_decode_attention launches its combine kernel: some sequence is cut
+    between two ranges of the split kernel's plan (the library's rule, restated)."""
+    nmax = max(1, (int(w.seq_lens.max()) + 15) // 16)
+    items = w.B * w.Hkv * ((w.Hq // w.Hkv + 3) // 4)
+    V = items * nmax
+    if S == 0:
+        halves = 2 * torch.cuda.get_device_properties(dev).multi_processor_count
+        R = max(1, -(-V // halves))
+    else:
+        R = max(1, -(-nmax // S))
+    return -(-V // R) > 1 and R % nmax != 0
+
+
 def cfg(w, l2):
     return {"workload": f"{w.name}: {w.B} seqs x {int(w.seq_lens[0])} tokens, {w.Hq} q / {w.Hkv} kv heads, "
                         f"d {w.d}, block 16, shuffled block tables, {w.append_tokens}-token append per seq",
@@ -418,7 +432,7 @@ def run_tq(args, rank, world, local):
                          "peak_source": f"{peak_kind} hbm_gbs"},
             "e2e": {"value": weak_scaling_value(kv, args.steps, world, e2e_s) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * (2 + (1 if S > 1 else 0)),
+            "gpu_launches": args.steps * (2 + (1 if combine_runs(w, S, dev) else 0)),
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
