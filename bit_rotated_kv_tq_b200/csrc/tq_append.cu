@@ -58,9 +58,14 @@ struct __align__(8) BinEntry {
 };
 
 // Build the per-head bin tables in shared memory (called by the whole CTA).
+// Without per-head tables every head uses the default table: one set of bins,
+// which every head then indexes as head 0.  Per bin, the midpoints below the
+// bin's extended range are counted by a binary search (the midpoints of a
+// strictly ascending table ascend too), and the one or more inside it follow.
 __device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t* k_tables,
                            const uint16_t* default_table) {
-    for (int h = threadIdx.x; h < Hkv; h += blockDim.x) {
+    const int nh = k_tables ? Hkv : 1;
+    for (int h = threadIdx.x; h < nh; h += blockDim.x) {
         const uint16_t* src = k_tables ? k_tables + 16 * h : default_table;
         for (int k = 0; k < 16; k++) hb[h].c[k] = half_bits_to_float(src[k]);
         hb[h].dense = 0;
@@ -68,17 +73,25 @@ __device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t
     __syncthreads();
     const float delta = 2.0f * kKeyMargin;
     const float w = 1.0f / kBinScale;
-    for (int e = threadIdx.x; e < Hkv * kBins; e += blockDim.x) {
+    for (int e = threadIdx.x; e < nh * kBins; e += blockDim.x) {
         const int h = e / kBins, bin = e % kBins;
         const float* c = hb[h].c;
         const float ext_lo = -1.0f + bin * w - delta;
         const float ext_hi = -1.0f + (bin + 1) * w + delta;
-        int below = 0, inside = 0;
+        // below = #{k < 15 : m_k < ext_lo}, m_k = (c_k + c_k+1) / 2 (exact: fp16 values)
+        int below = 0;
+#pragma unroll
+        for (int step = 8; step >= 1; step >>= 1) {
+            const int k = below + step - 1;
+            if (k < 15 && 0.5f * (c[k] + c[k + 1]) < ext_lo) below += step;
+        }
+        int inside = 0;
         float m_in = __int_as_float(0x7f800000);
-        for (int k = 0; k < 15; k++) {
-            const float m = 0.5f * (c[k] + c[k + 1]);  // exact: fp16 values
-            if (m < ext_lo) below++;
-            else if (m <= ext_hi) { inside++; m_in = m; }
+        for (int k = below; k < 15; k++) {
+            const float m = 0.5f * (c[k] + c[k + 1]);
+            if (m > ext_hi) break;
+            inside++;
+            m_in = m;
         }
         bins[e].mid = m_in;
         bins[e].k_lo = below;
@@ -86,7 +99,6 @@ __device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t
     }
     __syncthreads();
 }
-
 
 // fp32 neighbours of 1/15: the value rounded up and rounded down.
 __device__ __forceinline__ float inv15_up() { return __uint_as_float(0x3d888889u); }
@@ -145,11 +157,10 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a
 constexpr float kRound = 12582912.0f;
 
 template <int D>
-__global__ void __launch_bounds__(256, 2) append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
     HeadBins* hb = reinterpret_cast<HeadBins*>(smem);
     BinEntry* bins = reinterpret_cast<BinEntry*>(hb + a.Hkv);
-    build_bins(hb, bins, a.Hkv, a.k_tables, a.default_table);
 
     constexpr int LPV = D / 8;     // lanes per vector
     constexpr int VPW = 32 / LPV;  // vectors per warp pass
@@ -162,9 +173,11 @@ __global__ void __launch_bounds__(256, 2) append_kernel(AppendArgs a) {
     const uint32_t nwarps = gridDim.x * (blockDim.x / 32);
     const uint32_t cap = (uint32_t)(a.max_blocks * kBlock);
 
+    // the first pass's loads go out before the bins are built, so the two overlap
     Pass cur, nxt;
     uint32_t pass = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     load_pass<D>(a, pass, npass, total, grp, sub, cur);
+    build_bins(hb, bins, a.Hkv, a.k_tables, a.default_table);
     fetch_block(a, cur);
 
     for (; pass < npass; pass += nwarps) {
@@ -218,8 +231,9 @@ __global__ void __launch_bounds__(256, 2) append_kernel(AppendArgs a) {
         const float inv = ss > 0.f ? rsqrtf(ss * (float)D) : 0.f;
 
         // ---- key: nearest centroid through the per-head bins
-        const HeadBins& B = hb[h];
-        const BinEntry* hbins = bins + h * kBins;
+        const int hs = a.k_tables ? h : 0;  // whose bins (one shared set without per-head tables)
+        const HeadBins& B = hb[hs];
+        const BinEntry* hbins = bins + hs * kBins;
         uint32_t kw = 0;
         float y[8];
         {
@@ -311,6 +325,10 @@ __global__ void __launch_bounds__(256, 2) append_kernel(AppendArgs a) {
                 }
             }
         }
+
+        // the next pass's block-table entry: its slot has arrived by now, and the
+        // lookup overlaps this pass's value work and stores
+        fetch_block(a, nxt);
 
         // ---- values: group of 32 = 4 lanes
         float2 V2[4];
@@ -408,7 +426,6 @@ __global__ void __launch_bounds__(256, 2) append_kernel(AppendArgs a) {
             }
         }
 
-        fetch_block(a, nxt);  // its slot has arrived by now
         cur = nxt;
     }
 }
