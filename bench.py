@@ -342,52 +342,124 @@ def run_tq(args, rank, world, local):
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
 
+    # per call: CUDA events around each library call, launched one by one from Python
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
-    with ClockSampler(smi_id(local)) as clk:
-        clk.mark_start()
-        start.record(stream)
-        for i in range(args.steps):
-            step(evs[i])
-        end.record(stream)
-        torch.cuda.synchronize(dev)
-        clk.mark_end()
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize(dev)
     barrier(world)
-    total_ms = start.elapsed_time(end)
     app_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    total_ms = max_over_ranks(total_ms, world)
     dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
     app_avg = max_over_ranks(sum(app_ms) / len(app_ms), world)
 
-    # end to end through the same public calls with host buffers
+    # whole steps: the step (append, then decode) captured once as a CUDA graph, the way
+    # a serving engine launches a decode step, and replayed; CUDA events around K replays
+    gs = torch.cuda.Stream(dev)
+    gs.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(gs):
+        tq.quantize_append(aK, aV, aS, cache, block_table=bt, status=status, stream=gs)
+        tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws, num_splits=S,
+                            status=status, stream=gs)
+        gs.synchronize()
+        step_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(step_graph, stream=gs):
+            tq.quantize_append(aK, aV, aS, cache, block_table=bt, status=status, stream=gs)
+            tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws,
+                                num_splits=S, status=status, stream=gs)
+        for _ in range(max(args.warmup, 3)):
+            step_graph.replay()
+        gs.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        with ClockSampler(smi_id(local)) as clk:
+            clk.mark_start()
+            start.record(gs)
+            for _ in range(args.steps):
+                step_graph.replay()
+            end.record(gs)
+            gs.synchronize()
+            clk.mark_end()
+    barrier(world)
+    total_ms = max_over_ranks(start.elapsed_time(end), world)
+
+    # end to end through the same public calls with host buffers, driven the way a
+    # serving engine drives them: one CUDA graph per step.  Every step copies one set
+    # of inputs in from pinned host memory and reads one result back.  The graph of
+    # step k runs step k on the compute stream while it copies step k + 1's inputs
+    # into the other device buffer set on a copy stream, then reads step k's result
+    # back on a third stream; the timed region ends when the last read-back has landed.
+    nbuf = 2
     h_q = w.q().pin_memory()
     h_K, h_V, h_S = aK.cpu().pin_memory(), aV.cpu().pin_memory(), aS.cpu().pin_memory()
-    h_out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32).pin_memory()
-    d_q, d_K, d_V, d_S = torch.empty_like(q), torch.empty_like(aK), torch.empty_like(aV), torch.empty_like(aS)
+    h_outs = [torch.empty((w.B, w.Hq, w.d), dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    d_in = [(torch.empty_like(q), torch.empty_like(aK), torch.empty_like(aV), torch.empty_like(aS))
+            for _ in range(nbuf)]
+    d_out = [torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev) for _ in range(nbuf)]
+    cs = torch.cuda.Stream(dev)  # the stream the graphs are captured and replayed on
+    copy_s, read_s = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
+    def copy_in(i):
+        d_q, d_K, d_V, d_S = d_in[i]
         d_q.copy_(h_q, non_blocking=True)
         d_K.copy_(h_K, non_blocking=True)
         d_V.copy_(h_V, non_blocking=True)
         d_S.copy_(h_S, non_blocking=True)
-        tq.quantize_append(d_K, d_V, d_S, cache, block_table=bt, status=status, stream=stream)
-        tq.decode_attention(d_q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws, num_splits=S,
-                            status=status, stream=stream)
-        h_out.copy_(out, non_blocking=True)
-        stream.synchronize()
 
-    for _ in range(3):
-        e2e_step()
-    barrier(world)
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        e2e_step()
-    e2e_s = max_over_ranks(time.perf_counter() - t0, world)
+    def read_out(i):
+        with torch.cuda.stream(read_s):
+            h_outs[i].copy_(d_out[i], non_blocking=True)
+
+    def step_body(i):  # captured: step on set i, next step's inputs into set 1 - i,
+        # and the previous step's result (set 1 - i) read back, both beside the step
+        copy_s.wait_stream(cs)
+        with torch.cuda.stream(copy_s):
+            copy_in(1 - i)
+        read_s.wait_stream(cs)
+        read_out(1 - i)
+        d_q, d_K, d_V, d_S = d_in[i]
+        tq.quantize_append(d_K, d_V, d_S, cache, block_table=bt, status=status, stream=cs)
+        tq.decode_attention(d_q, cache, bt, lens, max_len, w.scale, out=d_out[i], workspace=ws,
+                            num_splits=S, status=status, stream=cs)
+        cs.wait_stream(copy_s)  # the graph ends when both side branches are done, so the
+        cs.wait_stream(read_s)  # next step may reuse what they read and write
+
+    cs.wait_stream(torch.cuda.current_stream(dev))
+    graphs = []
+    with torch.cuda.stream(cs):
+        for i in range(nbuf):
+            copy_in(i)  # every buffer set holds real inputs before any step reads one
+        for i in range(nbuf):
+            step_body(i)  # once outside capture (first-use setup of the library)
+        cs.synchronize()
+        for i in range(nbuf):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cs):
+                step_body(i)
+            graphs.append(g)
+        copy_in(0)
+        for k in range(4):
+            graphs[k % nbuf].replay()
+        cs.synchronize()
+        barrier(world)
+        t0 = time.perf_counter()
+        # steps 0 .. K-1; graph k reads back step k - 1's result, and the last result
+        # is read back after the loop, inside the timed region
+        for k in range(args.steps):
+            graphs[k % nbuf].replay()
+        read_s.wait_stream(cs)
+        read_out((args.steps - 1) % nbuf)
+        read_s.synchronize()
+        cs.synchronize()
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world)
+    torch.cuda.synchronize(dev)
+    # the read-back results are the device-timed path's (same inputs, same cache state)
+    assert torch.equal(h_outs[(args.steps - 1) % nbuf], out.cpu()), "end-to-end result differs"
+    assert torch.equal(h_outs[(args.steps - 2) % nbuf], out.cpu()), "end-to-end result differs"
     h2d = h_q.numel() * 2 + h_K.numel() * 2 + h_V.numel() * 2 + h_S.numel() * 4
-    d2h = h_out.numel() * 4
+    d2h = h_outs[0].numel() * 4
 
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
