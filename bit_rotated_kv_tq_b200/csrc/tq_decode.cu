@@ -82,9 +82,9 @@ __device__ __forceinline__ float ldsf(uint32_t a) {
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
     return v;
 }
-// barrier among the 256 threads of one half (ids 1, 2; 0 is __syncthreads)
+// barrier among the threads of one half (ids 1, 2; 0 is __syncthreads)
 __device__ __forceinline__ void half_sync(int half) {
-    asm volatile("bar.sync %0, 256;" ::"r"(1 + half) : "memory");
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + half), "n"(kNW * 32) : "memory");
 }
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
@@ -430,8 +430,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             first_seg = false;
             lut_tab = tab;
 #pragma unroll 1
-            for (int it = 0; it < 8; it++) {
-                const int row = 32 * warp + 4 * it + (lane >> 3);
+            for (int r4 = warp; r4 < 64; r4 += kNW) {  // 4 rows per warp and step
+                const int row = 4 * r4 + (lane >> 3);
                 const uint32_t lo = tab ? tab[row & 15] : a.default_table[row & 15];
                 const uint32_t hi = tab ? tab[row >> 4] : a.default_table[row >> 4];
                 sts128(P.lut + row * 256 + half * 128 + (lane & 7) * 16, lo | (hi << 16));
@@ -531,10 +531,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                     const uint32_t a2 = lds32(__byte_perm(w0, lanebase, sb));
                     const uint32_t a1 = lds32(__byte_perm(w1, lanebase, sa));
                     const uint32_t a3 = lds32(__byte_perm(w1, lanebase, sb));
+                    const uint32_t qb0 = qb[ks][0], qb1 = qb[ks][1];
                     if (ks == 0)
-                        mma16816_z(sc, a0, a1, a2, a3, qb[0][0], qb[0][1]);
+                        mma16816_z(sc, a0, a1, a2, a3, qb0, qb1);
                     else
-                        mma16816(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                        mma16816(sc, a0, a1, a2, a3, qb0, qb1);
                 }
                 // scores of head c at tokens g and g + 8 (base 2): columns 2c, 2c+1
                 // hold the high and low parts of the query
