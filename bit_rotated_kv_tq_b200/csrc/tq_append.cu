@@ -30,11 +30,6 @@
 
 namespace tq {
 
-// Absolute margin, in rotated unit-vector units, inside which an fp32
-// centroid decision is re-taken in fp64.  The fp32 butterfly of a bf16 key
-// followed by one scaling is accurate to ~1.3e-6 in the worst case
-// (7 stages, rsqrt within 2 ulp); typical errors are ~1e-7.
-constexpr float kKeyMargin = 3.0e-6f;
 // Relative margin on the norm before its fp16 rounding (fp32 sum of squares
 // of at most 128 exact products: error <= 11 ulp relative, 6.6e-7).
 constexpr float kNormMargin = 1.5e-6f;
@@ -42,62 +37,35 @@ constexpr float kNormMargin = 1.5e-6f;
 // (fp32 error <= 3 ulp of 15, i.e. 2.7e-6).
 constexpr float kValueMargin = 1.0f / 4096.0f;
 
-// Uniform bins over y in [-1, 1] (a unit vector's coordinates), width 1/64:
-// bin = (int)(64 y + 64) in [0, 128].
-constexpr int kBins = 129;
-constexpr float kBinScale = 64.0f;
-
-struct HeadBins {
-    float c[16];  // the head's table
-    int dense;    // 1: some bin holds more than one midpoint -> exact count path
-    int pad;      // keeps the BinEntry array that follows 8-byte aligned
-};
-struct __align__(8) BinEntry {
-    float mid;  // the one midpoint inside the bin (with margins), or +inf
-    int k_lo;   // number of midpoints strictly below the bin
-};
-
-// Build the per-head bin tables in shared memory (called by the whole CTA).
-// Without per-head tables every head uses the default table: one set of bins,
-// which every head then indexes as head 0.  Per bin, the midpoints below the
-// bin's extended range are counted by a binary search (the midpoints of a
-// strictly ascending table ascend too), and the one or more inside it follow.
-__device__ void build_bins(HeadBins* hb, BinEntry* bins, int Hkv, const uint16_t* k_tables,
-                           const uint16_t* default_table) {
-    const int nh = k_tables ? Hkv : 1;
-    for (int h = threadIdx.x; h < nh; h += blockDim.x) {
-        const uint16_t* src = k_tables ? k_tables + 16 * h : default_table;
-        for (int k = 0; k < 16; k++) hb[h].c[k] = half_bits_to_float(src[k]);
+// Bin tables in shared memory (called by the whole CTA).  Without per-head
+// tables every head uses the default table, whose bins the launcher computed
+// once on the host: they are copied, and every head indexes them as head 0.
+// Per-head tables are binned here, one thread per (head, bin).
+__device__ void build_bins(HeadBins* hb, BinEntry* bins, const AppendArgs& a) {
+    if (!a.k_tables) {
+        for (int e = threadIdx.x; e < kBins; e += blockDim.x) bins[e] = a.default_bins[e];
+        if (threadIdx.x == 0) hb[0] = a.default_hb;
+        __syncthreads();
+        return;
+    }
+    for (int h = threadIdx.x; h < a.Hkv; h += blockDim.x) {
+        for (int k = 0; k < 16; k++) hb[h].c[k] = half_bits_to_float(a.k_tables[16 * h + k]);
         hb[h].dense = 0;
     }
     __syncthreads();
-    const float delta = 2.0f * kKeyMargin;
-    const float w = 1.0f / kBinScale;
-    for (int e = threadIdx.x; e < nh * kBins; e += blockDim.x) {
+    for (int e = threadIdx.x; e < a.Hkv * kBins; e += blockDim.x) {
         const int h = e / kBins, bin = e % kBins;
-        const float* c = hb[h].c;
-        const float ext_lo = -1.0f + bin * w - delta;
-        const float ext_hi = -1.0f + (bin + 1) * w + delta;
-        // below = #{k < 15 : m_k < ext_lo}, m_k = (c_k + c_k+1) / 2 (exact: fp16 values)
-        int below = 0;
-#pragma unroll
-        for (int step = 8; step >= 1; step >>= 1) {
-            const int k = below + step - 1;
-            if (k < 15 && 0.5f * (c[k] + c[k + 1]) < ext_lo) below += step;
-        }
-        int inside = 0;
-        float m_in = __int_as_float(0x7f800000);
-        for (int k = below; k < 15; k++) {
-            const float m = 0.5f * (c[k] + c[k + 1]);
-            if (m > ext_hi) break;
-            inside++;
-            m_in = m;
-        }
-        bins[e].mid = m_in;
-        bins[e].k_lo = below;
-        if (inside > 1) hb[h].dense = 1;  // benign race: every writer stores 1
+        if (bin_entry(hb[h].c, bin, bins[e])) hb[h].dense = 1;  // benign race: all store 1
     }
     __syncthreads();
+}
+
+// 1/x by the hardware approximation (relative error ~2^-22): (v - z) * (1/s)
+// then errs by < 15 * 2^-21 code units, far inside kValueMargin
+__device__ __forceinline__ float fast_rcp(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // fp32 neighbours of 1/15: the value rounded up and rounded down.
@@ -177,7 +145,7 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
     Pass cur, nxt;
     uint32_t pass = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
     load_pass<D>(a, pass, npass, total, grp, sub, cur);
-    build_bins(hb, bins, a.Hkv, a.k_tables, a.default_table);
+    build_bins(hb, bins, a);
     fetch_block(a, cur);
 
     for (; pass < npass; pass += nwarps) {
@@ -362,7 +330,7 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         const float sf = half_bits_to_float(s16);
         uint32_t vw = 0;
         if (sf > 0.f) {
-            const float inv_s = __frcp_rn(sf);
+            const float inv_s = fast_rcp(sf);  // its error is far inside kValueMargin
             const float2 z2 = make_float2(zf, zf), is2 = make_float2(inv_s, inv_s);
             const float2 rnd = make_float2(kRound, kRound);
             uint32_t qb[8];
@@ -449,8 +417,28 @@ static int resident_ctas(int num_sms, size_t smem) {
     return per_sm[key] * num_sms;
 }
 
+// The bins of the default table of head_dim d, computed once per process.
+static void default_bins(int d, const uint16_t* table16, HeadBins& hb, BinEntry* bins) {
+    static HeadBins cached_hb[2];
+    static BinEntry cached[2][kBins];
+    static bool ready[2] = {false, false};
+    const int key = d == 128 ? 1 : 0;
+    if (!ready[key]) {
+        HeadBins& h = cached_hb[key];
+        for (int k = 0; k < 16; k++) h.c[k] = __half2float(__ushort_as_half(table16[k]));
+        h.dense = 0;
+        h.pad = 0;
+        for (int b = 0; b < kBins; b++)
+            if (bin_entry(h.c, b, cached[key][b])) h.dense = 1;
+        ready[key] = true;
+    }
+    hb = cached_hb[key];
+    memcpy(bins, cached[key], sizeof cached[key]);
+}
+
 cudaError_t launch_append(const AppendArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
     AppendArgs a = args;
+    if (!a.k_tables) default_bins(head_dim, a.default_table, a.default_hb, a.default_bins);
     a.div_hkv = div_magic((uint32_t)a.Hkv);
     a.div_cap = div_magic((uint32_t)(a.max_blocks > 0 ? a.max_blocks * kBlock : 1));
     const int threads = 256;

@@ -2,9 +2,60 @@
 // (internal to the library; the public interface is include/tq.h).
 #pragma once
 
+#include <math.h>
+
 #include "tq_common.cuh"
 
 namespace tq {
+
+// ---- key binning of the append: uniform bins over y in [-1, 1] (a unit
+// vector's rotated coordinates), width 1/64, bin = (int)(64 y + 64) in [0, 128]
+constexpr int kBins = 129;
+constexpr float kBinScale = 64.0f;
+// Absolute margin, in rotated unit-vector units, inside which an fp32
+// centroid decision is re-taken in fp64.  The fp32 butterfly of a bf16 key
+// followed by one scaling is accurate to ~1.3e-6 in the worst case
+// (7 stages, rsqrt within 2 ulp); typical errors are ~1e-7.
+constexpr float kKeyMargin = 3.0e-6f;
+
+struct HeadBins {
+    float c[16];  // the head's table
+    int dense;    // 1: some bin holds more than one midpoint -> exact count path
+    int pad;      // keeps the BinEntry array that follows 8-byte aligned
+};
+struct __align__(8) BinEntry {
+    float mid;  // the one midpoint inside the bin (with margins), or +inf
+    int k_lo;   // number of midpoints strictly below the bin
+};
+
+// One bin of a strictly ascending 16-entry table c: the midpoints below the
+// bin's range widened by 2 kKeyMargin on each side are counted by a binary
+// search (the midpoints ascend too), and the one or more inside it follow.
+// Returns true when more than one midpoint falls inside (the exact count path).
+// The host (default table) and the device (per-head tables) both use it; the
+// margins make the result insensitive to their float contraction differing.
+__host__ __device__ inline bool bin_entry(const float* c, int bin, BinEntry& e) {
+    const float delta = 2.0f * kKeyMargin;
+    const float w = 1.0f / kBinScale;
+    const float ext_lo = -1.0f + bin * w - delta;
+    const float ext_hi = -1.0f + (bin + 1) * w + delta;
+    int below = 0;  // #{k < 15 : m_k < ext_lo}, m_k = (c_k + c_k+1) / 2 (exact: fp16 values)
+    for (int step = 8; step >= 1; step >>= 1) {
+        const int k = below + step - 1;
+        if (k < 15 && 0.5f * (c[k] + c[k + 1]) < ext_lo) below += step;
+    }
+    int inside = 0;
+    float m_in = INFINITY;
+    for (int k = below; k < 15; k++) {
+        const float m = 0.5f * (c[k] + c[k + 1]);
+        if (m > ext_hi) break;
+        inside++;
+        m_in = m;
+    }
+    e.mid = m_in;
+    e.k_lo = below;
+    return inside > 1;
+}
 
 struct AppendArgs {
     const uint16_t* K;          // bf16 [T][Hkv][D]
@@ -19,6 +70,8 @@ struct AppendArgs {
     uint16_t default_table[16]; // fp16
     int32_t* status;
     uint64_t div_hkv, div_cap;  // fast-division multipliers (set by the launcher)
+    HeadBins default_hb;        // bins of default_table (set by the launcher)
+    BinEntry default_bins[kBins];
 };
 
 struct DecodeArgs {
