@@ -355,21 +355,20 @@ def run_tq(args, rank, world, local):
     dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
     app_avg = max_over_ranks(sum(app_ms) / len(app_ms), world)
 
-    # whole steps: the step -- the append and the decode in one launch, tq_append_decode --
-    # captured once as a CUDA graph, the way a serving engine launches a decode step, and
-    # replayed; CUDA events around K replays
-    def fused_step(K_, V_, S_, q_, out_, st_):
-        tq.append_decode(K_, V_, S_, q_, cache, bt, lens, max_len, w.scale, out=out_, workspace=ws,
-                         num_splits=S, append_block_table=bt, status=status, stream=st_)
-
+    # whole steps: the step (append, then decode) captured once as a CUDA graph, the way
+    # a serving engine launches a decode step, and replayed; CUDA events around K replays
     gs = torch.cuda.Stream(dev)
     gs.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(gs):
-        fused_step(aK, aV, aS, q, out, gs)
+        tq.quantize_append(aK, aV, aS, cache, block_table=bt, status=status, stream=gs)
+        tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws, num_splits=S,
+                            status=status, stream=gs)
         gs.synchronize()
         step_graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(step_graph, stream=gs):
-            fused_step(aK, aV, aS, q, out, gs)
+            tq.quantize_append(aK, aV, aS, cache, block_table=bt, status=status, stream=gs)
+            tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws,
+                                num_splits=S, status=status, stream=gs)
         for _ in range(max(args.warmup, 3)):
             step_graph.replay()
         gs.synchronize()
@@ -421,7 +420,9 @@ def run_tq(args, rank, world, local):
         read_s.wait_stream(cs)
         read_out(1 - i)
         d_q, d_K, d_V, d_S = d_in[i]
-        fused_step(d_K, d_V, d_S, d_q, d_out[i], cs)
+        tq.quantize_append(d_K, d_V, d_S, cache, block_table=bt, status=status, stream=cs)
+        tq.decode_attention(d_q, cache, bt, lens, max_len, w.scale, out=d_out[i], workspace=ws,
+                            num_splits=S, status=status, stream=cs)
         cs.wait_stream(copy_s)  # the graph ends when both side branches are done, so the
         cs.wait_stream(read_s)  # next step may reuse what they read and write
 
@@ -503,7 +504,7 @@ def run_tq(args, rank, world, local):
                          "peak_source": f"{peak_kind} hbm_gbs"},
             "e2e": {"value": weak_scaling_value(kv, args.steps, world, e2e_s) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": args.steps * (1 + (1 if combine_runs(w, S, dev) else 0)),
+            "gpu_launches": args.steps * (2 + (1 if combine_runs(w, S, dev) else 0)),
             "clocks": clocks,
             "cpu_baseline": cpu,
         }

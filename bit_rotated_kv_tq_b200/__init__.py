@@ -70,8 +70,6 @@ def load(path: str | None = None):
                                              _P, _I, _P, _P]
     L.tq_decode_static_scratch_bytes.restype = _Z
     L.tq_decode_static_scratch_bytes.argtypes = []
-    L.tq_append_decode.argtypes = [_P, _P, _P, _I, _I, _P, _I, _P, ctypes.POINTER(_Cache), _P, _P, _I,
-                                   _P, _I, _I, _I, _F, _P, _P, _Z, _I, _P, _P]
     L.tq_last_error.restype = ctypes.c_char_p
     L.tq_last_error.argtypes = []
     _lib = L
@@ -206,38 +204,6 @@ def decode_attention(q, cache: Cache, block_tables, seq_lens, max_seq_len: int, 
                                       block_tables.shape[1], _ptr(seq_lens), B, Hq, int(max_seq_len),
                                       float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                       int(num_splits), _ptr(status), _stream(stream)))
-    return out
-
-
-def append_decode(K, V, slot_mapping, q, cache: Cache, block_tables, seq_lens, max_seq_len: int,
-                  scale: float, out=None, workspace=None, num_splits: int = 0, append_block_table=None,
-                  k_tables=None, status=None, stream=None):
-    """quantize_append(K, V, slot_mapping, cache, append_block_table) then decode_attention(q, ...)
-    in one launch (tq_append_decode); returns fp32 [B][H_q][d]."""
-    _dev(K, torch.bfloat16, "K")
-    _dev(V, torch.bfloat16, "V")
-    _dev(slot_mapping, torch.int32, "slot_mapping")
-    _dev(append_block_table, torch.int32, "append_block_table")
-    _dev(q, torch.bfloat16, "q")
-    _dev(block_tables, torch.int32, "block_tables")
-    _dev(seq_lens, torch.int32, "seq_lens")
-    _dev(k_tables, torch.float16, "k_tables")
-    _dev(status, torch.int32, "status")
-    B, Hq, d = q.shape
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
-    _dev(out, torch.float32, "out")
-    S = num_splits or default_splits(B, cache.num_kv_heads, max_seq_len)
-    if workspace is None:
-        nb = workspace_bytes(B, Hq, d, S)
-        workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=q.device)
-    ab = append_block_table
-    ns, mb = (0, 0) if ab is None else (ab.shape[0], ab.shape[1])
-    _check(load().tq_append_decode(_ptr(K), _ptr(V), _ptr(ab), ns, mb, _ptr(slot_mapping), K.shape[0],
-                                   _ptr(q), cache.c, _ptr(k_tables), _ptr(block_tables),
-                                   block_tables.shape[1], _ptr(seq_lens), B, Hq, int(max_seq_len),
-                                   float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
-                                   int(num_splits), _ptr(status), _stream(stream)))
     return out
 
 

@@ -224,32 +224,28 @@ TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim,
     return it;
 }
 
-// Checks and argument block of an append; *empty when there is nothing to do.
-static int prep_append(const void* K, const void* V, const int32_t* block_table, int num_seqs,
+TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block_table, int num_seqs,
                        int max_blocks, const int32_t* slot_mapping, int T,
                        const tq_cache_t* cache, const uint16_t* k_tables, int32_t* status,
-                       const char* who, tq::AppendArgs& a, bool* empty) {
+                       void* stream) {
     int err;
-    *empty = false;
     if (!check_cache(cache, &err)) return err;
-    if (T < 0) return fail(TQ_ERR_INVALID_ARG, "%s: T < 0", who);
-    if (T == 0) {
-        *empty = true;
-        return TQ_OK;
-    }
+    if (T < 0) return fail(TQ_ERR_INVALID_ARG, "tq_quantize_append: T < 0");
+    if (T == 0) return ok();
     if ((long long)T * cache->num_kv_heads >= 0x7fffffffLL)
-        return fail(TQ_ERR_UNSUPPORTED, "%s: T * H_kv must stay below 2^31", who);
+        return fail(TQ_ERR_UNSUPPORTED, "tq_quantize_append: T * H_kv must stay below 2^31");
     if (!K || !V || !slot_mapping)
-        return fail(TQ_ERR_INVALID_ARG, "%s: K, V and slot_mapping are required", who);
+        return fail(TQ_ERR_INVALID_ARG, "tq_quantize_append: K, V and slot_mapping are required");
     if (block_table && (num_seqs <= 0 || max_blocks <= 0))
-        return fail(TQ_ERR_INVALID_ARG, "%s: block_table needs num_seqs, max_blocks > 0", who);
+        return fail(TQ_ERR_INVALID_ARG, "tq_quantize_append: block_table needs num_seqs, max_blocks > 0");
     if ((long long)num_seqs * max_blocks * tq::kBlock > 0x7fffffffLL)
-        return fail(TQ_ERR_UNSUPPORTED, "%s: logical slots exceed int32", who);
+        return fail(TQ_ERR_UNSUPPORTED, "tq_quantize_append: logical slots exceed int32");
     if (!aligned(K, 16) || !aligned(V, 16))
-        return fail(TQ_ERR_ALIGNMENT, "%s: K and V must be 16-byte aligned", who);
+        return fail(TQ_ERR_ALIGNMENT, "tq_quantize_append: K and V must be 16-byte aligned");
     if (!aligned(slot_mapping, 4) || (block_table && !aligned(block_table, 4)) ||
         (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
-        return fail(TQ_ERR_ALIGNMENT, "%s: int32 arrays and tables must be 4-byte aligned", who);
+        return fail(TQ_ERR_ALIGNMENT, "tq_quantize_append: int32 arrays and tables must be 4-byte aligned");
+    tq::AppendArgs a;
     a.K = static_cast<const uint16_t*>(K);
     a.V = static_cast<const uint16_t*>(V);
     a.block_table = block_table;
@@ -263,19 +259,6 @@ static int prep_append(const void* K, const void* V, const int32_t* block_table,
     a.k_tables = k_tables;
     memcpy(a.default_table, default_table(cache->head_dim), sizeof a.default_table);
     a.status = status;
-    return TQ_OK;
-}
-
-TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block_table, int num_seqs,
-                       int max_blocks, const int32_t* slot_mapping, int T,
-                       const tq_cache_t* cache, const uint16_t* k_tables, int32_t* status,
-                       void* stream) {
-    tq::AppendArgs a;
-    bool empty;
-    const int rc = prep_append(K, V, block_table, num_seqs, max_blocks, slot_mapping, T, cache,
-                               k_tables, status, "tq_quantize_append", a, &empty);
-    if (rc != TQ_OK) return rc;
-    if (empty) return ok();
     cudaError_t e = tq::launch_append(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "tq_quantize_append launch");
     return ok();
@@ -297,38 +280,35 @@ TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_sp
     return (size_t)ranges * 2 * 4 * ((size_t)head_dim * sizeof(float) + sizeof(float2));
 }
 
-// Checks, plan and argument block of a decode; *empty when B == 0.
-static int prep_decode(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
-                       const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
-                       int B, int H_q, int max_seq_len, float scale, float* out,
-                       void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
-                       const char* who, tq::DecodeArgs& a, bool* empty) {
-    *empty = false;
+TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
+                        const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                        int B, int H_q, int max_seq_len, float scale, float* out,
+                        void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
+                        void* stream) {
     int err;
     if (!check_cache(cache, &err)) return err;
     if (B < 0 || H_q <= 0 || max_blocks <= 0 || max_seq_len < 0 ||
         (long long)max_seq_len > (long long)max_blocks * tq::kBlock)
-        return fail(TQ_ERR_INVALID_ARG, "%s: need B >= 0, H_q > 0, 0 <= max_seq_len <= max_blocks*16", who);
-    if (B == 0) {
-        *empty = true;
-        return TQ_OK;
-    }
-    if (B > 65535) return fail(TQ_ERR_UNSUPPORTED, "%s: B %d > 65535", who, B);
+        return fail(TQ_ERR_INVALID_ARG,
+                    "tq_decode_attention: need B >= 0, H_q > 0, 0 <= max_seq_len <= max_blocks*16");
+    if (B == 0) return ok();
+    if (B > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B %d > 65535", B);
     if (!q || !block_tables || !seq_lens || !out)
-        return fail(TQ_ERR_INVALID_ARG, "%s: q, block_tables, seq_lens, out required", who);
+        return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: q, block_tables, seq_lens, out required");
     const int Hkv = cache->num_kv_heads;
     if (H_q % Hkv)
-        return fail(TQ_ERR_UNSUPPORTED, "%s: H_q %d not a multiple of H_kv %d", who, H_q, Hkv);
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: H_q %d not a multiple of H_kv %d", H_q, Hkv);
     const int G = H_q / Hkv;
     if (G != 1 && G != 2 && G != 4 && G != 8)
-        return fail(TQ_ERR_UNSUPPORTED, "%s: GQA group %d (supported 1, 2, 4, 8)", who, G);
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: GQA group %d (supported 1, 2, 4, 8)", G);
     if (num_splits < 0 || num_splits > 1024)
-        return fail(TQ_ERR_UNSUPPORTED, "%s: num_splits %d (0..1024)", who, num_splits);
-    if (!isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "%s: scale not finite", who);
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: num_splits %d (0..1024)", num_splits);
+    if (!isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: scale not finite");
     if (!aligned(q, 4) || !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(seq_lens, 4) ||
         (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
-        return fail(TQ_ERR_ALIGNMENT, "%s: q/out/tables must be 4-byte aligned", who);
+        return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: q/out/tables must be 4-byte aligned");
     const int d = cache->head_dim;
+    tq::DecodeArgs a;
     a.q = static_cast<const uint16_t*>(q);
     a.cache = static_cast<const unsigned char*>(cache->data);
     a.num_blocks = cache->num_blocks;
@@ -345,70 +325,22 @@ static int prep_decode(const void* q, const tq_cache_t* cache, const uint16_t* k
     a.num_splits = num_splits;
     a.max_seq_len = max_seq_len;
     if (!tq::decode_plan(a, device_sms()))
-        return fail(TQ_ERR_UNSUPPORTED, "%s: B * H_kv * num_splits too large", who);
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * num_splits too large");
     const size_t need = tq::decode_workspace_for(a, d);
     if (need) {
         if (!workspace || ws_bytes < need)
-            return fail(TQ_ERR_WORKSPACE, "%s: workspace %zu bytes < %zu needed", who,
+            return fail(TQ_ERR_WORKSPACE, "tq_decode_attention: workspace %zu bytes < %zu needed",
                         workspace ? ws_bytes : (size_t)0, need);
         if (!aligned(workspace, 16))
-            return fail(TQ_ERR_ALIGNMENT, "%s: workspace must be 16-byte aligned", who);
+            return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: workspace must be 16-byte aligned");
     }
     a.ws_o = static_cast<float*>(workspace);
     a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
                                                (size_t)a.nranges * 2 * 4 * d)
                    : nullptr;
     a.status = status;
-    a.fuse = 0;
-    return TQ_OK;
-}
-
-TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
-                        const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
-                        int B, int H_q, int max_seq_len, float scale, float* out,
-                        void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
-                        void* stream) {
-    tq::DecodeArgs a;
-    bool empty;
-    const int rc = prep_decode(q, cache, k_tables, block_tables, max_blocks, seq_lens, B, H_q,
-                               max_seq_len, scale, out, workspace, ws_bytes, num_splits, status,
-                               "tq_decode_attention", a, &empty);
-    if (rc != TQ_OK) return rc;
-    if (empty) return ok();
-    cudaError_t e = tq::launch_decode(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
+    cudaError_t e = tq::launch_decode(a, d, device_sms(), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");
-    return ok();
-}
-
-TQ_API int tq_append_decode(const void* K, const void* V, const int32_t* append_block_table,
-                     int num_seqs, int append_max_blocks, const int32_t* slot_mapping, int T,
-                     const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
-                     const int32_t* block_tables, int max_blocks, const int32_t* seq_lens, int B,
-                     int H_q, int max_seq_len, float scale, float* out, void* workspace,
-                     size_t ws_bytes, int num_splits, int32_t* status, void* stream) {
-    tq::AppendArgs ap;
-    tq::DecodeArgs a;
-    bool app_empty, dec_empty;
-    int rc = prep_append(K, V, append_block_table, num_seqs, append_max_blocks, slot_mapping, T,
-                         cache, k_tables, status, "tq_append_decode", ap, &app_empty);
-    if (rc != TQ_OK) return rc;
-    rc = prep_decode(q, cache, k_tables, block_tables, max_blocks, seq_lens, B, H_q, max_seq_len,
-                     scale, out, workspace, ws_bytes, num_splits, status, "tq_append_decode", a,
-                     &dec_empty);
-    if (rc != TQ_OK) return rc;
-    const int d = cache->head_dim;
-    cudaError_t e = cudaSuccess;
-    if (dec_empty) {
-        if (!app_empty) e = tq::launch_append(ap, d, device_sms(), (cudaStream_t)stream);
-    } else {
-        if (!app_empty) {
-            tq::prepare_append(ap, d);
-            a.app = ap;
-            a.fuse = 1;
-        }
-        e = tq::launch_decode(a, d, device_sms(), (cudaStream_t)stream);
-    }
-    if (e != cudaSuccess) return cuda_fail(e, "tq_append_decode launch");
     return ok();
 }
 

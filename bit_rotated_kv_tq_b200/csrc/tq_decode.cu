@@ -33,7 +33,7 @@
 // accumulators are rescaled only when a running maximum moves.  Each unit
 // leaves an unnormalised partial (o, m, l) that the combine kernel merges; a
 // single split writes the output directly.
-#include "tq_append_impl.cuh"
+#include "tq_kernels.cuh"
 
 namespace tq {
 namespace {
@@ -322,47 +322,6 @@ __device__ __forceinline__ void ldw(uint32_t a, uint32_t (&w)[N]) {
     }
 }
 
-// ------------------------------------------------------------------ grid barrier
-// On each device: {arrivals of the current barrier, barrier generation}.  The
-// last CTA to arrive returns the count to zero and moves the generation on, so
-// every launch (a graph replay included) finds the count at zero.
-__device__ unsigned g_grid_bar[2];
-
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// All CTAs of the (cooperatively launched, so co-resident) grid meet; the wait
-// gives up after ~2^31 clocks and sets TQ_STATUS_TIMEOUT.  After it the CTA's
-// bulk copies see every global write made before the other CTAs arrived.
-__device__ void grid_barrier(const DecodeArgs& a, int tid) {
-    __syncthreads();
-    if (tid == 0) {
-        unsigned* count = a.gbar;
-        unsigned* gen = a.gbar + 1;
-        const unsigned g0 = ld_acquire_gpu(gen);  // read before arriving: it cannot move yet
-        __threadfence();
-        if (atomicAdd(count, 1u) == gridDim.x - 1) {
-            atomicExch(count, 0u);
-            __threadfence();
-            atomicAdd(gen, 1u);
-        } else {
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(gen) == g0) {
-                if (clock64() - t0 > (1LL << 31)) {
-                    flag_status(a.status, TQ_STATUS_TIMEOUT);
-                    break;
-                }
-                __nanosleep(64);
-            }
-        }
-    }
-    __syncthreads();
-    asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
 // ------------------------------------------------------------------ split kernel
 template <int D>
 __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
@@ -384,16 +343,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     if (P.end - s0 > a.smem_bytes) {  // cannot happen with the launcher's size; never touch memory
         if (tid == 0 && blockIdx.x == 0) flag_status(a.status, TQ_STATUS_INTERNAL);
         return;
-    }
-    if (a.fuse) {
-        // ---- fused append: every warp of the grid quantises its share of the new
-        // tokens (the bin tables borrow the start of the dynamic region, which the
-        // rings and the centroid table take over only after the barrier); then all
-        // CTAs meet, so that every record the decode reads is complete
-        HeadBins* hb = reinterpret_cast<HeadBins*>(dsm);
-        BinEntry* bins = reinterpret_cast<BinEntry*>(hb + a.app.Hkv);
-        app::append_warps<D>(a.app, hb, bins, blockIdx.x * kWarps + wa, gridDim.x * kWarps);
-        grid_barrier(a, tid);
     }
     const int G = a.Hq / a.Hkv;
     const int stride = kHalves * gridDim.x;  // ranges per round over all halves
@@ -781,25 +730,7 @@ cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
     a.smem_bytes = smem;
     const int halves = (a.nranges + kHalves - 1) / kHalves;
     const int grid = halves < num_sms ? halves : num_sms;
-    if (a.fuse) {
-        // the grid barrier needs every CTA resident: a cooperative launch either
-        // guarantees that or fails
-        static unsigned* bar[64] = {};
-        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-        if (!bar[dev]) {
-            void* p = nullptr;
-            e = cudaGetSymbolAddress(&p, g_grid_bar);
-            if (e != cudaSuccess) return e;
-            bar[dev] = static_cast<unsigned*>(p);
-        }
-        a.gbar = bar[dev];
-        void* params[] = {&a};
-        e = cudaLaunchCooperativeKernel((const void*)decode_split_kernel<D>, dim3(grid),
-                                        dim3(kWarps * 32), params, smem, stream);
-        if (e != cudaSuccess) return e;
-    } else {
-        decode_split_kernel<D><<<grid, kWarps * 32, smem, stream>>>(a);
-    }
+    decode_split_kernel<D><<<grid, kWarps * 32, smem, stream>>>(a);
     if (decode_needs_combine(a)) combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a);
     return cudaGetLastError();
 }

@@ -99,11 +99,6 @@ struct DecodeArgs {
     int nranges;
     uint64_t div_nmax, div_hkv, div_quads;  // fast_div multipliers
     uint32_t smem_bytes;  // dynamic shared memory of the split kernel
-    // fused append (tq_append_decode): the append runs first on every warp of the
-    // grid, then a grid barrier, then the decode
-    int fuse;
-    unsigned* gbar;       // {count, generation} of the grid barrier (set by the launcher)
-    AppendArgs app;
 };
 
 struct DequantArgs {
@@ -123,7 +118,6 @@ struct DequantArgs {
 size_t append_smem_bytes(int Hkv);
 int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
-void prepare_append(AppendArgs& a, int head_dim);  // fast-division multipliers, default bins
 cudaError_t launch_decode(const DecodeArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 uint32_t decode_smem_bytes(int head_dim);  // dynamic shared memory of the split kernel
 bool decode_plan(DecodeArgs& a, int num_sms);            // ranges; false: too many

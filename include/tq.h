@@ -158,24 +158,6 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
                         void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
                         void* stream);
 
-/* tq_quantize_append followed by tq_decode_attention on the same cache, in
- * one launch: the kernel quantises the new tokens on every warp of its grid,
- * all its CTAs meet at a grid barrier, and then it decodes, so the decode sees
- * every appended token.  Arguments, checks, results and status bits are those
- * of the two calls (append_block_table, num_seqs and append_max_blocks are
- * the append's block_table, num_seqs and max_blocks; the cache, k_tables and
- * status are shared).  T == 0 is a plain decode, B == 0 a plain append.
- * The kernel is launched cooperatively (all its CTAs resident at once) and
- * may be captured in a CUDA graph.  Fused calls on one device must be ordered
- * on the GPU (one stream, or events), as they share the barrier's counter.  A
- * barrier that waits ~1 s sets TQ_STATUS_TIMEOUT. */
-TQ_API int tq_append_decode(const void* K, const void* V, const int32_t* append_block_table,
-                     int num_seqs, int append_max_blocks, const int32_t* slot_mapping, int T,
-                     const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
-                     const int32_t* block_tables, int max_blocks, const int32_t* seq_lens, int B,
-                     int H_q, int max_seq_len, float scale, float* out, void* workspace,
-                     size_t ws_bytes, int num_splits, int32_t* status, void* stream);
-
 /* Decode attention without a caller workspace.  No page describes this call;
  * it exists for callers that cannot allocate device memory at all -- an
  * operator or plugin hosted by another runtime usually receives only the
