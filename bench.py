@@ -460,6 +460,17 @@ def run_tq(args, rank, world, local):
     assert torch.equal(h_outs[(args.steps - 2) % nbuf], out.cpu()), "end-to-end result differs"
     h2d = h_q.numel() * 2 + h_K.numel() * 2 + h_V.numel() * 2 + h_S.numel() * 4
     d2h = h_outs[0].numel() * 4
+    # the host link alone: one step's input copies with nothing else running, the floor
+    # under the end-to-end step time
+    l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(copy_s):
+        copy_in(0)
+        l0.record(copy_s)
+        for _ in range(5):
+            copy_in(0)
+        l1.record(copy_s)
+    copy_s.synchronize()
+    h2d_link_gbs = h2d * 5 / (l0.elapsed_time(l1) / 1e3) / 1e9
 
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
@@ -503,7 +514,8 @@ def run_tq(args, rank, world, local):
                          "kernel": "tq_decode_attention (split kernel + combine)",
                          "peak_source": f"{peak_kind} hbm_gbs"},
             "e2e": {"value": weak_scaling_value(kv, args.steps, world, e2e_s) / 1e9, "unit": "GB/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_s * 1e3 / args.steps, "h2d_link_gbs": h2d_link_gbs},
             "gpu_launches": args.steps * (2 + (1 if combine_runs(w, S, dev) else 0)),
             "clocks": clocks,
             "cpu_baseline": cpu,
