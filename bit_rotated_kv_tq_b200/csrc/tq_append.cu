@@ -10,37 +10,49 @@
 //   z = fp16 rounded down from min, s = fp16 rounded up from (max - z)/15,
 //   q = round-half-even((v - z)/s) in [0, 15].
 //
-// Work split: one vector (token, kv head) is spread over D/8 lanes holding 8
-// elements each, so a warp handles 2 (D=128) or 4 (D=64) vectors per pass;
-// loads are 16-byte per lane and fully coalesced.  The grid is persistent
-// (one wave of resident CTAs) and every warp loads its next pass before it
-// computes the current one, so the global-load latency overlaps the math.
-// The rotation is an in-register butterfly over 3 index bits plus
-// xor-shuffles over the lane bits (a sign-FMA per element and stage).
+// Work split: one vector (token, kv head) is spread over D/16 lanes holding 16
+// consecutive elements each, so a warp pass covers 8 (D=64) or 4 (D=128)
+// vectors, 1 KB of keys and 1 KB of values.  The grid is persistent (one wave
+// of resident CTAs); warp w takes passes w, w + W, w + 2W, ... (W warps in
+// all).  Every warp keeps its next kPrefetch passes requested into L2 with
+// bulk prefetches and loads its next pass into registers while it computes
+// the current one, so HBM sees the whole input stream early and the register
+// loads hit L2.  The rotation is an in-register butterfly over the 4 index
+// bits inside a lane plus xor-shuffles over the lane bits.
 //
-// Exactness: the fast path runs in fp32.  Every decision it takes (fp16
-// rounding of the norm, the nearest centroid, the rounding of (v - z)/s and
-// the fp16 rounding up of the scale) is re-taken in fp64 from the bf16
-// inputs whenever the fp32 input lies inside the fp32 error bound of the
-// decision threshold.  The fp64 recomputation forms the +-1 Hadamard sums
-// exactly and divides once by n*sqrt(D), which is the definition evaluated
-// with exact sums, so the stored codes are those of the exact-arithmetic
-// definition except within ~1e-15 of a threshold.
+// Nearest centroid: x = 63 y + 64 is rounded to 1/8 by one fma against a
+// 2^20 magic constant, whose low mantissa bits then address a 128-entry bin
+// table in shared memory (1 KB per table).  A bin holds at most one midpoint
+// of the default tables; its entry gives that midpoint and the count of
+// midpoints below, and the code is that count plus one fp32 comparison.
+// Tables with closer midpoints take an exact count over all 15 midpoints.
+//
+// Exactness: the fast path runs in fp32.  Every decision it takes is
+// re-taken exactly whenever the fp32 input lies inside the fp32 error bound
+// of the decision threshold: the fp16 rounding of the norm and the nearest
+// centroid in fp64 from the bf16 inputs (exact +-1 Hadamard sums, compared
+// against midpoint * n * sqrt(D)), the value codes by comparing v - z with
+// (k + 1/2) s in fp64, and the fp16 rounding up of the scale in fp64.  The
+// stored codes are therefore those of the exact-arithmetic definition except
+// within ~1e-15 (relative) of a key threshold.
 #include "tq_kernels.cuh"
 
 namespace tq {
 
-// Relative margin on the norm before its fp16 rounding (fp32 sum of squares
-// of at most 128 exact products: error <= 11 ulp relative, 6.6e-7).
-constexpr float kNormMargin = 1.5e-6f;
+// Relative margin on the norm before its fp16 rounding: twice the error bound
+// of the fast path's norm (fp32 sum of exact squares along a tree of depth
+// <= 8, then ss * rsqrt with one Newton step: <= 9 ulp).
+constexpr float kNormMargin = 1.1e-6f;
 // Margin, in value-code units, around the .5 rounding points of (v - z)/s
-// (fp32 error <= 3 ulp of 15, i.e. 2.7e-6).
-constexpr float kValueMargin = 1.0f / 4096.0f;
+// (v - z and 1/s are each correctly rounded and the product is fused with
+// the rounding, so the fp32 quotient errs by at most ~2^-19 code units).
+constexpr float kValueMargin = 1.0f / 65536.0f;
 
-// Bin tables in shared memory (called by the whole CTA).  Without per-head
-// tables every head uses the default table, whose bins the launcher computed
-// once on the host: they are copied, and every head indexes them as head 0.
-// Per-head tables are binned here, one thread per (head, bin).
+// Bin tables in shared memory (called by the whole CTA): the tables sit at
+// the start of the dynamic shared memory, 1 KB each, the HeadBins after them.
+// Without per-head tables every head uses the default table, whose bins the
+// launcher computed once on the host: they are copied, and every head
+// indexes them as head 0.  Per-head tables are binned here.
 __device__ void build_bins(HeadBins* hb, BinEntry* bins, const AppendArgs& a) {
     if (!a.k_tables) {
         for (int e = threadIdx.x; e < kBins; e += blockDim.x) bins[e] = a.default_bins[e];
@@ -60,11 +72,9 @@ __device__ void build_bins(HeadBins* hb, BinEntry* bins, const AppendArgs& a) {
     __syncthreads();
 }
 
-// 1/x by the hardware approximation (relative error ~2^-22): (v - z) * (1/s)
-// then errs by < 15 * 2^-21 code units, far inside kValueMargin
-__device__ __forceinline__ float fast_rcp(float x) {
+__device__ __forceinline__ float rsqrt_approx(float x) {  // x normal and positive
     float y;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
@@ -72,11 +82,46 @@ __device__ __forceinline__ float fast_rcp(float x) {
 __device__ __forceinline__ float inv15_up() { return __uint_as_float(0x3d888889u); }
 __device__ __forceinline__ float inv15_dn() { return __uint_as_float(0x3d888888u); }
 
-// One warp pass's inputs (prefetched one pass ahead).
+// 16-byte read-only load that allocates in L1: a lane's two loads cover one
+// 32-byte sector, so the second one is served by the first one's fill.
+__device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Request [p, p + bytes) into L2 (p and bytes multiples of 16); no completion.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// passes each warp keeps requested into L2 ahead of its loads
+constexpr int kPrefetch = 4;
+
+template <int D>
+struct Geo {
+    static constexpr int LPV = D / 16;    // lanes per vector
+    static constexpr int VPW = 32 / LPV;  // vectors per warp pass
+};
+
+// keys and values of pass p into L2
+template <int D>
+__device__ __forceinline__ void prefetch_pass(const AppendArgs& a, uint32_t p, uint32_t npass,
+                                              uint32_t total) {
+    if (p >= npass) return;
+    const uint32_t v0 = p * Geo<D>::VPW;
+    const uint32_t nv = min((uint32_t)Geo<D>::VPW, total - v0);
+    prefetch_l2_bulk(a.K + (size_t)v0 * D, nv * D * 2);
+    prefetch_l2_bulk(a.V + (size_t)v0 * D, nv * D * 2);
+}
+
+// One warp pass's inputs (loaded one pass ahead).
 struct Pass {
-    uint4 k, v;  // this lane's 8 bf16 keys / values
-    int slot;    // slot_mapping entry of the token (-1: skip)
-    int pb;      // physical block read from the block table (when one is given)
+    uint4 k0, k1, v0, v1;  // this lane's 16 bf16 keys / values
+    int slot;              // slot_mapping entry of the token (-1: skip)
+    int pb;                // physical block read from the block table (when one is given)
     uint32_t vec;
     bool in;
 };
@@ -84,19 +129,19 @@ struct Pass {
 template <int D>
 __device__ __forceinline__ void load_pass(const AppendArgs& a, uint32_t p, uint32_t npass,
                                           uint32_t total, int grp, int sub, Pass& L) {
-    constexpr int VPW = 32 / (D / 8);
-    L.vec = p * VPW + grp;
+    L.vec = p * Geo<D>::VPW + grp;
     L.in = p < npass && L.vec < total;
     L.slot = -1;
     L.pb = -1;
-    L.k = make_uint4(0, 0, 0, 0);
-    L.v = make_uint4(0, 0, 0, 0);
+    L.k0 = L.k1 = L.v0 = L.v1 = make_uint4(0, 0, 0, 0);
     if (L.in) {
-        const uint32_t t = fast_div(L.vec, a.div_hkv);
+        const uint32_t t = fast_div32(L.vec, a.dv_hkv);
         L.slot = __ldg(a.slots + t);
-        const size_t eoff = (size_t)L.vec * D + sub * 8;  // vec = t * Hkv + h
-        L.k = ld_stream_u4(a.K + eoff);
-        L.v = ld_stream_u4(a.V + eoff);
+        const size_t eoff = (size_t)L.vec * D + sub * 16;  // vec = t * Hkv + h
+        L.k0 = ld_nc_u4(a.K + eoff);
+        L.k1 = ld_nc_u4(a.K + eoff + 8);
+        L.v0 = ld_nc_u4(a.V + eoff);
+        L.v1 = ld_nc_u4(a.V + eoff + 8);
     }
 }
 
@@ -105,7 +150,7 @@ __device__ __forceinline__ void load_pass(const AppendArgs& a, uint32_t p, uint3
 __device__ __forceinline__ void fetch_block(const AppendArgs& a, Pass& L) {
     if (a.block_table && L.in && L.slot >= 0) {
         const uint32_t s = (uint32_t)L.slot;
-        const uint32_t seq = fast_div(s, a.div_cap);
+        const uint32_t seq = fast_div32(s, a.dv_cap);
         const uint32_t pos = s - seq * (uint32_t)(a.max_blocks * kBlock);
         L.pb = seq < (uint32_t)a.num_seqs
                    ? __ldg(a.block_table + (size_t)seq * a.max_blocks + pos / kBlock)
@@ -118,7 +163,6 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
     return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a - b, one rounding
 }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // 1.5 * 2^23: x + kRound rounds x (0 <= x < 2^22) to the nearest integer,
 // ties to even, and leaves that integer in the low mantissa bits.
@@ -127,192 +171,57 @@ constexpr float kRound = 12582912.0f;
 template <int D>
 __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
     extern __shared__ __align__(16) unsigned char smem[];
-    HeadBins* hb = reinterpret_cast<HeadBins*>(smem);
-    BinEntry* bins = reinterpret_cast<BinEntry*>(hb + a.Hkv);
-
-    constexpr int LPV = D / 8;     // lanes per vector
-    constexpr int VPW = 32 / LPV;  // vectors per warp pass
+    constexpr int LPV = Geo<D>::LPV;
+    constexpr int VPW = Geo<D>::VPW;
     using R = Rec<D>;
+    const int ntab = a.k_tables ? a.Hkv : 1;
+    BinEntry* bins = reinterpret_cast<BinEntry*>(smem);
+    HeadBins* hb = reinterpret_cast<HeadBins*>(smem + (size_t)ntab * kBins * sizeof(BinEntry));
+
     const int lane = threadIdx.x & 31;
     const int sub = lane % LPV;
     const int grp = lane / LPV;
     const uint32_t total = (uint32_t)a.T * (uint32_t)a.Hkv;
     const uint32_t npass = (total + VPW - 1) / VPW;
     const uint32_t nwarps = gridDim.x * (blockDim.x / 32);
-    const uint32_t cap = (uint32_t)(a.max_blocks * kBlock);
+    const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.125f;  // fp32 of 1/sqrt(D)
 
-    // the first pass's loads go out before the bins are built, so the two overlap
-    Pass cur, nxt;
     uint32_t pass = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
+    // the warp's first passes into L2 (lane j: pass + j W), then its first loads;
+    // the bins are built while they are in flight
+    if (lane < kPrefetch) prefetch_pass<D>(a, pass + (uint32_t)lane * nwarps, npass, total);
+    Pass cur, nxt;
     load_pass<D>(a, pass, npass, total, grp, sub, cur);
     build_bins(hb, bins, a);
     fetch_block(a, cur);
 
     for (; pass < npass; pass += nwarps) {
+        if (lane == 0) prefetch_pass<D>(a, pass + (uint32_t)kPrefetch * nwarps, npass, total);
         load_pass<D>(a, pass + nwarps, npass, total, grp, sub, nxt);
-        const uint32_t t = fast_div(cur.vec, a.div_hkv);
+        const uint32_t t = fast_div32(cur.vec, a.dv_hkv);
         const int h = cur.in ? (int)(cur.vec - t * (uint32_t)a.Hkv) : 0;
 
-        // ---- key: norm (elements 2i, 2i+1 in P[i])
-        float2 P[4];
-        P[0] = make_float2(bf16_lo(cur.k.x), bf16_hi(cur.k.x));
-        P[1] = make_float2(bf16_lo(cur.k.y), bf16_hi(cur.k.y));
-        P[2] = make_float2(bf16_lo(cur.k.z), bf16_hi(cur.k.z));
-        P[3] = make_float2(bf16_lo(cur.k.w), bf16_hi(cur.k.w));
-        float2 q2 = mul2(P[0], P[0]);
-        q2 = __ffma2_rn(P[1], P[1], q2);
-        q2 = __ffma2_rn(P[2], P[2], q2);
-        q2 = __ffma2_rn(P[3], P[3], q2);
-        float ss = q2.x + q2.y;
+        // ---- values: group of 32 = this lane and lane ^ 1
+        const uint32_t vwd[8] = {cur.v0.x, cur.v0.y, cur.v0.z, cur.v0.w,
+                                 cur.v1.x, cur.v1.y, cur.v1.z, cur.v1.w};
+        __nv_bfloat162 mn2 = *reinterpret_cast<const __nv_bfloat162*>(&vwd[0]);
+        __nv_bfloat162 mx2 = mn2;
 #pragma unroll
-        for (int m = 1; m < LPV; m <<= 1) ss += __shfl_xor_sync(kFull, ss, m);
-        const float n = sqrtf(ss);
-        uint16_t n16 = __half_as_ushort(__float2half_rn(n));
-        bool near = __half_as_ushort(__float2half_rn(n * (1.0f - kNormMargin))) !=
-                    __half_as_ushort(__float2half_rn(n * (1.0f + kNormMargin)));
-        // squares that leave the normal fp32 range (or a non-finite key) lose the
-        // fp32 error bound: take the fp64 path
-        near |= !(ss >= 1e-30f && ss <= 1e30f) && ss != 0.f;
-
-        // ---- key: unnormalised Hadamard butterfly.  Index bit 0 lies inside a
-        // pair, bits 1-2 across pairs (packed adds), the rest across lanes.
-        float2 Q[4];
-#pragma unroll
-        for (int i = 0; i < 4; i++) Q[i] = make_float2(P[i].x + P[i].y, P[i].x - P[i].y);
+        for (int j = 1; j < 8; j++) {
+            const __nv_bfloat162 w = *reinterpret_cast<const __nv_bfloat162*>(&vwd[j]);
+            mn2 = __hmin2(mn2, w);
+            mx2 = __hmax2(mx2, w);
+        }
         {
-            const float2 a0 = add2(Q[0], Q[1]), a1 = sub2(Q[0], Q[1]);
-            const float2 a2 = add2(Q[2], Q[3]), a3 = sub2(Q[2], Q[3]);
-            Q[0] = add2(a0, a2); Q[2] = sub2(a0, a2);
-            Q[1] = add2(a1, a3); Q[3] = sub2(a1, a3);
+            const uint32_t pm = __shfl_xor_sync(kFull, *reinterpret_cast<const uint32_t*>(&mn2), 1);
+            const uint32_t px = __shfl_xor_sync(kFull, *reinterpret_cast<const uint32_t*>(&mx2), 1);
+            mn2 = __hmin2(mn2, *reinterpret_cast<const __nv_bfloat162*>(&pm));
+            mx2 = __hmax2(mx2, *reinterpret_cast<const __nv_bfloat162*>(&px));
         }
-#pragma unroll
-        for (int m = 1; m < LPV; m <<= 1) {
-            const float sg = (sub & m) ? -1.f : 1.f;  // upper half: partner - own
-            const float2 sg2 = make_float2(sg, sg);
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float2 pr = make_float2(__shfl_xor_sync(kFull, Q[i].x, m),
-                                              __shfl_xor_sync(kFull, Q[i].y, m));
-                Q[i] = __ffma2_rn(sg2, Q[i], pr);
-            }
-        }
-        const float inv = ss > 0.f ? rsqrtf(ss * (float)D) : 0.f;
-
-        // ---- key: nearest centroid through the per-head bins
-        const int hs = a.k_tables ? h : 0;  // whose bins (one shared set without per-head tables)
-        const HeadBins& B = hb[hs];
-        const BinEntry* hbins = bins + hs * kBins;
-        uint32_t kw = 0;
-        float y[8];
-        {
-            const float2 inv2 = make_float2(inv, inv);
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float2 yy = mul2(Q[i], inv2);
-                y[2 * i] = yy.x;
-                y[2 * i + 1] = yy.y;
-            }
-        }
-        if (!B.dense) {
-            uint32_t nib[8];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float2 ps = __ffma2_rn(make_float2(y[2 * i], y[2 * i + 1]),
-                                            make_float2(kBinScale, kBinScale),
-                                            make_float2(kBinScale, kBinScale));
-                const int b0 = max(min((int)ps.x, kBins - 1), 0);
-                const int b1 = max(min((int)ps.y, kBins - 1), 0);
-                const BinEntry e0 = hbins[b0], e1 = hbins[b1];
-                const float d0 = y[2 * i] - e0.mid, d1 = y[2 * i + 1] - e1.mid;
-                nib[2 * i] = (uint32_t)(e0.k_lo + (d0 > 0.f ? 1 : 0));
-                nib[2 * i + 1] = (uint32_t)(e1.k_lo + (d1 > 0.f ? 1 : 0));
-                near |= fmaxf(fabsf(d0), fabsf(d1)) < kKeyMargin;
-            }
-            // bytes (nib[2j] | nib[2j+1] << 4), j = 0..3, into one word
-            const uint32_t b01 = __byte_perm(nib[0] | (nib[1] << 4), nib[2] | (nib[3] << 4), 0x0040);
-            const uint32_t b23 = __byte_perm(nib[4] | (nib[5] << 4), nib[6] | (nib[7] << 4), 0x0040);
-            kw = __byte_perm(b01, b23, 0x5410);
-        } else {
-#pragma unroll
-            for (int e = 0; e < 8; e++) {
-                int idx = 0;
-                for (int j = 0; j < 15; j++) {
-                    const float dm = y[e] - 0.5f * (B.c[j] + B.c[j + 1]);
-                    idx += dm > 0.f ? 1 : 0;
-                    near |= fabsf(dm) < kKeyMargin;
-                }
-                kw |= (uint32_t)idx << (4 * e);
-            }
-        }
-        near = near && cur.in && cur.slot >= 0;
-
-        // ---- key: fp64 recomputation when any decision of the warp is close
-        if (__any_sync(kFull, near)) {
-            double Sd[8];
-            double ssd = 0.0;
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                Sd[2 * i] = (double)P[i].x;
-                Sd[2 * i + 1] = (double)P[i].y;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; e++) ssd = fma(Sd[e], Sd[e], ssd);
-#pragma unroll
-            for (int m = 1; m < LPV; m <<= 1) ssd += __shfl_xor_sync(kFull, ssd, m);
-            const double nd = sqrt(ssd);
-#pragma unroll
-            for (int b = 1; b < 8; b <<= 1) {
-#pragma unroll
-                for (int e = 0; e < 8; e++)
-                    if (!(e & b)) {
-                        const double x = Sd[e], yv = Sd[e | b];
-                        Sd[e] = x + yv;
-                        Sd[e | b] = x - yv;
-                    }
-            }
-#pragma unroll
-            for (int m = 1; m < LPV; m <<= 1) {
-                const bool upper = sub & m;
-#pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    const double p = __shfl_xor_sync(kFull, Sd[e], m);
-                    Sd[e] = upper ? p - Sd[e] : Sd[e] + p;
-                }
-            }
-            if (cur.in) {
-                n16 = __half_as_ushort(__double2half(nd));
-                const double denom = nd * sqrt((double)D);
-                kw = 0;
-#pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    const double yd = nd > 0.0 ? Sd[e] / denom : 0.0;
-                    int idx = 0;
-                    for (int j = 0; j < 15; j++)
-                        idx += yd > 0.5 * ((double)B.c[j] + (double)B.c[j + 1]) ? 1 : 0;
-                    kw |= (uint32_t)idx << (4 * e);
-                }
-            }
-        }
-
-        // the next pass's block-table entry: its slot has arrived by now, and the
-        // lookup overlaps this pass's value work and stores
-        fetch_block(a, nxt);
-
-        // ---- values: group of 32 = 4 lanes
-        float2 V2[4];
-        V2[0] = make_float2(bf16_lo(cur.v.x), bf16_hi(cur.v.x));
-        V2[1] = make_float2(bf16_lo(cur.v.y), bf16_hi(cur.v.y));
-        V2[2] = make_float2(bf16_lo(cur.v.z), bf16_hi(cur.v.z));
-        V2[3] = make_float2(bf16_lo(cur.v.w), bf16_hi(cur.v.w));
-        float mn = fminf(fminf(fminf(V2[0].x, V2[0].y), fminf(V2[1].x, V2[1].y)),
-                         fminf(fminf(V2[2].x, V2[2].y), fminf(V2[3].x, V2[3].y)));
-        float mx = fmaxf(fmaxf(fmaxf(V2[0].x, V2[0].y), fmaxf(V2[1].x, V2[1].y)),
-                         fmaxf(fmaxf(V2[2].x, V2[2].y), fmaxf(V2[3].x, V2[3].y)));
-#pragma unroll
-        for (int m = 1; m < 4; m <<= 1) {
-            mn = fminf(mn, __shfl_xor_sync(kFull, mn, m));
-            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-        }
+        const uint32_t mnw = *reinterpret_cast<const uint32_t*>(&mn2);
+        const uint32_t mxw = *reinterpret_cast<const uint32_t*>(&mx2);
+        const float mn = fminf(bf16_lo(mnw), bf16_hi(mnw));
+        const float mx = fmaxf(bf16_lo(mxw), bf16_hi(mxw));
         const __half zh = __float2half_rd(mn);  // exact: mn is a bf16 value
         const float zf = __half2float(zh);
         // s = fp16 rounded up from (mx - z)/15: bracket the quotient in fp32 with
@@ -328,68 +237,273 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
             if (s_hi != s_lo) s16 = double_to_half_up_nonneg(((double)mx - (double)zf) / 15.0);
         }
         const float sf = half_bits_to_float(s16);
-        uint32_t vw = 0;
+        const bool vbad = !isfinite(sf) || !isfinite(zf);
+        const uint32_t sz = (uint32_t)s16 | ((uint32_t)__half_as_ushort(zh) << 16);  // scale, zero
+        uint32_t vw0 = 0, vw1 = 0;  // code bytes of elements 0-7, 8-15
         if (sf > 0.f) {
-            const float inv_s = fast_rcp(sf);  // its error is far inside kValueMargin
-            const float2 z2 = make_float2(zf, zf), is2 = make_float2(inv_s, inv_s);
+            const float is = __frcp_rn(sf);
+            const float2 z2 = make_float2(zf, zf), is2 = make_float2(is, is);
             const float2 rnd = make_float2(kRound, kRound);
-            uint32_t qb[8];
-            bool tie = false;
+            float dmax = 0.f;
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const float2 r = mul2(sub2(V2[i], z2), is2);  // (v - z) / s, in [0, 15]
-                const float2 tr = add2(r, rnd);               // round half to even
-                const float2 d = sub2(r, sub2(tr, rnd));      // r - round(r)
-                tie |= fmaxf(fabsf(d.x), fabsf(d.y)) > 0.5f - kValueMargin;
-                qb[2 * i] = __float_as_uint(tr.x);            // low byte = code
-                qb[2 * i + 1] = __float_as_uint(tr.y);
+            for (int j = 0; j < 8; j++) {
+                const float2 vz = sub2(make_float2(bf16_lo(vwd[j]), bf16_hi(vwd[j])), z2);
+                const float2 tr = __ffma2_rn(vz, is2, rnd);  // kRound + round-half-even(r)
+                const float2 ti = sub2(tr, rnd);             // that integer, exact
+                const float2 d = __ffma2_rn(vz, is2, make_float2(-ti.x, -ti.y));  // r - ti
+                dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+                // the codes are the low bytes of tr
+                const uint32_t byte = (__float_as_uint(tr.x) + (__float_as_uint(tr.y) << 4)) & 0xffu;
+                if (j < 4) vw0 |= byte << (8 * j);
+                else vw1 |= byte << (8 * (j - 4));
             }
-            if (tie) {  // a .5 point within the fp32 error: exact quotients in fp64
+            if (dmax > 0.5f - kValueMargin) {
+                // a .5 point within the fp32 error: decide every element exactly by
+                // comparing v - z with (k + 1/2) s in fp64 (both exact there), k the
+                // integer below the fp32 quotient, ties to even
+                vw0 = vw1 = 0;
 #pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    qb[2 * i] = (uint32_t)rint(((double)V2[i].x - (double)zf) / (double)sf);
-                    qb[2 * i + 1] = (uint32_t)rint(((double)V2[i].y - (double)zf) / (double)sf);
+                for (int e = 0; e < 16; e++) {
+                    const float vf = e & 1 ? bf16_hi(vwd[e >> 1]) : bf16_lo(vwd[e >> 1]);
+                    const float k = floorf((vf - zf) * is);
+                    const double v = (double)vf - (double)zf;
+                    const double bnd = ((double)k + 0.5) * (double)sf;
+                    const int ki = (int)k;
+                    const int q = v > bnd ? ki + 1 : (v < bnd ? ki : ki + (ki & 1));
+                    const uint32_t c = (uint32_t)min(max(q, 0), 15);
+                    if (e < 8) vw0 |= c << (4 * e);
+                    else vw1 |= c << (4 * (e - 8));
                 }
             }
-            const uint32_t even = __byte_perm(__byte_perm(qb[0], qb[2], 0x0040),
-                                              __byte_perm(qb[4], qb[6], 0x0040), 0x5410);
-            const uint32_t odd = __byte_perm(__byte_perm(qb[1], qb[3], 0x0040),
-                                             __byte_perm(qb[5], qb[7], 0x0040), 0x5410);
-            vw = ((even & 0x0f0f0f0fu) | ((odd & 0x0f0f0f0fu) << 4));
         }
 
+        // ---- key: norm and in-lane butterfly over element bits 0-3.  Q[j]
+        // holds elements (2j, 2j+1) of the lane's 16.
+        const uint32_t kwd[8] = {cur.k0.x, cur.k0.y, cur.k0.z, cur.k0.w,
+                                 cur.k1.x, cur.k1.y, cur.k1.z, cur.k1.w};
+        float2 Q[8];
+        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+        uint32_t kor = 0;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const float2 P = make_float2(bf16_lo(kwd[j]), bf16_hi(kwd[j]));
+            if (j & 1) sb = __ffma2_rn(P, P, sb);
+            else sa = __ffma2_rn(P, P, sa);
+            Q[j] = make_float2(P.x + P.y, P.x - P.y);
+            kor |= kwd[j];
+        }
+        float ss = (sa.x + sa.y) + (sb.x + sb.y);
+#pragma unroll
+        for (int m = 1; m < LPV; m <<= 1) ss += __shfl_xor_sync(kFull, ss, m);
+#pragma unroll
+        for (int b = 1; b < 8; b <<= 1) {
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (!(j & b)) {
+                    const float2 x = Q[j], y = Q[j | b];
+                    Q[j] = add2(x, y);
+                    Q[j | b] = sub2(x, y);
+                }
+        }
+        // ---- key: butterfly over the lane bits (upper half: partner - own)
+#pragma unroll
+        for (int m = 1; m < LPV; m <<= 1) {
+            const float sg = (sub & m) ? -1.f : 1.f;
+            const float2 sg2 = make_float2(sg, sg);
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const float2 pr = make_float2(__shfl_xor_sync(kFull, Q[j].x, m),
+                                              __shfl_xor_sync(kFull, Q[j].y, m));
+                Q[j] = __ffma2_rn(sg2, Q[j], pr);
+            }
+        }
+        // ---- key: norm (fp16) and the scale to unit-vector coordinates: rsqrt
+        // refined by one Newton step (relative error ~4 ulp whatever the
+        // approximation's), so n errs by <= 9 ulp and 1 / (n sqrt(D)) by <= 10 ulp
+        const float ssc = fmaxf(ss, 1.17549435e-38f);
+        const float rs0 = rsqrt_approx(ssc);
+        const float rs = rs0 * fmaf(-0.5f * ssc * rs0, rs0, 1.5f);
+        const float n = ss * rs;
+        uint16_t n16 = __half_as_ushort(__float2half_rn(n));
+        bool near = __half_as_ushort(__float2half_rn(n * (1.0f - kNormMargin))) !=
+                    __half_as_ushort(__float2half_rn(n * (1.0f + kNormMargin)));
+        // squares that leave the normal fp32 range (or a non-finite key) lose the
+        // fp32 error bound: every decision is re-taken (an all-zero key stays here)
+        const bool wild = !(ss >= 1e-30f && ss <= 1e30f) && (kor & 0x7fff7fffu) != 0u;
+        near |= wild;
+        const float inv = rs * inv_sqrt_d;              // 1 / (n sqrt(D))
+        const float A = rs * (inv_sqrt_d * kBinScale);  // kBinScale / (n sqrt(D))
+
+        // ---- key: nearest centroid
+        const int hs = a.k_tables ? h : 0;  // whose table
+        const HeadBins& B = hb[hs];
+        const unsigned char* tab = smem + (size_t)hs * (kBins * sizeof(BinEntry));
+        uint32_t kw0 = 0, kw1 = 0;  // codes of elements 0-7, 8-15
+        if (!B.dense) {
+            const float2 A2 = make_float2(A, A), M2 = make_float2(kBinMagic, kBinMagic);
+            float dmin = INFINITY;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const float2 x = __ffma2_rn(Q[j], A2, M2);
+                const BinEntry e0 = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x.x) & 0x3f8u));
+                const BinEntry e1 = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x.y) & 0x3f8u));
+                // y - mid with one rounding: its sign is the decision
+                const float d0 = fmaf(Q[j].x, inv, -e0.mid);
+                const float d1 = fmaf(Q[j].y, inv, -e1.mid);
+                dmin = fminf(dmin, fminf(fabsf(d0), fabsf(d1)));
+                // k_hi - 1 where y <= mid (sign bit set; y == mid is near anyway)
+                const uint32_t c0 = (uint32_t)(e0.k_hi + (__float_as_int(d0) >> 31));
+                const uint32_t c1 = (uint32_t)(e1.k_hi + (__float_as_int(d1) >> 31));
+                const uint32_t byte = c0 | (c1 << 4);
+                if (j < 4) kw0 |= byte << (8 * j);
+                else kw1 |= byte << (8 * (j - 4));
+            }
+            near |= dmin < kKeyMargin;
+        } else {  // midpoints closer than a bin: count them all
+#pragma unroll
+            for (int e = 0; e < 16; e++) {
+                const float y = (e & 1 ? Q[e >> 1].y : Q[e >> 1].x) * inv;
+                uint32_t idx = 0;
+#pragma unroll 1
+                for (int k = 0; k < 15; k++) {
+                    const float dm = y - 0.5f * (B.c[k] + B.c[k + 1]);
+                    idx += dm > 0.f ? 1u : 0u;
+                    near |= fabsf(dm) < kKeyMargin;
+                }
+                if (e < 8) kw0 |= idx << (4 * e);
+                else kw1 |= idx << (4 * (e - 8));
+            }
+        }
+        near = near && cur.in && cur.slot >= 0;
+
+        // ---- key: exact decisions when any decision of the warp is close
+        if (__any_sync(kFull, near)) {
+            // the elements whose fp32 decision lies within the margin (all of them
+            // when the fp32 scale is unusable)
+            uint32_t nm = 0;
+            if (near) {
+                if (wild) {
+                    nm = 0xffffu;
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; e++) {
+                        const float q = e & 1 ? Q[e >> 1].y : Q[e >> 1].x;
+                        bool nr = false;
+                        if (!B.dense) {
+                            const float x = fmaf(q, A, kBinMagic);
+                            const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
+                            nr = fabsf(fmaf(q, inv, -be.mid)) < kKeyMargin;
+                        } else {
+                            const float y = q * inv;
+#pragma unroll 1
+                            for (int k = 0; k < 15; k++) nr |= fabsf(y - 0.5f * (B.c[k] + B.c[k + 1])) < kKeyMargin;
+                        }
+                        nm |= (nr ? 1u : 0u) << e;
+                    }
+                }
+            }
+            // this lane's keys again (L1 hits: they came through L1 a pass ago) and
+            // the exact norm from their fp64 sum of squares
+            const uint16_t* kp = a.K + (size_t)(cur.in ? cur.vec : 0u) * D + sub * 16;
+            const uint4 ra = ld_nc_u4(kp), rb = ld_nc_u4(kp + 8);
+            const uint32_t w[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
+            double s0 = 0.0, s1 = 0.0;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const double x = (double)bf16_lo(w[j]), y = (double)bf16_hi(w[j]);
+                s0 = fma(x, x, s0);
+                s1 = fma(y, y, s1);
+            }
+            double ssd = s0 + s1;
+#pragma unroll
+            for (int m = 1; m < LPV; m <<= 1) ssd += __shfl_xor_sync(kFull, ssd, m);
+            const double nd = sqrt(ssd);
+            const double denom = nd * sqrt((double)D);  // y_e = (H k)_e / denom
+            if (near) n16 = __half_as_ushort(__double2half(nd));
+            if (near && ssd == 0.0) {
+                // an all-zero key: y = 0 exactly, every element takes the code of 0
+                uint32_t c0 = 0;
+                const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(kBinMagic) & 0x3f8u));
+                if (!B.dense) c0 = (uint32_t)be.k_hi - (0.f > be.mid ? 0u : 1u);
+                else
+                    for (int k = 0; k < 15; k++) c0 += 0.f > 0.5f * (B.c[k] + B.c[k + 1]) ? 1u : 0u;
+                kw0 = kw1 = c0 * 0x11111111u;
+                nm = 0;
+            }
+            const float rden = ssd > 0.0 ? (float)(1.0 / denom) : 0.f;
+            // one close element per vector per round: its row of the Hadamard sum,
+            // exact in fp64, decides it against midpoint * denom
+            const uint32_t gmask = ((1u << LPV) - 1u) << (grp * LPV);
+            while (__any_sync(kFull, nm != 0)) {
+                const uint32_t pend = __ballot_sync(kFull, nm != 0) & gmask;
+                const int owner = pend ? __ffs(pend) - 1 : lane;
+                const int mine = nm ? __ffs(nm) - 1 : 0;
+                const uint32_t r = (uint32_t)__shfl_sync(kFull, 16 * sub + mine, owner);
+                double part = 0.0;
+#pragma unroll
+                for (int e = 0; e < 16; e++) {
+                    const double x = (double)(e & 1 ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]));
+                    part += (__popc((r & 15u) & (uint32_t)e) & 1) ? -x : x;
+                }
+                if (__popc((r >> 4) & (uint32_t)sub) & 1) part = -part;
+#pragma unroll
+                for (int m = 1; m < LPV; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
+                if (pend && lane == owner) {
+                    uint32_t idx = 0;
+                    if (!B.dense) {
+                        const float x = fmaf((float)part * rden, kBinScale, kBinMagic);
+                        const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
+                        idx = (uint32_t)be.k_hi - (part > (double)be.mid * denom ? 0u : 1u);
+                    } else {
+#pragma unroll 1
+                        for (int k = 0; k < 15; k++)
+                            idx += part > 0.5 * ((double)B.c[k] + (double)B.c[k + 1]) * denom ? 1u : 0u;
+                    }
+                    const int sh = 4 * (mine & 7);
+                    if (mine < 8) kw0 = (kw0 & ~(0xfu << sh)) | (idx << sh);
+                    else kw1 = (kw1 & ~(0xfu << sh)) | (idx << sh);
+                    nm &= nm - 1u;
+                }
+            }
+        }
+
+        // the next pass's block-table entry: its slot has arrived by now, and the
+        // lookup overlaps this pass's value work and stores
+        fetch_block(a, nxt);
+
         // ---- where this vector goes (the block-table read was issued a pass ago)
-        int blk = -1, off = 0;
+        int blk = -1;
+        const int off = cur.slot & (kBlock - 1);  // table rows span whole blocks
         if (cur.in && cur.slot >= 0) {
             if (a.block_table) {
                 if (cur.pb >= 0 && cur.pb < a.num_blocks) {
                     blk = cur.pb;
-                    off = (int)(((uint32_t)cur.slot - fast_div((uint32_t)cur.slot, a.div_cap) * cap) %
-                                kBlock);
                 } else if (sub == 0) {
                     flag_status(a.status, cur.pb == -2 ? TQ_STATUS_BAD_SLOT : TQ_STATUS_BAD_BLOCK);
                 }
             } else if (cur.slot / kBlock < a.num_blocks) {
                 blk = cur.slot / kBlock;
-                off = cur.slot % kBlock;
             } else if (sub == 0) {
                 flag_status(a.status, TQ_STATUS_BAD_SLOT);
             }
         }
         if (blk >= 0) {
             unsigned char* rec = a.cache + ((size_t)blk * a.Hkv + h) * (size_t)R::kBytes;
-            *reinterpret_cast<uint32_t*>(rec + R::kKCodes + off * R::kCodeRow + sub * 4) = kw;
-            // bytes j = 4 sub + i share m = sub / 2 and spread over r = 4 (sub % 2) + i
-            unsigned char* vdst = rec + R::kVCodes + R::vcode_pos(off, 4 * sub);
+            *reinterpret_cast<uint2*>(rec + R::kKCodes + off * R::kCodeRow + sub * 8) =
+                make_uint2(kw0, kw1);
+            // code bytes j = 8 sub + r (r = 0..7) of this token: m = sub, chunk r
+            unsigned char* vdst = rec + R::kVCodes + R::vcode_pos(off, 8 * sub);
 #pragma unroll
-            for (int i = 0; i < 4; i++) vdst[i * R::kPairChunk] = (unsigned char)(vw >> (8 * i));
+            for (int r = 0; r < 4; r++) {
+                vdst[r * R::kPairChunk] = (unsigned char)(vw0 >> (8 * r));
+                vdst[(r + 4) * R::kPairChunk] = (unsigned char)(vw1 >> (8 * r));
+            }
             if (sub == 0) *reinterpret_cast<uint16_t*>(rec + R::kKNorm + off * 2) = n16;
-            if ((sub & 3) == 0) {
-                const int gp = R::group_pos(off, sub / 4);
-                *reinterpret_cast<uint16_t*>(rec + R::kVScale + gp) = s16;
-                *reinterpret_cast<uint16_t*>(rec + R::kVZero + gp) = __half_as_ushort(zh);
-                const bool bad = !isfinite(sf) || !isfinite(zf) ||
-                                 (sub == 0 && !isfinite(half_bits_to_float(n16)));
+            if ((sub & 1) == 0) {
+                const int gp = R::group_pos(off, sub / 2);
+                *reinterpret_cast<uint16_t*>(rec + R::kVScale + gp) = (uint16_t)sz;
+                *reinterpret_cast<uint16_t*>(rec + R::kVZero + gp) = (uint16_t)(sz >> 16);
+                const bool bad = vbad || (sub == 0 && !isfinite(half_bits_to_float(n16)));
                 if (bad) flag_status(a.status, TQ_STATUS_RANGE);
             }
         }
@@ -398,10 +512,9 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
     }
 }
 
-size_t append_smem_bytes(int Hkv) {
-    return (size_t)Hkv * sizeof(HeadBins) + (size_t)Hkv * kBins * sizeof(BinEntry);
+size_t append_smem_bytes(int ntab) {
+    return (size_t)ntab * kBins * sizeof(BinEntry) + (size_t)ntab * sizeof(HeadBins);
 }
-
 
 template <int D>
 static int resident_ctas(int num_sms, size_t smem) {
@@ -439,14 +552,14 @@ static void default_bins(int d, const uint16_t* table16, HeadBins& hb, BinEntry*
 cudaError_t launch_append(const AppendArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
     AppendArgs a = args;
     if (!a.k_tables) default_bins(head_dim, a.default_table, a.default_hb, a.default_bins);
-    a.div_hkv = div_magic((uint32_t)a.Hkv);
-    a.div_cap = div_magic((uint32_t)(a.max_blocks > 0 ? a.max_blocks * kBlock : 1));
+    a.dv_hkv = div32_magic((uint32_t)a.Hkv);
+    a.dv_cap = div32_magic((uint32_t)(a.max_blocks > 0 ? a.max_blocks * kBlock : 1));
     const int threads = 256;
     const long long vectors = (long long)a.T * a.Hkv;
-    const int vpw = 32 / (head_dim / 8);
+    const int vpw = 32 / (head_dim / 16);
     const long long warps_needed = (vectors + vpw - 1) / vpw;
     long long blocks = (warps_needed + threads / 32 - 1) / (threads / 32);
-    const size_t smem = append_smem_bytes(a.Hkv);
+    const size_t smem = append_smem_bytes(a.k_tables ? a.Hkv : 1);
     const long long cap = head_dim == 128 ? resident_ctas<128>(num_sms, smem)
                                           : resident_ctas<64>(num_sms, smem);
     if (blocks > cap) blocks = cap;  // one wave; warps loop over the passes

@@ -77,6 +77,22 @@ __device__ __forceinline__ uint32_t fast_div(uint32_t n, uint64_t M) {
 // the multiplier of fast_div for divisor d (0 for d == 1)
 inline uint64_t div_magic(uint32_t d) { return d <= 1 ? 0 : ~0ull / d + 1; }
 
+// n / d for n < 2^31 with one 32 x 32 -> 64-bit multiply: floor(n m / 2^s),
+// s = 31 + ceil(log2 d), m = ceil(2^s / d) < 2^32 (m d - 2^s < d <= 2^(s-31),
+// the round-up condition under which the quotient is exact for 31-bit n).
+struct Div32 {
+    uint32_t m, s;
+};
+__device__ __forceinline__ uint32_t fast_div32(uint32_t n, Div32 d) {
+    return (uint32_t)(((uint64_t)n * d.m) >> d.s);
+}
+inline Div32 div32_magic(uint32_t d) {
+    uint32_t l = 0;
+    while ((1ull << l) < d) l++;
+    const uint32_t s = 31 + l;
+    return Div32{(uint32_t)(((1ull << s) + d - 1) / d), s};
+}
+
 __device__ __forceinline__ void flag_status(int32_t* status, int bits) {
     if (status) atomicOr(status, bits);
 }

@@ -8,37 +8,45 @@
 
 namespace tq {
 
-// ---- key binning of the append: uniform bins over y in [-1, 1] (a unit
-// vector's rotated coordinates), width 1/64, bin = (int)(64 y + 64) in [0, 128]
-constexpr int kBins = 129;
-constexpr float kBinScale = 64.0f;
+// ---- key binning of the append.  A rotated unit-vector coordinate y in
+// [-1, 1] is mapped to x = S y + S + 1 (S = kBinScale) and rounded to 1/8 by
+// one fma against kBinMagic = 2^20 + S + 1 (floats in [2^20, 2^21) are spaced
+// 1/8 apart); bits 3-9 of the result are then bin * 8 with bin = floor(x) mod
+// 128, in [0, 127] for |y| <= 1.  Bin b is taken to cover x in
+// [b - 1/8, b + 1 + 1/8] (the rounding to 1/8 and the fp32 error of x stay
+// inside that slack), widened further by 2 kKeyMargin in y.
+constexpr int kBins = 128;
+constexpr float kBinScale = 63.0f;
+constexpr float kBinMagic = 1048576.0f + kBinScale + 1.0f;
 // Absolute margin, in rotated unit-vector units, inside which an fp32
-// centroid decision is re-taken in fp64.  The fp32 butterfly of a bf16 key
-// followed by one scaling is accurate to ~1.3e-6 in the worst case
-// (7 stages, rsqrt within 2 ulp); typical errors are ~1e-7.
-constexpr float kKeyMargin = 3.0e-6f;
+// centroid decision is re-taken exactly.  The fp32 butterfly of a bf16 key
+// (L <= 7 rounding stages; stage s adds rounding errors of 2-norm at most
+// 2^-24 of its output, and the later stages scale them with the vector)
+// errs by at most L 2^-24 in unit-vector units, and the normalisation by at
+// most 10 ulp of |y| <= 1, so the fast path's y is within 17 ulp (1.0e-6) of
+// the exact one; the margin is twice that.
+constexpr float kKeyMargin = 2.0e-6f;
 
 struct HeadBins {
     float c[16];  // the head's table
     int dense;    // 1: some bin holds more than one midpoint -> exact count path
-    int pad;      // keeps the BinEntry array that follows 8-byte aligned
+    int pad;
 };
 struct __align__(8) BinEntry {
     float mid;  // the one midpoint inside the bin (with margins), or +inf
-    int k_lo;   // number of midpoints strictly below the bin
+    int k_hi;   // 1 + the number of midpoints strictly below the bin
 };
 
 // One bin of a strictly ascending 16-entry table c: the midpoints below the
-// bin's range widened by 2 kKeyMargin on each side are counted by a binary
-// search (the midpoints ascend too), and the one or more inside it follow.
-// Returns true when more than one midpoint falls inside (the exact count path).
-// The host (default table) and the device (per-head tables) both use it; the
-// margins make the result insensitive to their float contraction differing.
+// bin's widened range are counted by a binary search (the midpoints ascend
+// too), and the one or more inside it follow.  Returns true when more than
+// one midpoint falls inside (the exact count path).  The host (default table)
+// and the device (per-head tables) both use it; the margins make the result
+// insensitive to their float contraction differing.
 __host__ __device__ inline bool bin_entry(const float* c, int bin, BinEntry& e) {
     const float delta = 2.0f * kKeyMargin;
-    const float w = 1.0f / kBinScale;
-    const float ext_lo = -1.0f + bin * w - delta;
-    const float ext_hi = -1.0f + (bin + 1) * w + delta;
+    const float ext_lo = ((float)bin - 1.125f - kBinScale) / kBinScale - delta;
+    const float ext_hi = ((float)bin + 0.125f - kBinScale) / kBinScale + delta;
     int below = 0;  // #{k < 15 : m_k < ext_lo}, m_k = (c_k + c_k+1) / 2 (exact: fp16 values)
     for (int step = 8; step >= 1; step >>= 1) {
         const int k = below + step - 1;
@@ -53,7 +61,7 @@ __host__ __device__ inline bool bin_entry(const float* c, int bin, BinEntry& e) 
         m_in = m;
     }
     e.mid = m_in;
-    e.k_lo = below;
+    e.k_hi = below + 1;
     return inside > 1;
 }
 
@@ -69,7 +77,7 @@ struct AppendArgs {
     const uint16_t* k_tables;   // fp16 [Hkv][16] or null
     uint16_t default_table[16]; // fp16
     int32_t* status;
-    uint64_t div_hkv, div_cap;  // fast-division multipliers (set by the launcher)
+    Div32 dv_hkv, dv_cap;       // division by H_kv and by max_blocks * 16 (set by the launcher)
     HeadBins default_hb;        // bins of default_table (set by the launcher)
     BinEntry default_bins[kBins];
 };
@@ -115,7 +123,7 @@ struct DequantArgs {
     int32_t* status;
 };
 
-size_t append_smem_bytes(int Hkv);
+size_t append_smem_bytes(int ntab);  // ntab bin tables (1, or H_kv per-head tables)
 int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int head_dim, int num_sms, cudaStream_t stream);
