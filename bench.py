@@ -301,6 +301,124 @@ def cfg(w, l2):
             "global_batch": w.B, "seq_len": int(w.seq_lens[0]), "l2": l2}
 
 
+# ---------------------------------------------------------------- the other workloads
+def other_workloads(dev, peak, reps: int = 20) -> dict:
+    """Per-call CUDA-event timings (median of `reps`) of the scope table's other
+    measured workloads, each on its own cache; L2 is flushed before every timed
+    call by reading a 512 MB buffer (the prefill chunk and its cache fit in L2).
+
+    long_context: decode over 4 x 131072 tokens with 64 splits per item (and the
+    even cut); agentic: decode over the shared-prefix batch with calibrated
+    per-head tables, as logical bytes (what the sequences attend over) and unique
+    bytes (distinct records); prefill_small_head: one 2048-token chunk appended to
+    every sequence, and decode at context 32768."""
+    import bit_rotated_kv_tq_b200 as tq
+
+    flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def timed(fn):
+        ts = []
+        for i in range(reps + 2):
+            flush.sum()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    def build(w, tables=None):
+        cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
+        bt = torch.from_numpy(w.block_tables).to(dev)
+        for K, V, slots in w.population():
+            tq.quantize_append(K.to(dev), V.to(dev), slots.to(dev), cache, block_table=bt,
+                               k_tables=tables, status=status)
+        return cache, bt
+
+    def decode(w, cache, bt, S, tables=None):
+        lens = torch.from_numpy(w.seq_lens).to(dev)
+        q = w.q().to(dev)
+        max_len = int(w.seq_lens.max())
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(16, tq.workspace_bytes(w.B, w.Hq, w.d, S)), dtype=torch.uint8, device=dev)
+        return timed(lambda: tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out,
+                                                 workspace=ws, num_splits=S, k_tables=tables,
+                                                 status=status))
+
+    res = {}
+    w = W.make("long_context")
+    cache, bt = build(w)
+    kv = decode_kv_bytes(w)
+    for S in (64, 0):
+        ms = decode(w, cache, bt, S)
+        res[f"long_context_decode_s{S}"] = {"ms": ms, "gbs": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / peak}
+    del cache
+
+    w = W.make("agentic")
+    keys = w.calibration_keys(20)
+    init = tq.lloyd_max_table(w.d)
+    tables = torch.from_numpy(np.stack([tq.fit_k_table(keys[h], init, 100)[0] for h in range(w.Hkv)])).to(dev)
+    cache, bt = build(w, tables)
+    ms = decode(w, cache, bt, 0, tables)
+    rec = tq.record_bytes(w.d)
+    logical = decode_kv_bytes(w)
+    nblk = (w.seq_lens + 15) // 16
+    used = np.unique(np.concatenate([w.block_tables[b, :nblk[b]] for b in range(w.B)]))
+    unique = int(used.size) * w.Hkv * rec
+    res["agentic_decode"] = {"ms": ms, "logical_gbs": logical / ms / 1e6, "unique_gbs": unique / ms / 1e6,
+                             "unique_hbm_frac": unique / ms / 1e6 / peak,
+                             "logical_mb": logical / 1e6, "unique_mb": unique / 1e6}
+    del cache
+
+    w = W.make("prefill_small_head")
+    cache, bt = build(w)
+    cap = w.max_blocks * 16
+    parts = [w.kv(b, 0, 2048) for b in range(w.B)]
+    K = torch.cat([p[0] for p in parts]).to(dev)
+    V = torch.cat([p[1] for p in parts]).to(dev)
+    slots = torch.cat([torch.arange(0, 2048, dtype=torch.int32) + b * cap for b in range(w.B)]).to(dev)
+    T = K.shape[0]
+    ms = timed(lambda: tq.quantize_append(K, V, slots, cache, block_table=bt, status=status))
+    ab = append_bytes(w, T)
+    res["prefill_chunk_append"] = {"ms": ms, "tokens": T, "tokens_per_s": T / ms * 1e3,
+                                   "gbs": ab / ms / 1e6, "hbm_frac": ab / ms / 1e6 / peak}
+    kv = decode_kv_bytes(w)
+    ms = decode(w, cache, bt, 0)
+    res["prefill_small_head_decode"] = {"ms": ms, "gbs": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / peak}
+    del cache
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0, f"device status {int(status.item())}"
+    return res
+
+
+def prefill_append_case(dev):
+    """One 2048-token chunk appended to each of the 16 sequences of
+    prefill_small_head (d 64, 2 kv heads), 3 warm-up calls then 1: the small,
+    self-contained case the append kernel is profiled on."""
+    import bit_rotated_kv_tq_b200 as tq
+
+    tq.load()
+    w = W.make("prefill_small_head")
+    cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    cap = w.max_blocks * 16
+    parts = [w.kv(b, 0, 2048) for b in range(w.B)]
+    K = torch.cat([p[0] for p in parts]).to(dev)
+    V = torch.cat([p[1] for p in parts]).to(dev)
+    slots = torch.cat([torch.arange(0, 2048, dtype=torch.int32) + b * cap for b in range(w.B)]).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(4):
+        flush.sum()
+        tq.quantize_append(K, V, slots, cache, block_table=bt, status=status)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0
+    print(json.dumps({"case": "prefill_append", "tokens": K.shape[0], "ok": True}))
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_tq(args, rank, world, local):
     import bit_rotated_kv_tq_b200 as tq
@@ -496,6 +614,10 @@ def run_tq(args, rank, world, local):
                "sample": f"1 of {w.B} sequences (8 kv heads x {s['L']} tokens + {w.append_tokens}-token append), "
                          f"{n_rep} passes, {dt:.2f} s each"}
 
+    others = None
+    if rank == 0 and world == 1 and not args.no_workloads:
+        others = other_workloads(dev, peak)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -520,6 +642,8 @@ def run_tq(args, rank, world, local):
             "clocks": clocks,
             "cpu_baseline": cpu,
         }
+        if others is not None:
+            line["workloads"] = others
         print(json.dumps(line), flush=True)
 
 
@@ -530,6 +654,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["prefill_append"], default=None,
+                    help="run one small profiling case instead of the bench")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the long-context, agentic and prefill-chunk measurements")
     ap.add_argument("--batch", type=int, default=0,
                     help="sequences per rank (default: the workload's 32); smaller values make the "
                          "profiling case, not a bench line")
@@ -538,6 +666,9 @@ def main():
         rank = int(os.environ.get("RANK", 0))
         world = int(os.environ.get("WORLD_SIZE", args.gpus))
         run_reference(args, rank, world)
+        return
+    if args.case == "prefill_append":
+        prefill_append_case(torch.device("cuda", 0))
         return
     rank, world, local = dist_setup(args.gpus)
     try:
