@@ -32,7 +32,8 @@
 // of the decision threshold: the fp16 rounding of the norm and the nearest
 // centroid in fp64 from the bf16 inputs (exact +-1 Hadamard sums, compared
 // against midpoint * n * sqrt(D)), the value codes by comparing v - z with
-// (k + 1/2) s in fp64, and the fp16 rounding up of the scale in fp64.  The
+// (k + 1/2) s in fp64, and the fp16 rounding up of the scale by an exact fp32
+// comparison of 15 s with max - z (fp64 when max - z is inexact in fp32).  The
 // stored codes are therefore those of the exact-arithmetic definition except
 // within ~1e-15 (relative) of a key threshold.
 #include "tq_kernels.cuh"
@@ -43,9 +44,9 @@ namespace tq {
 // of the fast path's norm (fp32 sum of exact squares along a tree of depth
 // <= 8, then ss * rsqrt with one Newton step: <= 9 ulp).
 constexpr float kNormMargin = 1.1e-6f;
-// Margin, in value-code units, around the .5 rounding points of (v - z)/s
-// (v - z and 1/s are each correctly rounded and the product is fused with
-// the rounding, so the fp32 quotient errs by at most ~2^-19 code units).
+// Margin, in value-code units, around the .5 rounding points of (v - z)/s:
+// the fp32 residual v - z - t s errs by at most 16 ulp of s (v - z rounded
+// once, the fused residual once), far inside 2^-16.
 constexpr float kValueMargin = 1.0f / 65536.0f;
 
 // Bin tables in shared memory (called by the whole CTA): the tables sit at
@@ -78,8 +79,7 @@ __device__ __forceinline__ float rsqrt_approx(float x) {  // x normal and positi
     return y;
 }
 
-// fp32 neighbours of 1/15: the value rounded up and rounded down.
-__device__ __forceinline__ float inv15_up() { return __uint_as_float(0x3d888889u); }
+// 1/15 rounded down to fp32
 __device__ __forceinline__ float inv15_dn() { return __uint_as_float(0x3d888888u); }
 
 // 16-byte read-only load that allocates in L1: a lane's two loads cover one
@@ -229,12 +229,18 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         // the answer, otherwise (an fp16 value inside the bracket) use fp64.
         uint16_t s16;
         {
-            const float hi = __fmul_ru(__fsub_ru(mx, zf), inv15_up());
-            const float lo = __fmul_rd(__fsub_rd(mx, zf), inv15_dn());
-            const uint16_t s_hi = __half_as_ushort(__float2half_ru(hi));
-            const uint16_t s_lo = __half_as_ushort(__float2half_ru(lo));
-            s16 = s_hi;
-            if (s_hi != s_lo) s16 = double_to_half_up_nonneg(((double)mx - (double)zf) / 15.0);
+            // s = fp16 rounded up from D / 15, D = max - z.  c, the smallest fp16 at or
+            // above a lower bound of D / 15 within one fp16 step of it, is s unless
+            // 15 c < D, and then s is the next fp16.  15 c is exact in fp32, and so is
+            // D when its two directed roundings agree (otherwise fp64 decides).
+            // (+0 in round-to-nearest turns the -0 that max - max gives toward -inf into +0)
+            const float Dd = __fsub_rd(mx, zf), Du = __fsub_ru(mx, zf);
+            const float lo = __fadd_rn(__fmul_rd(Dd, inv15_dn()), 0.0f);
+            const uint16_t c16 = __half_as_ushort(__float2half_ru(lo));
+            if (Dd == Du)
+                s16 = (uint16_t)(c16 + (half_bits_to_float(c16) * 15.f < Dd ? 1u : 0u));
+            else
+                s16 = double_to_half_up_nonneg(((double)mx - (double)zf) / 15.0);
         }
         const float sf = half_bits_to_float(s16);
         const bool vbad = !isfinite(sf) || !isfinite(zf);
@@ -242,37 +248,43 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         uint32_t vw0 = 0, vw1 = 0;  // code bytes of elements 0-7, 8-15
         if (sf > 0.f) {
             const float is = __frcp_rn(sf);
-            const float2 z2 = make_float2(zf, zf), is2 = make_float2(is, is);
+            const float2 z2 = make_float2(zf, zf), is2 = make_float2(is, is), s2 = make_float2(sf, sf);
             const float2 rnd = make_float2(kRound, kRound);
-            float dmax = 0.f;
+            float emax = 0.f;
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 const float2 vz = sub2(make_float2(bf16_lo(vwd[j]), bf16_hi(vwd[j])), z2);
                 const float2 tr = __ffma2_rn(vz, is2, rnd);  // kRound + round-half-even(r)
-                const float2 ti = sub2(tr, rnd);             // that integer, exact
-                const float2 d = __ffma2_rn(vz, is2, make_float2(-ti.x, -ti.y));  // r - ti
-                dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+                const float2 nti = sub2(rnd, tr);            // minus that integer t, exact
+                const float2 e = __ffma2_rn(nti, s2, vz);    // v - z - t s
+                emax = fmaxf(emax, fmaxf(fabsf(e.x), fabsf(e.y)));
                 // the codes are the low bytes of tr
                 const uint32_t byte = (__float_as_uint(tr.x) + (__float_as_uint(tr.y) << 4)) & 0xffu;
                 if (j < 4) vw0 |= byte << (8 * j);
                 else vw1 |= byte << (8 * (j - 4));
             }
-            if (dmax > 0.5f - kValueMargin) {
-                // a .5 point within the fp32 error: decide every element exactly by
-                // comparing v - z with (k + 1/2) s in fp64 (both exact there), k the
-                // integer below the fp32 quotient, ties to even
-                vw0 = vw1 = 0;
+            // |v - z - t s| >= s / 2 (less the fp32 error of v - z, <= 16 ulp of s)
+            // marks an exact .5 tie, or a quotient whose fp32 rounding may be on the
+            // wrong side of a .5 point: that element is decided exactly by comparing
+            // v - z with (k + 1/2) s in fp64, k the integer below, ties to even
+            const float thr = (0.5f - kValueMargin) * sf;
+            if (emax >= thr) {
 #pragma unroll
                 for (int e = 0; e < 16; e++) {
                     const float vf = e & 1 ? bf16_hi(vwd[e >> 1]) : bf16_lo(vwd[e >> 1]);
-                    const float k = floorf((vf - zf) * is);
-                    const double v = (double)vf - (double)zf;
-                    const double bnd = ((double)k + 0.5) * (double)sf;
-                    const int ki = (int)k;
-                    const int q = v > bnd ? ki + 1 : (v < bnd ? ki : ki + (ki & 1));
-                    const uint32_t c = (uint32_t)min(max(q, 0), 15);
-                    if (e < 8) vw0 |= c << (4 * e);
-                    else vw1 |= c << (4 * (e - 8));
+                    const float vz = vf - zf;
+                    const float tr = fmaf(vz, is, kRound);
+                    if (fabsf(fmaf(kRound - tr, sf, vz)) >= thr) {
+                        const float k = floorf(vz * is);
+                        const double v = (double)vf - (double)zf;
+                        const double bnd = ((double)k + 0.5) * (double)sf;
+                        const int ki = (int)k;
+                        const int q = v > bnd ? ki + 1 : (v < bnd ? ki : ki + (ki & 1));
+                        const uint32_t c = (uint32_t)min(max(q, 0), 15);
+                        const int sh = 4 * (e & 7);
+                        if (e < 8) vw0 = (vw0 & ~(0xfu << sh)) | (c << sh);
+                        else vw1 = (vw1 & ~(0xfu << sh)) | (c << sh);
+                    }
                 }
             }
         }

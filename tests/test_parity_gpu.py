@@ -253,9 +253,11 @@ def test_bad_block_and_slot_set_status(tq):
     assert int(st.item()) & tq.STATUS_BAD_LEN
 
 
-def test_value_and_key_edge_data(tq, orc):
-    """Zero keys, constant and integer-valued value groups (exact .5 ties), huge ranges."""
-    d, H = 128, 2
+@pytest.mark.parametrize("d", [64, 128])
+def test_value_and_key_edge_data(tq, orc, d):
+    """Zero keys, constant and integer-valued value groups (exact .5 ties), huge ranges,
+    groups whose (max - z)/15 is an fp16 value, and groups whose max - z is inexact in fp32."""
+    H = 2
     T = 64
     rng = np.random.default_rng(5)
     K = rng.standard_normal((T, H, d)).astype(np.float32)
@@ -265,10 +267,15 @@ def test_value_and_key_edge_data(tq, orc):
     K[1, :, 0] = K[1, :, 1] = 1.0                 # exact zeros after rotation
     V[2] = 3.25                                   # constant group
     V[3] = np.round(rng.uniform(-8, 8, (H, d)))   # integers: exact .5 ties
-    V[4] = np.tile(np.arange(32, dtype=np.float32), (H, 4))
+    V[4] = np.tile(np.arange(32, dtype=np.float32), (H, d // 32))
     V[5] *= 1000.0
     V[5, :, 7] = 1e-3                             # wide dynamic range in one group
     K[6] *= 1e-20                                 # tiny norm
+    # z = -1, max - z = 1.875 = 15 * 0.125 (s exact in fp16), every other value on a .5 point
+    V[7] = np.tile(-1.0 + 0.0625 * np.minimum(np.arange(32), 30), (H, d // 32))
+    V[8] = rng.uniform(0.0, 1.0, (H, d))
+    V[8, :, ::32] = 524288.0                      # max - z needs 29 bits: inexact in fp32
+    V[8, :, 1::32] = 2.0 ** -10
     Kt = torch.from_numpy(K).to(torch.bfloat16)
     Vt = torch.from_numpy(V).to(torch.bfloat16)
     cache = tq.Cache(4, H, d)
@@ -278,7 +285,20 @@ def test_value_and_key_edge_data(tq, orc):
     rc, ky, vr = orc.quantize_append(bf16_bits(Kt), bf16_bits(Vt), np.arange(T, dtype=np.int32), ocache,
                                      want_aux=True)
     assert rc == 0
-    assert np.array_equal(cache.data.cpu().numpy(), ocache)
+    got = cache.data.cpu().numpy()
+    if not np.array_equal(got, ocache):
+        msgs = []
+        for blk in range(4):
+            for h in range(H):
+                a = unpack_record(got[blk, h], d)
+                b = unpack_record(ocache[blk, h], d)
+                for name, x, y in zip(("kidx", "knorm", "vq", "vs", "vz"), a, b):
+                    bad = np.argwhere(x != y)
+                    if bad.size:
+                        t0 = tuple(bad[0])
+                        msgs.append(f"blk {blk} head {h} {name}: {len(bad)} differ, first at {t0}: "
+                                    f"gpu {x[t0]} oracle {y[t0]}")
+        raise AssertionError("records differ:\n" + "\n".join(msgs[:12]))
 
 
 # ---------------------------------------------------------------- full size, sampled
