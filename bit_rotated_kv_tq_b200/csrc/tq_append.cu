@@ -15,9 +15,9 @@
 // vectors, 1 KB of keys and 1 KB of values.  The grid is persistent (one wave
 // of resident CTAs); warp w takes passes w, w + W, w + 2W, ... (W warps in
 // all).  Every warp keeps its next kPrefetch passes requested into L2 with
-// bulk prefetches and loads its next pass into registers while it computes
-// the current one, so HBM sees the whole input stream early and the register
-// loads hit L2.  The rotation is an in-register butterfly over the 4 index
+// bulk prefetches, so HBM sees the whole input stream early; it loads its
+// next pass into registers after the current pass's key work and before its
+// stores, and looks up the pass's physical block at the top of the pass.  The rotation is an in-register butterfly over the 4 index
 // bits inside a lane plus xor-shuffles over the lane bits.
 //
 // Nearest centroid: x = 63 y + 64 is rounded to 1/8 by one fma against a
@@ -117,7 +117,7 @@ __device__ __forceinline__ void prefetch_pass(const AppendArgs& a, uint32_t p, u
     prefetch_l2_bulk(a.V + (size_t)v0 * D, nv * D * 2);
 }
 
-// One warp pass's inputs (loaded one pass ahead).
+// One warp pass's inputs (loaded during the pass before).
 struct Pass {
     uint4 k0, k1, v0, v1;  // this lane's 16 bf16 keys / values
     int slot;              // slot_mapping entry of the token (-1: skip)
@@ -145,8 +145,8 @@ __device__ __forceinline__ void load_pass(const AppendArgs& a, uint32_t p, uint3
     }
 }
 
-// With a block table, fetch the physical block of the pass's slot (issued one
-// pass before it is used).
+// With a block table, fetch the physical block of the pass's slot (issued at
+// the top of the pass, used by its stores at the end).
 __device__ __forceinline__ void fetch_block(const AppendArgs& a, Pass& L) {
     if (a.block_table && L.in && L.slot >= 0) {
         const uint32_t s = (uint32_t)L.slot;
@@ -193,11 +193,10 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
     Pass cur, nxt;
     load_pass<D>(a, pass, npass, total, grp, sub, cur);
     build_bins(hb, bins, a);
-    fetch_block(a, cur);
 
     for (; pass < npass; pass += nwarps) {
+        fetch_block(a, cur);  // its slot was loaded with the pass's inputs
         if (lane == 0) prefetch_pass<D>(a, pass + (uint32_t)kPrefetch * nwarps, npass, total);
-        load_pass<D>(a, pass + nwarps, npass, total, grp, sub, nxt);
         const uint32_t t = fast_div32(cur.vec, a.dv_hkv);
         const int h = cur.in ? (int)(cur.vec - t * (uint32_t)a.Hkv) : 0;
 
@@ -479,11 +478,11 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
             }
         }
 
-        // the next pass's block-table entry: its slot has arrived by now, and the
-        // lookup overlaps this pass's value work and stores
-        fetch_block(a, nxt);
+        // the next pass's inputs, issued after the key work so that they do not hold
+        // registers through it (they are L2 hits: prefetched passes ago)
+        load_pass<D>(a, pass + nwarps, npass, total, grp, sub, nxt);
 
-        // ---- where this vector goes (the block-table read was issued a pass ago)
+        // ---- where this vector goes (the block-table read was issued at the top)
         int blk = -1;
         const int off = cur.slot & (kBlock - 1);  // table rows span whole blocks
         if (cur.in && cur.slot >= 0) {
