@@ -78,6 +78,16 @@ __device__ __forceinline__ float rsqrt_approx(float x) {  // x normal and positi
     asm("rsqrt.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+__device__ __forceinline__ float rcp_approx(float x) {  // x normal
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// four bytes (the low byte of each argument) into one word
+__device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2, uint32_t b3) {
+    return __byte_perm(__byte_perm(b0, b1, 0x0040), __byte_perm(b2, b3, 0x0040), 0x5410);
+}
 
 // 1/15 rounded down to fp32
 __device__ __forceinline__ float inv15_dn() { return __uint_as_float(0x3d888888u); }
@@ -246,10 +256,14 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         const uint32_t sz = (uint32_t)s16 | ((uint32_t)__half_as_ushort(zh) << 16);  // scale, zero
         uint32_t vw0 = 0, vw1 = 0;  // code bytes of elements 0-7, 8-15
         if (sf > 0.f) {
-            const float is = __frcp_rn(sf);
+            // 1/s to ~1 ulp (approximation and one Newton step): it only picks the
+            // candidate code, whose exact residual is checked below
+            const float is0 = rcp_approx(sf);
+            const float is = fmaf(is0, fmaf(-sf, is0, 1.0f), is0);
             const float2 z2 = make_float2(zf, zf), is2 = make_float2(is, is), s2 = make_float2(sf, sf);
             const float2 rnd = make_float2(kRound, kRound);
             float emax = 0.f;
+            uint32_t by[8];
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 const float2 vz = sub2(make_float2(bf16_lo(vwd[j]), bf16_hi(vwd[j])), z2);
@@ -258,10 +272,10 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
                 const float2 e = __ffma2_rn(nti, s2, vz);    // v - z - t s
                 emax = fmaxf(emax, fmaxf(fabsf(e.x), fabsf(e.y)));
                 // the codes are the low bytes of tr
-                const uint32_t byte = (__float_as_uint(tr.x) + (__float_as_uint(tr.y) << 4)) & 0xffu;
-                if (j < 4) vw0 |= byte << (8 * j);
-                else vw1 |= byte << (8 * (j - 4));
+                by[j] = __float_as_uint(tr.x) + (__float_as_uint(tr.y) << 4);
             }
+            vw0 = pack4(by[0], by[1], by[2], by[3]);
+            vw1 = pack4(by[4], by[5], by[6], by[7]);
             // |v - z - t s| >= s / 2 (less the fp32 error of v - z, <= 16 ulp of s)
             // marks an exact .5 tie, or a quotient whose fp32 rounding may be on the
             // wrong side of a .5 point: that element is decided exactly by comparing
@@ -336,12 +350,12 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         const float rs = rs0 * fmaf(-0.5f * ssc * rs0, rs0, 1.5f);
         const float n = ss * rs;
         uint16_t n16 = __half_as_ushort(__float2half_rn(n));
-        bool near = __half_as_ushort(__float2half_rn(n * (1.0f - kNormMargin))) !=
-                    __half_as_ushort(__float2half_rn(n * (1.0f + kNormMargin)));
+        const bool nnorm = __half_as_ushort(__float2half_rn(n * (1.0f - kNormMargin))) !=
+                           __half_as_ushort(__float2half_rn(n * (1.0f + kNormMargin)));
         // squares that leave the normal fp32 range (or a non-finite key) lose the
         // fp32 error bound: every decision is re-taken (an all-zero key stays here)
         const bool wild = !(ss >= 1e-30f && ss <= 1e30f) && (kor & 0x7fff7fffu) != 0u;
-        near |= wild;
+        bool nkey = wild;  // some centroid decision is close (all of them when wild)
         const float inv = rs * inv_sqrt_d;              // 1 / (n sqrt(D))
         const float A = rs * (inv_sqrt_d * kBinScale);  // kBinScale / (n sqrt(D))
 
@@ -353,6 +367,7 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         if (!B.dense) {
             const float2 A2 = make_float2(A, A), M2 = make_float2(kBinMagic, kBinMagic);
             float dmin = INFINITY;
+            uint32_t by[8];
 #pragma unroll
             for (int j = 0; j < 8; j++) {
                 const float2 x = __ffma2_rn(Q[j], A2, M2);
@@ -365,11 +380,11 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
                 // k_hi - 1 where y <= mid (sign bit set; y == mid is near anyway)
                 const uint32_t c0 = (uint32_t)(e0.k_hi + (__float_as_int(d0) >> 31));
                 const uint32_t c1 = (uint32_t)(e1.k_hi + (__float_as_int(d1) >> 31));
-                const uint32_t byte = c0 | (c1 << 4);
-                if (j < 4) kw0 |= byte << (8 * j);
-                else kw1 |= byte << (8 * (j - 4));
+                by[j] = c0 | (c1 << 4);
             }
-            near |= dmin < kKeyMargin;
+            kw0 = pack4(by[0], by[1], by[2], by[3]);
+            kw1 = pack4(by[4], by[5], by[6], by[7]);
+            nkey |= dmin < kKeyMargin;
         } else {  // midpoints closer than a bin: count them all
 #pragma unroll
             for (int e = 0; e < 16; e++) {
@@ -379,13 +394,14 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
                 for (int k = 0; k < 15; k++) {
                     const float dm = y - 0.5f * (B.c[k] + B.c[k + 1]);
                     idx += dm > 0.f ? 1u : 0u;
-                    near |= fabsf(dm) < kKeyMargin;
+                    nkey |= fabsf(dm) < kKeyMargin;
                 }
                 if (e < 8) kw0 |= idx << (4 * e);
                 else kw1 |= idx << (4 * (e - 8));
             }
         }
-        near = near && cur.in && cur.slot >= 0;
+        nkey = nkey && cur.in && cur.slot >= 0;
+        const bool near = nkey || (nnorm && cur.in && cur.slot >= 0);
 
         // ---- key: exact decisions when any decision of the warp is close
         if (__any_sync(kFull, near)) {
@@ -441,7 +457,10 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
                 kw0 = kw1 = c0 * 0x11111111u;
                 nm = 0;
             }
-            const float rden = ssd > 0.0 ? (float)(1.0 / denom) : 0.f;
+            // 1 / denom, only to pick a bin: the fast path's fp32 scale, or from the
+            // exact norm when that scale is unusable
+            float rden = inv;
+            if (wild) rden = ssd > 0.0 ? (float)(1.0 / denom) : 0.f;
             // one close element per vector per round: its row of the Hadamard sum,
             // exact in fp64, decides it against midpoint * denom
             const uint32_t gmask = ((1u << LPV) - 1u) << (grp * LPV);
