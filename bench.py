@@ -419,6 +419,33 @@ def prefill_append_case(dev):
     print(json.dumps({"case": "prefill_append", "tokens": K.shape[0], "ok": True}))
 
 
+def prefill_decode_case(dev):
+    """Decode over the prefill_small_head cache (16 x 32768 tokens, 16 q / 2 kv
+    heads, d 64), 3 warm-up calls then 1, L2 flushed before each: the case the
+    d 64 decode kernel is profiled on."""
+    import bit_rotated_kv_tq_b200 as tq
+
+    tq.load()
+    w = W.make("prefill_small_head")
+    cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for K, V, slots in w.population():
+        tq.quantize_append(K.to(dev), V.to(dev), slots.to(dev), cache, block_table=bt, status=status)
+    lens = torch.from_numpy(w.seq_lens).to(dev)
+    q = w.q().to(dev)
+    max_len = int(w.seq_lens.max())
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, tq.workspace_bytes(w.B, w.Hq, w.d, 0)), dtype=torch.uint8, device=dev)
+    flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(4):
+        flush.sum()
+        tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out, workspace=ws, status=status)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0
+    print(json.dumps({"case": "prefill_decode", "ok": True}))
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_tq(args, rank, world, local):
     import bit_rotated_kv_tq_b200 as tq
@@ -654,7 +681,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["prefill_append"], default=None,
+    ap.add_argument("--case", choices=["prefill_append", "prefill_decode"], default=None,
                     help="run one small profiling case instead of the bench")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the long-context, agentic and prefill-chunk measurements")
@@ -669,6 +696,9 @@ def main():
         return
     if args.case == "prefill_append":
         prefill_append_case(torch.device("cuda", 0))
+        return
+    if args.case == "prefill_decode":
+        prefill_decode_case(torch.device("cuda", 0))
         return
     rank, world, local = dist_setup(args.gpus)
     try:

@@ -273,11 +273,16 @@ TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len) {
 
 TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_splits) {
     if (B <= 0 || H_q <= 0 || !supported_d(head_dim) || num_splits == 1 || num_splits < 0) return 0;
-    // ranges: at most two per SM half-pair with the even cut, else at most
-    // items * S + 1 with items <= B * H_q
+    // Even cut: at most two ranges per SM (one per half), each with partials of
+    // up to 8 heads per item at d = 64 (two groups of four) and 4 at d = 128.
+    // S splits: at most items * S + 1 ranges, and items * (heads per item) is at
+    // most B * H_kv * (G + 3) with 4 heads per item, B * H_kv * (G + 7) with 8
+    // (only when G > 4); both leave items * S * heads + heads within
+    // 4 (B * H_q * S + 1) head partials
     const long long ranges =
         num_splits == 0 ? 2LL * device_sms() : (long long)B * H_q * num_splits + 1;
-    return (size_t)ranges * 2 * 4 * ((size_t)head_dim * sizeof(float) + sizeof(float2));
+    const long long heads = num_splits == 0 && head_dim == 64 ? 8 : 4;
+    return (size_t)ranges * 2 * heads * ((size_t)head_dim * sizeof(float) + sizeof(float2));
 }
 
 TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
@@ -324,7 +329,7 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
     a.out = out;
     a.num_splits = num_splits;
     a.max_seq_len = max_seq_len;
-    if (!tq::decode_plan(a, device_sms()))
+    if (!tq::decode_plan(a, d, device_sms()))
         return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * num_splits too large");
     const size_t need = tq::decode_workspace_for(a, d);
     if (need) {
@@ -335,8 +340,9 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
             return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: workspace must be 16-byte aligned");
     }
     a.ws_o = static_cast<float*>(workspace);
+    // [ranges][2][heads per item][d] partial outputs, then [ranges][2][heads per item] (m, l)
     a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
-                                               (size_t)a.nranges * 2 * 4 * d)
+                                               (size_t)a.nranges * 2 * 4 * a.qpi * d)
                    : nullptr;
     a.status = status;
     cudaError_t e = tq::launch_decode(a, d, device_sms(), (cudaStream_t)stream);

@@ -43,7 +43,7 @@ constexpr int kHalves = 2;               // independent halves per CTA
 constexpr int kWarps = kNW * kHalves;    // 16 warps, 512 threads
 constexpr int kStages = 3;               // records in flight per warp
 constexpr int kSlots = kWarps * kStages;
-constexpr int kHeads = 4;                // query heads per item
+constexpr int kHeads = 4;                // query heads per mma group (an item holds 1 or 2)
 constexpr uint32_t kLutBytes = 1u << 16; // 256 byte values x (2 halves x 32 lanes x 4 B)
 constexpr uint32_t kOnes = 0x3C003C00u;  // fp16 (1, 1)
 
@@ -196,11 +196,11 @@ __device__ __forceinline__ uint32_t ps_part(uint32_t u, uint32_t w, uint32_t s) 
 // Shared-window addresses for a dynamic region that starts at s0.  The table
 // must sit on a 64 KB boundary so that one prmt can splice a code byte into
 // the address; whole warp rings fill the space below it first.
-template <int D>
+template <int D, int HPI>
 struct Plan {
     static constexpr uint32_t kRec = Rec<D>::kBytes;
     static constexpr uint32_t kRing = kStages * kRec;  // one warp's stages, contiguous
-    static constexpr uint32_t kMergeHalf = kNW * (kHeads * D + 2 * kHeads) * 4;
+    static constexpr uint32_t kMergeHalf = kNW * (HPI * D + 2 * HPI) * 4;
     uint32_t lut, low, hi, merge, qh, ql, ids, bars, end;
     __host__ __device__ explicit Plan(uint32_t s0) {
         lut = (s0 + kLutBytes - 1) & ~(kLutBytes - 1);
@@ -209,8 +209,8 @@ struct Plan {
         hi = lut + kLutBytes;
         merge = hi + (kWarps - low) * kRing;
         qh = merge + kHalves * kMergeHalf;
-        ql = qh + kHalves * kHeads * D * 2;
-        ids = ql + kHalves * kHeads * D * 2;
+        ql = qh + kHalves * HPI * D * 2;
+        ids = ql + kHalves * HPI * D * 2;
         bars = ids + kSlots * 4;
         end = bars + kSlots * 8;
     }
@@ -222,11 +222,11 @@ struct Plan {
 
 // Bytes to request so that the plan fits wherever the dynamic region starts
 // (the start depends on the reserved shared memory of the device).
-template <int D>
+template <int D, int HPI>
 uint32_t plan_bytes() {
     uint32_t worst = 0;
     for (uint32_t s0 = 0; s0 <= 8192; s0 += 16) {
-        const Plan<D> p(s0);
+        const Plan<D, HPI> p(s0);
         if (p.end - s0 > worst) worst = p.end - s0;
     }
     return worst;
@@ -323,8 +323,9 @@ __device__ __forceinline__ void ldw(uint32_t a, uint32_t (&w)[N]) {
 }
 
 // ------------------------------------------------------------------ split kernel
-template <int D>
+template <int D, int QPI>
 __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
+    constexpr int HPI = kHeads * QPI;  // query heads per item
     constexpr int KS = D / 16;   // k-steps of q.K = m-tiles of p.V
     constexpr int NG = D / 32;   // value groups
     constexpr int KB = D / 8;    // key bytes of a lane per token = bytes of a value chunk
@@ -339,7 +340,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     const int ht = tid - half * kNW * 32;  // thread index within the half
     const int g = lane >> 2, c = lane & 3;
     const uint32_t s0 = smem_u32(dsm);
-    const Plan<D> P(s0);
+    const Plan<D, HPI> P(s0);
     if (P.end - s0 > a.smem_bytes) {  // cannot happen with the launcher's size; never touch memory
         if (tid == 0 && blockIdx.x == 0) flag_status(a.status, TQ_STATUS_INTERNAL);
         return;
@@ -407,9 +408,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     const uint32_t lanebase = P.lut | ((uint32_t)half << 7) | ((uint32_t)lane << 2);
     const float lo_sel = (float)(g & 1);  // this lane feeds the low part of its head
     const uint32_t lo_mask = (g & 1) ? 0xffffffffu : 0u;
-    const uint32_t qsrc = ((g & 1) ? P.ql : P.qh) + (uint32_t)((half * kHeads + (g >> 1)) * D * 2);
-    const uint32_t mb = P.merge + half * Plan<D>::kMergeHalf;  // [warp][head][D] o, then m, l
-    const uint32_t mb_m = mb + kNW * kHeads * D * 4, mb_l = mb_m + kNW * kHeads * 4;
+    const uint32_t qsrc = ((g & 1) ? P.ql : P.qh) + (uint32_t)((half * HPI + (g >> 1)) * D * 2);
+    const uint32_t mb = P.merge + half * Plan<D, HPI>::kMergeHalf;  // [warp][head][D] o, then m, l
+    const uint32_t mb_m = mb + kNW * HPI * D * 4, mb_l = mb_m + kNW * HPI * 4;
     int stage = 0;
     uint32_t phase = 0;
     bool aborted = false;
@@ -420,8 +421,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     bool first_seg = true;
 #pragma unroll 1
     for (; cu.r < a.nranges; seg_next<D>(cu, stride, a, warp, warp == 0 && lane == 0)) {
-        const int h0 = cu.kv * G + cu.quad * kHeads;  // first query head of the item
-        const int nh = min(kHeads, G - cu.quad * kHeads);
+        const int h0 = cu.kv * G + cu.quad * HPI;  // first query head of the item
+        const int nh = min(HPI, G - cu.quad * HPI);
 
         // ---- the centroid-pair table of this kv head, on this half's side of
         // each 256-byte row: word (row, lane) = (C[row & 15], C[row >> 4])
@@ -438,7 +439,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             }
         }
         // ---- rotate this item's queries: q~ = H q * scale log2(e) / sqrt(D), as fp16 parts
-        if (warp < kHeads) {
+        if (warp < HPI) {
             float x[EPL];
             if (warp < nh) {
                 const uint16_t* src = a.q + ((size_t)cu.b * a.Hq + h0 + warp) * D + lane * EPL;
@@ -467,8 +468,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 }
             }
             const float sc = a.scale_log2 * rsqrtf((float)D);
-            const uint32_t dh = P.qh + (uint32_t)(((half * kHeads + warp) * D + lane * EPL) * 2);
-            const uint32_t dl = P.ql + (uint32_t)(((half * kHeads + warp) * D + lane * EPL) * 2);
+            const uint32_t dh = P.qh + (uint32_t)(((half * HPI + warp) * D + lane * EPL) * 2);
+            const uint32_t dl = P.ql + (uint32_t)(((half * HPI + warp) * D + lane * EPL) * 2);
 #pragma unroll
             for (int e = 0; e < EPL; e += 2) {
                 const float y0 = x[e] * sc, y1 = x[e + 1] * sc;
@@ -480,27 +481,34 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
         }
         half_sync(half);
 
-        // ---- q.K B fragments: column g is head g/2, its high fp16 part for even
-        // g and its low part for odd g; k = 2c, 2c+1 | 2c+8, 2c+9 of step ks are
-        // the dims of key bytes j = c*KB + 2ks and j + 1 (a fixed permutation)
-        uint32_t qb[KS][2];
+        // ---- q.K B fragments of each group q of four heads: column g is head
+        // 4q + g/2, its high fp16 part for even g and its low part for odd g;
+        // k = 2c, 2c+1 | 2c+8, 2c+9 of step ks are the dims of key bytes
+        // j = c*KB + 2ks and j + 1 (a fixed permutation)
+        uint32_t qb[QPI][KS][2];
 #pragma unroll
-        for (int ks = 0; ks < KS; ks++) {
-            const uint2 v2 = lds64(qsrc + 4 * (c * KB + 2 * ks));
-            qb[ks][0] = v2.x;
-            qb[ks][1] = v2.y;
-        }
+        for (int q = 0; q < QPI; q++)
+#pragma unroll
+            for (int ks = 0; ks < KS; ks++) {
+                const uint2 v2 = lds64(qsrc + (uint32_t)(q * kHeads * D * 2) + 4 * (c * KB + 2 * ks));
+                qb[q][ks][0] = v2.x;
+                qb[q][ks][1] = v2.y;
+            }
 
         // ---- this warp's records of the unit
-        float O[KS][4];  // p.V: rows = dims (16m + 2g, 16m + 2g + 1), cols = head c (hi, lo)
-        float Z[4];      // p.z: rows g = zero sums of group g, rows g + 8 = sum of p
+        float O[QPI][KS][4];  // p.V: rows = dims (16m + 2g, 16m + 2g + 1), cols = head c (hi, lo)
+        float Z[QPI][4];      // p.z: rows g = zero sums of group g, rows g + 8 = sum of p
+        float mrun[QPI];      // running maximum of head 4q + c
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            Z[i] = 0.f;
+        for (int q = 0; q < QPI; q++) {
+            mrun[q] = -INFINITY;
 #pragma unroll
-            for (int m = 0; m < KS; m++) O[m][i] = 0.f;
+            for (int i = 0; i < 4; i++) {
+                Z[q][i] = 0.f;
+#pragma unroll
+                for (int m = 0; m < KS; m++) O[q][m][i] = 0.f;
+            }
         }
-        float mrun = -INFINITY;  // running maximum of head c
         const int nk = aborted ? 0 : cu.nk;
         // tokens in this warp's last record of the unit (< 16 only at the end of the sequence)
         const int last_valid = cu.L - (cu.jb + warp + kNW * (nk - 1)) * kBlock;
@@ -516,11 +524,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             if (__all_sync(kFull, (uint32_t)id < (uint32_t)a.num_blocks)) {
                 const bool partial = k == nk - 1 && last_valid < kBlock;
 
-                // -------- q.K: A = centroids of tokens g (rows 0-7) and g + 8 (rows 8-15)
+                // -------- q.K: A = centroids of tokens g (rows 0-7) and g + 8 (rows 8-15),
+                // shared by the QPI groups of heads
                 uint32_t kw0[KW], kw1[KW];
                 ldw<KW>(rec + g * (D / 2) + c * KB, kw0);
                 ldw<KW>(rec + (g + 8) * (D / 2) + c * KB, kw1);
-                float sc[4];
+                float sc[QPI][4];
 #pragma unroll
                 for (int ks = 0; ks < KS; ks++) {
                     // table address: the code byte spliced into byte 1 of lanebase
@@ -531,53 +540,60 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                     const uint32_t a2 = lds32(__byte_perm(w0, lanebase, sb));
                     const uint32_t a1 = lds32(__byte_perm(w1, lanebase, sa));
                     const uint32_t a3 = lds32(__byte_perm(w1, lanebase, sb));
-                    const uint32_t qb0 = qb[ks][0], qb1 = qb[ks][1];
-                    if (ks == 0)
-                        mma16816_z(sc, a0, a1, a2, a3, qb0, qb1);
-                    else
-                        mma16816(sc, a0, a1, a2, a3, qb0, qb1);
+#pragma unroll
+                    for (int q = 0; q < QPI; q++) {
+                        if (ks == 0)
+                            mma16816_z(sc[q], a0, a1, a2, a3, qb[q][ks][0], qb[q][ks][1]);
+                        else
+                            mma16816(sc[q], a0, a1, a2, a3, qb[q][ks][0], qb[q][ks][1]);
+                    }
                 }
-                // scores of head c at tokens g and g + 8 (base 2): columns 2c, 2c+1
+                // scores of head 4q + c at tokens g and g + 8 (base 2): columns 2c, 2c+1
                 // hold the high and low parts of the query
                 const uint32_t nw = lds32(rec + R::kKNorm + 4 * (g >> 1));
                 const uint32_t nw8 = lds32(rec + R::kKNorm + 16 + 4 * (g >> 1));
                 const float na = __half2float(__ushort_as_half((uint16_t)((g & 1) ? nw >> 16 : nw)));
                 const float nb = __half2float(__ushort_as_half((uint16_t)((g & 1) ? nw8 >> 16 : nw8)));
-                float xa = (sc[0] + sc[1]) * na, xb = (sc[2] + sc[3]) * nb;
                 uint32_t mA = 0xffffffffu, mB = 0xffffffffu;  // valid tokens (fp16 lanes)
+                bool va_ok = true, vb_ok = true;               // tokens g, g + 8 valid
                 if (partial) {  // the last block of the sequence
                     const int t = 2 * c, nvalid = last_valid;
-                    xa = g < nvalid ? xa : -INFINITY;
-                    xb = g + 8 < nvalid ? xb : -INFINITY;
+                    va_ok = g < nvalid;
+                    vb_ok = g + 8 < nvalid;
                     mA = (t < nvalid ? 0xffffu : 0u) | (t + 1 < nvalid ? 0xffff0000u : 0u);
                     mB = (t + 8 < nvalid ? 0xffffu : 0u) | (t + 9 < nvalid ? 0xffff0000u : 0u);
                 }
 
-                // -------- online softmax (head c: lanes with the same c)
-                float mx = fmaxf(xa, xb);
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
-                mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
-                const float mn = fmaxf(mrun, mx);
-                if (__any_sync(kFull, mn > mrun)) {
-                    const float corr = ex2(mrun - mn);
-#pragma unroll
-                    for (int i = 0; i < 4; i++) {
-                        Z[i] *= corr;
-#pragma unroll
-                        for (int m = 0; m < KS; m++) O[m][i] *= corr;
-                    }
-                }
-                mrun = mn;
-                const float pa = ex2(xa - mn), pb = ex2(xb - mn);
-                // to the p.V operand: head g/2 at tokens 2c, 2c+1, 2c+8, 2c+9 lives in
-                // lanes (2c, g/2) and (2c+1, g/2), as their tokens g and g + 8
+                // -------- online softmax (head 4q + c: lanes with the same c), and the
+                // weights moved to the p.V operand: head g/2 at tokens 2c, 2c+1, 2c+8,
+                // 2c+9 lives in lanes (2c, g/2) and (2c+1, g/2), as their tokens g, g + 8
                 const int s_even = 8 * c + (g >> 1), s_odd = s_even + 4;
-                const float p0 = __shfl_sync(kFull, pa, s_even), p1 = __shfl_sync(kFull, pa, s_odd);
-                const float p2 = __shfl_sync(kFull, pb, s_even), p3 = __shfl_sync(kFull, pb, s_odd);
-                uint32_t u01, w01, u89, w89;
-                split_uw(p0, p1, lo_sel, lo_mask, u01, w01);
-                split_uw(p2, p3, lo_sel, lo_mask, u89, w89);
+                uint32_t u01[QPI], w01[QPI], u89[QPI], w89[QPI];
+#pragma unroll
+                for (int q = 0; q < QPI; q++) {
+                    const float xa = va_ok ? (sc[q][0] + sc[q][1]) * na : -INFINITY;
+                    const float xb = vb_ok ? (sc[q][2] + sc[q][3]) * nb : -INFINITY;
+                    float mx = fmaxf(xa, xb);
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
+                    const float mn = fmaxf(mrun[q], mx);
+                    if (__any_sync(kFull, mn > mrun[q])) {
+                        const float corr = ex2(mrun[q] - mn);
+#pragma unroll
+                        for (int i = 0; i < 4; i++) {
+                            Z[q][i] *= corr;
+#pragma unroll
+                            for (int m = 0; m < KS; m++) O[q][m][i] *= corr;
+                        }
+                    }
+                    mrun[q] = mn;
+                    const float pa = ex2(xa - mn), pb = ex2(xb - mn);
+                    const float p0 = __shfl_sync(kFull, pa, s_even), p1 = __shfl_sync(kFull, pa, s_odd);
+                    const float p2 = __shfl_sync(kFull, pb, s_even), p3 = __shfl_sync(kFull, pb, s_odd);
+                    split_uw(p0, p1, lo_sel, lo_mask, u01[q], w01[q]);
+                    split_uw(p2, p3, lo_sel, lo_mask, u89[q], w89[q]);
+                }
 
                 // -------- p.z and sum p
                 uint2 zz = lds64(rec + R::kVZero + (c * NG + (g & (NG - 1))) * 8);
@@ -598,7 +614,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                         sw[2 * G_ + 1] &= mB;
                     }
                 }
-                mma16816(Z, zz.x, kOnes, zz.y, kOnes, w01, w89);
+#pragma unroll
+                for (int q = 0; q < QPI; q++) mma16816(Z[q], zz.x, kOnes, zz.y, kOnes, w01[q], w89[q]);
 
                 // -------- p.V: word G of a chunk holds m-tiles 2G (bytes 0, 2) and
                 // 2G + 1 (bytes 1, 3) of tokens 2c, 2c+1 (va) and 2c+8, 2c+9 (vb)
@@ -607,13 +624,16 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 ldw<KW>(rec + R::kVCodes + ((c + 4) * 8 + g) * KB, vb);
 #pragma unroll
                 for (int G_ = 0; G_ < NG; G_++) {
-                    const uint32_t b0 = ps_part(u01, w01, sw[2 * G_]);
-                    const uint32_t b1 = ps_part(u89, w89, sw[2 * G_ + 1]);
                     const uint32_t A0 = va[G_], B0 = vb[G_], A1 = A0 >> 8, B1 = B0 >> 8;
-                    mma16816(O[2 * G_], A0 & 0x000F000Fu, A0 & 0x00F000F0u, B0 & 0x000F000Fu,
-                             B0 & 0x00F000F0u, b0, b1);
-                    mma16816(O[2 * G_ + 1], A1 & 0x000F000Fu, A1 & 0x00F000F0u, B1 & 0x000F000Fu,
-                             B1 & 0x00F000F0u, b0, b1);
+#pragma unroll
+                    for (int q = 0; q < QPI; q++) {
+                        const uint32_t b0 = ps_part(u01[q], w01[q], sw[2 * G_]);
+                        const uint32_t b1 = ps_part(u89[q], w89[q], sw[2 * G_ + 1]);
+                        mma16816(O[q][2 * G_], A0 & 0x000F000Fu, A0 & 0x00F000F0u, B0 & 0x000F000Fu,
+                                 B0 & 0x00F000F0u, b0, b1);
+                        mma16816(O[q][2 * G_ + 1], A1 & 0x000F000Fu, A1 & 0x00F000F0u,
+                                 B1 & 0x000F000Fu, B1 & 0x00F000F0u, b0, b1);
+                    }
                 }
             } else {
                 flag_lane0(a.status, TQ_STATUS_BAD_BLOCK, lane);
@@ -626,21 +646,23 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             }
         }
 
-        // ---- this warp's share -> merge buffer (o with the zero-point term, m, l of head c)
-        {
+        // ---- this warp's share -> merge buffer (o with the zero-point term, m, l of
+        // head 4q + c)
+#pragma unroll
+        for (int q = 0; q < QPI; q++) {
             float zs[NG];
 #pragma unroll
-            for (int G_ = 0; G_ < NG; G_++) zs[G_] = __shfl_sync(kFull, Z[0] + Z[1], 4 * G_ + c);
-            const uint32_t ro = mb + (uint32_t)((warp * kHeads + c) * D * 4);
+            for (int G_ = 0; G_ < NG; G_++) zs[G_] = __shfl_sync(kFull, Z[q][0] + Z[q][1], 4 * G_ + c);
+            const int hq = q * kHeads + c;
+            const uint32_t ro = mb + (uint32_t)((warp * HPI + hq) * D * 4);
 #pragma unroll
             for (int m = 0; m < KS; m++) {
-                stsf(ro + (16 * m + 2 * g) * 4, fmaf(O[m][0] + O[m][1], 0x1p24f, zs[m >> 1]));
-                stsf(ro + (16 * m + 2 * g + 1) * 4, fmaf(O[m][2] + O[m][3], 0x1p20f, zs[m >> 1]));
+                stsf(ro + (16 * m + 2 * g) * 4, fmaf(O[q][m][0] + O[q][m][1], 0x1p24f, zs[m >> 1]));
+                stsf(ro + (16 * m + 2 * g + 1) * 4, fmaf(O[q][m][2] + O[q][m][3], 0x1p20f, zs[m >> 1]));
             }
-            const float mh = mrun;  // head c
             if (g == 0) {
-                stsf(mb_m + (warp * kHeads + c) * 4, mh);
-                stsf(mb_l + (warp * kHeads + c) * 4, Z[2] + Z[3]);
+                stsf(mb_m + (warp * HPI + hq) * 4, mrun[q]);
+                stsf(mb_l + (warp * HPI + hq) * 4, Z[q][2] + Z[q][3]);
             }
         }
         half_sync(half);
@@ -651,20 +673,20 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             const int h = idx / D, i = idx % D;
             float M = -INFINITY;
 #pragma unroll
-            for (int w = 0; w < kNW; w++) M = fmaxf(M, ldsf(mb_m + (w * kHeads + h) * 4));
+            for (int w = 0; w < kNW; w++) M = fmaxf(M, ldsf(mb_m + (w * HPI + h) * 4));
             float o = 0.f, l = 0.f;
             if (M != -INFINITY) {
 #pragma unroll
                 for (int w = 0; w < kNW; w++) {
-                    const float f = ex2(ldsf(mb_m + (w * kHeads + h) * 4) - M);
-                    o = fmaf(f, ldsf(mb + ((w * kHeads + h) * D + i) * 4), o);
-                    l = fmaf(f, ldsf(mb_l + (w * kHeads + h) * 4), l);
+                    const float f = ex2(ldsf(mb_m + (w * HPI + h) * 4) - M);
+                    o = fmaf(f, ldsf(mb + ((w * HPI + h) * D + i) * 4), o);
+                    l = fmaf(f, ldsf(mb_l + (w * HPI + h) * 4), l);
                 }
             }
             if (cu.direct) {
                 a.out[((size_t)cu.b * a.Hq + h0 + h) * D + i] = l > 0.f ? o / l : 0.f;
             } else {
-                const size_t pr = ((size_t)cu.r * 2 + (cu.i == cu.i_first ? 0 : 1)) * kHeads + h;
+                const size_t pr = ((size_t)cu.r * 2 + (cu.i == cu.i_first ? 0 : 1)) * HPI + h;
                 a.ws_o[pr * D + i] = o;
                 if (i == 0) a.ws_ml[pr] = make_float2(M, l);
             }
@@ -683,20 +705,21 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
 // Items cut by range boundaries: out[b][h] = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r
 // over the ranges r that hold part of the item, M = max_r m_r.  Whole items
 // were written by the split kernel and are skipped.
-template <int D>
+template <int D, int QPI>
 __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
+    constexpr int HPI = kHeads * QPI;
     const int bh = blockIdx.x;
     const int i = threadIdx.x;
     const int G = a.Hq / a.Hkv;
     const int b = bh / a.Hq, hh = bh % a.Hq;
-    const int kv = hh / G, quad = (hh % G) / kHeads, h = (hh % G) % kHeads;
+    const int kv = hh / G, quad = (hh % G) / HPI, h = (hh % G) % HPI;
     const int item = (b * a.Hkv + kv) * a.quads + quad;
     const int base = item * a.nmax;
     const int rA = base / a.R, rB = (base + a.nmax - 1) / a.R;
     if (rA == rB) return;  // whole inside one range: already written
     auto part = [&](int r) {
         const int slot = r * a.R / a.nmax == item ? 0 : 1;
-        return ((size_t)r * 2 + slot) * kHeads + h;
+        return ((size_t)r * 2 + slot) * HPI + h;
     };
     float M = -INFINITY;
     for (int r = rA; r <= rB; r++) M = fmaxf(M, a.ws_ml[part(r)].x);
@@ -713,40 +736,43 @@ __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
     a.out[(size_t)bh * D + i] = l > 0.f ? o / l : 0.f;
 }
 
-template <int D>
+template <int D, int QPI>
 cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
     static uint32_t smem = 0;
     static bool configured[64] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (!smem) smem = plan_bytes<D>();
+    if (!smem) smem = plan_bytes<D, kHeads * QPI>();
     if (dev < 0 || dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
+        e = cudaFuncSetAttribute(decode_split_kernel<D, QPI>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         if (dev >= 0 && dev < 64) configured[dev] = true;
     }
     a.smem_bytes = smem;
     const int halves = (a.nranges + kHalves - 1) / kHalves;
     const int grid = halves < num_sms ? halves : num_sms;
-    decode_split_kernel<D><<<grid, kWarps * 32, smem, stream>>>(a);
-    if (decode_needs_combine(a)) combine_kernel<D><<<a.B * a.Hq, D, 0, stream>>>(a);
+    decode_split_kernel<D, QPI><<<grid, kWarps * 32, smem, stream>>>(a);
+    if (decode_needs_combine(a)) combine_kernel<D, QPI><<<a.B * a.Hq, D, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-uint32_t decode_smem_bytes(int head_dim) {
-    return head_dim == 128 ? plan_bytes<128>() : plan_bytes<64>();
+uint32_t decode_smem_bytes(int head_dim) {  // the largest plan of the head_dim's kernels
+    return head_dim == 128 ? plan_bytes<128, kHeads>() : plan_bytes<64, 2 * kHeads>();
 }
 
 // Ranges: with num_splits = 0 the virtual records are cut evenly over every
 // half of a full grid; with num_splits = S each range is ceil(nmax / S) records
 // (S = 1: one range per item, nothing to combine).
-bool decode_plan(DecodeArgs& a, int num_sms) {
+bool decode_plan(DecodeArgs& a, int head_dim, int num_sms) {
     const int G = a.Hq / a.Hkv;
-    a.quads = (G + kHeads - 1) / kHeads;
+    // at d = 64 an item takes two groups of four query heads when there are more
+    // than four per kv head: the record is staged and dequantised once for both
+    a.qpi = head_dim == 64 && G > kHeads ? 2 : 1;
+    a.quads = (G + kHeads * a.qpi - 1) / (kHeads * a.qpi);
     a.items = a.B * a.Hkv * a.quads;
     a.nmax = a.max_seq_len > 0 ? (a.max_seq_len + kBlock - 1) / kBlock : 1;
     const long long V = (long long)a.items * a.nmax;
@@ -772,14 +798,15 @@ bool decode_needs_combine(const DecodeArgs& a) { return a.nranges > 1 && a.R % a
 
 size_t decode_workspace_for(const DecodeArgs& a, int head_dim) {
     if (!decode_needs_combine(a)) return 0;
-    return (size_t)a.nranges * 2 * kHeads * (head_dim * sizeof(float) + sizeof(float2));
+    return (size_t)a.nranges * 2 * kHeads * a.qpi * (head_dim * sizeof(float) + sizeof(float2));
 }
 
 cudaError_t launch_decode(const DecodeArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
     DecodeArgs a = args;
     if (num_sms < 1) num_sms = 1;
-    if (!decode_plan(a, num_sms)) return cudaErrorInvalidValue;
-    return head_dim == 128 ? launch_d<128>(a, num_sms, stream) : launch_d<64>(a, num_sms, stream);
+    if (!decode_plan(a, head_dim, num_sms)) return cudaErrorInvalidValue;
+    if (head_dim == 128) return launch_d<128, 1>(a, num_sms, stream);
+    return a.qpi == 2 ? launch_d<64, 2>(a, num_sms, stream) : launch_d<64, 1>(a, num_sms, stream);
 }
 
 }  // namespace tq

@@ -99,7 +99,8 @@ struct DecodeArgs {
     int max_seq_len;
     int32_t* status;
     // set by decode_plan
-    int quads;            // groups of four query heads per kv head
+    int qpi;              // groups of four query heads per item (1, or 2 at d = 64 with G > 4)
+    int quads;            // items per kv head
     int items;            // B * Hkv * quads
     int nmax;             // blocks of the longest sequence (>= 1)
     int vrec;             // virtual records items x nmax (< 2^30)
@@ -128,7 +129,7 @@ int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 uint32_t decode_smem_bytes(int head_dim);  // dynamic shared memory of the split kernel
-bool decode_plan(DecodeArgs& a, int num_sms);            // ranges; false: too many
+bool decode_plan(DecodeArgs& a, int head_dim, int num_sms);  // ranges; false: too many
 bool decode_needs_combine(const DecodeArgs& a);          // some item is cut by a range
 size_t decode_workspace_for(const DecodeArgs& a, int head_dim);  // partials, bytes
 cudaError_t launch_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);
