@@ -304,8 +304,8 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
     if (H_q % Hkv)
         return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: H_q %d not a multiple of H_kv %d", H_q, Hkv);
     const int G = H_q / Hkv;
-    if (G != 1 && G != 2 && G != 4 && G != 8)
-        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: GQA group %d (supported 1, 2, 4, 8)", G);
+    if (G > 64)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: GQA group %d (supported 1..64)", G);
     if (num_splits < 0 || num_splits > 1024)
         return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: num_splits %d (0..1024)", num_splits);
     if (!isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: scale not finite");

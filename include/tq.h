@@ -143,7 +143,8 @@ TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_sp
  * h / (H_q / H_kv).  The query is rotated by the same Hadamard transform
  * once, so scores are computed in the rotated domain against the stored
  * centroids; K and V are dequantised in registers and never written out.
- *   q            (device) bf16 [B][H_q][d]
+ *   q            (device) bf16 [B][H_q][d]; H_q a multiple of H_kv, at most 64 query
+ *                heads per kv head (TQ_ERR_UNSUPPORTED otherwise)
  *   block_tables (device) int32 [B][max_blocks]
  *   seq_lens     (device) int32 [B], each in [0, max_blocks*16]
  *   max_seq_len  (host)   upper bound of seq_lens (sizes the split grid); a

@@ -94,7 +94,8 @@ def test_argument_validation_without_launch(lib):
     assert rc == tq.TQ_ERR_INVALID_ARG
     rc = lib.tq_quantize_append(None, None, None, 0, 0, None, 0, ctypes.byref(c), None, None, None)
     assert rc == tq.TQ_OK  # T == 0 is a no-op
-    # decode: GQA group 3 unsupported; workspace too small; bad split count
+    # decode: H_q not a multiple of H_kv, or a GQA group above 64, unsupported; workspace
+    # too small; bad split count
     c = _cache_struct(heads=2)
     args = dict(q=P(16), k=None, bt=P(16), mb=4, sl=P(16), B=1, Hq=6, L=64, scale=0.1, out=P(16),
                 ws=None, wsb=0, S=0)
@@ -105,7 +106,8 @@ def test_argument_validation_without_launch(lib):
                                        a["Hq"], a["L"], ctypes.c_float(a["scale"]), a["out"], a["ws"],
                                        a["wsb"], a["S"], None, None)
 
-    assert dec() == tq.TQ_ERR_UNSUPPORTED
+    assert dec(Hq=5) == tq.TQ_ERR_UNSUPPORTED
+    assert dec(Hq=2 * 65) == tq.TQ_ERR_UNSUPPORTED
     assert dec(Hq=4, S=4) == tq.TQ_ERR_WORKSPACE
     assert dec(Hq=4, S=2000) == tq.TQ_ERR_UNSUPPORTED
     assert dec(Hq=4, L=65) == tq.TQ_ERR_INVALID_ARG  # max_seq_len beyond max_blocks * 16

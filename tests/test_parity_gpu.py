@@ -165,6 +165,13 @@ def test_dequantize_matches_oracle(tq, orc):
     ("qwen3_8b_layer", dict(B=2, ctx=300, Hq=16), 0), # GQA 2
     ("qwen3_8b_layer", dict(B=2, ctx=300, Hq=64), 2), # GQA 8 at d = 128
     ("prefill_small_head", dict(B=2, ctx=200, Hq=8), 1),  # GQA 4 at d = 64
+    # d = 64 items of two groups of four heads, the second one partly or wholly used
+    ("prefill_small_head", dict(B=2, ctx=333, Hq=10), 0),  # GQA 5: 4 + 1
+    ("prefill_small_head", dict(B=2, ctx=250, Hq=12), 3),  # GQA 6: 4 + 2, splits
+    ("prefill_small_head", dict(B=2, ctx=180, Hq=24), 0),  # GQA 12: items of 8 and 4 heads
+    ("prefill_small_head", dict(B=1, ctx=520, Hq=32), 2),  # GQA 16: two items of 8 heads
+    ("qwen3_8b_layer", dict(B=2, ctx=200, Hq=48), 0),      # GQA 6 at d = 128: 4 + 2
+    ("qwen3_8b_layer", dict(B=2, ctx=150, Hq=24), 2),      # GQA 3 at d = 128
 ])
 def test_reduced_configs(tq, orc, name, over, S):
     w = W.make(name, **over)
