@@ -7,14 +7,18 @@
 // Values: v_hat = code * s + z per group of 32, so
 //   o = sum_t p_t v_hat_t = sum_t (p_t s_t,g) code_t + sum_t p_t z_t,g.
 //
-// Work.  An item is (sequence, kv head, group of four query heads); a unit is
-// (item, split of the context).  The grid is persistent: one CTA of 16 warps
-// per SM, made of two independent halves of 8 warps, each half walking its
-// own list of units.  Within a unit the 8 warps take the split's 16-token
-// blocks round-robin.  Each warp streams its records through a private ring
-// of shared-memory stages with bulk asynchronous copies (cp.async.bulk +
-// mbarrier); the ring runs across unit boundaries, so the next unit's first
-// records are in flight while a unit's partial results are merged.
+// Work.  An item is (sequence, kv head, group of four query heads), or at d = 64
+// with more than four query heads per kv head two such groups, whose records are
+// then staged and unpacked once for both.  The virtual record space items x
+// nmax (nmax = blocks of the longest sequence) is cut into ranges: evenly over
+// every half of a full grid, or into ceil(nmax / S) records per range with S
+// splits.  The grid is persistent: one CTA of 16 warps per SM, made of two
+// independent halves of 8 warps, half h taking ranges h, h + H, ...  Within a
+// range's part of an item (a segment) the 8 warps take its 16-token blocks
+// round-robin.  Each warp streams its records through a private ring of
+// shared-memory stages with bulk asynchronous copies (cp.async.bulk +
+// mbarrier); the ring runs across segment boundaries, so the next segment's
+// first records are in flight while a segment's partial results are merged.
 //
 // Per record every product runs on the tensor cores (mma.sync m16n8k16, fp32
 // accumulate), with exact fp16 operands only:
@@ -30,9 +34,9 @@
 //   p.z  A = fp16 zero points (rows 0-7) and ones (rows 8-15), B = p as fp16
 //        parts: gives sum_t p_t z_t,g and the softmax denominator.
 // Softmax runs online in base 2 (scale * log2 e is folded into q~) and the
-// accumulators are rescaled only when a running maximum moves.  Each unit
-// leaves an unnormalised partial (o, m, l) that the combine kernel merges; a
-// single split writes the output directly.
+// accumulators are rescaled only when a running maximum moves.  An item
+// that lies wholly inside one range is written directly; the others leave an
+// unnormalised partial (o, m, l) per range that the combine kernel merges.
 #include "tq_kernels.cuh"
 
 namespace tq {
@@ -89,13 +93,6 @@ __device__ __forceinline__ void half_sync(int half) {
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
     uint32_t ok;
     asm volatile(
@@ -128,16 +125,6 @@ __device__ __forceinline__ void flag_lane0(int32_t* status, int bits, int lane) 
     const uint32_t p = (uint32_t)(lane == 0 && status != nullptr);
     asm volatile("{\n .reg .pred p;\n setp.ne.u32 p, %0, 0;\n @p red.global.or.b32 [%1], %2;\n}\n"
                  ::"r"(p), "l"(status), "r"(bits) : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
-                                         uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
-        : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
