@@ -303,9 +303,11 @@ def cfg(w, l2):
 
 # ---------------------------------------------------------------- the other workloads
 def other_workloads(dev, peak, reps: int = 20) -> dict:
-    """Per-call CUDA-event timings (median of `reps`) of the scope table's other
-    measured workloads, each on its own cache; L2 is flushed before every timed
-    call by reading a 512 MB buffer (the prefill chunk and its cache fit in L2).
+    """Device time per call (graphs of `reps` calls, CUDA events) of the scope
+    table's other measured workloads, each on its own cache.  The long-context and
+    agentic decodes read more than L2 per call; the prefill chunk and its cache fit
+    in L2, so each of those calls follows a 512 MB read that evicts it, and the
+    read's own time is subtracted.
 
     long_context: decode over 4 x 131072 tokens with 64 splits per item (and the
     even cut); agentic: decode over the shared-prefix batch with calibrated
@@ -317,18 +319,37 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
     flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
-    def timed(fn):
-        ts = []
-        for i in range(reps + 2):
-            flush.sum()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
+    def graph_time(fn, n):
+        """ms per fn() on the device: n calls captured as one CUDA graph, the median of
+        three replays timed with CUDA events on the replay stream"""
+        s_ = torch.cuda.Stream(dev)
+        s_.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s_):
             fn()
-            e1.record()
-            torch.cuda.synchronize(dev)
-            if i >= 2:
+            s_.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s_):
+                for _ in range(n):
+                    fn()
+            g.replay()
+            s_.synchronize()
+            ts = []
+            for _ in range(3):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(s_)
+                g.replay()
+                e1.record(s_)
+                s_.synchronize()
                 ts.append(e0.elapsed_time(e1))
-        return statistics.median(ts)
+        del g
+        return statistics.median(ts) / n
+
+    def timed(fn, cold):
+        """ms per call on the device, without the host's launch latency; with cold,
+        every call follows an L2 flush (a 512 MB read) whose own time is subtracted"""
+        if not cold:
+            return graph_time(fn, reps)
+        return graph_time(lambda: (flush.sum(), fn()), reps) - graph_time(lambda: flush.sum(), reps)
 
     def build(w, tables=None):
         cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
@@ -338,7 +359,7 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
                                k_tables=tables, status=status)
         return cache, bt
 
-    def decode(w, cache, bt, S, tables=None):
+    def decode(w, cache, bt, S, tables=None, cold=False):
         lens = torch.from_numpy(w.seq_lens).to(dev)
         q = w.q().to(dev)
         max_len = int(w.seq_lens.max())
@@ -346,7 +367,7 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
         ws = torch.empty(max(16, tq.workspace_bytes(w.B, w.Hq, w.d, S)), dtype=torch.uint8, device=dev)
         return timed(lambda: tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out,
                                                  workspace=ws, num_splits=S, k_tables=tables,
-                                                 status=status))
+                                                 status=status), cold)
 
     res = {}
     w = W.make("long_context")
@@ -381,12 +402,12 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
     V = torch.cat([p[1] for p in parts]).to(dev)
     slots = torch.cat([torch.arange(0, 2048, dtype=torch.int32) + b * cap for b in range(w.B)]).to(dev)
     T = K.shape[0]
-    ms = timed(lambda: tq.quantize_append(K, V, slots, cache, block_table=bt, status=status))
+    ms = timed(lambda: tq.quantize_append(K, V, slots, cache, block_table=bt, status=status), True)
     ab = append_bytes(w, T)
     res["prefill_chunk_append"] = {"ms": ms, "tokens": T, "tokens_per_s": T / ms * 1e3,
                                    "gbs": ab / ms / 1e6, "hbm_frac": ab / ms / 1e6 / peak}
     kv = decode_kv_bytes(w)
-    ms = decode(w, cache, bt, 0)
+    ms = decode(w, cache, bt, 0, cold=True)
     res["prefill_small_head_decode"] = {"ms": ms, "gbs": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / peak}
     del cache
     torch.cuda.synchronize(dev)
@@ -497,8 +518,40 @@ def run_tq(args, rank, world, local):
     barrier(world)
     app_ms = [e[0].elapsed_time(e[1]) for e in evs]
     dec_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
-    app_avg = max_over_ranks(sum(app_ms) / len(app_ms), world)
+    dec_call = max_over_ranks(sum(dec_ms) / len(dec_ms), world)
+    app_call = max_over_ranks(sum(app_ms) / len(app_ms), world)
+
+    # the decode alone on the device: K calls captured as one CUDA graph and replayed,
+    # CUDA events around the replay on its stream, so the host's launch latency (the
+    # per-call events above include it) is not counted; 306 MB per call exceeds L2
+    def graph_ms(fn):
+        s_ = torch.cuda.Stream(dev)
+        s_.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s_):
+            fn(s_)
+            s_.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s_):
+                for _ in range(args.steps):
+                    fn(s_)
+            g.replay()
+            s_.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            barrier(world)
+            e0.record(s_)
+            g.replay()
+            e1.record(s_)
+            s_.synchronize()
+        ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        del g
+        return ms
+
+    dec_avg = graph_ms(lambda s_: tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out,
+                                                      workspace=ws, num_splits=S, status=status,
+                                                      stream=s_))
+    # the append's inputs (4.4 MB) would stay in L2 over back-to-back calls, so its
+    # figure stays the per-call one, taken right after a decode has streamed 306 MB
+    app_avg = app_call
 
     # whole steps: the step (append, then decode) captured once as a CUDA graph, the way
     # a serving engine launches a decode step, and replayed; CUDA events around K replays
@@ -653,7 +706,7 @@ def run_tq(args, rank, world, local):
             "config": cfg(w, f"inputs larger than L2: {kv / 1e6:.0f} MB cache read per rank vs 126 MB L2, no flush"),
             "decode_gbs": kv / (dec_avg / 1e3) / 1e9,
             "decode_hbm_frac": kv / (dec_avg / 1e3) / 1e9 / peak,
-            "decode_ms": dec_avg, "append_ms": app_avg,
+            "decode_ms": dec_avg, "append_ms": app_avg, "decode_call_ms": dec_call,
             "append_tokens_per_s": T / (app_avg / 1e3),
             "append_hbm_frac": append_bytes(w, T) / (app_avg / 1e3) / 1e9 / peak,
             "num_splits": S,
