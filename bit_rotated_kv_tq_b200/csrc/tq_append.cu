@@ -231,11 +231,9 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         const uint32_t mxw = *reinterpret_cast<const uint32_t*>(&mx2);
         const float mn = fminf(bf16_lo(mnw), bf16_hi(mnw));
         const float mx = fmaxf(bf16_lo(mxw), bf16_hi(mxw));
-        const __half zh = __float2half_rd(mn);  // exact: mn is a bf16 value
+        // z = fp16 rounded down from the minimum (exact when it lies in fp16's normal range)
+        const __half zh = __float2half_rd(mn);
         const float zf = __half2float(zh);
-        // s = fp16 rounded up from (mx - z)/15: bracket the quotient in fp32 with
-        // directed roundings; if both ends round up to the same fp16 value it is
-        // the answer, otherwise (an fp16 value inside the bracket) use fp64.
         uint16_t s16;
         {
             // s = fp16 rounded up from D / 15, D = max - z.  c, the smallest fp16 at or
@@ -353,8 +351,15 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         const bool nnorm = __half_as_ushort(__float2half_rn(n * (1.0f - kNormMargin))) !=
                            __half_as_ushort(__float2half_rn(n * (1.0f + kNormMargin)));
         // squares that leave the normal fp32 range (or a non-finite key) lose the
-        // fp32 error bound: every decision is re-taken (an all-zero key stays here)
-        const bool wild = !(ss >= 1e-30f && ss <= 1e30f) && (kor & 0x7fff7fffu) != 0u;
+        // fp32 error bound: every decision is re-taken.  An all-zero key stays here;
+        // whether any element is nonzero is asked of the whole vector, since one
+        // lane's 16 elements may all be zero while the others' are not.
+        const bool small = !(ss >= 1e-30f && ss <= 1e30f);
+        if (__any_sync(kFull, small)) {
+#pragma unroll
+            for (int m = 1; m < LPV; m <<= 1) kor |= __shfl_xor_sync(kFull, kor, m);
+        }
+        const bool wild = small && (kor & 0x7fff7fffu) != 0u;
         bool nkey = wild;  // some centroid decision is close (all of them when wild)
         const float inv = rs * inv_sqrt_d;              // 1 / (n sqrt(D))
         const float A = rs * (inv_sqrt_d * kBinScale);  // kBinScale / (n sqrt(D))

@@ -278,6 +278,8 @@ def test_value_and_key_edge_data(tq, orc, d):
     V[5] *= 1000.0
     V[5, :, 7] = 1e-3                             # wide dynamic range in one group
     K[6] *= 1e-20                                 # tiny norm
+    K[9] *= 1e-20
+    K[9, :, :16] = 0.0                            # tiny norm, one lane's elements all zero
     # z = -1, max - z = 1.875 = 15 * 0.125 (s exact in fp16), every other value on a .5 point
     V[7] = np.tile(-1.0 + 0.0625 * np.minimum(np.arange(32), 30), (H, d // 32))
     V[8] = rng.uniform(0.0, 1.0, (H, d))
