@@ -708,6 +708,20 @@ __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
         const int slot = r * a.R / a.nmax == item ? 0 : 1;
         return ((size_t)r * 2 + slot) * HPI + h;
     };
+    if (rB == rA + 1) {  // the usual cut: two ranges, their loads issued together
+        const size_t p0 = part(rA), p1 = part(rB);
+        const float2 ml0 = a.ws_ml[p0], ml1 = a.ws_ml[p1];
+        const float o0 = a.ws_o[p0 * D + i], o1 = a.ws_o[p1 * D + i];
+        const float M = fmaxf(fmaxf(-INFINITY, ml0.x), ml1.x);
+        float o = 0.f, l = 0.f;
+        if (M != -INFINITY) {
+            const float f0 = ex2(ml0.x - M), f1 = ex2(ml1.x - M);
+            o = fmaf(f1, o1, fmaf(f0, o0, 0.f));
+            l = fmaf(f1, ml1.y, fmaf(f0, ml0.y, 0.f));
+        }
+        a.out[(size_t)bh * D + i] = l > 0.f ? o / l : 0.f;
+        return;
+    }
     float M = -INFINITY;
     for (int r = rA; r <= rB; r++) M = fmaxf(M, a.ws_ml[part(r)].x);
     float o = 0.f, l = 0.f;
