@@ -14,6 +14,7 @@ Parity rule (the TQ4/4 statement of what must match):
 from __future__ import annotations
 
 import numpy as np
+import torch
 
 CODE_TOL = 1e-6
 COUNT_TOL = 1e-5
@@ -83,6 +84,86 @@ def fp16_midpoint_rel_distance(n: np.ndarray) -> np.ndarray:
     dn = np.nextafter(n.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
     mids = np.stack([(h + up) / 2, (h + dn) / 2], axis=-1)
     return np.min(np.abs(mids - n[..., None]), axis=-1) / np.maximum(n, 1e-300)
+
+
+def bf16_values(lo_exp: int, hi_exp: int) -> np.ndarray:
+    """Every positive bf16 value in [2^lo_exp, 2^hi_exp), ascending."""
+    e = np.arange(lo_exp, hi_exp, dtype=np.float64)
+    m = np.arange(128, dtype=np.float64)
+    return ((1.0 + m[None, :] / 128.0) * 2.0 ** e[:, None]).ravel()
+
+
+def near_threshold_pairs(d: int, table: np.ndarray, count: int, which: str):
+    """Pairs (a, b) of positive bf16 values for two-entry keys k = a e_i + b e_j.
+
+    The Sylvester rotation of such a key has coordinates (+-a +- b) / (|k| sqrt d),
+    with |k| = sqrt(a^2 + b^2).  The pairs are ranked by how close those
+    coordinates come to a midpoint of `table` (which="key"), or by how close
+    |k| comes, relatively, to an fp16 rounding midpoint (which="norm"), and the
+    `count` closest are returned with their distances.  a spans [1, 2), b spans
+    [2^-8, 2): about 147 000 candidates, so the closest sit far inside 1e-6.
+    """
+    A, B = np.meshgrid(bf16_values(0, 1), bf16_values(-8, 1), indexing="ij")
+    A, B = A.ravel(), B.ravel()
+    n = np.sqrt(A * A + B * B)
+    if which == "key":
+        t = np.sort(table.astype(np.float64))
+        mids = 0.5 * (t[:-1] + t[1:])
+        dist = np.full(A.shape, np.inf)
+        dist[A == B] = -1.0  # a = b: coordinates exactly 0, a tie pinned elsewhere; not taken
+        for s in (1.0, -1.0):
+            y = np.abs(A + s * B) / (n * np.sqrt(d))
+            dist = np.minimum(dist, np.min(np.abs(y[:, None] - np.abs(mids)[None, :]), axis=1))
+    elif which == "norm":
+        dist = fp16_midpoint_rel_distance(n)
+    else:
+        raise ValueError(which)
+    order = np.argsort(np.where(dist < 0, np.inf, dist), kind="stable")[:count]
+    return A[order], B[order], dist[order]
+
+
+def two_entry_keys(d: int, a: np.ndarray, b: np.ndarray, rng) -> np.ndarray:
+    """fp32 keys [len(a)][d], key t = a[t] e_i + b[t] e_j (signs and i != j at random).
+
+    a and b must be bf16 values, so the keys are exact in bf16."""
+    K = np.zeros((len(a), d), np.float32)
+    for t in range(len(a)):
+        i, j = rng.choice(d, 2, replace=False)
+        K[t, i] = a[t] * rng.choice((-1.0, 1.0))
+        K[t, j] = b[t] * rng.choice((-1.0, 1.0))
+    return K
+
+
+def near_threshold_keys(d: int, table: np.ndarray, count: int, which: str, seed: int,
+                        within: float = 1e-6, pool: int = 4096, max_pools: int = 64):
+    """bf16-exact fp32 keys [count][d] with a rotated unit coordinate within `within` of
+    a midpoint of `table` (which="key") or a norm within `within` (relative) of an fp16
+    rounding midpoint (which="norm"), drawn from pools of N(0, 1) keys; the 8 closest
+    two-entry keys of `near_threshold_pairs` come first.  Returns keys, distances."""
+    rng = np.random.default_rng(seed)
+    a, b, dist2 = near_threshold_pairs(d, table, 8, which)
+    keys, dists = [two_entry_keys(d, a, b, rng)], [dist2]
+    have = len(a)
+    Hs = np.array([[(-1.0) ** bin(i & j).count("1") for j in range(d)] for i in range(d)])
+    t = np.sort(table.astype(np.float64))
+    mids = 0.5 * (t[:-1] + t[1:])
+    for _ in range(max_pools):
+        if have >= count:
+            break
+        K = torch.from_numpy(rng.standard_normal((pool, d)).astype(np.float32)).to(
+            torch.bfloat16).float().numpy()
+        Kd = K.astype(np.float64)
+        n = np.sqrt(np.sum(Kd * Kd, axis=1))
+        if which == "key":
+            y = (Kd @ Hs.T) / (n[:, None] * np.sqrt(d))
+            dist = np.min(np.abs(y[..., None] - mids), axis=-1).min(axis=1)
+        else:
+            dist = fp16_midpoint_rel_distance(n)
+        sel = np.flatnonzero(dist < within)[: count - have]
+        keys.append(K[sel])
+        dists.append(dist[sel])
+        have += len(sel)
+    return np.concatenate(keys)[:count], np.concatenate(dists)[:count]
 
 
 class CodeReport:

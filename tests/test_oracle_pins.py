@@ -7,6 +7,7 @@ quadrature), a published table (Max 1960), a hand-derived worked example,
 an invariant, or brute force on tiny inputs.
 """
 import math
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -17,6 +18,7 @@ import scipy.stats
 import torch
 
 from conftest import read_golden
+from parity_util import near_threshold_keys
 
 RNG = np.random.default_rng(12345)
 
@@ -193,6 +195,92 @@ def test_key_rotation_matches_scipy_and_keeps_norm(orc, d):
         # brute force: the chosen level is at least as close as every other level
         dist = np.abs(y[:, None] - table[None, :].astype(np.float64))
         assert np.all(dist[np.arange(d), idx] <= dist.min(axis=1))
+
+
+def _exact_code(N, nsq, d, mids):
+    """Code of y = N / sqrt(nsq d) against sorted midpoints, all exact rationals:
+    the count of midpoints strictly below y (a tie keeps the lower index), and
+    whether y equals one of them.  y > m is decided on squares: N > m sqrt(nsq d)
+    with both sides' signs known."""
+    code, tie = 0, False
+    for m in mids:
+        tie |= (N > 0) == (m > 0) and N * N == m * m * nsq * d
+        if m == 0:
+            above = N > 0
+        elif (N >= 0) != (m > 0):
+            above = N >= 0  # opposite signs (or N = 0): y > m exactly when m < 0
+        elif m > 0:
+            above = N * N > m * m * nsq * d
+        else:
+            above = N * N < m * m * nsq * d
+        code += above
+    return code, tie
+
+
+def _exact_fp16_of_sqrt(nsq):
+    """fp16 nearest (ties to even) to sqrt(nsq), nsq an exact positive rational, and
+    whether sqrt(nsq) lies exactly on the midpoint of two fp16 values."""
+    lo = np.float16(math.sqrt(float(nsq)))
+    while Fraction(float(lo)) ** 2 > nsq:
+        lo = np.nextafter(lo, np.float16(-np.inf))
+    while Fraction(float(np.nextafter(lo, np.float16(np.inf)))) ** 2 <= nsq:
+        lo = np.nextafter(lo, np.float16(np.inf))
+    hi = np.nextafter(lo, np.float16(np.inf))
+    mid = (Fraction(float(lo)) + Fraction(float(hi))) / 2
+    if nsq != mid * mid:
+        return int((hi if nsq > mid * mid else lo).view(np.uint16)), False
+    even = lo if int(lo.view(np.uint16)) % 2 == 0 else hi
+    return int(even.view(np.uint16)), True
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("which", ["key", "norm"])
+def test_key_decisions_near_thresholds_match_exact_arithmetic(orc, d, which):
+    """bf16 keys chosen so that a rotated coordinate lies within 1e-6 of a centroid
+    midpoint, or the norm within 1e-6 (relative) of an fp16 rounding midpoint (two-entry
+    keys a e_i + b e_j searched for closeness, then N(0, 1) keys filtered).  With
+    N = (S k)_i exact (S = scipy's +-1 Hadamard matrix) and nsq = |k|^2 exact, each
+    coordinate y = N / sqrt(nsq d) is placed against the midpoints, and the norm
+    sqrt(nsq) against the fp16 grid, in exact rational arithmetic on squares.  The
+    oracle's binary64 codes and fp16 norms must agree wherever binary64 resolves the
+    question (distance >= 1e-14) and wherever the exact value sits on the threshold (a
+    tie: ties to even for the norm, to the lower index for a code).  Other cases
+    closer than 1e-14 are the binary64 reading itself (the norm and coordinates are
+    binary64 values before they are rounded or compared) and are only counted."""
+    table = orc.default_table(d)
+    t = np.sort(table.astype(np.float64))
+    mids = [(Fraction(float(t[j])) + Fraction(float(t[j + 1]))) / 2 for j in range(15)]
+    K, dist = near_threshold_keys(d, table, 40, which, seed=71 + d)
+    assert len(K) == 40 and dist.max() < 1e-6
+    S = scipy.linalg.hadamard(d)
+    checked_near = unresolved = 0
+    for k in K:
+        idx, n16, y = orc.encode_k(bf16_bits_of(k), table)
+        nz = np.flatnonzero(k)
+        nsq = sum(Fraction(float(k[j])) ** 2 for j in nz)
+        # norm
+        n = math.sqrt(float(nsq))
+        h = np.float16(n)
+        cand = [np.nextafter(h, np.float16(-np.inf)), h, np.nextafter(h, np.float16(np.inf))]
+        ndist = min(abs(n - (float(cand[i]) + float(cand[i + 1])) / 2) for i in range(2)) / n
+        n_exact, n_tie = _exact_fp16_of_sqrt(nsq)
+        if ndist >= 1e-14 or n_tie:
+            assert n16 == n_exact, (k[nz], n16, n_tie)
+            checked_near += which == "norm" and ndist < 1e-6
+        else:
+            unresolved += which == "norm"
+        # codes: every coordinate
+        for i in range(d):
+            N = sum(int(S[i, j]) * Fraction(float(k[j])) for j in nz)
+            kdist = float(np.min(np.abs(y[i] - np.asarray([float(m) for m in mids]))))
+            code, tie = _exact_code(N, nsq, d, mids)
+            if kdist >= 1e-14 or tie:
+                assert idx[i] == code, (k[nz], i, y[i], idx[i], tie)
+                checked_near += which == "key" and kdist < 1e-6
+            else:
+                unresolved += which == "key"
+    # the selection reaches the thresholds: nearly every chosen key was decided within 1e-6
+    assert checked_near >= 36, (checked_near, unresolved)
 
 
 @pytest.mark.parametrize("d", [64, 128])

@@ -12,7 +12,8 @@ import torch
 
 import workloads as W
 from parity_util import (CodeReport, check_attention, fp16_midpoint_rel_distance,
-                         key_boundary_distance, unpack_record, value_boundary_distance)
+                         key_boundary_distance, near_threshold_keys, unpack_record,
+                         value_boundary_distance)
 from workloads import bf16_bits
 
 pytestmark = pytest.mark.gpu
@@ -308,6 +309,60 @@ def test_value_and_key_edge_data(tq, orc, d):
                         msgs.append(f"blk {blk} head {h} {name}: {len(bad)} differ, first at {t0}: "
                                     f"gpu {x[t0]} oracle {y[t0]}")
         raise AssertionError("records differ:\n" + "\n".join(msgs[:12]))
+
+
+@pytest.mark.parametrize("d,dense", [(64, False), (128, False), (128, True)],
+                         ids=["d64", "d128", "d128-dense-table"])
+def test_keys_near_decision_thresholds(tq, orc, d, dense):
+    """Keys whose rotated unit coordinates lie within 1e-6 of a centroid midpoint (kv
+    head 0) or whose norms lie within 1e-6 (relative) of an fp16 rounding midpoint,
+    exact ties included (kv head 1): every one of them takes the append's exact
+    re-decision.  The records must equal the oracle's byte for byte; a differing code
+    or norm is accepted only below 1e-12 of its threshold, where the two sides' binary64
+    rounding orders (y - C against product with the midpoint) may split a case."""
+    T, H = 64, 2
+    t = orc.default_table(d)
+    if dense:  # midpoints 7 and 8 in one bin: the exact counting path
+        t = t.astype(np.float64)
+        t[7], t[8], t[9] = -1e-4, 0.0, 1e-4
+        t = t.astype(np.float16)
+    Kk, dk = near_threshold_keys(d, t, T, "key", seed=301 + d)
+    Kn, dn = near_threshold_keys(d, t, T, "norm", seed=401 + d)
+    K = np.stack([Kk, Kn], axis=1)
+    V = np.random.default_rng(7).standard_normal((T, H, d)).astype(np.float32)
+    Kt = torch.from_numpy(K).to(torch.bfloat16)
+    Vt = torch.from_numpy(V).to(torch.bfloat16)
+    assert torch.equal(Kt.float(), torch.from_numpy(K))  # the keys are bf16 values
+    tables = np.tile(t, (H, 1))
+    cache = tq.Cache(T // 16, H, d)
+    tq.quantize_append(Kt.cuda(), Vt.cuda(), torch.arange(T, dtype=torch.int32).cuda(), cache,
+                       k_tables=torch.from_numpy(np.ascontiguousarray(tables, np.float16)).cuda())
+    torch.cuda.synchronize()
+    ocache = np.zeros((T // 16, H, orc.record_bytes(d)), np.uint8)
+    rc, ky, vr = orc.quantize_append(bf16_bits(Kt), bf16_bits(Vt), np.arange(T, dtype=np.int32),
+                                     ocache, tables=tables, want_aux=True)
+    assert rc == 0
+    got = cache.data.cpu().numpy()
+    if np.array_equal(got, ocache):
+        return
+    ky = ky.reshape(T, H, d)
+    n = np.linalg.norm(Kt.double().numpy(), axis=-1)
+    bad = []
+    for blk in range(T // 16):
+        for h in range(H):
+            a = unpack_record(got[blk, h], d)
+            b = unpack_record(ocache[blk, h], d)
+            rows = slice(16 * blk, 16 * blk + 16)
+            kd = key_boundary_distance(ky[rows, h], t)
+            nd = fp16_midpoint_rel_distance(n[rows, h])
+            for name, x, y, dist in zip(("kidx", "knorm", "vq", "vs", "vz"), a, b,
+                                        (kd, nd, None, None, None)):
+                for pos in np.argwhere(x != y):
+                    pos = tuple(pos)
+                    if dist is None or dist[pos] >= 1e-12:
+                        bad.append(f"blk {blk} head {h} {name} {pos}: gpu {x[pos]} oracle {y[pos]}"
+                                   + ("" if dist is None else f" distance {dist[pos]:.3e}"))
+    assert not bad, "records differ:\n" + "\n".join(bad[:12])
 
 
 # ---------------------------------------------------------------- full size, sampled
