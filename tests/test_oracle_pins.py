@@ -348,6 +348,22 @@ def test_value_constant_group_is_exact(orc):
     assert np.all(orc.decode_v(q, s, z) == 3.25)
 
 
+def test_value_near_ties_below_half_round_down(orc):
+    """Worked example of near-ties: a group with minimum 2^-24, maximum 15/16 and the
+    elements (2k + 1)/32 (all bf16 values).  z = fp16 down of 2^-24 = 2^-24 (0x0001),
+    s = fp16 up of (15/16 - 2^-24)/15, just below 1/16, = 1/16 (0x2C00), and
+    ((2k + 1)/32 - z)/s = k + 1/2 - 2^-20: 9.5e-7 below a .5 point, so every such
+    element takes code k (an exact tie would send odd k up to k + 1)."""
+    k = np.arange(15)
+    v = np.concatenate([[2.0 ** -24, 15 / 16], (2 * k + 1) / 32, (2 * k[::-1] + 1) / 32])
+    assert v.size == 32
+    q, s, z, r = orc.encode_v(bf16_bits_of(v))
+    assert int(z[0]) == 0x0001 and int(s[0]) == 0x2C00
+    assert q[0] == 0 and q[1] == 15
+    assert np.array_equal(q[2:17], k) and np.array_equal(q[17:], k[::-1])
+    assert np.allclose(r[2:17], k + 0.5 - 2.0 ** -20, rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- record format
 def test_record_size_and_nibble_order(orc):
     g = {r[0]: r[1:] for r in read_golden("worked_examples.txt")}

@@ -264,7 +264,8 @@ def test_bad_block_and_slot_set_status(tq):
 @pytest.mark.parametrize("d", [64, 128])
 def test_value_and_key_edge_data(tq, orc, d):
     """Zero keys, constant and integer-valued value groups (exact .5 ties), huge ranges,
-    groups whose (max - z)/15 is an fp16 value, and groups whose max - z is inexact in fp32."""
+    groups whose (max - z)/15 is an fp16 value, groups whose max - z is inexact in fp32,
+    and groups whose quotients lie 2^-20 off a .5 point."""
     H = 2
     T = 64
     rng = np.random.default_rng(5)
@@ -286,6 +287,12 @@ def test_value_and_key_edge_data(tq, orc, d):
     V[8] = rng.uniform(0.0, 1.0, (H, d))
     V[8, :, ::32] = 524288.0                      # max - z needs 29 bits: inexact in fp32
     V[8, :, 1::32] = 2.0 ** -10
+    # minimum 2^-24, maximum 15/16, elements (2k + 1)/32: s = 1/16 and every quotient
+    # 2^-20 below a .5 point (near-ties that round down)
+    k15 = np.arange(15)
+    near = np.concatenate([[2.0 ** -24, 15 / 16], (2 * k15 + 1) / 32, (2 * k15[::-1] + 1) / 32])
+    V[10] = np.tile(near, (H, d // 32))
+    V[11] = -np.tile(near[::-1], (H, d // 32))  # mirrored: minimum -15/16
     Kt = torch.from_numpy(K).to(torch.bfloat16)
     Vt = torch.from_numpy(V).to(torch.bfloat16)
     cache = tq.Cache(4, H, d)
