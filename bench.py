@@ -684,10 +684,12 @@ def run_tq(args, rank, world, local):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         s = oracle_sample(w, 1)
         oracle_step(w, s)
-        n_rep = 3
+        # passes until about 10 s of CPU work (at least 3, at most 60)
+        n_rep = 0
         t0 = time.perf_counter()
-        for _ in range(n_rep):
+        while n_rep < 3 or (n_rep < 60 and time.perf_counter() - t0 < 10.0):
             oracle_step(w, s)
+            n_rep += 1
         dt = (time.perf_counter() - t0) / n_rep
         cpu = {"value": s["L"] * w.Hkv * tq.record_bytes(w.d) // 16 / dt / 1e9, "unit": "GB/s", "cores": 1,
                "kind": "oracle",
