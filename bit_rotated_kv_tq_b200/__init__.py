@@ -91,6 +91,8 @@ def _stream(stream):
 
 
 def _dev(t, dtype, name):
+    """A contiguous CUDA tensor of `dtype` on the current device (the one the
+    library launches on), or None."""
     if t is None:
         return None
     if not t.is_cuda:
@@ -99,7 +101,33 @@ def _dev(t, dtype, name):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}; the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     return t
+
+
+def _shape(t, shape, name):
+    """The library sees bare pointers: every extent it will read or write is
+    checked here.  None in `shape` matches any size."""
+    if t is None:
+        return
+    if t.dim() != len(shape) or any(w is not None and int(g) != w for g, w in zip(t.shape, shape)):
+        want = "[" + "][".join("*" if w is None else str(w) for w in shape) + "]"
+        raise ValueError(f"{name} has shape {list(t.shape)}, expected {want}")
+
+
+def _tables(k_tables, cache):
+    """k_tables: [H_kv][16] values (any shape holding exactly that many)."""
+    if k_tables is not None and k_tables.numel() != cache.num_kv_heads * 16:
+        raise ValueError(f"k_tables holds {k_tables.numel()} values, expected "
+                         f"{cache.num_kv_heads} x 16")
+
+
+def _status(status):
+    """The library writes status[0] only."""
+    if status is not None and status.numel() < 1:
+        raise ValueError("status must hold at least one int32")
 
 
 # ------------------------------------------------------------------ sizes, tables
@@ -163,13 +191,20 @@ def quantize_append(K, V, slot_mapping, cache: Cache, block_table=None, k_tables
     With block_table (int32 [num_seqs][max_blocks]) the slots are logical:
     seq * max_blocks * 16 + position.
     """
+    T = K.shape[0] if K.dim() == 3 else -1
+    _shape(K, (T, cache.num_kv_heads, cache.head_dim), "K")
+    _shape(V, (T, cache.num_kv_heads, cache.head_dim), "V")
+    _shape(slot_mapping, (T,), "slot_mapping")
+    _shape(block_table, (None, None), "block_table")
+    _tables(k_tables, cache)
+    _status(status)
     _dev(K, torch.bfloat16, "K")
     _dev(V, torch.bfloat16, "V")
     _dev(slot_mapping, torch.int32, "slot_mapping")
     _dev(block_table, torch.int32, "block_table")
     _dev(k_tables, torch.float16, "k_tables")
     _dev(status, torch.int32, "status")
-    T = K.shape[0]
+    _dev(cache.data, torch.uint8, "cache.data")
     ns, mb = (0, 0) if block_table is None else (block_table.shape[0], block_table.shape[1])
     _check(load().tq_quantize_append(_ptr(K), _ptr(V), _ptr(block_table), ns, mb, _ptr(slot_mapping),
                                      T, cache.c, _ptr(k_tables), _ptr(status), _stream(stream)))
@@ -187,39 +222,50 @@ def decode_attention(q, cache: Cache, block_tables, seq_lens, max_seq_len: int, 
                      out=None, workspace=None, num_splits: int = 0, k_tables=None, status=None,
                      stream=None):
     """Split-K decode attention over the compressed cache; returns fp32 [B][H_q][d]."""
-    _dev(q, torch.bfloat16, "q")
-    _dev(block_tables, torch.int32, "block_tables")
-    _dev(seq_lens, torch.int32, "seq_lens")
-    _dev(k_tables, torch.float16, "k_tables")
-    _dev(status, torch.int32, "status")
-    B, Hq, d = q.shape
+    B, Hq, d = _decode_checks(q, cache, block_tables, seq_lens, out, k_tables, status)
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
-    _dev(out, torch.float32, "out")
     S = num_splits or default_splits(B, cache.num_kv_heads, max_seq_len)
     if workspace is None:
         nb = workspace_bytes(B, Hq, d, S)
         workspace = torch.empty(max(nb, 16), dtype=torch.uint8, device=q.device)
+    _dev(workspace, workspace.dtype, "workspace")
     _check(load().tq_decode_attention(_ptr(q), cache.c, _ptr(k_tables), _ptr(block_tables),
                                       block_tables.shape[1], _ptr(seq_lens), B, Hq, int(max_seq_len),
-                                      float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                      float(scale), _ptr(out), _ptr(workspace),
+                                      workspace.numel() * workspace.element_size(),
                                       int(num_splits), _ptr(status), _stream(stream)))
     return out
+
+
+def _decode_checks(q, cache, block_tables, seq_lens, out, k_tables, status):
+    """Shapes first (any device), then placement; returns (B, H_q, d)."""
+    if q.dim() != 3:
+        raise ValueError(f"q has shape {list(q.shape)}, expected [B][H_q][d]")
+    B, Hq, d = (int(x) for x in q.shape)
+    _shape(q, (B, Hq, cache.head_dim), "q")
+    _shape(block_tables, (B, None), "block_tables")
+    _shape(seq_lens, (B,), "seq_lens")
+    _shape(out, (B, Hq, d), "out")
+    _tables(k_tables, cache)
+    _status(status)
+    _dev(q, torch.bfloat16, "q")
+    _dev(block_tables, torch.int32, "block_tables")
+    _dev(seq_lens, torch.int32, "seq_lens")
+    _dev(out, torch.float32, "out")
+    _dev(k_tables, torch.float16, "k_tables")
+    _dev(status, torch.int32, "status")
+    _dev(cache.data, torch.uint8, "cache.data")
+    return B, Hq, d
 
 
 def decode_attention_static(q, cache: Cache, block_tables, seq_lens, max_seq_len: int, scale: float,
                             out=None, num_splits: int = 0, k_tables=None, status=None, stream=None):
     """decode_attention for callers that cannot allocate: no workspace argument; the split
     partials use the library's fixed device array (see tq_decode_attention_static)."""
-    _dev(q, torch.bfloat16, "q")
-    _dev(block_tables, torch.int32, "block_tables")
-    _dev(seq_lens, torch.int32, "seq_lens")
-    _dev(k_tables, torch.float16, "k_tables")
-    _dev(status, torch.int32, "status")
-    B, Hq, d = q.shape
+    B, Hq, d = _decode_checks(q, cache, block_tables, seq_lens, out, k_tables, status)
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
-    _dev(out, torch.float32, "out")
     _check(load().tq_decode_attention_static(_ptr(q), cache.c, _ptr(k_tables), _ptr(block_tables),
                                              block_tables.shape[1], _ptr(seq_lens), B, Hq,
                                              int(max_seq_len), float(scale), _ptr(out), int(num_splits),
@@ -230,6 +276,11 @@ def decode_attention_static(q, cache: Cache, block_tables, seq_lens, max_seq_len
 def dequantize(cache: Cache, block_tables, seq_lens, max_len: int, k_tables=None, status=None,
                stream=None):
     """(K_hat, V_hat) fp32 [B][max_len][H_kv][d] in the original domain (checks only)."""
+    _shape(block_tables, (None, None), "block_tables")
+    _shape(seq_lens, (block_tables.shape[0],), "seq_lens")
+    _tables(k_tables, cache)
+    _status(status)
+    _dev(cache.data, torch.uint8, "cache.data")
     _dev(block_tables, torch.int32, "block_tables")
     _dev(seq_lens, torch.int32, "seq_lens")
     _dev(k_tables, torch.float16, "k_tables")

@@ -122,8 +122,53 @@ def test_argument_validation_without_launch(lib):
     assert rc == tq.TQ_ERR_ALIGNMENT
 
 
+def _host_cache(num_kv_heads=2, head_dim=128, num_blocks=1):
+    rec = tq.record_bytes(head_dim)
+    return tq.Cache(num_blocks, num_kv_heads, head_dim,
+                    data=torch.zeros((num_blocks, num_kv_heads, rec), dtype=torch.uint8))
+
+
 def test_binding_refuses_host_tensors(lib):
-    c = tq.Cache.__new__(tq.Cache)
+    c = _host_cache()
     K = torch.zeros((1, 2, 128), dtype=torch.bfloat16)
-    with pytest.raises(ValueError):
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
         tq.quantize_append(K, K, torch.zeros(1, dtype=torch.int32), c)
+
+
+def test_binding_checks_extents_before_anything_runs(lib):
+    """The library reads and writes through bare pointers, so the binding refuses every
+    tensor whose extent differs from what the call would touch (before placement)."""
+    c = _host_cache()  # 2 kv heads, d 128
+
+    def bf(*shape):
+        return torch.zeros(shape, dtype=torch.bfloat16)
+
+    def i32(*shape):
+        return torch.zeros(shape, dtype=torch.int32)
+
+    f16 = torch.zeros(16, dtype=torch.float16)
+    cases = [
+        (lambda: tq.quantize_append(bf(4, 1, 128), bf(4, 1, 128), i32(4), c), "K has shape"),
+        (lambda: tq.quantize_append(bf(4, 2, 128), bf(4, 2, 64), i32(4), c), "V has shape"),
+        (lambda: tq.quantize_append(bf(4, 256), bf(4, 256), i32(4), c), "K has shape"),
+        (lambda: tq.quantize_append(bf(4, 2, 128), bf(4, 2, 128), i32(3), c), "slot_mapping has shape"),
+        (lambda: tq.quantize_append(bf(4, 2, 128), bf(4, 2, 128), i32(4), c, k_tables=f16),
+         "k_tables holds 16 values"),
+        (lambda: tq.decode_attention(bf(2, 8, 64), c, i32(2, 4), i32(2), 64, 0.1), "q has shape"),
+        (lambda: tq.decode_attention(bf(2, 8, 128), c, i32(3, 4), i32(2), 64, 0.1),
+         "block_tables has shape"),
+        (lambda: tq.decode_attention(bf(2, 8, 128), c, i32(2, 4), i32(3), 64, 0.1), "seq_lens has shape"),
+        (lambda: tq.decode_attention(bf(2, 8, 128), c, i32(2, 4), i32(2), 64, 0.1,
+                                     out=torch.zeros((2, 8, 64))), "out has shape"),
+        (lambda: tq.decode_attention(bf(2, 8, 128), c, i32(2, 4), i32(2), 64, 0.1, status=i32(0)),
+         "status must hold"),
+        (lambda: tq.decode_attention_static(bf(2, 8, 128), c, i32(2, 4), i32(1), 64, 0.1),
+         "seq_lens has shape"),
+        (lambda: tq.dequantize(c, i32(2, 4), i32(3), 64), "seq_lens has shape"),
+    ]
+    for call, msg in cases:
+        with pytest.raises(ValueError, match=msg):
+            call()
+    # the right extents on the host are refused for their placement
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        tq.decode_attention(bf(2, 8, 128), c, i32(2, 4), i32(2), 64, 0.1)
