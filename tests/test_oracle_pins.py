@@ -489,6 +489,67 @@ def test_attention_special_cases(orc):
     assert np.all(empty == 0.0)
 
 
+def test_attention_split_then_combine_equals_whole(orc):
+    """Attention over disjoint token ranges, merged by their softmax masses
+    (o = sum_s l_s o_s / sum_s l_s, l_s = sum over range s of exp(a_t - M)), equals the
+    attention over the whole sequence: the identity a split-K decode relies on."""
+    q, Kh, Vh = _attn_case(B=1, Hq=2, Hkv=1, L=61)
+    scale = 0.7
+    whole = orc.attention(q, Kh, Vh, np.array([61], np.int32), scale)
+    qd = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).double().numpy()
+    cuts = [0, 5, 6, 30, 61]  # ranges of 5, 1, 24 and 31 tokens
+    for h in range(2):
+        a = scale * Kh[0, :, 0] @ qd[0, h]
+        M = a.max()
+        o, l = 0.0, 0.0
+        for c0, c1 in zip(cuts[:-1], cuts[1:]):
+            part = orc.attention(q, Kh[:, c0:c1], Vh[:, c0:c1], np.array([c1 - c0], np.int32), scale)
+            ls = np.exp(a[c0:c1] - M).sum()
+            o, l = o + ls * part[0, h], l + ls
+        assert np.allclose(o / l, whole[0, h], rtol=0, atol=1e-14)
+
+
+def test_shared_prefix_tables_equal_private_copies(orc):
+    """Two sequences whose first two blocks are one physical copy (block tables share
+    them) dequantise, and attend, exactly as with private copies of those blocks."""
+    H, d, L = 2, 64, 48
+    K, V = _rand_kv(L, H, d)
+    rec = orc.record_bytes(d)
+    lens = np.array([L, L], np.int32)
+    q = bf16_bits_of(RNG.standard_normal((2, 4, d)))
+
+    def run(bt, seq1_positions):
+        cache = np.zeros((int(bt.max()) + 1, H, rec), np.uint8)
+        cap = bt.shape[1] * 16
+        orc.quantize_append(K, V, np.arange(L, dtype=np.int32), cache, block_table=bt)
+        p = np.asarray(seq1_positions)
+        orc.quantize_append(K[p], V[p], (cap + p).astype(np.int32), cache, block_table=bt)
+        Kh, Vh = orc.dequantize(cache, H, d, bt, lens, L)
+        return Kh, Vh, orc.attention(q, Kh, Vh, lens, 0.125)
+
+    shared = run(np.array([[0, 1, 2], [0, 1, 3]], np.int32), np.arange(32, L))
+    private = run(np.array([[0, 1, 2], [4, 5, 3]], np.int32), np.arange(L))
+    for x, y in zip(shared, private):
+        assert np.array_equal(x, y)
+    assert np.array_equal(shared[0][0], shared[0][1])  # both sequences hold the same tokens
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_scores_in_rotated_domain_equal_original_domain(orc, d):
+    """H is symmetric and orthonormal, so q . k_hat = (H q) . (n16 C[idx]): the scores can
+    be taken against the stored centroids once the query is rotated (H from scipy)."""
+    table = orc.default_table(d).astype(np.float64)
+    Hs = scipy.linalg.hadamard(d) / math.sqrt(d)
+    for _ in range(20):
+        kb = bf16_bits_of(RNG.standard_normal(d) * 3.0)
+        idx, n16, _ = orc.encode_k(kb, orc.default_table(d))
+        khat = orc.decode_k(idx, n16, orc.default_table(d))
+        qd = RNG.standard_normal(d)
+        n = float(np.uint16(n16).view(np.float16))
+        rot = (Hs @ qd) @ (n * table[idx])
+        assert abs(qd @ khat - rot) <= 1e-12 * np.linalg.norm(qd) * np.linalg.norm(khat)
+
+
 def test_attention_invariant_to_token_order(orc):
     q, Kh, Vh = _attn_case(B=1, L=30)
     p = RNG.permutation(30)
