@@ -233,8 +233,10 @@ def dequantize(cache, Hkv, d, block_tables, seq_lens, max_len, tables=None):
     bt = _c(block_tables, np.int32)
     sl = _c(seq_lens, np.int32)
     B, max_blocks = bt.shape
-    Kh = np.zeros((B, max_len, Hkv, d), np.float64)
-    Vh = np.zeros((B, max_len, Hkv, d), np.float64)
+    # filled with NaN so that the oracle's own clearing of rows past each length is
+    # what a caller sees (a missed row would show as NaN, not as a lucky 0)
+    Kh = np.full((B, max_len, Hkv, d), np.nan, np.float64)
+    Vh = np.full((B, max_len, Hkv, d), np.nan, np.float64)
     tb = None if tables is None else _h(tables)
     rc = lib().orc_dequantize(_ptr(cache), cache.shape[0], Hkv, d, _ptr(tb), _ptr(bt), max_blocks,
                               _ptr(sl), B, max_len, _ptr(Kh), _ptr(Vh))

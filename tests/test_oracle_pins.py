@@ -627,3 +627,110 @@ def test_record_placement_round_trip(orc, d):
         k2, n2, v2, s2, z2 = orc.unpack_token(record, d, t)
         assert np.array_equal(k2, kidx[t]) and n2 == kn[t] and np.array_equal(v2, vq[t])
         assert np.array_equal(s2, vs[t]) and np.array_equal(z2, vz[t])
+
+
+# ---------------------------------------------------------------- cache glue
+def _glue_case(orc):
+    """2 sequences x 3 kv heads at d 64, ragged lengths 37 and 50, shuffled
+    physical blocks, three different per-head key tables: the default, one
+    re-fitted by k-means, and the default scaled by 1.25 (still fp16-exact
+    and strictly ascending)."""
+    d, H = 64, 3
+    r = np.random.default_rng(2024)
+    lens = np.array([37, 50], np.int32)
+    nblk = (lens + 15) // 16
+    max_blocks = int(nblk.max()) + 1  # one spare column, never read
+    perm = r.permutation(int(nblk.sum()) + 2).astype(np.int32)  # two physical blocks unused
+    bt = np.full((2, max_blocks), -1, np.int32)
+    bt[0, :nblk[0]] = perm[:nblk[0]]
+    bt[1, :nblk[1]] = perm[nblk[0]:nblk[0] + nblk[1]]
+    t0 = orc.default_table(d)
+    kb = bf16_bits_of(r.standard_t(4, (20, d)))
+    fitted, _ = orc.kmeans_table(orc.rotated_unit_samples(kb), t0, 100)
+    scaled = (t0.astype(np.float64) * 1.25).astype(np.float16)
+    tables = np.stack([t0, fitted, scaled]).astype(np.float16)
+    assert not np.array_equal(tables[0], tables[1]) and not np.array_equal(tables[0], tables[2])
+    T = int(lens.sum())
+    K = bf16_bits_of(r.standard_normal((T, H, d)) * r.lognormal(0, 1, (1, H, d)))
+    V = bf16_bits_of(r.standard_normal((T, H, d)) * 3.0)
+    seq = np.repeat(np.arange(2), lens)
+    pos = np.concatenate([np.arange(L) for L in lens])
+    logical = (seq * max_blocks * 16 + pos).astype(np.int32)
+    cache = np.zeros((len(perm), H, orc.record_bytes(d)), np.uint8)
+    assert orc.quantize_append(K, V, logical, cache, tables=tables, block_table=bt)[0] == 0
+    return dict(d=d, H=H, lens=lens, bt=bt, tables=tables, K=K, V=V, seq=seq, pos=pos,
+                cache=cache, max_len=int(lens.max()) + 3)
+
+
+def _expected_rows(orc, c):
+    """Per (b, t, h): decode_k(encode_k(k, table[h])) and decode_v(encode_v(v)),
+    the already pinned per-vector codecs, with no record, block or stride in between."""
+    d, H = c["d"], c["H"]
+    Ke = np.zeros((2, c["max_len"], H, d))
+    Ve = np.zeros((2, c["max_len"], H, d))
+    for i in range(len(c["seq"])):
+        b, t = c["seq"][i], c["pos"][i]
+        for h in range(H):
+            idx, n16, _ = orc.encode_k(c["K"][i, h], c["tables"][h])
+            Ke[b, t, h] = orc.decode_k(idx, n16, c["tables"][h])
+            q, s, z, _ = orc.encode_v(c["V"][i, h])
+            Ve[b, t, h] = orc.decode_v(q, s, z)
+    return Ke, Ve
+
+
+def _check_glue(c, Kh, Vh, Ke, Ve):
+    """Every valid row equals the per-vector codecs' row (bit for bit); every row
+    at or past a sequence's length is exactly 0."""
+    for b, L in enumerate(c["lens"]):
+        assert np.array_equal(Kh[b, :L], Ke[b, :L]), f"keys of sequence {b}"
+        assert np.array_equal(Vh[b, :L], Ve[b, :L]), f"values of sequence {b}"
+        assert np.all(Kh[b, L:] == 0) and np.all(Vh[b, L:] == 0), f"rows past length {L}"
+
+
+def test_dequantize_with_per_head_tables_equals_per_vector_codecs(orc):
+    """orc_dequantize and the per-head-table branch of orc_quantize_append, pinned
+    against encode/decode of each vector alone (which are pinned to scipy, Max 1960,
+    brute force and exact arithmetic above)."""
+    c = _glue_case(orc)
+    Ke, Ve = _expected_rows(orc, c)
+    Kh, Vh = orc.dequantize(c["cache"], c["H"], c["d"], c["bt"], c["lens"], c["max_len"],
+                            tables=c["tables"])
+    _check_glue(c, Kh, Vh, Ke, Ve)
+    # the records themselves, read by the test-side reader of the documented layout,
+    # hold the per-vector codes of each head's own table
+    from parity_util import unpack_record
+
+    for i in range(len(c["seq"])):
+        b, t = c["seq"][i], c["pos"][i]
+        blk = c["bt"][b, t // 16]
+        for h in range(c["H"]):
+            kidx, kn, vq, vs, vz = unpack_record(c["cache"][blk, h], c["d"])
+            idx, n16, _ = orc.encode_k(c["K"][i, h], c["tables"][h])
+            q, s, z, _ = orc.encode_v(c["V"][i, h])
+            assert np.array_equal(kidx[t % 16], idx) and kn[t % 16] == n16
+            assert np.array_equal(vq[t % 16], q) and np.array_equal(vs[t % 16], s)
+            assert np.array_equal(vz[t % 16], z)
+
+
+def test_glue_check_catches_planted_mistakes(orc):
+    """The check above fails under each plausible mistake of the glue, planted in
+    the oracle's result here on the CPU: the token and head strides swapped, every
+    head decoded with head 0's table, rows past the length left stale."""
+    c = _glue_case(orc)
+    Ke, Ve = _expected_rows(orc, c)
+    d, H, ml = c["d"], c["H"], c["max_len"]
+    Kh, Vh = orc.dequantize(c["cache"], H, d, c["bt"], c["lens"], ml, tables=c["tables"])
+    # [b][t][h][d] written as [b][h][t][d]
+    swapped = np.ascontiguousarray(Kh.transpose(0, 2, 1, 3)).reshape(Kh.shape)
+    with pytest.raises(AssertionError):
+        _check_glue(c, swapped, Vh, Ke, Ve)
+    # head_table ignoring h
+    Kw, Vw = orc.dequantize(c["cache"], H, d, c["bt"], c["lens"], ml,
+                            tables=np.stack([c["tables"][0]] * H))
+    with pytest.raises(AssertionError):
+        _check_glue(c, Kw, Vw, Ke, Ve)
+    # rows past the length not cleared (a buffer reused from a longer call)
+    stale_K, stale_V = Kh.copy(), Vh.copy()
+    stale_K[0, c["lens"][0]:] = 0.5
+    with pytest.raises(AssertionError):
+        _check_glue(c, stale_K, stale_V, Ke, Ve)
