@@ -131,6 +131,73 @@ bool check_cache(const tq_cache_t* c, int* err) {
 namespace tq {
 // Record a failure for tq_last_error() from another translation unit.
 int set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
+// Every host check of a decode call, then its split plan.  On TQ_OK with B > 0,
+// `a` is ready for decode_launch and `need` holds the workspace bytes the plan
+// uses (0 when nothing has to be combined); nothing has been enqueued.
+int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
+                   const int32_t* block_tables, int max_blocks, const int32_t* seq_lens, int B,
+                   int H_q, int max_seq_len, float scale, float* out, int num_splits,
+                   int32_t* status, DecodeArgs& a, size_t& need) {
+    int err;
+    need = 0;
+    if (!check_cache(cache, &err)) return err;
+    if (B < 0 || H_q <= 0 || max_blocks <= 0 || max_seq_len < 0 ||
+        (long long)max_seq_len > (long long)max_blocks * kBlock)
+        return fail(TQ_ERR_INVALID_ARG,
+                    "tq_decode_attention: need B >= 0, H_q > 0, 0 <= max_seq_len <= max_blocks*16");
+    if (num_splits < 0 || num_splits > 1024)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: num_splits %d (0..1024)", num_splits);
+    if (B == 0) return ok();
+    if (B > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B %d > 65535", B);
+    if (!q || !block_tables || !seq_lens || !out)
+        return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: q, block_tables, seq_lens, out required");
+    const int Hkv = cache->num_kv_heads;
+    if (H_q % Hkv)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: H_q %d not a multiple of H_kv %d", H_q, Hkv);
+    const int G = H_q / Hkv;
+    if (G > 64)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: GQA group %d (supported 1..64)", G);
+    if (!isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: scale not finite");
+    if (!aligned(q, 4) || !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(seq_lens, 4) ||
+        (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
+        return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: q/out/tables must be 4-byte aligned");
+    const int d = cache->head_dim;
+    a = DecodeArgs{};
+    a.q = static_cast<const uint16_t*>(q);
+    a.cache = static_cast<const unsigned char*>(cache->data);
+    a.num_blocks = cache->num_blocks;
+    a.Hkv = Hkv;
+    a.Hq = H_q;
+    a.B = B;
+    a.k_tables = k_tables;
+    memcpy(a.default_table, default_table(d), sizeof a.default_table);
+    a.block_tables = block_tables;
+    a.max_blocks = max_blocks;
+    a.seq_lens = seq_lens;
+    a.scale_log2 = scale * 1.44269504088896340736f;
+    a.out = out;
+    a.num_splits = num_splits;
+    a.max_seq_len = max_seq_len;
+    a.status = status;
+    if (!decode_plan(a, d, device_sms()))
+        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * num_splits too large");
+    need = decode_workspace_for(a, d);
+    return ok();
+}
+
+// Launch a prepared decode with its partials in `workspace` (the plan's
+// decode_workspace_for bytes, 16-byte aligned; unused when that is 0).
+int decode_launch(DecodeArgs& a, int head_dim, void* workspace, void* stream) {
+    a.ws_o = static_cast<float*>(workspace);
+    // [ranges][2][heads per item][d] partial outputs, then [ranges][2][heads per item] (m, l)
+    a.ws_ml = workspace ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
+                                                    (size_t)a.nranges * 2 * 4 * a.qpi * head_dim)
+                        : nullptr;
+    cudaError_t e = launch_decode(a, head_dim, device_sms(), (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");
+    return ok();
+}
 }  // namespace tq
 
 extern "C" {
@@ -290,48 +357,11 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
                         int B, int H_q, int max_seq_len, float scale, float* out,
                         void* workspace, size_t ws_bytes, int num_splits, int32_t* status,
                         void* stream) {
-    int err;
-    if (!check_cache(cache, &err)) return err;
-    if (B < 0 || H_q <= 0 || max_blocks <= 0 || max_seq_len < 0 ||
-        (long long)max_seq_len > (long long)max_blocks * tq::kBlock)
-        return fail(TQ_ERR_INVALID_ARG,
-                    "tq_decode_attention: need B >= 0, H_q > 0, 0 <= max_seq_len <= max_blocks*16");
-    if (B == 0) return ok();
-    if (B > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B %d > 65535", B);
-    if (!q || !block_tables || !seq_lens || !out)
-        return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: q, block_tables, seq_lens, out required");
-    const int Hkv = cache->num_kv_heads;
-    if (H_q % Hkv)
-        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: H_q %d not a multiple of H_kv %d", H_q, Hkv);
-    const int G = H_q / Hkv;
-    if (G > 64)
-        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: GQA group %d (supported 1..64)", G);
-    if (num_splits < 0 || num_splits > 1024)
-        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: num_splits %d (0..1024)", num_splits);
-    if (!isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: scale not finite");
-    if (!aligned(q, 4) || !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(seq_lens, 4) ||
-        (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
-        return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: q/out/tables must be 4-byte aligned");
-    const int d = cache->head_dim;
     tq::DecodeArgs a;
-    a.q = static_cast<const uint16_t*>(q);
-    a.cache = static_cast<const unsigned char*>(cache->data);
-    a.num_blocks = cache->num_blocks;
-    a.Hkv = Hkv;
-    a.Hq = H_q;
-    a.B = B;
-    a.k_tables = k_tables;
-    memcpy(a.default_table, default_table(d), sizeof a.default_table);
-    a.block_tables = block_tables;
-    a.max_blocks = max_blocks;
-    a.seq_lens = seq_lens;
-    a.scale_log2 = scale * 1.44269504088896340736f;
-    a.out = out;
-    a.num_splits = num_splits;
-    a.max_seq_len = max_seq_len;
-    if (!tq::decode_plan(a, d, device_sms()))
-        return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * num_splits too large");
-    const size_t need = tq::decode_workspace_for(a, d);
+    size_t need = 0;
+    const int err = tq::decode_prepare(q, cache, k_tables, block_tables, max_blocks, seq_lens, B, H_q,
+                                       max_seq_len, scale, out, num_splits, status, a, need);
+    if (err != TQ_OK || B == 0) return err;
     if (need) {
         if (!workspace || ws_bytes < need)
             return fail(TQ_ERR_WORKSPACE, "tq_decode_attention: workspace %zu bytes < %zu needed",
@@ -339,15 +369,7 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
         if (!aligned(workspace, 16))
             return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: workspace must be 16-byte aligned");
     }
-    a.ws_o = static_cast<float*>(workspace);
-    // [ranges][2][heads per item][d] partial outputs, then [ranges][2][heads per item] (m, l)
-    a.ws_ml = need ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
-                                               (size_t)a.nranges * 2 * 4 * a.qpi * d)
-                   : nullptr;
-    a.status = status;
-    cudaError_t e = tq::launch_decode(a, d, device_sms(), (cudaStream_t)stream);
-    if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");
-    return ok();
+    return tq::decode_launch(a, cache->head_dim, need ? workspace : nullptr, stream);
 }
 
 TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, const int32_t* block_tables,

@@ -36,6 +36,8 @@
 // comparison of 15 s with max - z (fp64 when max - z is inexact in fp32).  The
 // stored codes are therefore those of the exact-arithmetic definition except
 // within ~1e-15 (relative) of a key threshold.
+#include <mutex>
+
 #include "tq_kernels.cuh"
 
 namespace tq {
@@ -219,13 +221,13 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         for (int j = 1; j < 8; j++) {
             const __nv_bfloat162 w = *reinterpret_cast<const __nv_bfloat162*>(&vwd[j]);
             mn2 = __hmin2(mn2, w);
-            mx2 = __hmax2(mx2, w);
+            mx2 = __hmax2_nan(mx2, w);  // a NaN reaches the scale and flags the group
         }
         {
             const uint32_t pm = __shfl_xor_sync(kFull, *reinterpret_cast<const uint32_t*>(&mn2), 1);
             const uint32_t px = __shfl_xor_sync(kFull, *reinterpret_cast<const uint32_t*>(&mx2), 1);
             mn2 = __hmin2(mn2, *reinterpret_cast<const __nv_bfloat162*>(&pm));
-            mx2 = __hmax2(mx2, *reinterpret_cast<const __nv_bfloat162*>(&px));
+            mx2 = __hmax2_nan(mx2, *reinterpret_cast<const __nv_bfloat162*>(&px));
         }
         const uint32_t mnw = *reinterpret_cast<const uint32_t*>(&mn2);
         const uint32_t mxw = *reinterpret_cast<const uint32_t*>(&mx2);
@@ -551,35 +553,38 @@ size_t append_smem_bytes(int ntab) {
     return (size_t)ntab * kBins * sizeof(BinEntry) + (size_t)ntab * sizeof(HeadBins);
 }
 
+// CTAs of append_kernel<D> resident per SM with this much dynamic shared memory,
+// by size class, computed once per process.
 template <int D>
 static int resident_ctas(int num_sms, size_t smem) {
-    static int per_sm[2] = {0, 0};  // by (smem size class); set once per process
+    static std::once_flag once[2];
+    static int per_sm[2] = {0, 0};
     const int key = smem > 16384 ? 1 : 0;
-    if (!per_sm[key]) {
+    std::call_once(once[key], [&] {
         int n = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_kernel<D>, 256, smem) !=
                 cudaSuccess || n <= 0)
             n = 1;
         per_sm[key] = n;
-    }
+    });
     return per_sm[key] * num_sms;
 }
 
-// The bins of the default table of head_dim d, computed once per process.
+// The bins of the default table of head_dim d, computed once per process
+// (every caller waits until they are complete).
 static void default_bins(int d, const uint16_t* table16, HeadBins& hb, BinEntry* bins) {
+    static std::once_flag once[2];
     static HeadBins cached_hb[2];
     static BinEntry cached[2][kBins];
-    static bool ready[2] = {false, false};
     const int key = d == 128 ? 1 : 0;
-    if (!ready[key]) {
+    std::call_once(once[key], [&] {
         HeadBins& h = cached_hb[key];
         for (int k = 0; k < 16; k++) h.c[k] = __half2float(__ushort_as_half(table16[k]));
         h.dense = 0;
         h.pad = 0;
         for (int b = 0; b < kBins; b++)
             if (bin_entry(h.c, b, cached[key][b])) h.dense = 1;
-        ready[key] = true;
-    }
+    });
     hb = cached_hb[key];
     memcpy(bins, cached[key], sizeof cached[key]);
 }

@@ -37,6 +37,8 @@
 // accumulators are rescaled only when a running maximum moves.  An item
 // that lies wholly inside one range is written directly; the others leave an
 // unnormalised partial (o, m, l) per range that the combine kernel merges.
+#include <mutex>
+
 #include "tq_kernels.cuh"
 
 namespace tq {
@@ -739,17 +741,22 @@ __global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
 
 template <int D, int QPI>
 cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
-    static uint32_t smem = 0;
+    // the kernel's shared-memory size, set once per device (under a lock: the
+    // library may be called from several host threads)
+    static std::mutex mu;
     static bool configured[64] = {};
+    static const uint32_t smem = plan_bytes<D, kHeads * QPI>();
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (!smem) smem = plan_bytes<D, kHeads * QPI>();
-    if (dev < 0 || dev >= 64 || !configured[dev]) {
-        e = cudaFuncSetAttribute(decode_split_kernel<D, QPI>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        if (dev >= 0 && dev < 64) configured[dev] = true;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (dev < 0 || dev >= 64 || !configured[dev]) {
+            e = cudaFuncSetAttribute(decode_split_kernel<D, QPI>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) configured[dev] = true;
+        }
     }
     a.smem_bytes = smem;
     const int halves = (a.nranges + kHalves - 1) / kHalves;

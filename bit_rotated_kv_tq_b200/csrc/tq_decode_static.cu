@@ -12,7 +12,10 @@
 // The array lives in device memory of every GPU that loads the library, for
 // the life of the process, so it is kept small (kScratchBytes).  Its host-side
 // name is only a stand-in for the symbol; the device address is looked up
-// once per device with cudaGetSymbolAddress and cached.
+// once per device with cudaGetSymbolAddress and cached.  A device reset
+// (cudaDeviceReset, or anything else that destroys the primary context)
+// unloads the module and leaves that cached address stale: a process that
+// resets a device must not call tq_decode_attention_static on it afterwards.
 #include <stdio.h>
 
 #include <mutex>
@@ -55,35 +58,35 @@ TQ_API int tq_decode_attention_static(const void* q, const tq_cache_t* cache,
                                       int max_blocks, const int32_t* seq_lens, int B, int H_q,
                                       int max_seq_len, float scale, float* out, int num_splits,
                                       int32_t* status, void* stream) {
-    if (!cache || B < 0 || H_q <= 0 || num_splits < 0) {
-        // let the full checks of tq_decode_attention report the problem
-        return tq_decode_attention(q, cache, k_tables, block_tables, max_blocks, seq_lens, B, H_q,
-                                   max_seq_len, scale, out, nullptr, 0, num_splits, status, stream);
-    }
-    const size_t need = tq_decode_workspace_bytes(B, H_q, cache->head_dim, num_splits);
+    // every check of tq_decode_attention first, so a bad argument gets its own code
+    tq::DecodeArgs a;
+    size_t need = 0;
+    const int err = tq::decode_prepare(q, cache, k_tables, block_tables, max_blocks, seq_lens, B,
+                                       H_q, max_seq_len, scale, out, num_splits, status, a, need);
+    if (err != TQ_OK || B == 0) return err;
     if (need > kScratchBytes) {
         char msg[256];
         snprintf(msg, sizeof msg,
-                 "tq_decode_attention_static: num_splits %d may need %zu bytes of partials, more "
-                 "than the library's fixed %zu-byte scratch; pass 0 or fewer splits, or use "
-                 "tq_decode_attention",
+                 "tq_decode_attention_static: this split plan (num_splits %d) needs %zu bytes of "
+                 "partials, more than the library's fixed %zu-byte scratch; pass fewer splits "
+                 "(1 needs none) or use tq_decode_attention",
                  num_splits, need, kScratchBytes);
         return tq::set_last_error(TQ_ERR_WORKSPACE, msg);
     }
-    cudaError_t e = cudaSuccess;
-    void* ws = scratch_on_current_device(&e);
-    if (!ws) {
-        char msg[256];
-        snprintf(msg, sizeof msg, "tq_decode_attention_static: scratch address lookup failed: %s",
-                 cudaGetErrorString(e));
-        return tq::set_last_error(TQ_ERR_CUDA, msg);
+    void* ws = nullptr;
+    if (need) {
+        cudaError_t e = cudaSuccess;
+        ws = scratch_on_current_device(&e);
+        if (!ws) {
+            char msg[256];
+            snprintf(msg, sizeof msg, "tq_decode_attention_static: scratch address lookup failed: %s",
+                     cudaGetErrorString(e));
+            return tq::set_last_error(TQ_ERR_CUDA, msg);
+        }
     }
-    // Every partial slot is written by the split kernel before the combine reads
-    // it, so nothing in the scratch has to start at zero; the bound above covers
-    // the plan tq_decode_attention makes from the same num_splits.
-    return tq_decode_attention(q, cache, k_tables, block_tables, max_blocks, seq_lens, B, H_q,
-                               max_seq_len, scale, out, ws, kScratchBytes, num_splits, status,
-                               stream);
+    // Every partial slot the plan uses is written by the split kernel before the
+    // combine reads it, so nothing in the scratch has to start at zero.
+    return tq::decode_launch(a, cache->head_dim, ws, stream);
 }
 
 }  // extern "C"

@@ -124,6 +124,13 @@ struct DequantArgs {
     int32_t* status;
 };
 
+// Host checks and split plan of a decode call (the checks of tq_decode_attention
+// except the workspace ones); on TQ_OK with B > 0, `need` is the plan's workspace.
+int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
+                   const int32_t* block_tables, int max_blocks, const int32_t* seq_lens, int B,
+                   int H_q, int max_seq_len, float scale, float* out, int num_splits,
+                   int32_t* status, DecodeArgs& a, size_t& need);
+int decode_launch(DecodeArgs& a, int head_dim, void* workspace, void* stream);
 size_t append_smem_bytes(int ntab);  // ntab bin tables (1, or H_kv per-head tables)
 int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);

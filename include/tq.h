@@ -165,16 +165,19 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
  * tensors of the call while the host runtime owns (and pools) every other
  * byte of device memory, so it has no way to hand over a workspace.
  * Same arguments, result and checks as tq_decode_attention minus workspace /
- * ws_bytes; the split partials go to a fixed array compiled into the library
+ * ws_bytes (those checks run first, with the same error codes); the split
+ * partials go to a fixed array compiled into the library
  * (tq_decode_static_scratch_bytes() bytes, 8 MiB, present on every GPU that
  * loads the library until the process exits).  The call allocates and frees
- * nothing.  A split plan whose partials exceed the array
- * (tq_decode_workspace_bytes(B, H_q, d, splits) > 8 MiB) is rejected with
- * TQ_ERR_WORKSPACE before anything is enqueued; pass fewer splits (1 needs
- * none) or use tq_decode_attention.
- * The first call on a device looks the array's address up
- * (cudaGetSymbolAddress) and caches it; make that first call before any
- * stream capture.  All calls share the one array and it keeps the last
+ * nothing.  A split plan whose partials exceed the array is rejected with
+ * TQ_ERR_WORKSPACE before anything is enqueued (tq_decode_workspace_bytes
+ * bounds a plan's partials from above); pass fewer splits (1 needs none) or
+ * use tq_decode_attention.
+ * The first call on a device that needs partials looks the array's address
+ * up (cudaGetSymbolAddress) and caches it; make that first call before any
+ * stream capture.  A device reset (cudaDeviceReset) makes the cached address
+ * stale: do not use this call on a device after resetting it.  All calls
+ * share the one array and it keeps the last
  * call's contents (nothing in it needs to start at zero): calls that overlap
  * on the GPU -- on different streams, or from different threads -- race on
  * it and must be ordered by the caller. */

@@ -117,6 +117,19 @@ def test_argument_validation_without_launch(lib):
     assert lib.tq_decode_workspace_bytes(2, 8, 128, 4) == (2 * 8 * 4 + 1) * 2 * 4 * (128 * 4 + 8)
     assert lib.tq_decode_workspace_bytes(2, 8, 64, 3) == (2 * 8 * 3 + 1) * 2 * 4 * (64 * 4 + 8)
     assert lib.tq_decode_workspace_bytes(2, 8, 128, 1) == 0
+    # the fixed-scratch entry runs the same checks first, with the same codes
+    def dec_static(**kw):
+        a = {**args, **kw}
+        return lib.tq_decode_attention_static(a["q"], ctypes.byref(c), a["k"], a["bt"], a["mb"],
+                                              a["sl"], a["B"], a["Hq"], a["L"],
+                                              ctypes.c_float(a["scale"]), a["out"], a["S"], None, None)
+
+    assert dec_static(Hq=4, S=1025) == tq.TQ_ERR_UNSUPPORTED
+    assert dec_static(Hq=4, S=1025, B=4096) == tq.TQ_ERR_UNSUPPORTED
+    assert dec_static(Hq=5) == tq.TQ_ERR_UNSUPPORTED
+    assert dec_static(Hq=4, L=65) == tq.TQ_ERR_INVALID_ARG
+    assert dec_static(Hq=4, q=None) == tq.TQ_ERR_INVALID_ARG
+    assert dec_static(Hq=4, B=0) == tq.TQ_OK
     # dequantize: misaligned output
     rc = lib.tq_dequantize(ctypes.byref(c), None, P(16), 4, P(16), 1, 8, P(20), P(16), None, None)
     assert rc == tq.TQ_ERR_ALIGNMENT

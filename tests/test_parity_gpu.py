@@ -173,11 +173,28 @@ def test_dequantize_matches_oracle(tq, orc):
     ("prefill_small_head", dict(B=1, ctx=520, Hq=32), 2),  # GQA 16: two items of 8 heads
     ("qwen3_8b_layer", dict(B=2, ctx=200, Hq=48), 0),      # GQA 6 at d = 128: 4 + 2
     ("qwen3_8b_layer", dict(B=2, ctx=150, Hq=24), 2),      # GQA 3 at d = 128
+    # the largest GQA groups the library accepts: several 8-head items per kv head at d = 64,
+    # 8 and 16 four-head items per kv head at d = 128
+    ("prefill_small_head", dict(B=2, ctx=300, Hq=64), 0),   # GQA 32 at d = 64
+    ("prefill_small_head", dict(B=1, ctx=260, Hq=128), 3),  # GQA 64 at d = 64
+    ("qwen3_8b_layer", dict(B=2, ctx=180, Hq=32, Hkv=1), 2),  # GQA 32 at d = 128
+    ("qwen3_8b_layer", dict(B=2, ctx=200, Hq=64, Hkv=1), 0),  # GQA 64 at d = 128
+    # the most kv heads the cache accepts
+    ("qwen3_8b_layer", dict(B=2, ctx=150, Hq=32, Hkv=16), 0),  # H_kv 16
+    ("qwen3_8b_layer", dict(B=1, ctx=170, Hq=32, Hkv=32), 4),  # H_kv 32, GQA 1
+    ("prefill_small_head", dict(B=2, ctx=140, Hq=64, Hkv=32), 0),  # H_kv 32 at d = 64
 ])
 def test_reduced_configs(tq, orc, name, over, S):
     w = W.make(name, **over)
     pairs = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
     check_pairs(tq, orc, w, pairs, num_splits=S)
+
+
+def test_calibrated_tables_for_32_kv_heads(tq, orc):
+    """Per-head re-fitted tables at the most kv heads the cache takes: the append builds
+    one bin table per head in shared memory, the decode one centroid table per head."""
+    w = W.make("qwen3_8b_layer", B=2, ctx=120, Hq=64, Hkv=32)
+    check_pairs(tq, orc, w, [(b, h) for b in range(w.B) for h in range(0, 32, 3)], calibrated=True)
 
 
 def test_agentic_reduced_calibrated(tq, orc):
@@ -259,6 +276,52 @@ def test_bad_block_and_slot_set_status(tq):
     tq.decode_attention(w.q().cuda(), g.cache, g.bt, lens, 32, w.scale, num_splits=1, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) & tq.STATUS_BAD_LEN
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_out_of_range_inputs_set_status(tq, orc, d):
+    """Inputs whose stored fields cannot hold them set TQ_STATUS_RANGE: a key whose norm
+    exceeds 65504 (the largest fp16), a value group whose range needs a scale above 65504,
+    a value group whose minimum rounds down past -65504, a NaN in a value and a NaN in a
+    key.  Every other token's record still equals the oracle's byte for byte."""
+    H, T = 2, 48
+    rng = np.random.default_rng(31 + d)
+    K = rng.standard_normal((T, H, d)).astype(np.float32)
+    V = rng.standard_normal((T, H, d)).astype(np.float32)
+    K[3, 0, 5] = 70000.0            # norm > 65504: the fp16 norm overflows
+    V[5, 1, :32] = np.linspace(-1.0, 1.0e6, 32)  # (max - z) / 15 > 65504
+    V[9, 0, 32:64] = -1.0e5         # z = fp16 rounded down from -1e5: overflows
+    V[20, 1, 40] = np.nan           # a NaN among the values
+    K[33, 0, 7] = np.nan            # a NaN among the keys
+    flagged = {3, 5, 9, 20, 33}
+    Kt = torch.from_numpy(K).to(torch.bfloat16)
+    Vt = torch.from_numpy(V).to(torch.bfloat16)
+    cache = tq.Cache(T // 16, H, d)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    tq.quantize_append(Kt.cuda(), Vt.cuda(), torch.arange(T, dtype=torch.int32).cuda(), cache, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == tq.STATUS_RANGE
+    # one overflow at a time sets the bit too
+    for t in sorted(flagged):
+        c1 = tq.Cache(1, H, d)
+        st.zero_()
+        tq.quantize_append(Kt[t:t + 1].cuda(), Vt[t:t + 1].cuda(),
+                           torch.zeros(1, dtype=torch.int32).cuda(), c1, status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == tq.STATUS_RANGE, f"token {t}"
+    # the oracle on the tokens it can encode (a NaN has no defined code)
+    keep = np.array([t not in flagged for t in range(T)])
+    slots = np.where(keep, np.arange(T), -1).astype(np.int32)
+    ocache = np.zeros((T // 16, H, orc.record_bytes(d)), np.uint8)
+    assert orc.quantize_append(bf16_bits(Kt), bf16_bits(Vt), slots, ocache)[0] == 0
+    got = cache.data.cpu().numpy()
+    for blk in range(T // 16):
+        for h in range(H):
+            a = unpack_record(got[blk, h], d)
+            b = unpack_record(ocache[blk, h], d)
+            rows = [r for r in range(16) if keep[16 * blk + r]]
+            for name, x, y in zip(("kidx", "knorm", "vq", "vs", "vz"), a, b):
+                assert np.array_equal(x[rows], y[rows]), f"blk {blk} head {h} {name}"
 
 
 @pytest.mark.parametrize("d", [64, 128])

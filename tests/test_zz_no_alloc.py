@@ -13,7 +13,6 @@ import pytest
 import torch
 
 import workloads as W
-from parity_util import check_attention
 
 pytestmark = pytest.mark.gpu
 
@@ -56,7 +55,9 @@ def test_static_matches_workspace_entry_point_twice(tq, name, over, S):
         assert rc == tq.TQ_OK, tq.load().tq_last_error()
         torch.cuda.synchronize()
         assert int(status.item()) == 0
-        check_attention(out.cpu().numpy(), want, f"{name} call {call}")
+        # the same plan and the same kernels, only another home for the partials:
+        # the outputs must be identical bit for bit
+        assert torch.equal(out.cpu(), torch.from_numpy(want)), f"{name} call {call}"
 
 
 def test_static_rejects_plans_beyond_its_scratch(tq):
