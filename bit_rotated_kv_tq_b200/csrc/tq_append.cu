@@ -232,7 +232,8 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
         const uint32_t mnw = *reinterpret_cast<const uint32_t*>(&mn2);
         const uint32_t mxw = *reinterpret_cast<const uint32_t*>(&mx2);
         const float mn = fminf(bf16_lo(mnw), bf16_hi(mnw));
-        const float mx = fmaxf(bf16_lo(mxw), bf16_hi(mxw));
+        // the maximum of the two halves keeps a NaN (fmaxf would drop it)
+        const float mx = __bfloat162float(__hmax_nan(__low2bfloat16(mx2), __high2bfloat16(mx2)));
         // z = fp16 rounded down from the minimum (exact when it lies in fp16's normal range)
         const __half zh = __float2half_rd(mn);
         const float zf = __half2float(zh);
