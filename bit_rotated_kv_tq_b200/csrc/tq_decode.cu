@@ -44,11 +44,12 @@
 namespace tq {
 namespace {
 
-constexpr int kNW = 8;                   // warps per half (per unit)
+constexpr int kNW = 6;                   // warps per half (per range)
 constexpr int kHalves = 2;               // independent halves per CTA
-constexpr int kWarps = kNW * kHalves;    // 16 warps, 512 threads
-constexpr int kStages = 3;               // records in flight per warp
-constexpr int kSlots = kWarps * kStages;
+constexpr int kWarps = kNW * kHalves;    // 12 warps, 384 threads
+constexpr int kStages = 4;               // records per warp ring: two pairs
+constexpr int kPairs = kStages / 2;      // pair slots per ring (one mbarrier each)
+constexpr int kMergeSlots = kNW / 2;     // partials a half's merge tree holds at once
 constexpr int kHeads = 4;                // query heads per mma group (an item holds 1 or 2)
 constexpr uint32_t kLutBytes = 1u << 16; // 256 byte values x (2 halves x 32 lanes x 4 B)
 constexpr uint32_t kOnes = 0x3C003C00u;  // fp16 (1, 1)
@@ -79,14 +80,6 @@ __device__ __forceinline__ void sts32(uint32_t a, uint32_t v) {
 }
 __device__ __forceinline__ void sts128(uint32_t a, uint32_t v) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(a), "r"(v));
-}
-__device__ __forceinline__ void stsf(uint32_t a, float v) {
-    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v));
-}
-__device__ __forceinline__ float ldsf(uint32_t a) {
-    float v;
-    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
-    return v;
 }
 // barrier among the threads of one half (ids 1, 2; 0 is __syncthreads)
 __device__ __forceinline__ void half_sync(int half) {
@@ -182,40 +175,53 @@ __device__ __forceinline__ uint32_t ps_part(uint32_t u, uint32_t w, uint32_t s) 
 }
 
 // ------------------------------------------------------------------ shared memory plan
+// Floats of one warp's partial per lane, for one item: per group of four heads,
+// 2 D/16 output values (two dims per m-tile) plus the head's sum l and maximum m,
+// padded to whole 16-byte vectors.
+template <int D, int QPI>
+struct Part {
+    static constexpr int kPerQ = 2 * (D / 16) + 2;
+    static constexpr int kFloats = (QPI * kPerQ + 3) / 4 * 4;
+    static constexpr uint32_t kSlotBytes = 32u * kFloats * 4u;  // [vector][lane][4 floats]
+};
+
 // Shared-window addresses for a dynamic region that starts at s0.  The table
 // must sit on a 64 KB boundary so that one prmt can splice a code byte into
-// the address; whole warp rings fill the space below it first.
-template <int D, int HPI>
+// the address.  The small buffers come first, whole warp rings fill the space
+// below the table, and the remaining rings follow it.
+template <int D, int QPI>
 struct Plan {
+    static constexpr int HPI = kHeads * QPI;
     static constexpr uint32_t kRec = Rec<D>::kBytes;
     static constexpr uint32_t kRing = kStages * kRec;  // one warp's stages, contiguous
-    static constexpr uint32_t kMergeHalf = kNW * (HPI * D + 2 * HPI) * 4;
-    uint32_t lut, low, hi, merge, qh, ql, ids, bars, end;
+    static constexpr uint32_t kMergeHalf = kMergeSlots * Part<D, QPI>::kSlotBytes;
+    uint32_t merge, qh, ql, ids, bars, rings, lut, low, hi, end;
     __host__ __device__ explicit Plan(uint32_t s0) {
-        lut = (s0 + kLutBytes - 1) & ~(kLutBytes - 1);
-        const uint32_t n = (lut - s0) / kRing;
-        low = n < (uint32_t)kWarps ? n : (uint32_t)kWarps;
-        hi = lut + kLutBytes;
-        merge = hi + (kWarps - low) * kRing;
+        merge = (s0 + 15) & ~15u;
         qh = merge + kHalves * kMergeHalf;
         ql = qh + kHalves * HPI * D * 2;
         ids = ql + kHalves * HPI * D * 2;
-        bars = ids + kSlots * 4;
-        end = bars + kSlots * 8;
+        bars = ids + kWarps * kStages * 4;
+        rings = (bars + kWarps * kPairs * 8 + 127) & ~127u;
+        lut = (rings + kLutBytes - 1) & ~(kLutBytes - 1);
+        const uint32_t n = (lut - rings) / kRing;
+        low = n < (uint32_t)kWarps ? n : (uint32_t)kWarps;
+        hi = lut + kLutBytes;
+        end = hi + (kWarps - low) * kRing;
     }
     // first stage of warp w's ring
-    __host__ __device__ uint32_t ring(uint32_t s0, int w) const {
-        return (uint32_t)w < low ? s0 + w * kRing : hi + (w - low) * kRing;
+    __host__ __device__ uint32_t ring(int w) const {
+        return (uint32_t)w < low ? rings + w * kRing : hi + (w - low) * kRing;
     }
 };
 
 // Bytes to request so that the plan fits wherever the dynamic region starts
 // (the start depends on the reserved shared memory of the device).
-template <int D, int HPI>
+template <int D, int QPI>
 uint32_t plan_bytes() {
     uint32_t worst = 0;
     for (uint32_t s0 = 0; s0 <= 8192; s0 += 16) {
-        const Plan<D, HPI> p(s0);
+        const Plan<D, QPI> p(s0);
         if (p.end - s0 > worst) worst = p.end - s0;
     }
     return worst;
@@ -311,25 +317,185 @@ __device__ __forceinline__ void ldw(uint32_t a, uint32_t (&w)[N]) {
     }
 }
 
+// ------------------------------------------------------------------ merge tree
+// The warps of a half merge their partials in rounds: in a round over `act`
+// warps, warps [h, act) (h = ceil(act / 2)) hand their partials to warps
+// [0, act - h) through the merge slots, and the next round is over h warps.  A
+// writer uses the slot it read itself in an earlier round (else its own index
+// minus h), so a slot is never overwritten while another warp may still be
+// reading it, and one barrier per round suffices.
+__host__ __device__ constexpr int tree_act(int k) {
+    int act = kNW;
+    for (int r = 0; r < k; r++) act = (act + 1) / 2;
+    return act;
+}
+__host__ __device__ constexpr int tree_rounds() {
+    int k = 0;
+    while (tree_act(k) > 1) k++;
+    return k;
+}
+// The slot each writer of round k uses, 4 bits per warp.
+__host__ __device__ constexpr uint32_t tree_wslot(int k) {
+    int rd[16] = {-1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1, -1};
+    for (int r = 0;; r++) {
+        const int act = tree_act(r), h = (act + 1) / 2;
+        uint32_t ws = 0;
+        for (int w = h; w < act; w++) {
+            const int sl = rd[w] >= 0 ? rd[w] : w - h;
+            ws |= (uint32_t)sl << (4 * w);
+            rd[w - h] = sl;
+        }
+        if (r == k) return ws;
+    }
+}
+// Checks of the schedule: every slot index is below kMergeSlots, and no writer
+// of round k uses a slot that a reader of round k - 1 other than itself read.
+__host__ __device__ constexpr bool tree_ok() {
+    for (int k = 0; k < tree_rounds(); k++) {
+        const int act = tree_act(k), h = (act + 1) / 2;
+        for (int w = h; w < act; w++) {
+            const int sl = (int)((tree_wslot(k) >> (4 * w)) & 15u);
+            if (sl >= kMergeSlots) return false;
+            if (k > 0) {
+                const int pa = tree_act(k - 1), ph = (pa + 1) / 2;
+                for (int r = 0; r < pa - ph; r++)
+                    if (r != w && (int)((tree_wslot(k - 1) >> (4 * (r + ph))) & 15u) == sl) return false;
+            }
+        }
+    }
+    return true;
+}
+static_assert(kNW <= 16 && tree_ok(), "merge tree schedule");
+
 // ------------------------------------------------------------------ split kernel
+// The scores of one record for QPI groups of four heads: s[q] rows g (token g)
+// and g + 8 (token g + 8), columns 2c, 2c+1 (head 4q + c, high and low part of q~).
+template <int D, int QPI>
+__device__ __forceinline__ void record_scores(uint32_t rec, int g, int c, uint32_t lanebase,
+                                              const uint32_t (&qb)[QPI][D / 16][2],
+                                              float (&sc)[QPI][4]) {
+    constexpr int KS = D / 16, KB = D / 8, KW = KB / 4;
+    uint32_t kw0[KW], kw1[KW];
+    ldw<KW>(rec + g * (D / 2) + c * KB, kw0);
+    ldw<KW>(rec + (g + 8) * (D / 2) + c * KB, kw1);
+#pragma unroll
+    for (int ks = 0; ks < KS; ks++) {
+        // table address: the code byte spliced into byte 1 of lanebase
+        const uint32_t sa = (ks & 1) ? 0x7624u : 0x7604u;
+        const uint32_t sb = (ks & 1) ? 0x7634u : 0x7614u;
+        const uint32_t w0 = kw0[ks >> 1], w1 = kw1[ks >> 1];
+        const uint32_t a0 = lds32(__byte_perm(w0, lanebase, sa));
+        const uint32_t a2 = lds32(__byte_perm(w0, lanebase, sb));
+        const uint32_t a1 = lds32(__byte_perm(w1, lanebase, sa));
+        const uint32_t a3 = lds32(__byte_perm(w1, lanebase, sb));
+#pragma unroll
+        for (int q = 0; q < QPI; q++) {
+            if (ks == 0)
+                mma16816_z(sc[q], a0, a1, a2, a3, qb[q][ks][0], qb[q][ks][1]);
+            else
+                mma16816(sc[q], a0, a1, a2, a3, qb[q][ks][0], qb[q][ks][1]);
+        }
+    }
+}
+
+// p.z (and sum p) and p.V of one record for QPI groups of heads, given this
+// lane's fp16 parts of the weights (u, w: tokens 2c, 2c+1 | 2c+8, 2c+9 of head
+// g/2 of each group) and the valid-token masks of the fp16 lanes (mA: tokens
+// 2c, 2c+1; mB: tokens 2c+8, 2c+9; all ones for a full record).
+template <int D, int QPI>
+__device__ __forceinline__ void record_values(uint32_t rec, int g, int c, uint32_t mA, uint32_t mB,
+                                              const uint32_t (&u01)[QPI], const uint32_t (&w01)[QPI],
+                                              const uint32_t (&u89)[QPI], const uint32_t (&w89)[QPI],
+                                              float (&O)[QPI][D / 16][4], float (&Z)[QPI][4]) {
+    constexpr int NG = D / 32, KB = D / 8, KW = KB / 4;
+    using R = Rec<D>;
+    uint2 zz = lds64(rec + R::kVZero + (c * NG + (g & (NG - 1))) * 8);
+    uint32_t sw[2 * NG];
+#pragma unroll
+    for (int i = 0; i < 2 * NG; i += 4) {
+        uint32_t t4[4];
+        ldw<4>(rec + R::kVScale + c * NG * 8 + 4 * i, t4);
+#pragma unroll
+        for (int e = 0; e < 4; e++) sw[i + e] = t4[e];
+    }
+    // stale fields of unwritten tokens must not reach the products
+    zz.x &= mA;
+    zz.y &= mB;
+#pragma unroll
+    for (int G_ = 0; G_ < NG; G_++) {
+        sw[2 * G_] &= mA;
+        sw[2 * G_ + 1] &= mB;
+    }
+#pragma unroll
+    for (int q = 0; q < QPI; q++) mma16816(Z[q], zz.x, kOnes, zz.y, kOnes, w01[q], w89[q]);
+    // word G of a chunk holds m-tiles 2G (bytes 0, 2) and 2G + 1 (bytes 1, 3) of
+    // tokens 2c, 2c+1 (va) and 2c+8, 2c+9 (vb)
+    uint32_t va[KW], vb[KW];
+    ldw<KW>(rec + R::kVCodes + (c * 8 + g) * KB, va);
+    ldw<KW>(rec + R::kVCodes + ((c + 4) * 8 + g) * KB, vb);
+#pragma unroll
+    for (int G_ = 0; G_ < NG; G_++) {
+        const uint32_t A0 = va[G_], B0 = vb[G_], A1 = A0 >> 8, B1 = B0 >> 8;
+#pragma unroll
+        for (int q = 0; q < QPI; q++) {
+            const uint32_t b0 = ps_part(u01[q], w01[q], sw[2 * G_]);
+            const uint32_t b1 = ps_part(u89[q], w89[q], sw[2 * G_ + 1]);
+            mma16816(O[q][2 * G_], A0 & 0x000F000Fu, A0 & 0x00F000F0u, B0 & 0x000F000Fu,
+                     B0 & 0x00F000F0u, b0, b1);
+            mma16816(O[q][2 * G_ + 1], A1 & 0x000F000Fu, A1 & 0x00F000F0u, B1 & 0x000F000Fu,
+                     B1 & 0x00F000F0u, b0, b1);
+        }
+    }
+}
+
+// Token masks of a record with n valid tokens (n = 16: everything valid):
+// tokens g, g + 8 of the score rows, and the fp16 lanes of tokens 2c, 2c+1 |
+// 2c+8, 2c+9 of the value operands.
+struct Mask {
+    bool va, vb;
+    uint32_t mA, mB;
+};
+__device__ __forceinline__ Mask token_mask(int n, int g, int c) {
+    const int t = 2 * c;
+    Mask m;
+    m.va = g < n;
+    m.vb = g + 8 < n;
+    m.mA = (t < n ? 0xffffu : 0u) | (t + 1 < n ? 0xffff0000u : 0u);
+    m.mB = (t + 8 < n ? 0xffffu : 0u) | (t + 9 < n ? 0xffff0000u : 0u);
+    return m;
+}
+
+// Merge partial (pm, pl, po) into (m, l, o): both relative to their own maxima
+// in base 2; an empty partial has maximum -inf and contributes nothing.
+template <int N>
+__device__ __forceinline__ void merge_into(float& m, float& l, float (&o)[N], float pm, float pl,
+                                           const float* po) {
+    const float M = fmaxf(m, pm);
+    const float f0 = m == -INFINITY ? 0.f : ex2(m - M);
+    const float f1 = pm == -INFINITY ? 0.f : ex2(pm - M);
+#pragma unroll
+    for (int j = 0; j < N; j++) o[j] = fmaf(f1, po[j], f0 * o[j]);
+    l = fmaf(f1, pl, f0 * l);
+    m = M;
+}
+
 template <int D, int QPI>
 __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs a) {
     constexpr int HPI = kHeads * QPI;  // query heads per item
     constexpr int KS = D / 16;   // k-steps of q.K = m-tiles of p.V
-    constexpr int NG = D / 32;   // value groups
     constexpr int KB = D / 8;    // key bytes of a lane per token = bytes of a value chunk
-    constexpr int KW = KB / 4;   // words of those (= NG)
     constexpr int EPL = D / 32;  // query elements per lane in the rotation
+    constexpr int PQ = 2 * KS;   // output values of a lane per group of heads
     constexpr uint32_t REC = Rec<D>::kBytes;
     using R = Rec<D>;
+    using PT = Part<D, QPI>;
     extern __shared__ __align__(128) unsigned char dsm[];
 
     const int tid = threadIdx.x, lane = tid & 31, wa = tid >> 5;
     const int half = wa / kNW, warp = wa % kNW;
-    const int ht = tid - half * kNW * 32;  // thread index within the half
     const int g = lane >> 2, c = lane & 3;
     const uint32_t s0 = smem_u32(dsm);
-    const Plan<D, HPI> P(s0);
+    const Plan<D, QPI> P(s0);
     if (P.end - s0 > a.smem_bytes) {  // cannot happen with the launcher's size; never touch memory
         if (tid == 0 && blockIdx.x == 0) flag_status(a.status, TQ_STATUS_INTERNAL);
         return;
@@ -338,59 +504,78 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     const int stride = kHalves * gridDim.x;  // ranges per round over all halves
     const int v = kHalves * blockIdx.x + half;
 
-    // ---- this warp's ring: slots, barriers, and the block id of each stage
-    const uint32_t bar0 = P.bars + wa * kStages * 8;
+    // ---- this warp's ring: kStages record stages, one mbarrier per pair of
+    // stages, and the block ids of each stage
+    const uint32_t bar0 = P.bars + wa * kPairs * 8;
     const uint32_t idw = P.ids + wa * kStages * 4;
-    const uint32_t ringw = P.ring(s0, wa);
+    const uint32_t ringw = P.ring(wa);
     if (lane == 0) {
 #pragma unroll
-        for (int s = 0; s < kStages; s++) mbar_init(bar0 + 8 * s, 1);
+        for (int s = 0; s < kPairs; s++) mbar_init(bar0 + 8 * s, 1);
         fence_mbar_init();
     }
     __syncwarp();
 
     const long long rec_stride = (long long)a.Hkv * REC;  // bytes between blocks of one kv head
-    // ---- issue cursor: the next record of this warp's stream (all its segments, in order)
+    // ---- issue cursor: the next pair of records of this warp's stream (all its
+    // segments in order; a pair never spans two segments, so a segment with an
+    // odd number of records ends with a single record)
     Seg is;
     seg_range<D>(is, v, a, warp, false);
     while (is.r < a.nranges && is.nk == 0) seg_next<D>(is, stride, a, warp, false);
-    int irem = is.nk, istage = 0;
+    int irem = is.nk, ipair = 0, issued = 0;
     const int32_t* ibt = is.bt;
-    int nid = is.r < a.nranges ? *ibt : -1;
-    // Copy the record of block nid into stage istage (one elected lane, no branch),
-    // note its id for the consumer, and move the cursor on.
+    int nid0 = -1, nid1 = -1;
+    if (is.r < a.nranges) {
+        nid0 = ibt[0];
+        if (irem > 1) nid1 = ibt[kNW];
+    }
+    // Copy the next pair into pair slot ipair (one elected lane, no branch), note
+    // the block ids for the consumer, and move the cursor on.
     auto issue = [&]() {
         if (is.r >= a.nranges) return;
-        const uint32_t bar = bar0 + 8 * istage;
-        const uint32_t valid = (uint32_t)((uint32_t)nid < (uint32_t)a.num_blocks);
+        const int n = irem > 1 ? 2 : 1;
+        const uint32_t bar = bar0 + 8 * ipair;
+        const uint32_t v0 = (uint32_t)((uint32_t)nid0 < (uint32_t)a.num_blocks);
+        const uint32_t v1 = (uint32_t)(n == 2 && (uint32_t)nid1 < (uint32_t)a.num_blocks);
         const uint32_t me = (uint32_t)(lane == 0);
-        const unsigned char* src = is.src + (long long)nid * rec_stride;  // used only if valid
+        const uint32_t dst = ringw + (2 * ipair) * REC;
+        const unsigned char* src0 = is.src + (long long)nid0 * rec_stride;  // used only if v0
+        const unsigned char* src1 = is.src + (long long)nid1 * rec_stride;  // used only if v1
         asm volatile(
-            "{\n .reg .pred pc, pa, pm;\n"
+            "{\n .reg .pred pm, pa, pz, p0, p1;\n"
             " setp.ne.u32 pm, %0, 0;\n"
-            " setp.ne.and.u32 pc, %1, 0, pm;\n"
-            " setp.eq.and.u32 pa, %1, 0, pm;\n"
-            " @pc fence.proxy.async.shared::cta;\n"
-            " @pc mbarrier.arrive.expect_tx.shared::cta.b64 _, [%2], %3;\n"
-            " @pc cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%4], [%5], %3, [%2];\n"
-            " @pa mbarrier.arrive.shared::cta.b64 _, [%2];\n"
-            " @pm st.shared.b32 [%6], %7;\n"
-            "}\n" ::"r"(me), "r"(valid), "r"(bar), "r"(REC), "r"(ringw + istage * REC), "l"(src),
-            "r"(idw + 4 * istage), "r"(nid)
+            " setp.ne.and.u32 pa, %9, 0, pm;\n"
+            " setp.eq.and.u32 pz, %9, 0, pm;\n"
+            " setp.ne.and.u32 p0, %1, 0, pm;\n"
+            " setp.ne.and.u32 p1, %2, 0, pm;\n"
+            " @pa fence.proxy.async.shared::cta;\n"
+            " @pa mbarrier.arrive.expect_tx.shared::cta.b64 _, [%3], %9;\n"
+            " @pz mbarrier.arrive.shared::cta.b64 _, [%3];\n"
+            " @p0 cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%4], [%5], %10, [%3];\n"
+            " @p1 cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%6], [%7], %10, [%3];\n"
+            " @pm st.shared.v2.b32 [%8], {%11, %12};\n"
+            "}\n" ::"r"(me), "r"(v0), "r"(v1), "r"(bar), "r"(dst), "l"(src0), "r"(dst + REC),
+            "l"(src1), "r"(idw + 8 * ipair), "r"((v0 + v1) * REC), "r"(REC), "r"(nid0), "r"(nid1)
             : "memory");
-        istage = istage == kStages - 1 ? 0 : istage + 1;
-        if (--irem == 0) {
+        ipair ^= 1;
+        issued++;
+        irem -= n;
+        if (irem == 0) {
             do seg_next<D>(is, stride, a, warp, false);
             while (is.r < a.nranges && is.nk == 0);
             irem = is.nk;
             ibt = is.bt;
         } else {
-            ibt += kNW;
+            ibt += 2 * kNW;
         }
-        nid = is.r < a.nranges ? *ibt : -1;
+        if (is.r < a.nranges) {
+            nid0 = ibt[0];
+            nid1 = irem > 1 ? ibt[kNW] : -1;
+        }
     };
 #pragma unroll 1
-    for (int k = 0; k < kStages; k++) issue();
+    for (int k = 0; k < kPairs; k++) issue();
     __syncwarp();
 
     // ---- per-lane constants of the consumer
@@ -398,12 +583,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
     const float lo_sel = (float)(g & 1);  // this lane feeds the low part of its head
     const uint32_t lo_mask = (g & 1) ? 0xffffffffu : 0u;
     const uint32_t qsrc = ((g & 1) ? P.ql : P.qh) + (uint32_t)((half * HPI + (g >> 1)) * D * 2);
-    const uint32_t mb = P.merge + half * Plan<D, HPI>::kMergeHalf;  // [warp][head][D] o, then m, l
-    const uint32_t mb_m = mb + kNW * HPI * D * 4, mb_l = mb_m + kNW * HPI * 4;
-    int stage = 0;
+    const uint32_t mslots = P.merge + half * Plan<D, QPI>::kMergeHalf;
+    int slot = 0, consumed = 0;
     uint32_t phase = 0;
     bool aborted = false;
     const uint16_t* lut_tab = nullptr;  // table held by this half's side of the LUT
+    const int s_even = 8 * c + (g >> 1), s_odd = s_even + 4;  // weight sources of the p.V operand
 
     Seg cu;
     seg_range<D>(cu, v, a, warp, warp == 0 && lane == 0);
@@ -427,11 +612,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 sts128(P.lut + row * 256 + half * 128 + (lane & 7) * 16, lo | (hi << 16));
             }
         }
-        // ---- rotate this item's queries: q~ = H q * scale log2(e) / sqrt(D), as fp16 parts
-        if (warp < HPI) {
+        // ---- rotate this item's queries: q~ = H q * scale log2(e) / sqrt(D), as
+        // fp16 parts (the half's warps take the heads in turn)
+#pragma unroll 1
+        for (int hw = warp; hw < HPI; hw += kNW) {
             float x[EPL];
-            if (warp < nh) {
-                const uint16_t* src = a.q + ((size_t)cu.b * a.Hq + h0 + warp) * D + lane * EPL;
+            if (hw < nh) {
+                const uint16_t* src = a.q + ((size_t)cu.b * a.Hq + h0 + hw) * D + lane * EPL;
 #pragma unroll
                 for (int e = 0; e < EPL; e++) x[e] = __uint_as_float((uint32_t)src[e] << 16);
             } else {
@@ -457,8 +644,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 }
             }
             const float sc = a.scale_log2 * rsqrtf((float)D);
-            const uint32_t dh = P.qh + (uint32_t)(((half * HPI + warp) * D + lane * EPL) * 2);
-            const uint32_t dl = P.ql + (uint32_t)(((half * HPI + warp) * D + lane * EPL) * 2);
+            const uint32_t dh = P.qh + (uint32_t)(((half * HPI + hw) * D + lane * EPL) * 2);
+            const uint32_t dl = P.ql + (uint32_t)(((half * HPI + hw) * D + lane * EPL) * 2);
 #pragma unroll
             for (int e = 0; e < EPL; e += 2) {
                 const float y0 = x[e] * sc, y1 = x[e + 1] * sc;
@@ -484,7 +671,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 qb[q][ks][1] = v2.y;
             }
 
-        // ---- this warp's records of the unit
+        // ---- this warp's records of the segment, two per iteration
         float O[QPI][KS][4];  // p.V: rows = dims (16m + 2g, 16m + 2g + 1), cols = head c (hi, lo)
         float Z[QPI][4];      // p.z: rows g = zero sums of group g, rows g + 8 = sum of p
         float mrun[QPI];      // running maximum of head 4q + c
@@ -499,70 +686,57 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
             }
         }
         const int nk = aborted ? 0 : cu.nk;
-        // tokens in this warp's last record of the unit (< 16 only at the end of the sequence)
+        // tokens in this warp's last record of the segment (< 16 only at the end of the sequence)
         const int last_valid = cu.L - (cu.jb + warp + kNW * (nk - 1)) * kBlock;
 #pragma unroll 1
-        for (int k = 0; k < nk; k++) {
-            const uint32_t rec = ringw + stage * REC;
-            if (!mbar_wait_warp(bar0 + 8 * stage, phase)) {
+        for (int k = 0; k < nk; k += 2) {
+            if (!mbar_wait_warp(bar0 + 8 * slot, phase)) {
                 flag_lane0(a.status, TQ_STATUS_TIMEOUT, lane);
                 aborted = true;
                 break;
             }
-            const int id = (int)lds32(idw + 4 * stage);
-            if (__all_sync(kFull, (uint32_t)id < (uint32_t)a.num_blocks)) {
-                const bool partial = k == nk - 1 && last_valid < kBlock;
-
-                // -------- q.K: A = centroids of tokens g (rows 0-7) and g + 8 (rows 8-15),
-                // shared by the QPI groups of heads
-                uint32_t kw0[KW], kw1[KW];
-                ldw<KW>(rec + g * (D / 2) + c * KB, kw0);
-                ldw<KW>(rec + (g + 8) * (D / 2) + c * KB, kw1);
-                float sc[QPI][4];
-#pragma unroll
-                for (int ks = 0; ks < KS; ks++) {
-                    // table address: the code byte spliced into byte 1 of lanebase
-                    const uint32_t sa = (ks & 1) ? 0x7624u : 0x7604u;
-                    const uint32_t sb = (ks & 1) ? 0x7634u : 0x7614u;
-                    const uint32_t w0 = kw0[ks >> 1], w1 = kw1[ks >> 1];
-                    const uint32_t a0 = lds32(__byte_perm(w0, lanebase, sa));
-                    const uint32_t a2 = lds32(__byte_perm(w0, lanebase, sb));
-                    const uint32_t a1 = lds32(__byte_perm(w1, lanebase, sa));
-                    const uint32_t a3 = lds32(__byte_perm(w1, lanebase, sb));
-#pragma unroll
-                    for (int q = 0; q < QPI; q++) {
-                        if (ks == 0)
-                            mma16816_z(sc[q], a0, a1, a2, a3, qb[q][ks][0], qb[q][ks][1]);
-                        else
-                            mma16816(sc[q], a0, a1, a2, a3, qb[q][ks][0], qb[q][ks][1]);
-                    }
-                }
-                // scores of head 4q + c at tokens g and g + 8 (base 2): columns 2c, 2c+1
-                // hold the high and low parts of the query
-                const uint32_t nw = lds32(rec + R::kKNorm + 4 * (g >> 1));
-                const uint32_t nw8 = lds32(rec + R::kKNorm + 16 + 4 * (g >> 1));
-                const float na = __half2float(__ushort_as_half((uint16_t)((g & 1) ? nw >> 16 : nw)));
-                const float nb = __half2float(__ushort_as_half((uint16_t)((g & 1) ? nw8 >> 16 : nw8)));
-                uint32_t mA = 0xffffffffu, mB = 0xffffffffu;  // valid tokens (fp16 lanes)
-                bool va_ok = true, vb_ok = true;               // tokens g, g + 8 valid
-                if (partial) {  // the last block of the sequence
-                    const int t = 2 * c, nvalid = last_valid;
-                    va_ok = g < nvalid;
-                    vb_ok = g + 8 < nvalid;
-                    mA = (t < nvalid ? 0xffffu : 0u) | (t + 1 < nvalid ? 0xffff0000u : 0u);
-                    mB = (t + 8 < nvalid ? 0xffffu : 0u) | (t + 9 < nvalid ? 0xffff0000u : 0u);
+            const uint2 ids = lds64(idw + 8 * slot);
+            const bool has1 = k + 1 < nk;
+            const bool ok0 = (uint32_t)ids.x < (uint32_t)a.num_blocks;
+            const bool ok1 = has1 && (uint32_t)ids.y < (uint32_t)a.num_blocks;
+            if (!ok0 || (has1 && !ok1)) flag_lane0(a.status, TQ_STATUS_BAD_BLOCK, lane);
+            // valid tokens of the two records (a bad or missing record has none)
+            const int n0 = ok0 ? (k == nk - 1 ? last_valid : kBlock) : 0;
+            const int n1 = ok1 ? (k + 1 == nk - 1 ? last_valid : kBlock) : 0;
+            if (n0 + n1 > 0) {
+                const uint32_t rec0 = ringw + (2 * slot) * REC, rec1 = rec0 + REC;
+                // -------- q.K of both records
+                float sc0[QPI][4], sc1[QPI][4];
+                record_scores<D, QPI>(rec0, g, c, lanebase, qb, sc0);
+                record_scores<D, QPI>(rec1, g, c, lanebase, qb, sc1);
+                // scores of head 4q + c at tokens g and g + 8 (base 2): columns 2c,
+                // 2c+1 hold the high and low parts of the query; the norm after the dot
+                const uint32_t nw0 = lds32(rec0 + R::kKNorm + 4 * (g >> 1));
+                const uint32_t nw0b = lds32(rec0 + R::kKNorm + 16 + 4 * (g >> 1));
+                const uint32_t nw1 = lds32(rec1 + R::kKNorm + 4 * (g >> 1));
+                const uint32_t nw1b = lds32(rec1 + R::kKNorm + 16 + 4 * (g >> 1));
+                const int sh = (g & 1) * 16;
+                const float na0 = __half2float(__ushort_as_half((uint16_t)(nw0 >> sh)));
+                const float nb0 = __half2float(__ushort_as_half((uint16_t)(nw0b >> sh)));
+                const float na1 = __half2float(__ushort_as_half((uint16_t)(nw1 >> sh)));
+                const float nb1 = __half2float(__ushort_as_half((uint16_t)(nw1b >> sh)));
+                Mask m0 = {true, true, 0xffffffffu, 0xffffffffu}, m1 = m0;
+                if (n0 < kBlock || n1 < kBlock) {  // the last block of a sequence, or a bad block
+                    m0 = token_mask(n0, g, c);
+                    m1 = token_mask(n1, g, c);
                 }
 
-                // -------- online softmax (head 4q + c: lanes with the same c), and the
-                // weights moved to the p.V operand: head g/2 at tokens 2c, 2c+1, 2c+8,
-                // 2c+9 lives in lanes (2c, g/2) and (2c+1, g/2), as their tokens g, g + 8
-                const int s_even = 8 * c + (g >> 1), s_odd = s_even + 4;
-                uint32_t u01[QPI], w01[QPI], u89[QPI], w89[QPI];
+                // -------- online softmax over the 32 tokens (head 4q + c: lanes with
+                // the same c), and the weights moved to the p.V operand: head g/2 at
+                // tokens 2c, 2c+1, 2c+8, 2c+9 lives in lanes (2c, g/2) and (2c+1, g/2)
+                uint32_t u01[2][QPI], w01[2][QPI], u89[2][QPI], w89[2][QPI];
 #pragma unroll
                 for (int q = 0; q < QPI; q++) {
-                    const float xa = va_ok ? (sc[q][0] + sc[q][1]) * na : -INFINITY;
-                    const float xb = vb_ok ? (sc[q][2] + sc[q][3]) * nb : -INFINITY;
-                    float mx = fmaxf(xa, xb);
+                    const float xa0 = m0.va ? (sc0[q][0] + sc0[q][1]) * na0 : -INFINITY;
+                    const float xb0 = m0.vb ? (sc0[q][2] + sc0[q][3]) * nb0 : -INFINITY;
+                    const float xa1 = m1.va ? (sc1[q][0] + sc1[q][1]) * na1 : -INFINITY;
+                    const float xb1 = m1.vb ? (sc1[q][2] + sc1[q][3]) * nb1 : -INFINITY;
+                    float mx = fmaxf(fmaxf(xa0, xb0), fmaxf(xa1, xb1));
                     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 4));
                     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 8));
                     mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 16));
@@ -577,117 +751,117 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                         }
                     }
                     mrun[q] = mn;
-                    const float pa = ex2(xa - mn), pb = ex2(xb - mn);
-                    const float p0 = __shfl_sync(kFull, pa, s_even), p1 = __shfl_sync(kFull, pa, s_odd);
-                    const float p2 = __shfl_sync(kFull, pb, s_even), p3 = __shfl_sync(kFull, pb, s_odd);
-                    split_uw(p0, p1, lo_sel, lo_mask, u01[q], w01[q]);
-                    split_uw(p2, p3, lo_sel, lo_mask, u89[q], w89[q]);
+                    const float pa0 = ex2(xa0 - mn), pb0 = ex2(xb0 - mn);
+                    const float pa1 = ex2(xa1 - mn), pb1 = ex2(xb1 - mn);
+                    split_uw(__shfl_sync(kFull, pa0, s_even), __shfl_sync(kFull, pa0, s_odd), lo_sel,
+                             lo_mask, u01[0][q], w01[0][q]);
+                    split_uw(__shfl_sync(kFull, pb0, s_even), __shfl_sync(kFull, pb0, s_odd), lo_sel,
+                             lo_mask, u89[0][q], w89[0][q]);
+                    split_uw(__shfl_sync(kFull, pa1, s_even), __shfl_sync(kFull, pa1, s_odd), lo_sel,
+                             lo_mask, u01[1][q], w01[1][q]);
+                    split_uw(__shfl_sync(kFull, pb1, s_even), __shfl_sync(kFull, pb1, s_odd), lo_sel,
+                             lo_mask, u89[1][q], w89[1][q]);
                 }
 
-                // -------- p.z and sum p
-                uint2 zz = lds64(rec + R::kVZero + (c * NG + (g & (NG - 1))) * 8);
-                uint32_t sw[2 * NG];
-#pragma unroll
-                for (int i = 0; i < 2 * NG; i += 4) {
-                    uint32_t t4[4];
-                    ldw<4>(rec + R::kVScale + c * NG * 8 + 4 * i, t4);
-#pragma unroll
-                    for (int e = 0; e < 4; e++) sw[i + e] = t4[e];
-                }
-                if (partial) {  // stale fields of unwritten tokens must not reach the products
-                    zz.x &= mA;
-                    zz.y &= mB;
-#pragma unroll
-                    for (int G_ = 0; G_ < NG; G_++) {
-                        sw[2 * G_] &= mA;
-                        sw[2 * G_ + 1] &= mB;
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < QPI; q++) mma16816(Z[q], zz.x, kOnes, zz.y, kOnes, w01[q], w89[q]);
-
-                // -------- p.V: word G of a chunk holds m-tiles 2G (bytes 0, 2) and
-                // 2G + 1 (bytes 1, 3) of tokens 2c, 2c+1 (va) and 2c+8, 2c+9 (vb)
-                uint32_t va[KW], vb[KW];
-                ldw<KW>(rec + R::kVCodes + (c * 8 + g) * KB, va);
-                ldw<KW>(rec + R::kVCodes + ((c + 4) * 8 + g) * KB, vb);
-#pragma unroll
-                for (int G_ = 0; G_ < NG; G_++) {
-                    const uint32_t A0 = va[G_], B0 = vb[G_], A1 = A0 >> 8, B1 = B0 >> 8;
-#pragma unroll
-                    for (int q = 0; q < QPI; q++) {
-                        const uint32_t b0 = ps_part(u01[q], w01[q], sw[2 * G_]);
-                        const uint32_t b1 = ps_part(u89[q], w89[q], sw[2 * G_ + 1]);
-                        mma16816(O[q][2 * G_], A0 & 0x000F000Fu, A0 & 0x00F000F0u, B0 & 0x000F000Fu,
-                                 B0 & 0x00F000F0u, b0, b1);
-                        mma16816(O[q][2 * G_ + 1], A1 & 0x000F000Fu, A1 & 0x00F000F0u,
-                                 B1 & 0x000F000Fu, B1 & 0x00F000F0u, b0, b1);
-                    }
-                }
-            } else {
-                flag_lane0(a.status, TQ_STATUS_BAD_BLOCK, lane);
+                // -------- p.z, sum p and p.V of both records
+                record_values<D, QPI>(rec0, g, c, m0.mA, m0.mB, u01[0], w01[0], u89[0], w89[0], O, Z);
+                record_values<D, QPI>(rec1, g, c, m1.mA, m1.mB, u01[1], w01[1], u89[1], w89[1], O, Z);
             }
             __syncwarp();
-            issue();  // the record after the ring's last: into the slot just read
-            if (++stage == kStages) {
-                stage = 0;
-                phase ^= 1u;
-            }
+            consumed++;
+            issue();  // the pair after the ring's last: into the slot just read
+            slot ^= 1;
+            if (slot == 0) phase ^= 1u;
         }
 
-        // ---- this warp's share -> merge buffer (o with the zero-point term, m, l of
-        // head 4q + c)
+        // ---- this warp's partial, per group q of heads: the outputs of head
+        // 4q + c at dims 16m + 2g, 16m + 2g + 1 (zero-point term added), its
+        // sum of weights and its running maximum
+        float po[QPI][PQ], pl[QPI];
 #pragma unroll
         for (int q = 0; q < QPI; q++) {
-            float zs[NG];
+            float zs[KS / 2];
 #pragma unroll
-            for (int G_ = 0; G_ < NG; G_++) zs[G_] = __shfl_sync(kFull, Z[q][0] + Z[q][1], 4 * G_ + c);
-            const int hq = q * kHeads + c;
-            const uint32_t ro = mb + (uint32_t)((warp * HPI + hq) * D * 4);
+            for (int G_ = 0; G_ < KS / 2; G_++) zs[G_] = __shfl_sync(kFull, Z[q][0] + Z[q][1], 4 * G_ + c);
 #pragma unroll
             for (int m = 0; m < KS; m++) {
-                stsf(ro + (16 * m + 2 * g) * 4, fmaf(O[q][m][0] + O[q][m][1], 0x1p24f, zs[m >> 1]));
-                stsf(ro + (16 * m + 2 * g + 1) * 4, fmaf(O[q][m][2] + O[q][m][3], 0x1p20f, zs[m >> 1]));
+                po[q][2 * m] = fmaf(O[q][m][0] + O[q][m][1], 0x1p24f, zs[m >> 1]);
+                po[q][2 * m + 1] = fmaf(O[q][m][2] + O[q][m][3], 0x1p20f, zs[m >> 1]);
             }
-            if (g == 0) {
-                stsf(mb_m + (warp * HPI + hq) * 4, mrun[q]);
-                stsf(mb_l + (warp * HPI + hq) * 4, Z[q][2] + Z[q][3]);
+            pl[q] = Z[q][2] + Z[q][3];
+        }
+
+        // ---- merge the half's warps in a tree; warp 0 ends with the sum
+#pragma unroll
+        for (int k = 0; k < tree_rounds(); k++) {
+            const int act = tree_act(k), h = (act + 1) / 2;
+            const uint32_t ws = tree_wslot(k);
+            if (warp >= h && warp < act) {
+                const int sl = (int)((ws >> (4 * warp)) & 15u);
+                const uint32_t base = mslots + sl * PT::kSlotBytes + lane * 16;
+                float buf[PT::kFloats];
+#pragma unroll
+                for (int q = 0; q < QPI; q++) {
+#pragma unroll
+                    for (int j = 0; j < PQ; j++) buf[q * (PQ + 2) + j] = po[q][j];
+                    buf[q * (PQ + 2) + PQ] = pl[q];
+                    buf[q * (PQ + 2) + PQ + 1] = mrun[q];
+                }
+#pragma unroll
+                for (int j = QPI * (PQ + 2); j < PT::kFloats; j++) buf[j] = 0.f;
+#pragma unroll
+                for (int j = 0; j < PT::kFloats; j += 4)
+                    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(base + (j / 4) * 512),
+                                 "f"(buf[j]), "f"(buf[j + 1]), "f"(buf[j + 2]), "f"(buf[j + 3])
+                                 : "memory");
+            }
+            half_sync(half);
+            if (warp < act - h) {
+                const int sl = (int)((ws >> (4 * (warp + h))) & 15u);
+                const uint32_t base = mslots + sl * PT::kSlotBytes + lane * 16;
+                float buf[PT::kFloats];
+#pragma unroll
+                for (int j = 0; j < PT::kFloats; j += 4)
+                    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                 : "=f"(buf[j]), "=f"(buf[j + 1]), "=f"(buf[j + 2]), "=f"(buf[j + 3])
+                                 : "r"(base + (j / 4) * 512)
+                                 : "memory");
+#pragma unroll
+                for (int q = 0; q < QPI; q++)
+                    merge_into<PQ>(mrun[q], pl[q], po[q], buf[q * (PQ + 2) + PQ + 1],
+                                   buf[q * (PQ + 2) + PQ], &buf[q * (PQ + 2)]);
             }
         }
-        half_sync(half);
 
-        // ---- merge the 8 warps and write the unit's partial (or the output)
-#pragma unroll 1
-        for (int idx = ht; idx < nh * D; idx += kNW * 32) {
-            const int h = idx / D, i = idx % D;
-            float M = -INFINITY;
+        // ---- warp 0 writes the segment's output (a whole item) or its partial
+        if (warp == 0) {
 #pragma unroll
-            for (int w = 0; w < kNW; w++) M = fmaxf(M, ldsf(mb_m + (w * HPI + h) * 4));
-            float o = 0.f, l = 0.f;
-            if (M != -INFINITY) {
+            for (int q = 0; q < QPI; q++) {
+                const int hq = q * kHeads + c;
+                if (hq < nh) {
+                    if (cu.direct) {
+                        float* dst = a.out + ((size_t)cu.b * a.Hq + h0 + hq) * D + 2 * g;
 #pragma unroll
-                for (int w = 0; w < kNW; w++) {
-                    const float f = ex2(ldsf(mb_m + (w * HPI + h) * 4) - M);
-                    o = fmaf(f, ldsf(mb + ((w * HPI + h) * D + i) * 4), o);
-                    l = fmaf(f, ldsf(mb_l + (w * HPI + h) * 4), l);
+                        for (int m = 0; m < KS; m++)
+                            *reinterpret_cast<float2*>(dst + 16 * m) =
+                                pl[q] > 0.f ? make_float2(po[q][2 * m] / pl[q], po[q][2 * m + 1] / pl[q])
+                                            : make_float2(0.f, 0.f);
+                    } else {
+                        const size_t pr = ((size_t)cu.r * 2 + (cu.i == cu.i_first ? 0 : 1)) * HPI + hq;
+                        float* dst = a.ws_o + pr * D + 2 * g;
+#pragma unroll
+                        for (int m = 0; m < KS; m++)
+                            *reinterpret_cast<float2*>(dst + 16 * m) = make_float2(po[q][2 * m], po[q][2 * m + 1]);
+                        if (g == 0) a.ws_ml[pr] = make_float2(mrun[q], pl[q]);
+                    }
                 }
-            }
-            if (cu.direct) {
-                a.out[((size_t)cu.b * a.Hq + h0 + h) * D + i] = l > 0.f ? o / l : 0.f;
-            } else {
-                const size_t pr = ((size_t)cu.r * 2 + (cu.i == cu.i_first ? 0 : 1)) * HPI + h;
-                a.ws_o[pr * D + i] = o;
-                if (i == 0) a.ws_ml[pr] = make_float2(M, l);
             }
         }
     }
 
-    if (aborted) {  // give copies still in flight a bounded chance to land
+    if (aborted) {  // give the copies still in flight a bounded chance to land
 #pragma unroll 1
-        for (int s = 0; s < kStages; s++) {
-            mbar_wait(bar0 + 8 * s, 0);
-            mbar_wait(bar0 + 8 * s, 1);
-        }
+        for (int j = consumed; j < issued; j++) mbar_wait(bar0 + 8 * (j & 1), (uint32_t)(j >> 1) & 1u);
     }
 }
 
@@ -745,7 +919,7 @@ cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
     // library may be called from several host threads)
     static std::mutex mu;
     static bool configured[64] = {};
-    static const uint32_t smem = plan_bytes<D, kHeads * QPI>();
+    static const uint32_t smem = plan_bytes<D, QPI>();
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -769,7 +943,7 @@ cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
 }  // namespace
 
 uint32_t decode_smem_bytes(int head_dim) {  // the largest plan of the head_dim's kernels
-    return head_dim == 128 ? plan_bytes<128, kHeads>() : plan_bytes<64, 2 * kHeads>();
+    return head_dim == 128 ? plan_bytes<128, 1>() : plan_bytes<64, 2>();
 }
 
 // Ranges: with num_splits = 0 the virtual records are cut evenly over every
