@@ -230,7 +230,6 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
             mx2 = __hmax2_nan(mx2, *reinterpret_cast<const __nv_bfloat162*>(&px));
         }
         const uint32_t mnw = *reinterpret_cast<const uint32_t*>(&mn2);
-        const uint32_t mxw = *reinterpret_cast<const uint32_t*>(&mx2);
         const float mn = fminf(bf16_lo(mnw), bf16_hi(mnw));
         // the maximum of the two halves keeps a NaN (fmaxf would drop it)
         const float mx = __bfloat162float(__hmax_nan(__low2bfloat16(mx2), __high2bfloat16(mx2)));

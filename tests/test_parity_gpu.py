@@ -190,6 +190,34 @@ def test_reduced_configs(tq, orc, name, over, S):
     check_pairs(tq, orc, w, pairs, num_splits=S)
 
 
+@pytest.mark.parametrize("B,ctx,plans", [
+    (3, 700, (5, 0, 3, 64, 1, 0, 7)),
+    (8, 2000, (1024, 0, 1024, 9, 0)),  # 8000 one-block ranges with 1024 splits
+])
+def test_workspace_reused_across_plans(tq, orc, B, ctx, plans):
+    """One workspace serves calls with different split plans back to back, holding the
+    last call's partials: every partial a plan reads is written by the same call, so each
+    result equals the one from a fresh workspace bit for bit (and the oracle's)."""
+    w = W.make("qwen3_8b_layer", B=B, ctx=ctx)
+    g = GpuState(tq, w)
+    L = int(w.seq_lens.max())
+    nbytes = max(tq.workspace_bytes(w.B, w.Hq, w.d, S) for S in plans)
+    ws = torch.full((nbytes,), 0xff, dtype=torch.uint8, device="cuda")  # NaN floats to start
+    q = w.q().cuda()
+    for S in plans:
+        fresh = tq.decode_attention(q, g.cache, g.bt, g.seq_lens, L, w.scale, num_splits=S)
+        again = tq.decode_attention(q, g.cache, g.bt, g.seq_lens, L, w.scale, num_splits=S, workspace=ws)
+        torch.cuda.synchronize()
+        assert torch.equal(fresh, again), f"num_splits {S}"
+    q_bits = bf16_bits(w.q())
+    t = orc.default_table(w.d)
+    out = again.cpu().numpy()
+    for b, h in ((0, 0), (w.B - 1, 7)):
+        o = OracleSeq(orc, w, b, h, t)
+        heads = slice(h * w.G, (h + 1) * w.G)
+        check_attention(out[b, heads], o.attention(orc, q_bits[b, heads], w.scale), f"b={b} h={h}")
+
+
 def test_calibrated_tables_for_32_kv_heads(tq, orc):
     """Per-head re-fitted tables at the most kv heads the cache takes: the append builds
     one bin table per head in shared memory, the decode one centroid table per head."""
