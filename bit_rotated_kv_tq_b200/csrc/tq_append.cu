@@ -94,67 +94,62 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2,
 // 1/15 rounded down to fp32
 __device__ __forceinline__ float inv15_dn() { return __uint_as_float(0x3d888888u); }
 
-// 16-byte read-only load that allocates in L1: a lane's two loads cover one
-// 32-byte sector, so the second one is served by the first one's fill.
-__device__ __forceinline__ uint4 ld_nc_u4(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
-}
-
-// Request [p, p + bytes) into L2 (p and bytes multiples of 16); no completion.
-__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-// passes each warp keeps requested into L2 ahead of its loads
-constexpr int kPrefetch = 4;
+constexpr int kAppWarps = 16;   // warps per CTA (one persistent CTA per SM)
+constexpr int kAppStages = 4;   // passes in flight per warp
 
 template <int D>
 struct Geo {
     static constexpr int LPV = D / 16;    // lanes per vector
     static constexpr int VPW = 32 / LPV;  // vectors per warp pass
+    static constexpr uint32_t kPass = VPW * D * 2;  // bytes of one pass's keys (or values)
+    static constexpr uint32_t kStage = 2 * kPass;   // a ring stage: keys, then values
 };
 
-// keys and values of pass p into L2
-template <int D>
-__device__ __forceinline__ void prefetch_pass(const AppendArgs& a, uint32_t p, uint32_t npass,
-                                              uint32_t total) {
-    if (p >= npass) return;
-    const uint32_t v0 = p * Geo<D>::VPW;
-    const uint32_t nv = min((uint32_t)Geo<D>::VPW, total - v0);
-    prefetch_l2_bulk(a.K + (size_t)v0 * D, nv * D * 2);
-    prefetch_l2_bulk(a.V + (size_t)v0 * D, nv * D * 2);
+// ---- shared-memory helpers of the input ring
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint4 lds_u4(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a));
+    return v;
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t phase) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    return ok != 0;
+}
+// Wait for a phase of the barrier, giving up after ~2^31 clocks (about a second).
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t phase) {
+    if (mbar_try(bar, phase)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try(bar, phase))
+        if (clock64() - t0 > (1LL << 31)) return false;
+    return true;
 }
 
-// One warp pass's inputs (loaded during the pass before).
+// The pass-level bookkeeping of one warp pass (its inputs sit in a ring stage).
 struct Pass {
-    uint4 k0, k1, v0, v1;  // this lane's 16 bf16 keys / values
-    int slot;              // slot_mapping entry of the token (-1: skip)
-    int pb;                // physical block read from the block table (when one is given)
-    uint32_t vec;
-    bool in;
+    int slot;      // slot_mapping entry of the token (-1: skip)
+    int pb;        // physical block read from the block table (when one is given)
+    uint32_t vec;  // this lane's vector (token * H_kv + head)
+    bool in;       // the vector exists
 };
 
 template <int D>
-__device__ __forceinline__ void load_pass(const AppendArgs& a, uint32_t p, uint32_t npass,
-                                          uint32_t total, int grp, int sub, Pass& L) {
+__device__ __forceinline__ void pass_slot(const AppendArgs& a, uint32_t p, uint32_t total, int grp,
+                                          Pass& L) {
     L.vec = p * Geo<D>::VPW + grp;
-    L.in = p < npass && L.vec < total;
-    L.slot = -1;
+    L.in = L.vec < total;
+    L.slot = L.in ? __ldg(a.slots + fast_div32(L.vec, a.dv_hkv)) : -1;
     L.pb = -1;
-    L.k0 = L.k1 = L.v0 = L.v1 = make_uint4(0, 0, 0, 0);
-    if (L.in) {
-        const uint32_t t = fast_div32(L.vec, a.dv_hkv);
-        L.slot = __ldg(a.slots + t);
-        const size_t eoff = (size_t)L.vec * D + sub * 16;  // vec = t * Hkv + h
-        L.k0 = ld_nc_u4(a.K + eoff);
-        L.k1 = ld_nc_u4(a.K + eoff + 8);
-        L.v0 = ld_nc_u4(a.V + eoff);
-        L.v1 = ld_nc_u4(a.V + eoff + 8);
-    }
 }
 
 // With a block table, fetch the physical block of the pass's slot (issued at
@@ -180,41 +175,100 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
 // ties to even, and leaves that integer in the low mantissa bits.
 constexpr float kRound = 12582912.0f;
 
+// Shared memory: the bin tables (ntab tables of kBins entries, then the
+// HeadBins), then each warp's ring of kAppStages stages (a pass's keys and
+// values, 128-byte aligned), then one mbarrier per stage.
 template <int D>
-__global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
-    extern __shared__ __align__(16) unsigned char smem[];
+struct AppPlan {
+    uint32_t rings, bars, end;
+    __host__ __device__ explicit AppPlan(int ntab) {
+        const uint32_t tab = (uint32_t)ntab * (kBins * sizeof(BinEntry) + sizeof(HeadBins));
+        rings = (tab + 127) & ~127u;
+        bars = rings + kAppWarps * kAppStages * Geo<D>::kStage;
+        end = bars + kAppWarps * kAppStages * 8;
+    }
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a) {
+    extern __shared__ __align__(128) unsigned char smem[];
     constexpr int LPV = Geo<D>::LPV;
     constexpr int VPW = Geo<D>::VPW;
+    constexpr uint32_t PB = Geo<D>::kPass;
     using R = Rec<D>;
     const int ntab = a.k_tables ? a.Hkv : 1;
     BinEntry* bins = reinterpret_cast<BinEntry*>(smem);
     HeadBins* hb = reinterpret_cast<HeadBins*>(smem + (size_t)ntab * kBins * sizeof(BinEntry));
+    const AppPlan<D> P(ntab);
 
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int sub = lane % LPV;
     const int grp = lane / LPV;
     const uint32_t total = (uint32_t)a.T * (uint32_t)a.Hkv;
     const uint32_t npass = (total + VPW - 1) / VPW;
-    const uint32_t nwarps = gridDim.x * (blockDim.x / 32);
+    const uint32_t nwarps = gridDim.x * kAppWarps;
     const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.125f;  // fp32 of 1/sqrt(D)
 
-    uint32_t pass = blockIdx.x * (blockDim.x / 32) + threadIdx.x / 32;
-    // the warp's first passes into L2 (lane j: pass + j W), then its first loads;
-    // the bins are built while they are in flight
-    if (lane < kPrefetch) prefetch_pass<D>(a, pass + (uint32_t)lane * nwarps, npass, total);
+    // ---- this warp's passes gw, gw + nwarps, ...: their keys and values stream
+    // through the warp's ring (one bulk copy each, one mbarrier per stage)
+    const uint32_t gw = blockIdx.x * kAppWarps + wid;
+    const int cnt = gw < npass ? (int)((npass - 1 - gw) / nwarps) + 1 : 0;
+    const uint32_t ring = smem_addr(smem) + P.rings + wid * kAppStages * Geo<D>::kStage;
+    const uint32_t bar0 = smem_addr(smem) + P.bars + wid * kAppStages * 8;
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kAppStages; s++)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8 * s) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    // Copy pass k of this warp into stage k % kAppStages (lane 0; nothing past the end).
+    auto issue = [&](int k) {
+        if (k >= cnt || lane != 0) return;
+        const uint32_t p = gw + (uint32_t)k * nwarps;
+        const uint32_t v0 = p * VPW;
+        const uint32_t bytes = min((uint32_t)VPW, total - v0) * D * 2;
+        const uint32_t st = ring + (uint32_t)(k % kAppStages) * Geo<D>::kStage;
+        const uint32_t bar = bar0 + 8 * (uint32_t)(k % kAppStages);
+        asm volatile(
+            "fence.proxy.async.shared::cta;\n"
+            "mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n"
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3], %4, [%0];\n"
+            "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%5], [%6], %4, [%0];\n"
+            ::"r"(bar), "r"(2 * bytes), "r"(st), "l"(a.K + (size_t)v0 * D), "r"(bytes), "r"(st + PB),
+            "l"(a.V + (size_t)v0 * D)
+            : "memory");
+    };
+#pragma unroll 1
+    for (int k = 0; k < kAppStages; k++) issue(k);
     Pass cur, nxt;
-    load_pass<D>(a, pass, npass, total, grp, sub, cur);
+    if (cnt > 0) pass_slot<D>(a, gw, total, grp, cur);
     build_bins(hb, bins, a);
 
-    for (; pass < npass; pass += nwarps) {
-        fetch_block(a, cur);  // its slot was loaded with the pass's inputs
-        if (lane == 0) prefetch_pass<D>(a, pass + (uint32_t)kPrefetch * nwarps, npass, total);
+    int issued = min(cnt, kAppStages), k = 0;
+    bool aborted = false;
+#pragma unroll 1
+    for (; k < cnt; k++) {
+        const uint32_t pass = gw + (uint32_t)k * nwarps;
+        fetch_block(a, cur);  // its slot was loaded a pass ago
+        if (k + 1 < cnt) pass_slot<D>(a, pass + nwarps, total, grp, nxt);
         const uint32_t t = fast_div32(cur.vec, a.dv_hkv);
         const int h = cur.in ? (int)(cur.vec - t * (uint32_t)a.Hkv) : 0;
+        const uint32_t stage = ring + (uint32_t)(k % kAppStages) * Geo<D>::kStage;
+        if (!__all_sync(kFull, mbar_wait_bounded(bar0 + 8 * (uint32_t)(k % kAppStages),
+                                                 (uint32_t)(k / kAppStages) & 1u))) {
+            if (lane == 0) flag_status(a.status, TQ_STATUS_TIMEOUT);
+            aborted = true;
+            break;
+        }
+        // this lane's 16 keys and values (a lane past the pass's last vector reads
+        // stale stage bytes; it stores nothing)
+        const uint32_t eoff = (uint32_t)(grp * D + sub * 16) * 2;
+        uint4 ck0 = lds_u4(stage + eoff), ck1 = lds_u4(stage + eoff + 16);
+        const uint4 cv0 = lds_u4(stage + PB + eoff), cv1 = lds_u4(stage + PB + eoff + 16);
 
         // ---- values: group of 32 = this lane and lane ^ 1
-        const uint32_t vwd[8] = {cur.v0.x, cur.v0.y, cur.v0.z, cur.v0.w,
-                                 cur.v1.x, cur.v1.y, cur.v1.z, cur.v1.w};
+        const uint32_t vwd[8] = {cv0.x, cv0.y, cv0.z, cv0.w, cv1.x, cv1.y, cv1.z, cv1.w};
         __nv_bfloat162 mn2 = *reinterpret_cast<const __nv_bfloat162*>(&vwd[0]);
         __nv_bfloat162 mx2 = mn2;
 #pragma unroll
@@ -304,8 +358,7 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
 
         // ---- key: norm and in-lane butterfly over element bits 0-3.  Q[j]
         // holds elements (2j, 2j+1) of the lane's 16.
-        const uint32_t kwd[8] = {cur.k0.x, cur.k0.y, cur.k0.z, cur.k0.w,
-                                 cur.k1.x, cur.k1.y, cur.k1.z, cur.k1.w};
+        const uint32_t kwd[8] = {ck0.x, ck0.y, ck0.z, ck0.w, ck1.x, ck1.y, ck1.z, ck1.w};
         float2 Q[8];
         float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
         uint32_t kor = 0;
@@ -436,10 +489,9 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
                     }
                 }
             }
-            // this lane's keys again (L1 hits: they came through L1 a pass ago) and
-            // the exact norm from their fp64 sum of squares
-            const uint16_t* kp = a.K + (size_t)(cur.in ? cur.vec : 0u) * D + sub * 16;
-            const uint4 ra = ld_nc_u4(kp), rb = ld_nc_u4(kp + 8);
+            // this lane's keys again (still in the stage) and the exact norm from
+            // their fp64 sum of squares
+            const uint4 ra = lds_u4(stage + eoff), rb = lds_u4(stage + eoff + 16);
             const uint32_t w[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
             double s0 = 0.0, s1 = 0.0;
 #pragma unroll
@@ -504,9 +556,10 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
             }
         }
 
-        // the next pass's inputs, issued after the key work so that they do not hold
-        // registers through it (they are L2 hits: prefetched passes ago)
-        load_pass<D>(a, pass + nwarps, npass, total, grp, sub, nxt);
+        // the stage is read: refill it with the pass kAppStages ahead
+        __syncwarp();
+        issue(k + kAppStages);
+        if (k + kAppStages < cnt) issued++;
 
         // ---- where this vector goes (the block-table read was issued at the top)
         int blk = -1;
@@ -547,27 +600,15 @@ __global__ void __launch_bounds__(256, 3) append_kernel(AppendArgs a) {
 
         cur = nxt;
     }
+    if (aborted) {  // give the copies still in flight a bounded chance to land
+#pragma unroll 1
+        for (int j = k; j < issued; j++)
+            mbar_wait_bounded(bar0 + 8 * (uint32_t)(j % kAppStages), (uint32_t)(j / kAppStages) & 1u);
+    }
 }
 
-size_t append_smem_bytes(int ntab) {
-    return (size_t)ntab * kBins * sizeof(BinEntry) + (size_t)ntab * sizeof(HeadBins);
-}
-
-// CTAs of append_kernel<D> resident per SM with this much dynamic shared memory,
-// by size class, computed once per process.
-template <int D>
-static int resident_ctas(int num_sms, size_t smem) {
-    static std::once_flag once[2];
-    static int per_sm[2] = {0, 0};
-    const int key = smem > 16384 ? 1 : 0;
-    std::call_once(once[key], [&] {
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, append_kernel<D>, 256, smem) !=
-                cudaSuccess || n <= 0)
-            n = 1;
-        per_sm[key] = n;
-    });
-    return per_sm[key] * num_sms;
+size_t append_smem_bytes(int ntab, int head_dim) {
+    return head_dim == 128 ? AppPlan<128>(ntab).end : AppPlan<64>(ntab).end;
 }
 
 // The bins of the default table of head_dim d, computed once per process
@@ -589,26 +630,41 @@ static void default_bins(int d, const uint16_t* table16, HeadBins& hb, BinEntry*
     memcpy(bins, cached[key], sizeof cached[key]);
 }
 
+template <int D>
+static cudaError_t launch_a(const AppendArgs& a, int num_sms, cudaStream_t stream) {
+    // the largest shared-memory size, set once per device (under a lock: the
+    // library may be called from several host threads)
+    static std::mutex mu;
+    static bool configured[64] = {};
+    static const size_t max_smem = AppPlan<D>(32).end;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (dev < 0 || dev >= 64 || !configured[dev]) {
+            e = cudaFuncSetAttribute(append_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)max_smem);
+            if (e != cudaSuccess) return e;
+            if (dev >= 0 && dev < 64) configured[dev] = true;
+        }
+    }
+    const long long vectors = (long long)a.T * a.Hkv;
+    const long long passes = (vectors + Geo<D>::VPW - 1) / Geo<D>::VPW;
+    long long blocks = (passes + kAppWarps - 1) / kAppWarps;
+    if (blocks > num_sms) blocks = num_sms;  // one persistent wave; warps loop over the passes
+    if (blocks < 1) blocks = 1;
+    const size_t smem = AppPlan<D>(a.k_tables ? a.Hkv : 1).end;
+    append_kernel<D><<<(unsigned)blocks, kAppWarps * 32, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_append(const AppendArgs& args, int head_dim, int num_sms, cudaStream_t stream) {
     AppendArgs a = args;
     if (!a.k_tables) default_bins(head_dim, a.default_table, a.default_hb, a.default_bins);
     a.dv_hkv = div32_magic((uint32_t)a.Hkv);
     a.dv_cap = div32_magic((uint32_t)(a.max_blocks > 0 ? a.max_blocks * kBlock : 1));
-    const int threads = 256;
-    const long long vectors = (long long)a.T * a.Hkv;
-    const int vpw = 32 / (head_dim / 16);
-    const long long warps_needed = (vectors + vpw - 1) / vpw;
-    long long blocks = (warps_needed + threads / 32 - 1) / (threads / 32);
-    const size_t smem = append_smem_bytes(a.k_tables ? a.Hkv : 1);
-    const long long cap = head_dim == 128 ? resident_ctas<128>(num_sms, smem)
-                                          : resident_ctas<64>(num_sms, smem);
-    if (blocks > cap) blocks = cap;  // one wave; warps loop over the passes
-    if (blocks < 1) blocks = 1;
-    if (head_dim == 128)
-        append_kernel<128><<<(unsigned)blocks, threads, smem, stream>>>(a);
-    else
-        append_kernel<64><<<(unsigned)blocks, threads, smem, stream>>>(a);
-    return cudaGetLastError();
+    return head_dim == 128 ? launch_a<128>(a, num_sms, stream) : launch_a<64>(a, num_sms, stream);
 }
 
 }  // namespace tq

@@ -402,7 +402,7 @@ __device__ __forceinline__ void record_scores(uint32_t rec, int g, int c, uint32
 // lane's fp16 parts of the weights (u, w: tokens 2c, 2c+1 | 2c+8, 2c+9 of head
 // g/2 of each group) and the valid-token masks of the fp16 lanes (mA: tokens
 // 2c, 2c+1; mB: tokens 2c+8, 2c+9; all ones for a full record).
-template <int D, int QPI>
+template <int D, int QPI, bool MASK>
 __device__ __forceinline__ void record_values(uint32_t rec, int g, int c, uint32_t mA, uint32_t mB,
                                               const uint32_t (&u01)[QPI], const uint32_t (&w01)[QPI],
                                               const uint32_t (&u89)[QPI], const uint32_t (&w89)[QPI],
@@ -418,13 +418,14 @@ __device__ __forceinline__ void record_values(uint32_t rec, int g, int c, uint32
 #pragma unroll
         for (int e = 0; e < 4; e++) sw[i + e] = t4[e];
     }
-    // stale fields of unwritten tokens must not reach the products
-    zz.x &= mA;
-    zz.y &= mB;
+    if (MASK) {  // stale fields of unwritten tokens must not reach the products
+        zz.x &= mA;
+        zz.y &= mB;
 #pragma unroll
-    for (int G_ = 0; G_ < NG; G_++) {
-        sw[2 * G_] &= mA;
-        sw[2 * G_ + 1] &= mB;
+        for (int G_ = 0; G_ < NG; G_++) {
+            sw[2 * G_] &= mA;
+            sw[2 * G_ + 1] &= mB;
+        }
     }
 #pragma unroll
     for (int q = 0; q < QPI; q++) mma16816(Z[q], zz.x, kOnes, zz.y, kOnes, w01[q], w89[q]);
@@ -721,7 +722,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 const float na1 = __half2float(__ushort_as_half((uint16_t)(nw1 >> sh)));
                 const float nb1 = __half2float(__ushort_as_half((uint16_t)(nw1b >> sh)));
                 Mask m0 = {true, true, 0xffffffffu, 0xffffffffu}, m1 = m0;
-                if (n0 < kBlock || n1 < kBlock) {  // the last block of a sequence, or a bad block
+                const bool masked = n0 < kBlock || n1 < kBlock;  // a sequence's last block, or a bad one
+                if (masked) {
                     m0 = token_mask(n0, g, c);
                     m1 = token_mask(n1, g, c);
                 }
@@ -764,8 +766,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
                 }
 
                 // -------- p.z, sum p and p.V of both records
-                record_values<D, QPI>(rec0, g, c, m0.mA, m0.mB, u01[0], w01[0], u89[0], w89[0], O, Z);
-                record_values<D, QPI>(rec1, g, c, m1.mA, m1.mB, u01[1], w01[1], u89[1], w89[1], O, Z);
+                if (masked) {
+                    record_values<D, QPI, true>(rec0, g, c, m0.mA, m0.mB, u01[0], w01[0], u89[0], w89[0], O, Z);
+                    record_values<D, QPI, true>(rec1, g, c, m1.mA, m1.mB, u01[1], w01[1], u89[1], w89[1], O, Z);
+                } else {
+                    record_values<D, QPI, false>(rec0, g, c, 0u, 0u, u01[0], w01[0], u89[0], w89[0], O, Z);
+                    record_values<D, QPI, false>(rec1, g, c, 0u, 0u, u01[1], w01[1], u89[1], w89[1], O, Z);
+                }
             }
             __syncwarp();
             consumed++;
@@ -867,50 +874,57 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
 
 // Items cut by range boundaries: out[b][h] = sum_r 2^(m_r - M) o_r / sum_r 2^(m_r - M) l_r
 // over the ranges r that hold part of the item, M = max_r m_r.  Whole items
-// were written by the split kernel and are skipped.
+// were written by the split kernel and are skipped.  One warp per (sequence,
+// query head) pair, each lane D / 32 dims; two ranges' loads in flight at once.
 template <int D, int QPI>
-__global__ void __launch_bounds__(D) combine_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(32) combine_kernel(DecodeArgs a) {
     constexpr int HPI = kHeads * QPI;
-    const int bh = blockIdx.x;
-    const int i = threadIdx.x;
+    constexpr int DPL = D / 32;
+    const int lane = threadIdx.x;
     const int G = a.Hq / a.Hkv;
-    const int b = bh / a.Hq, hh = bh % a.Hq;
-    const int kv = hh / G, quad = (hh % G) / HPI, h = (hh % G) % HPI;
-    const int item = (b * a.Hkv + kv) * a.quads + quad;
-    const int base = item * a.nmax;
-    const int rA = base / a.R, rB = (base + a.nmax - 1) / a.R;
-    if (rA == rB) return;  // whole inside one range: already written
-    auto part = [&](int r) {
-        const int slot = r * a.R / a.nmax == item ? 0 : 1;
-        return ((size_t)r * 2 + slot) * HPI + h;
-    };
-    if (rB == rA + 1) {  // the usual cut: two ranges, their loads issued together
-        const size_t p0 = part(rA), p1 = part(rB);
-        const float2 ml0 = a.ws_ml[p0], ml1 = a.ws_ml[p1];
-        const float o0 = a.ws_o[p0 * D + i], o1 = a.ws_o[p1 * D + i];
-        const float M = fmaxf(fmaxf(-INFINITY, ml0.x), ml1.x);
-        float o = 0.f, l = 0.f;
-        if (M != -INFINITY) {
-            const float f0 = ex2(ml0.x - M), f1 = ex2(ml1.x - M);
-            o = fmaf(f1, o1, fmaf(f0, o0, 0.f));
-            l = fmaf(f1, ml1.y, fmaf(f0, ml0.y, 0.f));
+#pragma unroll 1
+    for (int bh = blockIdx.x; bh < a.B * a.Hq; bh += gridDim.x) {
+        const int b = bh / a.Hq, hh = bh % a.Hq;
+        const int kv = hh / G, quad = (hh % G) / HPI, h = (hh % G) % HPI;
+        const int item = (b * a.Hkv + kv) * a.quads + quad;
+        const int base = item * a.nmax;
+        const int rA = base / a.R, rB = (base + a.nmax - 1) / a.R;
+        if (rA == rB) continue;  // whole inside one range: already written
+        float M = -INFINITY, l = 0.f, o[DPL];
+#pragma unroll
+        for (int j = 0; j < DPL; j++) o[j] = 0.f;
+#pragma unroll 1
+        for (int r0 = rA; r0 <= rB; r0 += 2) {  // two ranges' loads in flight at a time
+            float2 ml[2];
+            float po[2][DPL];
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const int r = r0 + u;
+                ml[u] = make_float2(-INFINITY, 0.f);
+#pragma unroll
+                for (int j = 0; j < DPL; j++) po[u][j] = 0.f;
+                if (r <= rB) {
+                    const int slot = r * a.R / a.nmax == item ? 0 : 1;
+                    const size_t pr = ((size_t)r * 2 + slot) * HPI + h;
+                    ml[u] = a.ws_ml[pr];
+#pragma unroll
+                    for (int j = 0; j < DPL; j++) po[u][j] = a.ws_o[pr * D + j * 32 + lane];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+                const float Mn = fmaxf(M, ml[u].x);
+                const float f0 = M == -INFINITY ? 0.f : ex2(M - Mn);
+                const float f1 = ml[u].x == -INFINITY ? 0.f : ex2(ml[u].x - Mn);
+#pragma unroll
+                for (int j = 0; j < DPL; j++) o[j] = fmaf(f1, po[u][j], f0 * o[j]);
+                l = fmaf(f1, ml[u].y, f0 * l);
+                M = Mn;
+            }
         }
-        a.out[(size_t)bh * D + i] = l > 0.f ? o / l : 0.f;
-        return;
+#pragma unroll
+        for (int j = 0; j < DPL; j++) a.out[(size_t)bh * D + j * 32 + lane] = l > 0.f ? o[j] / l : 0.f;
     }
-    float M = -INFINITY;
-    for (int r = rA; r <= rB; r++) M = fmaxf(M, a.ws_ml[part(r)].x);
-    float o = 0.f, l = 0.f;
-    if (M != -INFINITY) {
-        for (int r = rA; r <= rB; r++) {
-            const size_t pr = part(r);
-            const float2 ml = a.ws_ml[pr];
-            const float f = ex2(ml.x - M);
-            o = fmaf(f, a.ws_o[pr * D + i], o);
-            l = fmaf(f, ml.y, l);
-        }
-    }
-    a.out[(size_t)bh * D + i] = l > 0.f ? o / l : 0.f;
 }
 
 template <int D, int QPI>
@@ -936,7 +950,7 @@ cudaError_t launch_d(DecodeArgs a, int num_sms, cudaStream_t stream) {
     const int halves = (a.nranges + kHalves - 1) / kHalves;
     const int grid = halves < num_sms ? halves : num_sms;
     decode_split_kernel<D, QPI><<<grid, kWarps * 32, smem, stream>>>(a);
-    if (decode_needs_combine(a)) combine_kernel<D, QPI><<<a.B * a.Hq, D, 0, stream>>>(a);
+    if (decode_needs_combine(a)) combine_kernel<D, QPI><<<a.B * a.Hq, 32, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

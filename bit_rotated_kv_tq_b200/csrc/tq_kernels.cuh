@@ -131,7 +131,7 @@ int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tab
                    int H_q, int max_seq_len, float scale, float* out, int num_splits,
                    int32_t* status, DecodeArgs& a, size_t& need);
 int decode_launch(DecodeArgs& a, int head_dim, void* workspace, void* stream);
-size_t append_smem_bytes(int ntab);  // ntab bin tables (1, or H_kv per-head tables)
+size_t append_smem_bytes(int ntab, int head_dim);  // ntab bin tables (1, or H_kv per-head tables)
 int set_last_error(int code, const char* msg);
 cudaError_t launch_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, int head_dim, int num_sms, cudaStream_t stream);
