@@ -94,7 +94,7 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2,
 // 1/15 rounded down to fp32
 __device__ __forceinline__ float inv15_dn() { return __uint_as_float(0x3d888888u); }
 
-constexpr int kAppWarps = 16;   // warps per CTA (one persistent CTA per SM)
+constexpr int kAppWarps = 24;   // warps per CTA (one persistent CTA per SM, at most 85 registers)
 constexpr int kAppStages = 4;   // passes in flight per warp
 
 template <int D>
@@ -206,13 +206,16 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
     const int grp = lane / LPV;
     const uint32_t total = (uint32_t)a.T * (uint32_t)a.Hkv;
     const uint32_t npass = (total + VPW - 1) / VPW;
-    const uint32_t nwarps = gridDim.x * kAppWarps;
     const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.125f;  // fp32 of 1/sqrt(D)
 
-    // ---- this warp's passes gw, gw + nwarps, ...: their keys and values stream
-    // through the warp's ring (one bulk copy each, one mbarrier per stage)
-    const uint32_t gw = blockIdx.x * kAppWarps + wid;
-    const int cnt = gw < npass ? (int)((npass - 1 - gw) / nwarps) + 1 : 0;
+    // ---- the CTA's passes are an even share [p0, p1) of all of them (so every SM
+    // has the same work); warp wid takes p0 + wid, p0 + wid + kAppWarps, ...,
+    // and their keys and values stream through the warp's ring (one bulk copy
+    // each, one mbarrier per stage)
+    const uint32_t p0 = (uint32_t)(((unsigned long long)blockIdx.x * npass) / gridDim.x);
+    const uint32_t p1 = (uint32_t)(((unsigned long long)(blockIdx.x + 1) * npass) / gridDim.x);
+    const uint32_t gw = p0 + (uint32_t)wid;
+    const int cnt = gw < p1 ? (int)((p1 - 1 - gw) / kAppWarps) + 1 : 0;
     const uint32_t ring = smem_addr(smem) + P.rings + wid * kAppStages * Geo<D>::kStage;
     const uint32_t bar0 = smem_addr(smem) + P.bars + wid * kAppStages * 8;
     if (lane == 0) {
@@ -225,7 +228,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
     // Copy pass k of this warp into stage k % kAppStages (lane 0; nothing past the end).
     auto issue = [&](int k) {
         if (k >= cnt || lane != 0) return;
-        const uint32_t p = gw + (uint32_t)k * nwarps;
+        const uint32_t p = gw + (uint32_t)k * kAppWarps;
         const uint32_t v0 = p * VPW;
         const uint32_t bytes = min((uint32_t)VPW, total - v0) * D * 2;
         const uint32_t st = ring + (uint32_t)(k % kAppStages) * Geo<D>::kStage;
@@ -249,9 +252,9 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
     bool aborted = false;
 #pragma unroll 1
     for (; k < cnt; k++) {
-        const uint32_t pass = gw + (uint32_t)k * nwarps;
+        const uint32_t pass = gw + (uint32_t)k * kAppWarps;
         fetch_block(a, cur);  // its slot was loaded a pass ago
-        if (k + 1 < cnt) pass_slot<D>(a, pass + nwarps, total, grp, nxt);
+        if (k + 1 < cnt) pass_slot<D>(a, pass + kAppWarps, total, grp, nxt);
         const uint32_t t = fast_div32(cur.vec, a.dv_hkv);
         const int h = cur.in ? (int)(cur.vec - t * (uint32_t)a.Hkv) : 0;
         const uint32_t stage = ring + (uint32_t)(k % kAppStages) * Geo<D>::kStage;
