@@ -654,8 +654,10 @@ static cudaError_t launch_a(const AppendArgs& a, int num_sms, cudaStream_t strea
     }
     const long long vectors = (long long)a.T * a.Hkv;
     const long long passes = (vectors + Geo<D>::VPW - 1) / Geo<D>::VPW;
-    long long blocks = (passes + kAppWarps - 1) / kAppWarps;
-    if (blocks > num_sms) blocks = num_sms;  // one persistent wave; warps loop over the passes
+    // one persistent wave over every SM (each CTA takes an even share of the passes,
+    // so a small append spreads over the whole GPU rather than filling a few SMs)
+    long long blocks = passes;
+    if (blocks > num_sms) blocks = num_sms;
     if (blocks < 1) blocks = 1;
     const size_t smem = AppPlan<D>(a.k_tables ? a.Hkv : 1).end;
     append_kernel<D><<<(unsigned)blocks, kAppWarps * 32, smem, stream>>>(a);
