@@ -77,6 +77,7 @@ def _declare(L):
     L.orc_quantize_append.argtypes = [_P, _P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _I, _P, _P]
     L.orc_dequantize.argtypes = [_P, _I, _I, _I, _P, _P, _I, _P, _I, _I, _P, _P]
     L.orc_attention.argtypes = [_P, _I, _I, _I, _I, _P, _P, _I, _P, _D, _P]
+    L.orc_prefill_attention.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _D, _P]
     L.orc_kmeans_table.argtypes = [_P, _I, _P, _I, _P]
     L.orc_rotated_unit_samples.argtypes = [_P, _I, _I, _P]
 
@@ -251,6 +252,23 @@ def attention(q_bits, Khat, Vhat, seq_lens, scale):
     out = np.zeros((B, Hq, d), np.float64)
     _check(lib().orc_attention(_ptr(q), B, Hq, Hkv, d, _ptr(_c(Khat, np.float64)), _ptr(_c(Vhat, np.float64)),
                                max_len, _ptr(_c(seq_lens, np.int32)), float(scale), _ptr(out)), "attention")
+    return out
+
+
+def prefill_attention(q_bits, q_start, Khat, Vhat, seq_lens, scale):
+    """Chunked prefill: q_bits uint16 [T][Hq][d] (bf16), q_start int32 [B+1]; the chunk of
+    sequence b is its last q_start[b+1] - q_start[b] cached tokens, each attending causally.
+    Returns fp64 [T][Hq][d]."""
+    q = _c(q_bits, np.uint16)
+    T, Hq, d = q.shape
+    qs = _c(q_start, np.int32)
+    B = qs.shape[0] - 1
+    _, max_len, Hkv, _ = Khat.shape
+    out = np.zeros((T, Hq, d), np.float64)
+    _check(lib().orc_prefill_attention(_ptr(q), _ptr(qs), B, Hq, Hkv, d, _ptr(_c(Khat, np.float64)),
+                                       _ptr(_c(Vhat, np.float64)), max_len,
+                                       _ptr(_c(seq_lens, np.int32)), float(scale), _ptr(out)),
+           "prefill_attention")
     return out
 
 

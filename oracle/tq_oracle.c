@@ -616,6 +616,73 @@ int orc_attention(const uint16_t *q, int B, int Hq, int Hkv, int d, const double
     return 0;
 }
 
+/* Chunked-prefill attention -- the prompt chunks of multi-turn serving, whose
+ * reuse of a cached prefix is what the pages measure ("TurboQuant 在 AMD GPU 上把
+ * 長上下文延遲壓下來", summary table, prefix-cache hit rate; "UltraQuant：4-bit
+ * KV 快取加速長代理", 「它實際證明了什麼」, late-round TTFT from cache residency).
+ * Sequence b's q_len = q_start[b+1] - q_start[b]
+ * newest tokens are the chunk, already in the cache (seq_lens[b] tokens in
+ * all), and chunk token i (position p = seq_lens[b] - q_len + i) attends to
+ * the cached tokens [0, p] -- causal within the chunk.  q bf16 [T][Hq][d]
+ * with T = q_start[B]; out fp64 [T][Hq][d]. */
+int orc_prefill_attention(const uint16_t *q, const int32_t *q_start, int B, int Hq, int Hkv, int d,
+                          const double *Khat, const double *Vhat, int max_len,
+                          const int32_t *seq_lens, double scale, double *out)
+{
+    if (!q || !q_start || !Khat || !Vhat || !seq_lens || !out || Hkv <= 0 || Hq % Hkv)
+        return -1;
+    int G = Hq / Hkv;
+    double *a = malloc(sizeof(double) * (max_len > 0 ? max_len : 1));
+    double *qd = malloc(sizeof(double) * d);
+    int rc = 0;
+    for (int b = 0; b < B; b++) {
+        int qlen = q_start[b + 1] - q_start[b];
+        int L = seq_lens[b];
+        for (int i = 0; i < qlen; i++) {
+            int tok = q_start[b] + i;
+            int n = L - qlen + i + 1; /* keys this query sees: positions 0 .. L - qlen + i */
+            if (n > max_len || n < 1) {
+                rc = -3;
+                n = 0;
+            }
+            for (int h = 0; h < Hq; h++) {
+                int kv = h / G;
+                double *o = out + ((size_t)tok * Hq + h) * d;
+                for (int e = 0; e < d; e++) {
+                    qd[e] = orc_bf16_to_double(q[((size_t)tok * Hq + h) * d + e]);
+                    o[e] = 0.0;
+                }
+                if (n <= 0)
+                    continue;
+                double amax = -INFINITY;
+                for (int t = 0; t < n; t++) {
+                    const double *k = Khat + (((size_t)b * max_len + t) * Hkv + kv) * d;
+                    double acc = 0.0;
+                    for (int e = 0; e < d; e++)
+                        acc += qd[e] * k[e];
+                    a[t] = scale * acc;
+                    if (a[t] > amax)
+                        amax = a[t];
+                }
+                double denom = 0.0;
+                for (int t = 0; t < n; t++) {
+                    a[t] = exp(a[t] - amax);
+                    denom += a[t];
+                }
+                for (int t = 0; t < n; t++) {
+                    const double *v = Vhat + (((size_t)b * max_len + t) * Hkv + kv) * d;
+                    double pr = a[t] / denom;
+                    for (int e = 0; e < d; e++)
+                        o[e] += pr * v[e];
+                }
+            }
+        }
+    }
+    free(a);
+    free(qd);
+    return rc;
+}
+
 /* ------------------------------------------------------------------ */
 /* calibrated table                                                     */
 /* ------------------------------------------------------------------ */

@@ -99,6 +99,14 @@ int orc_attention(const uint16_t *q, int B, int Hq, int Hkv, int d, const double
                   const double *Vhat, int max_len, const int32_t *seq_lens, double scale,
                   double *out);
 
+/* Chunked-prefill attention over dequantised K/V: the last q_len = q_start[b+1] -
+ * q_start[b] of sequence b's seq_lens[b] cached tokens are the chunk, and chunk
+ * token i attends to positions 0 .. seq_lens[b] - q_len + i (causal within the
+ * chunk).  q bf16 [q_start[B]][Hq][d]; out fp64 [q_start[B]][Hq][d]. */
+int orc_prefill_attention(const uint16_t *q, const int32_t *q_start, int B, int Hq, int Hkv, int d,
+                          const double *Khat, const double *Vhat, int max_len,
+                          const int32_t *seq_lens, double scale, double *out);
+
 /* 1-D k-means (Lloyd) refit of a 16-entry table on n scalar samples, starting
  * from init; empty clusters keep their centroid; the result is sorted and
  * rounded to fp16.  Returns the number of iterations run (>= 0). */

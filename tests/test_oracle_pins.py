@@ -734,3 +734,59 @@ def test_glue_check_catches_planted_mistakes(orc):
     stale_K[0, c["lens"][0]:] = 0.5
     with pytest.raises(AssertionError):
         _check_glue(c, stale_K, stale_V, Ke, Ve)
+
+
+# ---------------------------------------------------------------- chunked prefill
+def _prefill_case(orc, B=3, Hq=8, Hkv=2, d=64, Ls=(37, 20, 64), qlens=(5, 20, 1)):
+    r = np.random.default_rng(77)
+    max_len = max(Ls)
+    q_start = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
+    q = bf16_bits_of(r.standard_normal((int(q_start[-1]), Hq, d)))
+    Kh = r.standard_normal((B, max_len, Hkv, d))
+    Vh = r.standard_normal((B, max_len, Hkv, d))
+    return q, q_start, Kh, Vh, np.array(Ls, np.int32)
+
+
+def test_prefill_rows_equal_decode_attention_at_their_positions(orc):
+    """Each chunk token's output equals the (pinned) decode attention of that query
+    over the cached tokens up to and including its own position."""
+    q, q_start, Kh, Vh, L = _prefill_case(orc)
+    scale = 1 / 8
+    out = orc.prefill_attention(q, q_start, Kh, Vh, L, scale)
+    for b in range(len(L)):
+        qlen = q_start[b + 1] - q_start[b]
+        for i in range(qlen):
+            tok = q_start[b] + i
+            n = L[b] - qlen + i + 1
+            want = orc.attention(q[tok][None], Kh[b:b + 1], Vh[b:b + 1], np.array([n], np.int32), scale)[0]
+            assert np.array_equal(out[tok], want), (b, i)
+
+
+def test_prefill_is_causal_and_first_position_returns_first_value(orc):
+    q, q_start, Kh, Vh, L = _prefill_case(orc, Ls=(20, 20, 64), qlens=(20, 3, 1))
+    scale = 1 / 8
+    out = orc.prefill_attention(q, q_start, Kh, Vh, L, scale)
+    # sequence 0 is all chunk: its first token sees only position 0
+    for h in range(8):
+        assert np.allclose(out[0, h], Vh[0, 0, h // 4], atol=1e-15)
+    # changing keys and values after a token's position leaves its output unchanged
+    Kp, Vp = Kh.copy(), Vh.copy()
+    Kp[0, 10:] += 5.0
+    Vp[0, 10:] -= 3.0
+    out2 = orc.prefill_attention(q, q_start, Kp, Vp, L, scale)
+    assert np.array_equal(out[:10], out2[:10])  # tokens 0..9 of sequence 0
+    assert not np.allclose(out[10:20], out2[10:20])
+
+
+def test_prefill_matches_scipy_softmax(orc):
+    q, q_start, Kh, Vh, L = _prefill_case(orc, B=1, Ls=(30,), qlens=(7,))
+    scale = 0.3
+    out = orc.prefill_attention(q, q_start, Kh, Vh, L, scale)
+    qd = torch.tensor(q.view(np.int16)).view(torch.bfloat16).double().numpy()
+    for i in range(7):
+        n = 30 - 7 + i + 1
+        for h in range(8):
+            kv = h // 4
+            a = scale * (Kh[0, :n, kv] @ qd[i, h])
+            want = scipy.special.softmax(a) @ Vh[0, :n, kv]
+            assert np.allclose(out[i, h], want, rtol=1e-12, atol=1e-13)
