@@ -70,6 +70,8 @@ def load(path: str | None = None):
                                              _P, _I, _P, _P]
     L.tq_decode_static_scratch_bytes.restype = _Z
     L.tq_decode_static_scratch_bytes.argtypes = []
+    L.tq_prefill_attention.argtypes = [_P, ctypes.POINTER(_Cache), _P, _P, _I, _P, _P, _I, _I, _I, _I, _F, _P,
+                                       _P, _P]
     L.tq_last_error.restype = ctypes.c_char_p
     L.tq_last_error.argtypes = []
     _lib = L
@@ -270,6 +272,37 @@ def decode_attention_static(q, cache: Cache, block_tables, seq_lens, max_seq_len
                                              block_tables.shape[1], _ptr(seq_lens), B, Hq,
                                              int(max_seq_len), float(scale), _ptr(out), int(num_splits),
                                              _ptr(status), _stream(stream)))
+    return out
+
+
+def prefill_attention(q, cache: Cache, block_tables, seq_lens, q_start, max_q_len: int, scale: float,
+                      out=None, k_tables=None, status=None, stream=None):
+    """Chunked-prefill attention over the compressed cache (the chunk appended first):
+    chunk token i of sequence b attends to cached positions 0 .. seq_lens[b] - q_len + i.
+    q bf16 [T][H_q][d]; chunk b is rows q_start[b] .. q_start[b+1]-1; returns fp32
+    [T][H_q][d].  max_q_len bounds the chunks (it sizes the grid)."""
+    if q.dim() != 3:
+        raise ValueError(f"q has shape {list(q.shape)}, expected [T][H_q][d]")
+    T, Hq, d = (int(x) for x in q.shape)
+    B = int(seq_lens.shape[0]) if seq_lens.dim() == 1 else -1
+    _shape(q, (T, Hq, cache.head_dim), "q")
+    _shape(seq_lens, (B,), "seq_lens")
+    _shape(block_tables, (B, None), "block_tables")
+    _shape(q_start, (B + 1,), "q_start")
+    _shape(out, (T, Hq, d), "out")
+    _tables(k_tables, cache)
+    _status(status)
+    for t, dt, name in ((q, torch.bfloat16, "q"), (block_tables, torch.int32, "block_tables"),
+                        (seq_lens, torch.int32, "seq_lens"), (q_start, torch.int32, "q_start"),
+                        (out, torch.float32, "out"), (k_tables, torch.float16, "k_tables"),
+                        (status, torch.int32, "status"), (cache.data, torch.uint8, "cache.data")):
+        _dev(t, dt, name)
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.float32, device=q.device)
+    _check(load().tq_prefill_attention(_ptr(q), cache.c, _ptr(k_tables), _ptr(block_tables),
+                                       block_tables.shape[1], _ptr(seq_lens), _ptr(q_start), B, Hq, T,
+                                       int(max_q_len), float(scale), _ptr(out), _ptr(status),
+                                       _stream(stream)))
     return out
 
 

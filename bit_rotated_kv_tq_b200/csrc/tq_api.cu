@@ -372,6 +372,39 @@ TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uin
     return tq::decode_launch(a, cache->head_dim, need ? workspace : nullptr, stream);
 }
 
+TQ_API int tq_prefill_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
+                                const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                                const int32_t* q_start, int B, int H_q, int T, int max_q_len, float scale,
+                                float* out, int32_t* status, void* stream) {
+    int err;
+    if (!check_cache(cache, &err)) return err;
+    if (B < 0 || H_q <= 0 || T < 0 || max_q_len < 0 || max_blocks <= 0)
+        return fail(TQ_ERR_INVALID_ARG,
+                    "tq_prefill_attention: need B, T, max_q_len >= 0, H_q > 0, max_blocks > 0");
+    if (B == 0 || T == 0 || max_q_len == 0) return ok();
+    if (B > 65535) return fail(TQ_ERR_UNSUPPORTED, "tq_prefill_attention: B %d > 65535", B);
+    if (!q || !block_tables || !seq_lens || !q_start || !out)
+        return fail(TQ_ERR_INVALID_ARG,
+                    "tq_prefill_attention: q, block_tables, seq_lens, q_start and out are required");
+    const int Hkv = cache->num_kv_heads;
+    if (H_q % Hkv)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_prefill_attention: H_q %d not a multiple of H_kv %d", H_q, Hkv);
+    if ((long long)max_q_len * (H_q / Hkv) > (1LL << 30))
+        return fail(TQ_ERR_UNSUPPORTED, "tq_prefill_attention: max_q_len * GQA group too large");
+    if (!isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "tq_prefill_attention: scale not finite");
+    if (!aligned(q, 16) || !aligned(out, 16))
+        return fail(TQ_ERR_ALIGNMENT, "tq_prefill_attention: q and out must be 16-byte aligned");
+    if (!aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(q_start, 4) ||
+        (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
+        return fail(TQ_ERR_ALIGNMENT, "tq_prefill_attention: int32 arrays and tables must be 4-byte aligned");
+    cudaError_t e = tq::launch_prefill(q, static_cast<const unsigned char*>(cache->data), cache->num_blocks, Hkv,
+                                       H_q, B, k_tables, default_table(cache->head_dim), block_tables, max_blocks,
+                                       seq_lens, q_start, T, max_q_len, scale, out, status, cache->head_dim,
+                                       (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention launch");
+    return ok();
+}
+
 TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, const int32_t* block_tables,
                   int max_blocks, const int32_t* seq_lens, int B, int max_len, float* K_hat,
                   float* V_hat, int32_t* status, void* stream) {

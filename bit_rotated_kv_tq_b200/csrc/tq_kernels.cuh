@@ -140,5 +140,11 @@ bool decode_plan(DecodeArgs& a, int head_dim, int num_sms);  // ranges; false: t
 bool decode_needs_combine(const DecodeArgs& a);          // some item is cut by a range
 size_t decode_workspace_for(const DecodeArgs& a, int head_dim);  // partials, bytes
 cudaError_t launch_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);
+cudaError_t launch_prefill(const void* q, const unsigned char* cache, int num_blocks, int Hkv, int Hq, int B,
+                           const uint16_t* k_tables, const uint16_t* default_table,
+                           const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                           const int32_t* q_start, int T, int max_q_len, float scale, float* out,
+                           int32_t* status, int head_dim, cudaStream_t stream);
+size_t prefill_smem_bytes(int head_dim);
 
 }  // namespace tq

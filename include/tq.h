@@ -189,6 +189,33 @@ TQ_API int tq_decode_attention_static(const void* q, const tq_cache_t* cache,
 /* Size in bytes of the fixed array tq_decode_attention_static uses. */
 TQ_API size_t tq_decode_static_scratch_bytes(void);
 
+/* Chunked-prefill attention over the compressed cache: the prompt chunks of
+ * multi-turn serving, whose reuse of a cached prefix the pages measure
+ * ("TurboQuant 在 AMD GPU 上把長上下文延遲壓下來", summary table: prefix-cache
+ * hit rate; "UltraQuant：4-bit KV 快取加速長代理", 「它實際證明了什麼」: late-round
+ * TTFT comes from cache residency).  The chunk is appended first
+ * (tq_quantize_append), as for the decode: sequence b's chunk is its last
+ * q_len = q_start[b+1] - q_start[b] of seq_lens[b] cached tokens, and chunk
+ * token i attends to positions 0 .. seq_lens[b] - q_len + i (causal):
+ *   out[q_start[b] + i][h] = sum_t softmax_t(scale <q, k_hat_t>) v_hat_t.
+ *   q            (device) bf16 [T][H_q][d], 16-byte aligned
+ *   block_tables (device) int32 [B][max_blocks]
+ *   seq_lens     (device) int32 [B]; seq_lens[b] < q_len or > max_blocks*16 sets
+ *                TQ_STATUS_BAD_LEN and that sequence's rows get 0
+ *   q_start      (device) int32 [B+1]: chunk b is rows q_start[b] .. q_start[b+1]-1
+ *                of q and out; a chunk outside [0, T) sets TQ_STATUS_BAD_LEN and is
+ *                skipped (nothing read or written)
+ *   T            (host)   rows of q and out
+ *   max_q_len    (host)   the largest q_len (sizes the grid); a longer chunk sets
+ *                TQ_STATUS_BAD_LEN and only its first max_q_len rows are written
+ *   out          (device) fp32 [T][H_q][d], 16-byte aligned
+ * Runs on the tcgen05 tensor cores: tiles of 128 (chunk token, query head)
+ * rows of one kv head; scores and the output accumulate in tensor memory. */
+TQ_API int tq_prefill_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
+                                const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
+                                const int32_t* q_start, int B, int H_q, int T, int max_q_len,
+                                float scale, float* out, int32_t* status, void* stream);
+
 /* Dequantise every valid token (checks only): K_hat and V_hat (device) fp32
  * [B][max_len][H_kv][d] in the original (unrotated) domain,
  * k_hat = fp16 norm * H * C[idx],  v_hat = code * scale + zero;
