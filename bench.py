@@ -43,6 +43,15 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def measured_tensor_peak() -> float:
+    """Dense bf16 TFLOP/s of this machine's B200s (burst), else the fallback figure."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return 1590.0
+
+
 def decode_bytes(w) -> int:
     """Algorithmic bytes of one decode launch: the quantised records of every
     valid token (record/16 per token-head), q, block tables read, output written."""
@@ -229,6 +238,18 @@ def oracle_step(w, s):
     return oracle.attention(s["q"], Kh, Vh, s["lens"], w.scale)
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (/proc/cpuinfo), for the CPU-baseline record."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, on a bounded sample."""
     if rank != 0:
@@ -249,7 +270,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": cfg(w, "oracle sample"),
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle", "cpu_model": cpu_model(),
                          "sample": f"{n_seqs} of {w.B} sequences (all 8 kv heads, 8192 tokens, "
                                    f"32-token append) per step"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -313,7 +334,9 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
     even cut); agentic: decode over the shared-prefix batch with calibrated
     per-head tables, as logical bytes (what the sequences attend over) and unique
     bytes (distinct records); prefill_small_head: one 2048-token chunk appended to
-    every sequence, and decode at context 32768."""
+    every sequence, and decode at context 32768; prefill_chunk_attention: the
+    chunked-prefill attention of every sequence's second 2048-token chunk (context
+    4096) on the tcgen05 tensor cores, as FLOP/s against the bf16 tensor peak."""
     import bit_rotated_kv_tq_b200 as tq
 
     flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
@@ -410,6 +433,28 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
     ms = decode(w, cache, bt, 0, cold=True)
     res["prefill_small_head_decode"] = {"ms": ms, "gbs": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / peak}
     del cache
+
+    # chunked-prefill attention (tcgen05): the second 2048-token chunk of every
+    # prefill_small_head sequence, attending causally over positions 0 .. 4095;
+    # algorithmic FLOPs = 4 d per (query head, key) pair (q.k and p.v)
+    w = W.make("prefill_small_head", ctx=4096)
+    cache, bt = build(w)
+    qlen = 2048
+    lens = torch.from_numpy(w.seq_lens).to(dev)
+    q_start = (torch.arange(w.B + 1, dtype=torch.int32) * qlen).to(dev)
+    rng = np.random.default_rng([w.seed, 99])
+    q = torch.from_numpy(rng.standard_normal((w.B * qlen, w.Hq, w.d), dtype=np.float32)).to(torch.bfloat16).to(dev)
+    out = torch.empty((w.B * qlen, w.Hq, w.d), dtype=torch.float32, device=dev)
+    L = int(w.seq_lens[0])
+    pairs = w.B * w.Hq * sum(L - qlen + i + 1 for i in range(qlen))
+    flops = 4 * w.d * pairs
+    ms = graph_time(lambda: tq.prefill_attention(q, cache, bt, lens, q_start, qlen, w.scale, out=out,
+                                                 status=status), 5)
+    tf_peak = measured_tensor_peak()
+    res["prefill_chunk_attention"] = {"ms": ms, "tokens": w.B * qlen, "context": L,
+                                      "tflops": flops / ms / 1e9, "tensor_frac": flops / ms / 1e9 / tf_peak,
+                                      "tensor_peak_tflops": tf_peak}
+    del cache
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
     return res
@@ -438,6 +483,31 @@ def prefill_append_case(dev):
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0
     print(json.dumps({"case": "prefill_append", "tokens": K.shape[0], "ok": True}))
+
+
+def prefill_attention_case(dev):
+    """Chunked-prefill attention of the second 2048-token chunk of 4 prefill_small_head
+    sequences (context 4096, d 64), 3 warm-up calls then 1: the case the tcgen05
+    prefill kernel is profiled on."""
+    import bit_rotated_kv_tq_b200 as tq
+
+    tq.load()
+    w = W.make("prefill_small_head", B=4, ctx=4096)
+    cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for K, V, slots in w.population():
+        tq.quantize_append(K.to(dev), V.to(dev), slots.to(dev), cache, block_table=bt, status=status)
+    qlen = 2048
+    lens = torch.from_numpy(w.seq_lens).to(dev)
+    q_start = (torch.arange(w.B + 1, dtype=torch.int32) * qlen).to(dev)
+    q = torch.randn((w.B * qlen, w.Hq, w.d), device=dev, generator=torch.Generator(dev).manual_seed(4)).to(
+        torch.bfloat16)
+    for _ in range(4):
+        tq.prefill_attention(q, cache, bt, lens, q_start, qlen, w.scale, status=status)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0
+    print(json.dumps({"case": "prefill_attention", "ok": True}))
 
 
 def prefill_decode_case(dev):
@@ -692,7 +762,7 @@ def run_tq(args, rank, world, local):
             n_rep += 1
         dt = (time.perf_counter() - t0) / n_rep
         cpu = {"value": s["L"] * w.Hkv * tq.record_bytes(w.d) // 16 / dt / 1e9, "unit": "GB/s", "cores": 1,
-               "kind": "oracle",
+               "kind": "oracle", "cpu_model": cpu_model(),
                "sample": f"1 of {w.B} sequences (8 kv heads x {s['L']} tokens + {w.append_tokens}-token append), "
                          f"{n_rep} passes, {dt:.2f} s each"}
 
@@ -736,7 +806,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["prefill_append", "prefill_decode"], default=None,
+    ap.add_argument("--case", choices=["prefill_append", "prefill_decode", "prefill_attention"], default=None,
                     help="run one small profiling case instead of the bench")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the long-context, agentic and prefill-chunk measurements")
@@ -754,6 +824,9 @@ def main():
         return
     if args.case == "prefill_decode":
         prefill_decode_case(torch.device("cuda", 0))
+        return
+    if args.case == "prefill_attention":
+        prefill_attention_case(torch.device("cuda", 0))
         return
     rank, world, local = dist_setup(args.gpus)
     try:

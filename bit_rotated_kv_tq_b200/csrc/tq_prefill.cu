@@ -274,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
         const uint32_t bar = sBars + 8 * (uint32_t)(s % kRecStages);
         int ids[4];
         uint32_t bytes = 0;
+#pragma unroll
         for (int j = 0; j < 4; j++) {
             const int jb = 4 * s + j;
             int id = jb < nblk ? bt[jb] : -1;
@@ -291,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
             asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
         else
             asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+#pragma unroll
         for (int j = 0; j < 4; j++)
             if (ids[j] >= 0) {
                 const unsigned char* src = a.cache + (long long)ids[j] * rec_stride + (long long)kv * REC;
@@ -375,9 +377,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
             return (int)(j == 0 ? idv.x : j == 1 ? idv.y : j == 2 ? idv.z : idv.w);
         };
         // ---- keys: token tt, dims 8c .. 8c+7 -> one 16-byte row of a core matrix
+        // (consecutive threads take consecutive tokens: eight of them fill one
+        // 128-byte core matrix, so the stores do not collide on banks)
 #pragma unroll 2
         for (int u = tid; u < kStep * (D / 8); u += kThreads) {
-            const int tt = u / (D / 8), c = u % (D / 8);
+            const int tt = u % kStep, c = u / kStep;
             const int j = tt >> 4, o = tt & 15;
             uint4 w4 = make_uint4(0, 0, 0, 0);
             if (id_of(j) >= 0 && kStep * s + tt < maxlim) {
@@ -393,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
         // (D/8) r + D/8 - 1 (dims 16m + 2r + e), high and low parts
 #pragma unroll 1
         for (int u = tid; u < kStep * 8; u += kThreads) {
-            const int tt = u >> 3, r = u & 7;
+            const int tt = u % kStep, r = u / kStep;  // consecutive tokens: bank-free stores
             const int j = tt >> 4, o = tt & 15;
             const bool valid = id_of(j) >= 0 && kStep * s + tt < maxlim;
             float v[D / 8];
@@ -477,6 +481,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
             for (int j = 0; j < 16; j++) x[c0 + j] = t16[j];
         }
         float mx = -INFINITY;
+        const bool whole = kStep * (s + 1) <= lim;  // the row sees every token of the step
 #pragma unroll
         for (int c0 = 0; c0 < kStep; c0 += 4) {
             const uint4 nw = ld_s128(sNorm + 4 * c0);
@@ -485,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
 #pragma unroll
             for (int j = 0; j < 4; j++) {
                 const int t = kStep * s + c0 + j;
-                x[c0 + j] = t < lim ? x[c0 + j] * nn[j] : -INFINITY;
+                x[c0 + j] = whole || t < lim ? x[c0 + j] * nn[j] : -INFINITY;
                 mx = fmaxf(mx, x[c0 + j]);
             }
         }

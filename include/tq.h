@@ -114,7 +114,11 @@ TQ_API int tq_lloyd_max_table(int head_dim, uint16_t out16[16]);
 TQ_API int tq_fit_k_table(const uint16_t* keys_bf16, int n, int head_dim,
                           const uint16_t init16[16], int max_iter, uint16_t out16[16]);
 
-/* Quantise T new tokens and write them into the cache (the TQ4/4 write path).
+/* Quantise T new tokens and write them into the cache (the TQ4/4 write path):
+ * keys by Walsh-Hadamard rotation and the 16-entry look-up table, values by
+ * uniform 4-bit codes ("TurboQuant 在 AMD GPU 上把長上下文延遲壓下來", section 2,
+ * TQ4/4, and section 4, Walsh-Hadamard rotation); the call follows the write
+ * step tq_quantize_append(K, V, block_table, slot_mapping) of the TQ4/4 cache.
  *   K, V        (device) bf16 [T][H_kv][d], 16-byte aligned
  *   block_table (device, may be NULL) int32 [num_seqs][max_blocks]
  *   slot_mapping(device) int32 [T]:
@@ -137,7 +141,10 @@ TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len);
  * outputs and softmax statistics per (sequence, query head, split)). */
 TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_splits);
 
-/* Decode attention over the compressed cache, one query per sequence:
+/* Decode attention over the compressed cache, one query per sequence -- the
+ * fused attention over 4-bit keys and values that the TurboQuant kernels run
+ * ("TurboQuant 在 AMD GPU 上把長上下文延遲壓下來", summary table and section 2:
+ * rotation + LUT keys, uniform values, dequantised inside the attention):
  *   out[b][h] = sum_t softmax_t(scale * <q[b][h], k_hat_t>) * v_hat_t,
  * t < seq_lens[b], with the keys/values the cache holds for kv head
  * h / (H_q / H_kv).  The query is rotated by the same Hadamard transform
@@ -216,7 +223,8 @@ TQ_API int tq_prefill_attention(const void* q, const tq_cache_t* cache, const ui
                                 const int32_t* q_start, int B, int H_q, int T, int max_q_len,
                                 float scale, float* out, int32_t* status, void* stream);
 
-/* Dequantise every valid token (checks only): K_hat and V_hat (device) fp32
+/* Dequantise every valid token (checks only; the inverse of the section 2
+ * encodings of "TurboQuant 在 AMD GPU 上把長上下文延遲壓下來"): K_hat and V_hat (device) fp32
  * [B][max_len][H_kv][d] in the original (unrotated) domain,
  * k_hat = fp16 norm * H * C[idx],  v_hat = code * scale + zero;
  * rows at or past seq_lens[b] are written as 0. */
