@@ -10,15 +10,17 @@
 //   z = fp16 rounded down from min, s = fp16 rounded up from (max - z)/15,
 //   q = round-half-even((v - z)/s) in [0, 15].
 //
-// Work split: one vector (token, kv head) is spread over D/16 lanes holding 16
-// consecutive elements each, so a warp pass covers 8 (D=64) or 4 (D=128)
-// vectors, 1 KB of keys and 1 KB of values.  The grid is persistent (one wave
-// of resident CTAs); warp w takes passes w, w + W, w + 2W, ... (W warps in
-// all).  Every warp keeps its next kPrefetch passes requested into L2 with
-// bulk prefetches, so HBM sees the whole input stream early; it loads its
-// next pass into registers after the current pass's key work and before its
-// stores, and looks up the pass's physical block at the top of the pass.  The rotation is an in-register butterfly over the 4 index
-// bits inside a lane plus xor-shuffles over the lane bits.
+// Work split: one vector (token, kv head) is spread over D/32 lanes holding 32
+// consecutive elements each (one value group per lane), so a warp pass covers
+// 16 (D=64) or 8 (D=128) vectors, 2 KB of keys and 2 KB of values.  The grid
+// is persistent (one CTA per SM); each CTA takes an even share of the passes
+// and deals them to its warps, and each warp streams its passes' keys and
+// values through a private ring of shared-memory stages filled by bulk copies
+// (one mbarrier per stage).  The rotation is an in-register butterfly over the
+// 5 element bits inside a lane plus xor-shuffles over the lane bits.  Decisions
+// inside their error margin are flagged per element pair in the main loop and
+// taken again afterwards by short loops over the flagged pairs only (the code
+// of the main loop stays small enough for the instruction cache).
 //
 // Nearest centroid: x = 63 y + 64 is rounded to 1/8 by one fma against a
 // 2^20 magic constant, whose low mantissa bits then address a 128-entry bin
@@ -94,12 +96,12 @@ __device__ __forceinline__ uint32_t pack4(uint32_t b0, uint32_t b1, uint32_t b2,
 // 1/15 rounded down to fp32
 __device__ __forceinline__ float inv15_dn() { return __uint_as_float(0x3d888888u); }
 
-constexpr int kAppWarps = 24;   // warps per CTA (one persistent CTA per SM, at most 85 registers)
-constexpr int kAppStages = 4;   // passes in flight per warp
+constexpr int kAppWarps = 16;   // warps per CTA (one persistent CTA per SM)
+constexpr int kAppStages = 3;   // passes in flight per warp
 
 template <int D>
 struct Geo {
-    static constexpr int LPV = D / 16;    // lanes per vector
+    static constexpr int LPV = D / 32;    // lanes per vector (one value group each)
     static constexpr int VPW = 32 / LPV;  // vectors per warp pass
     static constexpr uint32_t kPass = VPW * D * 2;  // bytes of one pass's keys (or values)
     static constexpr uint32_t kStage = 2 * kPass;   // a ring stage: keys, then values
@@ -115,6 +117,22 @@ __device__ __forceinline__ uint4 lds_u4(uint32_t a) {
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(a));
     return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+// the 32 bf16 elements (16 words) at a stage address
+__device__ __forceinline__ void lds_32(uint32_t a, uint32_t (&w)[16]) {
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+        const uint4 t = lds_u4(a + 16 * c);
+        w[4 * c] = t.x;
+        w[4 * c + 1] = t.y;
+        w[4 * c + 2] = t.z;
+        w[4 * c + 3] = t.w;
+    }
 }
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t phase) {
     uint32_t ok;
@@ -170,6 +188,12 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
     return __ffma2_rn(b, make_float2(-1.f, -1.f), a);  // a - b, one rounding
 }
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t w) {
+    return *reinterpret_cast<const __nv_bfloat162*>(&w);
+}
+__device__ __forceinline__ uint32_t bf2_bits(__nv_bfloat162 v) {
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
 
 // 1.5 * 2^23: x + kRound rounds x (0 <= x < 2^22) to the nearest integer,
 // ties to even, and leaves that integer in the low mantissa bits.
@@ -202,8 +226,8 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
     const AppPlan<D> P(ntab);
 
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int sub = lane % LPV;
-    const int grp = lane / LPV;
+    const int sub = lane % LPV;  // the lane's 32 elements: 32 sub .. 32 sub + 31
+    const int grp = lane / LPV;  // the lane's vector within the pass
     const uint32_t total = (uint32_t)a.T * (uint32_t)a.Hkv;
     const uint32_t npass = (total + VPW - 1) / VPW;
     const float inv_sqrt_d = D == 128 ? 0.08838834764831845f : 0.125f;  // fp32 of 1/sqrt(D)
@@ -264,29 +288,20 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
             aborted = true;
             break;
         }
-        // this lane's 16 keys and values (a lane past the pass's last vector reads
+        // the lane's elements in the stage (a lane past the pass's last vector reads
         // stale stage bytes; it stores nothing)
-        const uint32_t eoff = (uint32_t)(grp * D + sub * 16) * 2;
-        uint4 ck0 = lds_u4(stage + eoff), ck1 = lds_u4(stage + eoff + 16);
-        const uint4 cv0 = lds_u4(stage + PB + eoff), cv1 = lds_u4(stage + PB + eoff + 16);
+        const uint32_t eoff = (uint32_t)(grp * D + sub * 32) * 2;
 
-        // ---- values: group of 32 = this lane and lane ^ 1
-        const uint32_t vwd[8] = {cv0.x, cv0.y, cv0.z, cv0.w, cv1.x, cv1.y, cv1.z, cv1.w};
-        __nv_bfloat162 mn2 = *reinterpret_cast<const __nv_bfloat162*>(&vwd[0]);
-        __nv_bfloat162 mx2 = mn2;
+        // ---- values: the lane's 32 elements are one group
+        uint32_t vwd[16];
+        lds_32(stage + PB + eoff, vwd);
+        __nv_bfloat162 mn2 = as_bf2(vwd[0]), mx2 = mn2;
 #pragma unroll
-        for (int j = 1; j < 8; j++) {
-            const __nv_bfloat162 w = *reinterpret_cast<const __nv_bfloat162*>(&vwd[j]);
-            mn2 = __hmin2(mn2, w);
-            mx2 = __hmax2_nan(mx2, w);  // a NaN reaches the scale and flags the group
+        for (int j = 1; j < 16; j++) {
+            mn2 = __hmin2(mn2, as_bf2(vwd[j]));
+            mx2 = __hmax2_nan(mx2, as_bf2(vwd[j]));  // a NaN reaches the scale and flags the group
         }
-        {
-            const uint32_t pm = __shfl_xor_sync(kFull, *reinterpret_cast<const uint32_t*>(&mn2), 1);
-            const uint32_t px = __shfl_xor_sync(kFull, *reinterpret_cast<const uint32_t*>(&mx2), 1);
-            mn2 = __hmin2(mn2, *reinterpret_cast<const __nv_bfloat162*>(&pm));
-            mx2 = __hmax2_nan(mx2, *reinterpret_cast<const __nv_bfloat162*>(&px));
-        }
-        const uint32_t mnw = *reinterpret_cast<const uint32_t*>(&mn2);
+        const uint32_t mnw = bf2_bits(mn2);
         const float mn = fminf(bf16_lo(mnw), bf16_hi(mnw));
         // the maximum of the two halves keeps a NaN (fmaxf would drop it)
         const float mx = __bfloat162float(__hmax_nan(__low2bfloat16(mx2), __high2bfloat16(mx2)));
@@ -310,8 +325,11 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
         }
         const float sf = half_bits_to_float(s16);
         const bool vbad = !isfinite(sf) || !isfinite(zf);
-        const uint32_t sz = (uint32_t)s16 | ((uint32_t)__half_as_ushort(zh) << 16);  // scale, zero
-        uint32_t vw0 = 0, vw1 = 0;  // code bytes of elements 0-7, 8-15
+        // sv[r]: the record's 16-bit chunk r of this lane, the code bytes of its
+        // element pairs r (low byte) and 8 + r (high byte)
+        uint32_t sv[8];
+#pragma unroll
+        for (int r = 0; r < 8; r++) sv[r] = 0;
         if (sf > 0.f) {
             // 1/s to ~1 ulp (approximation and one Newton step): it only picks the
             // candidate code, whose exact residual is checked below
@@ -319,67 +337,82 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
             const float is = fmaf(is0, fmaf(-sf, is0, 1.0f), is0);
             const float2 z2 = make_float2(zf, zf), is2 = make_float2(is, is), s2 = make_float2(sf, sf);
             const float2 rnd = make_float2(kRound, kRound);
-            float emax = 0.f;
-            uint32_t by[8];
+            // |v - z - t s| >= s / 2 (less the fp32 error of v - z, <= 16 ulp of s)
+            // marks an exact .5 tie, or a quotient whose fp32 rounding may be on the
+            // wrong side of a .5 point: such pairs are flagged in vpm
+            const float thr = (0.5f - kValueMargin) * sf;
+            uint32_t vpm = 0;
+            uint32_t by[16];
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
+            for (int j = 0; j < 16; j++) {
                 const float2 vz = sub2(make_float2(bf16_lo(vwd[j]), bf16_hi(vwd[j])), z2);
                 const float2 tr = __ffma2_rn(vz, is2, rnd);  // kRound + round-half-even(r)
                 const float2 nti = sub2(rnd, tr);            // minus that integer t, exact
                 const float2 e = __ffma2_rn(nti, s2, vz);    // v - z - t s
-                emax = fmaxf(emax, fmaxf(fabsf(e.x), fabsf(e.y)));
+                if (fmaxf(fabsf(e.x), fabsf(e.y)) >= thr) vpm |= 1u << j;
                 // the codes are the low bytes of tr
                 by[j] = __float_as_uint(tr.x) + (__float_as_uint(tr.y) << 4);
             }
-            vw0 = pack4(by[0], by[1], by[2], by[3]);
-            vw1 = pack4(by[4], by[5], by[6], by[7]);
-            // |v - z - t s| >= s / 2 (less the fp32 error of v - z, <= 16 ulp of s)
-            // marks an exact .5 tie, or a quotient whose fp32 rounding may be on the
-            // wrong side of a .5 point: that element is decided exactly by comparing
-            // v - z with (k + 1/2) s in fp64, k the integer below, ties to even
-            const float thr = (0.5f - kValueMargin) * sf;
-            if (emax >= thr) {
 #pragma unroll
-                for (int e = 0; e < 16; e++) {
-                    const float vf = e & 1 ? bf16_hi(vwd[e >> 1]) : bf16_lo(vwd[e >> 1]);
+            for (int r = 0; r < 8; r++) sv[r] = __byte_perm(by[r], by[8 + r], 0x0040);
+            // a flagged pair's elements are decided exactly: v - z against (k + 1/2) s
+            // in fp64, k the integer below, ties to even (its word is read again from
+            // the stage)
+#pragma unroll 1
+            while (vpm) {
+                const int j = __ffs(vpm) - 1;
+                vpm &= vpm - 1u;
+                const uint32_t wv = lds_u32(stage + PB + eoff + 4 * j);
+                uint32_t pb = 0;
+#pragma unroll
+                for (int hh = 0; hh < 2; hh++) {
+                    const float vf = hh ? bf16_hi(wv) : bf16_lo(wv);
                     const float vz = vf - zf;
                     const float tr = fmaf(vz, is, kRound);
+                    uint32_t c = __float_as_uint(tr) & 15u;
                     if (fabsf(fmaf(kRound - tr, sf, vz)) >= thr) {
-                        const float k = floorf(vz * is);
+                        const float kf = floorf(vz * is);
                         const double v = (double)vf - (double)zf;
-                        const double bnd = ((double)k + 0.5) * (double)sf;
-                        const int ki = (int)k;
+                        const double bnd = ((double)kf + 0.5) * (double)sf;
+                        const int ki = (int)kf;
                         const int q = v > bnd ? ki + 1 : (v < bnd ? ki : ki + (ki & 1));
-                        const uint32_t c = (uint32_t)min(max(q, 0), 15);
-                        const int sh = 4 * (e & 7);
-                        if (e < 8) vw0 = (vw0 & ~(0xfu << sh)) | (c << sh);
-                        else vw1 = (vw1 & ~(0xfu << sh)) | (c << sh);
+                        c = (uint32_t)min(max(q, 0), 15);
                     }
+                    pb |= c << (4 * hh);
                 }
+                // pair j is byte j / 8 of chunk j % 8
+                const int sh = 8 * (j >> 3);
+                const uint32_t jr = (uint32_t)j & 7u, cm = ~(0xffu << sh), cv = pb << sh;
+#pragma unroll
+                for (int r = 0; r < 8; r++) sv[r] = jr == (uint32_t)r ? (sv[r] & cm) | cv : sv[r];
             }
         }
 
-        // ---- key: norm and in-lane butterfly over element bits 0-3.  Q[j]
-        // holds elements (2j, 2j+1) of the lane's 16.
-        const uint32_t kwd[8] = {ck0.x, ck0.y, ck0.z, ck0.w, ck1.x, ck1.y, ck1.z, ck1.w};
-        float2 Q[8];
-        float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
-        uint32_t kor = 0;
+        // ---- key: norm and in-lane butterfly over element bits 0-4.  Q[j]
+        // holds elements (2j, 2j+1) of the lane's 32.
+        float2 Q[16];
+        float ss;
+        {
+            uint32_t kwd[16];
+            lds_32(stage + eoff, kwd);
+            float2 s4[4];
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            const float2 P = make_float2(bf16_lo(kwd[j]), bf16_hi(kwd[j]));
-            if (j & 1) sb = __ffma2_rn(P, P, sb);
-            else sa = __ffma2_rn(P, P, sa);
-            Q[j] = make_float2(P.x + P.y, P.x - P.y);
-            kor |= kwd[j];
+            for (int i = 0; i < 4; i++) s4[i] = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int j = 0; j < 16; j++) {
+                const float2 P = make_float2(bf16_lo(kwd[j]), bf16_hi(kwd[j]));
+                s4[j & 3] = __ffma2_rn(P, P, s4[j & 3]);
+                Q[j] = make_float2(P.x + P.y, P.x - P.y);
+            }
+            const float2 s2 = add2(add2(s4[0], s4[1]), add2(s4[2], s4[3]));
+            ss = s2.x + s2.y;
         }
-        float ss = (sa.x + sa.y) + (sb.x + sb.y);
 #pragma unroll
         for (int m = 1; m < LPV; m <<= 1) ss += __shfl_xor_sync(kFull, ss, m);
 #pragma unroll
-        for (int b = 1; b < 8; b <<= 1) {
+        for (int b = 1; b < 16; b <<= 1) {
 #pragma unroll
-            for (int j = 0; j < 8; j++)
+            for (int j = 0; j < 16; j++)
                 if (!(j & b)) {
                     const float2 x = Q[j], y = Q[j | b];
                     Q[j] = add2(x, y);
@@ -392,7 +425,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
             const float sg = (sub & m) ? -1.f : 1.f;
             const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
+            for (int j = 0; j < 16; j++) {
                 const float2 pr = make_float2(__shfl_xor_sync(kFull, Q[j].x, m),
                                               __shfl_xor_sync(kFull, Q[j].y, m));
                 Q[j] = __ffma2_rn(sg2, Q[j], pr);
@@ -411,99 +444,87 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
         // squares that leave the normal fp32 range (or a non-finite key) lose the
         // fp32 error bound: every decision is re-taken.  An all-zero key stays here;
         // whether any element is nonzero is asked of the whole vector, since one
-        // lane's 16 elements may all be zero while the others' are not.
+        // lane's 32 elements may all be zero while the others' are not.
         const bool small = !(ss >= 1e-30f && ss <= 1e30f);
+        bool wild = false;
         if (__any_sync(kFull, small)) {
+            uint32_t kor = 0;
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                const uint4 t4 = lds_u4(stage + eoff + 16 * c);
+                kor |= t4.x | t4.y | t4.z | t4.w;
+            }
 #pragma unroll
             for (int m = 1; m < LPV; m <<= 1) kor |= __shfl_xor_sync(kFull, kor, m);
+            wild = small && (kor & 0x7fff7fffu) != 0u;
         }
-        const bool wild = small && (kor & 0x7fff7fffu) != 0u;
-        bool nkey = wild;  // some centroid decision is close (all of them when wild)
         const float inv = rs * inv_sqrt_d;              // 1 / (n sqrt(D))
         const float A = rs * (inv_sqrt_d * kBinScale);  // kBinScale / (n sqrt(D))
 
-        // ---- key: nearest centroid
+        // ---- key: nearest centroid.  kc[i] holds the codes of elements 8i .. 8i+7;
+        // kpm flags the pairs with a decision inside the margin.
         const int hs = a.k_tables ? h : 0;  // whose table
         const HeadBins& B = hb[hs];
         const unsigned char* tab = smem + (size_t)hs * (kBins * sizeof(BinEntry));
-        uint32_t kw0 = 0, kw1 = 0;  // codes of elements 0-7, 8-15
+        uint32_t kc[4] = {0u, 0u, 0u, 0u};
+        uint32_t kpm = 0;
         if (!B.dense) {
             const float2 A2 = make_float2(A, A), M2 = make_float2(kBinMagic, kBinMagic);
-            float dmin = INFINITY;
-            uint32_t by[8];
+            uint32_t by[16];
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
+            for (int j = 0; j < 16; j++) {
                 const float2 x = __ffma2_rn(Q[j], A2, M2);
                 const BinEntry e0 = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x.x) & 0x3f8u));
                 const BinEntry e1 = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x.y) & 0x3f8u));
                 // y - mid with one rounding: its sign is the decision
                 const float d0 = fmaf(Q[j].x, inv, -e0.mid);
                 const float d1 = fmaf(Q[j].y, inv, -e1.mid);
-                dmin = fminf(dmin, fminf(fabsf(d0), fabsf(d1)));
+                if (fminf(fabsf(d0), fabsf(d1)) < kKeyMargin) kpm |= 1u << j;
                 // k_hi - 1 where y <= mid (sign bit set; y == mid is near anyway)
                 const uint32_t c0 = (uint32_t)(e0.k_hi + (__float_as_int(d0) >> 31));
                 const uint32_t c1 = (uint32_t)(e1.k_hi + (__float_as_int(d1) >> 31));
                 by[j] = c0 | (c1 << 4);
             }
-            kw0 = pack4(by[0], by[1], by[2], by[3]);
-            kw1 = pack4(by[4], by[5], by[6], by[7]);
-            nkey |= dmin < kKeyMargin;
+#pragma unroll
+            for (int i = 0; i < 4; i++) kc[i] = pack4(by[4 * i], by[4 * i + 1], by[4 * i + 2], by[4 * i + 3]);
         } else {  // midpoints closer than a bin: count them all
 #pragma unroll
-            for (int e = 0; e < 16; e++) {
-                const float y = (e & 1 ? Q[e >> 1].y : Q[e >> 1].x) * inv;
-                uint32_t idx = 0;
+            for (int j = 0; j < 16; j++) {
+                uint32_t pc = 0;
+                bool nr = false;
 #pragma unroll 1
                 for (int k = 0; k < 15; k++) {
-                    const float dm = y - 0.5f * (B.c[k] + B.c[k + 1]);
-                    idx += dm > 0.f ? 1u : 0u;
-                    nkey |= fabsf(dm) < kKeyMargin;
+                    const float m = 0.5f * (B.c[k] + B.c[k + 1]);
+                    const float dx = Q[j].x * inv - m, dy = Q[j].y * inv - m;
+                    pc += (dx > 0.f ? 1u : 0u) + (dy > 0.f ? 16u : 0u);
+                    nr |= fminf(fabsf(dx), fabsf(dy)) < kKeyMargin;
                 }
-                if (e < 8) kw0 |= idx << (4 * e);
-                else kw1 |= idx << (4 * (e - 8));
+                if (nr) kpm |= 1u << j;
+                kc[j >> 2] |= pc << (8 * (j & 3));
             }
         }
-        nkey = nkey && cur.in && cur.slot >= 0;
-        const bool near = nkey || (nnorm && cur.in && cur.slot >= 0);
+        const bool live = cur.in && cur.slot >= 0;
+        const bool near = live && (wild || kpm != 0 || nnorm);
 
         // ---- key: exact decisions when any decision of the warp is close
         if (__any_sync(kFull, near)) {
-            // the elements whose fp32 decision lies within the margin (all of them
-            // when the fp32 scale is unusable)
-            uint32_t nm = 0;
-            if (near) {
-                if (wild) {
-                    nm = 0xffffu;
-                } else {
+            // the pairs to decide again (all of them when the fp32 scale is unusable)
+            uint32_t nm = near ? (wild ? 0xffffu : kpm) : 0u;
+            // the exact norm from the fp64 sum of squares of this lane's keys (still
+            // in the stage)
+            double ssd = 0.0;
+            {
+                uint32_t w[16];
+                lds_32(stage + eoff, w);
+                double s0 = 0.0, s1 = 0.0;
 #pragma unroll
-                    for (int e = 0; e < 16; e++) {
-                        const float q = e & 1 ? Q[e >> 1].y : Q[e >> 1].x;
-                        bool nr = false;
-                        if (!B.dense) {
-                            const float x = fmaf(q, A, kBinMagic);
-                            const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
-                            nr = fabsf(fmaf(q, inv, -be.mid)) < kKeyMargin;
-                        } else {
-                            const float y = q * inv;
-#pragma unroll 1
-                            for (int k = 0; k < 15; k++) nr |= fabsf(y - 0.5f * (B.c[k] + B.c[k + 1])) < kKeyMargin;
-                        }
-                        nm |= (nr ? 1u : 0u) << e;
-                    }
+                for (int j = 0; j < 16; j++) {
+                    const double x = (double)bf16_lo(w[j]), y = (double)bf16_hi(w[j]);
+                    s0 = fma(x, x, s0);
+                    s1 = fma(y, y, s1);
                 }
+                ssd = s0 + s1;
             }
-            // this lane's keys again (still in the stage) and the exact norm from
-            // their fp64 sum of squares
-            const uint4 ra = lds_u4(stage + eoff), rb = lds_u4(stage + eoff + 16);
-            const uint32_t w[8] = {ra.x, ra.y, ra.z, ra.w, rb.x, rb.y, rb.z, rb.w};
-            double s0 = 0.0, s1 = 0.0;
-#pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const double x = (double)bf16_lo(w[j]), y = (double)bf16_hi(w[j]);
-                s0 = fma(x, x, s0);
-                s1 = fma(y, y, s1);
-            }
-            double ssd = s0 + s1;
 #pragma unroll
             for (int m = 1; m < LPV; m <<= 1) ssd += __shfl_xor_sync(kFull, ssd, m);
             const double nd = sqrt(ssd);
@@ -516,44 +537,66 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
                 if (!B.dense) c0 = (uint32_t)be.k_hi - (0.f > be.mid ? 0u : 1u);
                 else
                     for (int k = 0; k < 15; k++) c0 += 0.f > 0.5f * (B.c[k] + B.c[k + 1]) ? 1u : 0u;
-                kw0 = kw1 = c0 * 0x11111111u;
+#pragma unroll
+                for (int i = 0; i < 4; i++) kc[i] = c0 * 0x11111111u;
                 nm = 0;
             }
             // 1 / denom, only to pick a bin: the fast path's fp32 scale, or from the
             // exact norm when that scale is unusable
             float rden = inv;
             if (wild) rden = ssd > 0.0 ? (float)(1.0 / denom) : 0.f;
-            // one close element per vector per round: its row of the Hadamard sum,
-            // exact in fp64, decides it against midpoint * denom
+            // one flagged pair per vector per round.  Its rows 2p and 2p + 1 of the
+            // Hadamard sum share their signs on each element pair (row 2p + 1 flips
+            // the odd elements), so the sums over the even and the odd elements, exact
+            // in fp64, give both: E + O and E - O.  Each is decided against
+            // midpoint * denom.
             const uint32_t gmask = ((1u << LPV) - 1u) << (grp * LPV);
+#pragma unroll 1
             while (__any_sync(kFull, nm != 0)) {
                 const uint32_t pend = __ballot_sync(kFull, nm != 0) & gmask;
                 const int owner = pend ? __ffs(pend) - 1 : lane;
                 const int mine = nm ? __ffs(nm) - 1 : 0;
-                const uint32_t r = (uint32_t)__shfl_sync(kFull, 16 * sub + mine, owner);
-                double part = 0.0;
-#pragma unroll
-                for (int e = 0; e < 16; e++) {
-                    const double x = (double)(e & 1 ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]));
-                    part += (__popc((r & 15u) & (uint32_t)e) & 1) ? -x : x;
+                const uint32_t pr = (uint32_t)__shfl_sync(kFull, 16 * sub + mine, owner);  // pair of the vector
+                double pe = 0.0, po = 0.0;
+#pragma unroll 4
+                for (int j = 0; j < 16; j++) {
+                    const uint32_t wv = lds_u32(stage + eoff + 4 * j);
+                    const double x0 = (double)bf16_lo(wv), x1 = (double)bf16_hi(wv);
+                    const bool neg = __popc((pr & 15u) & (uint32_t)j) & 1;
+                    pe += neg ? -x0 : x0;
+                    po += neg ? -x1 : x1;
                 }
-                if (__popc((r >> 4) & (uint32_t)sub) & 1) part = -part;
+                if (__popc((pr >> 4) & (uint32_t)sub) & 1) {
+                    pe = -pe;
+                    po = -po;
+                }
 #pragma unroll
-                for (int m = 1; m < LPV; m <<= 1) part += __shfl_xor_sync(kFull, part, m);
+                for (int m = 1; m < LPV; m <<= 1) {
+                    pe += __shfl_xor_sync(kFull, pe, m);
+                    po += __shfl_xor_sync(kFull, po, m);
+                }
                 if (pend && lane == owner) {
-                    uint32_t idx = 0;
-                    if (!B.dense) {
-                        const float x = fmaf((float)part * rden, kBinScale, kBinMagic);
-                        const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
-                        idx = (uint32_t)be.k_hi - (part > (double)be.mid * denom ? 0u : 1u);
-                    } else {
+                    uint32_t pc = 0;
+#pragma unroll
+                    for (int hh = 0; hh < 2; hh++) {
+                        const double part = hh ? pe - po : pe + po;
+                        uint32_t idx = 0;
+                        if (!B.dense) {
+                            const float x = fmaf((float)part * rden, kBinScale, kBinMagic);
+                            const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
+                            idx = (uint32_t)be.k_hi - (part > (double)be.mid * denom ? 0u : 1u);
+                        } else {
 #pragma unroll 1
-                        for (int k = 0; k < 15; k++)
-                            idx += part > 0.5 * ((double)B.c[k] + (double)B.c[k + 1]) * denom ? 1u : 0u;
+                            for (int k = 0; k < 15; k++)
+                                idx += part > 0.5 * ((double)B.c[k] + (double)B.c[k + 1]) * denom ? 1u : 0u;
+                        }
+                        pc |= idx << (4 * hh);
                     }
-                    const int sh = 4 * (mine & 7);
-                    if (mine < 8) kw0 = (kw0 & ~(0xfu << sh)) | (idx << sh);
-                    else kw1 = (kw1 & ~(0xfu << sh)) | (idx << sh);
+                    // pair mine is byte mine % 4 of word mine / 4
+                    const int sh = 8 * (mine & 3);
+                    const uint32_t wi = (uint32_t)mine >> 2, cm = ~(0xffu << sh), cv = pc << sh;
+#pragma unroll
+                    for (int i = 0; i < 4; i++) kc[i] = wi == (uint32_t)i ? (kc[i] & cm) | cv : kc[i];
                     nm &= nm - 1u;
                 }
             }
@@ -582,23 +625,20 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
         }
         if (blk >= 0) {
             unsigned char* rec = a.cache + ((size_t)blk * a.Hkv + h) * (size_t)R::kBytes;
-            *reinterpret_cast<uint2*>(rec + R::kKCodes + off * R::kCodeRow + sub * 8) =
-                make_uint2(kw0, kw1);
-            // code bytes j = 8 sub + r (r = 0..7) of this token: m = sub, chunk r
-            unsigned char* vdst = rec + R::kVCodes + R::vcode_pos(off, 8 * sub);
+            *reinterpret_cast<uint4*>(rec + R::kKCodes + off * R::kCodeRow + sub * 16) =
+                make_uint4(kc[0], kc[1], kc[2], kc[3]);
+            // code bytes 16 sub + r (m = 2 sub) and 16 sub + 8 + r (m = 2 sub + 1) of
+            // this token sit side by side in chunk r
+            unsigned char* vdst = rec + R::kVCodes + R::vcode_pos(off, 16 * sub);
 #pragma unroll
-            for (int r = 0; r < 4; r++) {
-                vdst[r * R::kPairChunk] = (unsigned char)(vw0 >> (8 * r));
-                vdst[(r + 4) * R::kPairChunk] = (unsigned char)(vw1 >> (8 * r));
-            }
+            for (int r = 0; r < 8; r++)
+                *reinterpret_cast<uint16_t*>(vdst + r * R::kPairChunk) = (uint16_t)sv[r];
             if (sub == 0) *reinterpret_cast<uint16_t*>(rec + R::kKNorm + off * 2) = n16;
-            if ((sub & 1) == 0) {
-                const int gp = R::group_pos(off, sub / 2);
-                *reinterpret_cast<uint16_t*>(rec + R::kVScale + gp) = (uint16_t)sz;
-                *reinterpret_cast<uint16_t*>(rec + R::kVZero + gp) = (uint16_t)(sz >> 16);
-                const bool bad = vbad || (sub == 0 && !isfinite(half_bits_to_float(n16)));
-                if (bad) flag_status(a.status, TQ_STATUS_RANGE);
-            }
+            const int gp = R::group_pos(off, sub);
+            *reinterpret_cast<uint16_t*>(rec + R::kVScale + gp) = s16;
+            *reinterpret_cast<uint16_t*>(rec + R::kVZero + gp) = __half_as_ushort(zh);
+            const bool bad = vbad || (sub == 0 && !isfinite(half_bits_to_float(n16)));
+            if (bad) flag_status(a.status, TQ_STATUS_RANGE);
         }
 
         cur = nxt;
