@@ -619,9 +619,14 @@ def run_tq(args, rank, world, local):
     dec_avg = graph_ms(lambda s_: tq.decode_attention(q, cache, bt, lens, max_len, w.scale, out=out,
                                                       workspace=ws, num_splits=S, status=status,
                                                       stream=s_))
-    # the append's inputs (4.4 MB) would stay in L2 over back-to-back calls, so its
-    # figure stays the per-call one, taken right after a decode has streamed 306 MB
-    app_avg = app_call
+    # the append alone on the device, each call right after a 512 MB read that evicts
+    # L2 (its inputs, 4.4 MB, would otherwise stay there over back-to-back calls):
+    # graph-replayed (read + append) less graph-replayed reads
+    flush = torch.ones(512 << 20, dtype=torch.uint8, device=dev)
+    app_flush = graph_ms(lambda s_: (flush.sum(), tq.quantize_append(aK, aV, aS, cache, block_table=bt,
+                                                                     status=status, stream=s_)))
+    app_avg = app_flush - graph_ms(lambda s_: flush.sum())
+    del flush
 
     # whole steps: the step (append, then decode) captured once as a CUDA graph, the way
     # a serving engine launches a decode step, and replayed; CUDA events around K replays
@@ -778,7 +783,7 @@ def run_tq(args, rank, world, local):
             "config": cfg(w, f"inputs larger than L2: {kv / 1e6:.0f} MB cache read per rank vs 126 MB L2, no flush"),
             "decode_gbs": kv / (dec_avg / 1e3) / 1e9,
             "decode_hbm_frac": kv / (dec_avg / 1e3) / 1e9 / peak,
-            "decode_ms": dec_avg, "append_ms": app_avg, "decode_call_ms": dec_call,
+            "decode_ms": dec_avg, "append_ms": app_avg, "decode_call_ms": dec_call, "append_call_ms": app_call,
             "append_tokens_per_s": T / (app_avg / 1e3),
             "append_hbm_frac": append_bytes(w, T) / (app_avg / 1e3) / 1e9 / peak,
             "num_splits": S,
