@@ -427,8 +427,15 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
     T = K.shape[0]
     ms = timed(lambda: tq.quantize_append(K, V, slots, cache, block_table=bt, status=status), True)
     ab = append_bytes(w, T)
+    # what a plain device copy moving the same bytes (half read, half written) reaches
+    # at this size, L2 evicted the same way: the ceiling of a streaming kernel this short
+    cbuf = torch.randint(0, 256, (ab // 2 // 16 * 16,), dtype=torch.uint8, device=dev)
+    cdst = torch.zeros_like(cbuf)
+    cms = timed(lambda: cdst.copy_(cbuf), True)
+    del cbuf, cdst
     res["prefill_chunk_append"] = {"ms": ms, "tokens": T, "tokens_per_s": T / ms * 1e3,
-                                   "gbs": ab / ms / 1e6, "hbm_frac": ab / ms / 1e6 / peak}
+                                   "gbs": ab / ms / 1e6, "hbm_frac": ab / ms / 1e6 / peak,
+                                   "same_bytes_copy_ms": cms, "same_bytes_copy_hbm_frac": ab / cms / 1e6 / peak}
     kv = decode_kv_bytes(w)
     ms = decode(w, cache, bt, 0, cold=True)
     res["prefill_small_head_decode"] = {"ms": ms, "gbs": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / peak}
@@ -457,7 +464,68 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
     del cache
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0, f"device status {int(status.item())}"
+    res["quality"] = quality_study(dev)
     return res
+
+
+def sphere_coordinate_mse(table16: np.ndarray, d: int) -> float:
+    """E[(y - C[nearest(y)])^2] for a coordinate y of a uniform unit vector in R^d
+    (density proportional to (1 - y^2)^((d-3)/2)): the key error of Gaussian keys."""
+    import scipy.integrate
+
+    c = table16.view(np.float16).astype(np.float64)
+    edges = np.concatenate([[-1.0], (c[:-1] + c[1:]) / 2, [1.0]])
+    dens = lambda y: (1.0 - y * y) ** ((d - 3) / 2.0)
+    Z = scipy.integrate.quad(dens, -1, 1, limit=400)[0]
+    return sum(scipy.integrate.quad(lambda y, ci=ci: (y - ci) ** 2 * dens(y), edges[i], edges[i + 1],
+                                    limit=400)[0] for i, ci in enumerate(c)) / Z
+
+
+def quality_study(dev) -> dict:
+    """Table-quality study on the library's own kernels: per-element K MSE of the unit
+    key vector, ((k - k_hat) / ||k||)^2 averaged, for the Lloyd-Max table, tables
+    re-fitted (tq_fit_k_table) on 20 calibration vectors per head, and the unrotated
+    cache; V MSE (v - v_hat)^2.  Evaluated on sequences other than the calibration one."""
+    import bit_rotated_kv_tq_b200 as tq
+
+    out = {}
+    cases = [("qwen3_8b_layer", dict(B=2, ctx=8192)), ("tiny", dict(B=2)),
+             ("prefill_small_head", dict(B=2, ctx=8192)), ("iid_normal", dict(B=2))]
+    for name, over in cases:
+        w = W.make(name, **over)
+        T = int(w.seq_lens[1])
+        K, V = w.kv(1, 0, T)
+        Kd, Vd = K.to(dev), V.to(dev)
+        keys = w.calibration_keys(20)
+        tabs = np.stack([tq.fit_k_table(keys[h], tq.lloyd_max_table(w.d), 100)[0] for h in range(w.Hkv)])
+        nblk = (T + 15) // 16
+        bt = torch.arange(nblk, dtype=torch.int32, device=dev)[None]
+        lens = torch.tensor([T], dtype=torch.int32, device=dev)
+        slots = torch.arange(T, dtype=torch.int32, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        Kf, Vf = Kd.double(), Vd.double()
+        n2 = (Kf * Kf).sum(-1, keepdim=True)
+        live = n2[..., 0] > 0
+        row = {"tokens": T, "kv_heads": w.Hkv, "d": w.d, "dist": w.dist}
+        for label, tables, rotate in (("lloyd_max", None, True), ("calibrated", tabs, True),
+                                      ("unrotated", None, False)):
+            cache = tq.Cache(nblk, w.Hkv, w.d, device=dev, rotate=rotate)
+            kt = None if tables is None else torch.from_numpy(np.ascontiguousarray(tables)).to(dev)
+            tq.quantize_append(Kd, Vd, slots, cache, k_tables=kt, status=st)
+            Kh, Vh = tq.dequantize(cache, bt, lens, T, k_tables=kt, status=st)
+            ek = ((Kf - Kh[0].double()) ** 2) / torch.where(n2 > 0, n2, torch.ones_like(n2))
+            row["k_mse_" + label] = float(ek[live].mean())
+            if label == "lloyd_max":
+                row["v_mse"] = float(((Vf - Vh[0].double()) ** 2).mean())
+                row["v_rel_mse"] = float(((Vf - Vh[0].double()) ** 2).sum() / (Vf * Vf).sum())
+            del cache, Kh, Vh
+        torch.cuda.synchronize(dev)
+        assert int(st.item()) == 0, f"device status {int(st.item())}"
+        row["calibrated_vs_lloyd_max"] = row["k_mse_calibrated"] / row["k_mse_lloyd_max"] - 1
+        row["unrotated_vs_lloyd_max"] = row["k_mse_unrotated"] / row["k_mse_lloyd_max"] - 1
+        row["k_mse_gaussian_keys"] = sphere_coordinate_mse(tq.lloyd_max_table(w.d), w.d)
+        out[name] = row
+    return out
 
 
 def prefill_append_case(dev):

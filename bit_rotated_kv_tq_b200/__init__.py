@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
 
 BLOCK = 16
 VALUE_GROUP = 32
+TQ_CACHE_UNROTATED = 1  # cache flag: keys quantised without the rotation
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_ALIGNMENT, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(6)
 STATUS_BAD_SLOT, STATUS_BAD_BLOCK, STATUS_RANGE, STATUS_BAD_LEN, STATUS_TIMEOUT, STATUS_INTERNAL = \
@@ -36,7 +37,7 @@ class TQError(RuntimeError):
 
 class _Cache(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
-                ("head_dim", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("data", ctypes.c_void_p)]
 
 
@@ -164,9 +165,14 @@ def fit_k_table(keys: torch.Tensor, init: np.ndarray, max_iter: int = 100):
 
 # ------------------------------------------------------------------ cache
 class Cache:
-    """A paged TQ4/4 cache: uint8 [num_blocks][num_kv_heads][record] in device memory."""
+    """A paged TQ4/4 cache: uint8 [num_blocks][num_kv_heads][record] in device memory.
 
-    def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, device="cuda", data=None):
+    rotate=False makes an unrotated cache (TQ_CACHE_UNROTATED: keys quantised without
+    the Walsh-Hadamard rotation, the baseline the rotation is measured against).
+    """
+
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, device="cuda", data=None,
+                 rotate: bool = True):
         nbytes = int(load().tq_cache_bytes(num_blocks, num_kv_heads, head_dim))
         if nbytes == 0:
             raise TQError(TQ_ERR_UNSUPPORTED, f"cache shape ({num_blocks}, {num_kv_heads}, {head_dim})")
@@ -177,7 +183,9 @@ class Cache:
             raise ValueError("cache data has the wrong shape or dtype")
         self.data = data
         self.num_blocks, self.num_kv_heads, self.head_dim = num_blocks, num_kv_heads, head_dim
-        self._c = _Cache(num_blocks, num_kv_heads, head_dim, 0, data.data_ptr())
+        self.rotate = bool(rotate)
+        self._c = _Cache(num_blocks, num_kv_heads, head_dim, 0 if rotate else TQ_CACHE_UNROTATED,
+                         data.data_ptr())
 
     @property
     def c(self):

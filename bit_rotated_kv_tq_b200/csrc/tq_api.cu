@@ -107,8 +107,12 @@ const uint16_t* default_table(int d) {
 }
 
 bool check_cache(const tq_cache_t* c, int* err) {
-    if (!c || !c->data || c->num_blocks <= 0 || c->num_kv_heads <= 0 || c->reserved != 0) {
+    if (!c || !c->data || c->num_blocks <= 0 || c->num_kv_heads <= 0) {
         *err = fail(TQ_ERR_INVALID_ARG, "cache: null data or non-positive num_blocks/num_kv_heads");
+        return false;
+    }
+    if (c->flags & ~TQ_CACHE_UNROTATED) {
+        *err = fail(TQ_ERR_INVALID_ARG, "cache: unknown flags 0x%x", (unsigned)c->flags);
         return false;
     }
     if (!supported_d(c->head_dim)) {
@@ -176,6 +180,7 @@ int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tab
     a.max_blocks = max_blocks;
     a.seq_lens = seq_lens;
     a.scale_log2 = scale * 1.44269504088896340736f;
+    a.rotate = (cache->flags & TQ_CACHE_UNROTATED) ? 0 : 1;
     a.out = out;
     a.num_splits = num_splits;
     a.max_seq_len = max_seq_len;
@@ -326,6 +331,7 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
     a.k_tables = k_tables;
     memcpy(a.default_table, default_table(cache->head_dim), sizeof a.default_table);
     a.status = status;
+    a.rotate = (cache->flags & TQ_CACHE_UNROTATED) ? 0 : 1;
     cudaError_t e = tq::launch_append(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "tq_quantize_append launch");
     return ok();
@@ -400,7 +406,7 @@ TQ_API int tq_prefill_attention(const void* q, const tq_cache_t* cache, const ui
     cudaError_t e = tq::launch_prefill(q, static_cast<const unsigned char*>(cache->data), cache->num_blocks, Hkv,
                                        H_q, B, k_tables, default_table(cache->head_dim), block_tables, max_blocks,
                                        seq_lens, q_start, T, max_q_len, scale, out, status, cache->head_dim,
-                                       (cudaStream_t)stream);
+                                       (cache->flags & TQ_CACHE_UNROTATED) ? 0 : 1, (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "tq_prefill_attention launch");
     return ok();
 }
@@ -431,6 +437,7 @@ TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, cons
     a.K_hat = K_hat;
     a.V_hat = V_hat;
     a.status = status;
+    a.rotate = (cache->flags & TQ_CACHE_UNROTATED) ? 0 : 1;
     cudaError_t e = tq::launch_dequant(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "tq_dequantize launch");
     return ok();

@@ -213,7 +213,8 @@ struct AppPlan {
     }
 };
 
-template <int D>
+// ROT = false: keys quantised without the rotation (an unrotated cache).
+template <int D, bool ROT>
 __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a) {
     extern __shared__ __align__(128) unsigned char smem[];
     constexpr int LPV = Geo<D>::LPV;
@@ -402,7 +403,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
             for (int j = 0; j < 16; j++) {
                 const float2 P = make_float2(bf16_lo(kwd[j]), bf16_hi(kwd[j]));
                 s4[j & 3] = __ffma2_rn(P, P, s4[j & 3]);
-                Q[j] = make_float2(P.x + P.y, P.x - P.y);
+                Q[j] = ROT ? make_float2(P.x + P.y, P.x - P.y) : P;
             }
             const float2 s2 = add2(add2(s4[0], s4[1]), add2(s4[2], s4[3]));
             ss = s2.x + s2.y;
@@ -410,7 +411,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
 #pragma unroll
         for (int m = 1; m < LPV; m <<= 1) ss += __shfl_xor_sync(kFull, ss, m);
 #pragma unroll
-        for (int b = 1; b < 16; b <<= 1) {
+        for (int b = 1; b < (ROT ? 16 : 1); b <<= 1) {
 #pragma unroll
             for (int j = 0; j < 16; j++)
                 if (!(j & b)) {
@@ -421,7 +422,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
         }
         // ---- key: butterfly over the lane bits (upper half: partner - own)
 #pragma unroll
-        for (int m = 1; m < LPV; m <<= 1) {
+        for (int m = 1; m < (ROT ? LPV : 1); m <<= 1) {
             const float sg = (sub & m) ? -1.f : 1.f;
             const float2 sg2 = make_float2(sg, sg);
 #pragma unroll
@@ -458,8 +459,9 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
             for (int m = 1; m < LPV; m <<= 1) kor |= __shfl_xor_sync(kFull, kor, m);
             wild = small && (kor & 0x7fff7fffu) != 0u;
         }
-        const float inv = rs * inv_sqrt_d;              // 1 / (n sqrt(D))
-        const float A = rs * (inv_sqrt_d * kBinScale);  // kBinScale / (n sqrt(D))
+        // y = Q / (n sqrt(D)) after the +-1 butterfly, Q / n without it
+        const float inv = ROT ? rs * inv_sqrt_d : rs;
+        const float A = ROT ? rs * (inv_sqrt_d * kBinScale) : rs * kBinScale;
 
         // ---- key: nearest centroid.  kc[i] holds the codes of elements 8i .. 8i+7;
         // kpm flags the pairs with a decision inside the margin.
@@ -528,7 +530,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
 #pragma unroll
             for (int m = 1; m < LPV; m <<= 1) ssd += __shfl_xor_sync(kFull, ssd, m);
             const double nd = sqrt(ssd);
-            const double denom = nd * sqrt((double)D);  // y_e = (H k)_e / denom
+            const double denom = ROT ? nd * sqrt((double)D) : nd;  // y_e = (H k)_e / denom, or k_e / denom
             if (near) n16 = __half_as_ushort(__double2half(nd));
             if (near && ssd == 0.0) {
                 // an all-zero key: y = 0 exactly, every element takes the code of 0
@@ -545,59 +547,74 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
             // exact norm when that scale is unusable
             float rden = inv;
             if (wild) rden = ssd > 0.0 ? (float)(1.0 / denom) : 0.f;
-            // one flagged pair per vector per round.  Its rows 2p and 2p + 1 of the
-            // Hadamard sum share their signs on each element pair (row 2p + 1 flips
-            // the odd elements), so the sums over the even and the odd elements, exact
-            // in fp64, give both: E + O and E - O.  Each is decided against
-            // midpoint * denom.
-            const uint32_t gmask = ((1u << LPV) - 1u) << (grp * LPV);
-#pragma unroll 1
-            while (__any_sync(kFull, nm != 0)) {
-                const uint32_t pend = __ballot_sync(kFull, nm != 0) & gmask;
-                const int owner = pend ? __ffs(pend) - 1 : lane;
-                const int mine = nm ? __ffs(nm) - 1 : 0;
-                const uint32_t pr = (uint32_t)__shfl_sync(kFull, 16 * sub + mine, owner);  // pair of the vector
-                double pe = 0.0, po = 0.0;
-#pragma unroll 4
-                for (int j = 0; j < 16; j++) {
-                    const uint32_t wv = lds_u32(stage + eoff + 4 * j);
-                    const double x0 = (double)bf16_lo(wv), x1 = (double)bf16_hi(wv);
-                    const bool neg = __popc((pr & 15u) & (uint32_t)j) & 1;
-                    pe += neg ? -x0 : x0;
-                    po += neg ? -x1 : x1;
-                }
-                if (__popc((pr >> 4) & (uint32_t)sub) & 1) {
-                    pe = -pe;
-                    po = -po;
-                }
+            // Pair pj's two decisions from their exact numerators (y times denom):
+            // each against midpoint * denom, then the pair's byte of kc
+            auto decide_pair = [&](int pj, double part0, double part1) {
+                uint32_t pc = 0;
 #pragma unroll
-                for (int m = 1; m < LPV; m <<= 1) {
-                    pe += __shfl_xor_sync(kFull, pe, m);
-                    po += __shfl_xor_sync(kFull, po, m);
-                }
-                if (pend && lane == owner) {
-                    uint32_t pc = 0;
-#pragma unroll
-                    for (int hh = 0; hh < 2; hh++) {
-                        const double part = hh ? pe - po : pe + po;
-                        uint32_t idx = 0;
-                        if (!B.dense) {
-                            const float x = fmaf((float)part * rden, kBinScale, kBinMagic);
-                            const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
-                            idx = (uint32_t)be.k_hi - (part > (double)be.mid * denom ? 0u : 1u);
-                        } else {
+                for (int hh = 0; hh < 2; hh++) {
+                    const double part = hh ? part1 : part0;
+                    uint32_t idx = 0;
+                    if (!B.dense) {
+                        const float x = fmaf((float)part * rden, kBinScale, kBinMagic);
+                        const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
+                        idx = (uint32_t)be.k_hi - (part > (double)be.mid * denom ? 0u : 1u);
+                    } else {
 #pragma unroll 1
-                            for (int k = 0; k < 15; k++)
-                                idx += part > 0.5 * ((double)B.c[k] + (double)B.c[k + 1]) * denom ? 1u : 0u;
-                        }
-                        pc |= idx << (4 * hh);
+                        for (int k = 0; k < 15; k++)
+                            idx += part > 0.5 * ((double)B.c[k] + (double)B.c[k + 1]) * denom ? 1u : 0u;
                     }
-                    // pair mine is byte mine % 4 of word mine / 4
-                    const int sh = 8 * (mine & 3);
-                    const uint32_t wi = (uint32_t)mine >> 2, cm = ~(0xffu << sh), cv = pc << sh;
+                    pc |= idx << (4 * hh);
+                }
+                // pair pj is byte pj % 4 of word pj / 4
+                const int sh = 8 * (pj & 3);
+                const uint32_t wi = (uint32_t)pj >> 2, cm = ~(0xffu << sh), cv = pc << sh;
 #pragma unroll
-                    for (int i = 0; i < 4; i++) kc[i] = wi == (uint32_t)i ? (kc[i] & cm) | cv : kc[i];
+                for (int i = 0; i < 4; i++) kc[i] = wi == (uint32_t)i ? (kc[i] & cm) | cv : kc[i];
+            };
+            if constexpr (ROT) {
+                // one flagged pair per vector per round.  Its rows 2p and 2p + 1 of
+                // the Hadamard sum share their signs on each element pair (row 2p + 1
+                // flips the odd elements), so the sums over the even and the odd
+                // elements, exact in fp64, give both: E + O and E - O.
+                const uint32_t gmask = ((1u << LPV) - 1u) << (grp * LPV);
+#pragma unroll 1
+                while (__any_sync(kFull, nm != 0)) {
+                    const uint32_t pend = __ballot_sync(kFull, nm != 0) & gmask;
+                    const int owner = pend ? __ffs(pend) - 1 : lane;
+                    const int mine = nm ? __ffs(nm) - 1 : 0;
+                    const uint32_t pr = (uint32_t)__shfl_sync(kFull, 16 * sub + mine, owner);  // pair of the vector
+                    double pe = 0.0, po = 0.0;
+#pragma unroll 4
+                    for (int j = 0; j < 16; j++) {
+                        const uint32_t wv = lds_u32(stage + eoff + 4 * j);
+                        const double x0 = (double)bf16_lo(wv), x1 = (double)bf16_hi(wv);
+                        const bool neg = __popc((pr & 15u) & (uint32_t)j) & 1;
+                        pe += neg ? -x0 : x0;
+                        po += neg ? -x1 : x1;
+                    }
+                    if (__popc((pr >> 4) & (uint32_t)sub) & 1) {
+                        pe = -pe;
+                        po = -po;
+                    }
+#pragma unroll
+                    for (int m = 1; m < LPV; m <<= 1) {
+                        pe += __shfl_xor_sync(kFull, pe, m);
+                        po += __shfl_xor_sync(kFull, po, m);
+                    }
+                    if (pend && lane == owner) {
+                        decide_pair(mine, pe + po, pe - po);
+                        nm &= nm - 1u;
+                    }
+                }
+            } else {
+                // unrotated: a coordinate's numerator is the key element itself
+#pragma unroll 1
+                while (nm) {
+                    const int pj = __ffs(nm) - 1;
                     nm &= nm - 1u;
+                    const uint32_t wv = lds_u32(stage + eoff + 4 * pj);
+                    decide_pair(pj, (double)bf16_lo(wv), (double)bf16_hi(wv));
                 }
             }
         }
@@ -673,7 +690,7 @@ static void default_bins(int d, const uint16_t* table16, HeadBins& hb, BinEntry*
     memcpy(bins, cached[key], sizeof cached[key]);
 }
 
-template <int D>
+template <int D, bool ROT>
 static cudaError_t launch_a(const AppendArgs& a, int num_sms, cudaStream_t stream) {
     // the largest shared-memory size, set once per device (under a lock: the
     // library may be called from several host threads)
@@ -686,7 +703,7 @@ static cudaError_t launch_a(const AppendArgs& a, int num_sms, cudaStream_t strea
     {
         std::lock_guard<std::mutex> lk(mu);
         if (dev < 0 || dev >= 64 || !configured[dev]) {
-            e = cudaFuncSetAttribute(append_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(append_kernel<D, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      (int)max_smem);
             if (e != cudaSuccess) return e;
             if (dev >= 0 && dev < 64) configured[dev] = true;
@@ -700,7 +717,7 @@ static cudaError_t launch_a(const AppendArgs& a, int num_sms, cudaStream_t strea
     if (blocks > num_sms) blocks = num_sms;
     if (blocks < 1) blocks = 1;
     const size_t smem = AppPlan<D>(a.k_tables ? a.Hkv : 1).end;
-    append_kernel<D><<<(unsigned)blocks, kAppWarps * 32, smem, stream>>>(a);
+    append_kernel<D, ROT><<<(unsigned)blocks, kAppWarps * 32, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -709,7 +726,8 @@ cudaError_t launch_append(const AppendArgs& args, int head_dim, int num_sms, cud
     if (!a.k_tables) default_bins(head_dim, a.default_table, a.default_hb, a.default_bins);
     a.dv_hkv = div32_magic((uint32_t)a.Hkv);
     a.dv_cap = div32_magic((uint32_t)(a.max_blocks > 0 ? a.max_blocks * kBlock : 1));
-    return head_dim == 128 ? launch_a<128>(a, num_sms, stream) : launch_a<64>(a, num_sms, stream);
+    if (head_dim == 128) return a.rotate ? launch_a<128, true>(a, num_sms, stream) : launch_a<128, false>(a, num_sms, stream);
+    return a.rotate ? launch_a<64, true>(a, num_sms, stream) : launch_a<64, false>(a, num_sms, stream);
 }
 
 }  // namespace tq

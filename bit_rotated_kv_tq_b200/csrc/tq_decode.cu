@@ -626,25 +626,28 @@ __global__ void __launch_bounds__(kWarps * 32, 1) decode_split_kernel(DecodeArgs
 #pragma unroll
                 for (int e = 0; e < EPL; e++) x[e] = 0.f;
             }
+            if (a.rotate) {
 #pragma unroll
-            for (int m = 1; m < EPL; m <<= 1)
+                for (int m = 1; m < EPL; m <<= 1)
 #pragma unroll
-                for (int e = 0; e < EPL; e++)
-                    if (!(e & m)) {
-                        const float p = x[e], q = x[e | m];
-                        x[e] = p + q;
-                        x[e | m] = p - q;
+                    for (int e = 0; e < EPL; e++)
+                        if (!(e & m)) {
+                            const float p = x[e], q = x[e | m];
+                            x[e] = p + q;
+                            x[e | m] = p - q;
+                        }
+#pragma unroll
+                for (int m = 1; m < 32; m <<= 1) {
+                    const bool upper = lane & m;
+#pragma unroll
+                    for (int e = 0; e < EPL; e++) {
+                        const float p = __shfl_xor_sync(kFull, x[e], m);
+                        x[e] = upper ? p - x[e] : x[e] + p;
                     }
-#pragma unroll
-            for (int m = 1; m < 32; m <<= 1) {
-                const bool upper = lane & m;
-#pragma unroll
-                for (int e = 0; e < EPL; e++) {
-                    const float p = __shfl_xor_sync(kFull, x[e], m);
-                    x[e] = upper ? p - x[e] : x[e] + p;
                 }
             }
-            const float sc = a.scale_log2 * rsqrtf((float)D);
+            // the +-1 butterfly leaves a factor sqrt(D) that the scale takes out
+            const float sc = a.rotate ? a.scale_log2 * rsqrtf((float)D) : a.scale_log2;
             const uint32_t dh = P.qh + (uint32_t)(((half * HPI + hw) * D + lane * EPL) * 2);
             const uint32_t dl = P.ql + (uint32_t)(((half * HPI + hw) * D + lane * EPL) * 2);
 #pragma unroll

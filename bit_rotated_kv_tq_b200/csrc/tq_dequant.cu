@@ -1,6 +1,7 @@
 // tq_dequant.cu -- gather and dequantise the cache back to fp32 (checks only).
 //   k_hat = fp16 norm * H_d * C[idx]   (H_d symmetric and involutive, so the
-//                                      same butterfly undoes the rotation)
+//                                      same butterfly undoes the rotation;
+//                                      fp16 norm * C[idx] for an unrotated cache)
 //   v_hat = code * scale + zero
 // One vector (sequence, position, kv head) per D/8 lanes, 8 elements per lane.
 #include "tq_kernels.cuh"
@@ -66,28 +67,31 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
             kx[e] = C[(kw >> (4 * e)) & 15];
             vx[e] = fmaf((float)((vw >> (4 * e)) & 15), s, z);
         }
-        // inverse rotation: the same +-1 butterfly, then 1/sqrt(D)
+        // inverse rotation: the same +-1 butterfly, then 1/sqrt(D) (none for an
+        // unrotated cache; the branch is uniform over the grid)
+        if (a.rotate) {
 #pragma unroll
-        for (int m = 1; m < 8; m <<= 1) {
+            for (int m = 1; m < 8; m <<= 1) {
 #pragma unroll
-            for (int e = 0; e < 8; e++)
-                if (!(e & m)) {
-                    float x = kx[e], y = kx[e | m];
-                    kx[e] = x + y;
-                    kx[e | m] = x - y;
+                for (int e = 0; e < 8; e++)
+                    if (!(e & m)) {
+                        float x = kx[e], y = kx[e | m];
+                        kx[e] = x + y;
+                        kx[e | m] = x - y;
+                    }
+            }
+#pragma unroll
+            for (int m = 1; m < LPV; m <<= 1) {
+                const bool upper = sub & m;
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    float p = __shfl_xor_sync(kFull, kx[e], m);
+                    kx[e] = upper ? p - kx[e] : kx[e] + p;
                 }
-        }
-#pragma unroll
-        for (int m = 1; m < LPV; m <<= 1) {
-            const bool upper = sub & m;
-#pragma unroll
-            for (int e = 0; e < 8; e++) {
-                float p = __shfl_xor_sync(kFull, kx[e], m);
-                kx[e] = upper ? p - kx[e] : kx[e] + p;
             }
         }
         if (in) {
-            const float f = rec ? nrm * inv_sqrt_d : 0.f;
+            const float f = rec ? (a.rotate ? nrm * inv_sqrt_d : nrm) : 0.f;
             const size_t o = (size_t)vec * D + sub * 8;
             float4* kd = reinterpret_cast<float4*>(a.K_hat + o);
             float4* vd = reinterpret_cast<float4*>(a.V_hat + o);

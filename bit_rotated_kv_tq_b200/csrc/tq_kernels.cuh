@@ -77,6 +77,7 @@ struct AppendArgs {
     const uint16_t* k_tables;   // fp16 [Hkv][16] or null
     uint16_t default_table[16]; // fp16
     int32_t* status;
+    int rotate;                 // 1: keys rotated (the TQ4/4 format); 0: TQ_CACHE_UNROTATED
     Div32 dv_hkv, dv_cap;       // division by H_kv and by max_blocks * 16 (set by the launcher)
     HeadBins default_hb;        // bins of default_table (set by the launcher)
     BinEntry default_bins[kBins];
@@ -98,6 +99,7 @@ struct DecodeArgs {
     int num_splits;              // 0: even cut over the grid; S: ranges of nmax/S blocks
     int max_seq_len;
     int32_t* status;
+    int rotate;                  // 0: TQ_CACHE_UNROTATED (the query is not rotated)
     // set by decode_plan
     int qpi;              // groups of four query heads per item (1, or 2 at d = 64 with G > 4)
     int quads;            // items per kv head
@@ -122,6 +124,7 @@ struct DequantArgs {
     float* K_hat;  // [B][max_len][Hkv][D]
     float* V_hat;
     int32_t* status;
+    int rotate;    // 0: TQ_CACHE_UNROTATED (no inverse rotation)
 };
 
 // Host checks and split plan of a decode call (the checks of tq_decode_attention
@@ -144,7 +147,7 @@ cudaError_t launch_prefill(const void* q, const unsigned char* cache, int num_bl
                            const uint16_t* k_tables, const uint16_t* default_table,
                            const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
                            const int32_t* q_start, int T, int max_q_len, float scale, float* out,
-                           int32_t* status, int head_dim, cudaStream_t stream);
+                           int32_t* status, int head_dim, int rotate, cudaStream_t stream);
 size_t prefill_smem_bytes(int head_dim);
 
 }  // namespace tq

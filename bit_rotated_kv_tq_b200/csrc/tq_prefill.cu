@@ -188,6 +188,7 @@ struct PrefillArgs {
     float scale_log2;             // scale * log2(e)
     float* out;                   // [T][Hq][D]
     int32_t* status;
+    int rotate;                   // 0: TQ_CACHE_UNROTATED (the query is not rotated)
 };
 
 template <int D>
@@ -320,25 +321,28 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
 #pragma unroll
             for (int e = 0; e < EPL; e++) x[e] = 0.f;
         }
+        if (a.rotate) {
 #pragma unroll
-        for (int m = 1; m < EPL; m <<= 1)
+            for (int m = 1; m < EPL; m <<= 1)
 #pragma unroll
-            for (int e = 0; e < EPL; e++)
-                if (!(e & m)) {
-                    const float p = x[e], q = x[e | m];
-                    x[e] = p + q;
-                    x[e | m] = p - q;
+                for (int e = 0; e < EPL; e++)
+                    if (!(e & m)) {
+                        const float p = x[e], q = x[e | m];
+                        x[e] = p + q;
+                        x[e | m] = p - q;
+                    }
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const bool upper = lane & m;
+#pragma unroll
+                for (int e = 0; e < EPL; e++) {
+                    const float p = __shfl_xor_sync(kFull, x[e], m);
+                    x[e] = upper ? p - x[e] : x[e] + p;
                 }
-#pragma unroll
-        for (int m = 1; m < 32; m <<= 1) {
-            const bool upper = lane & m;
-#pragma unroll
-            for (int e = 0; e < EPL; e++) {
-                const float p = __shfl_xor_sync(kFull, x[e], m);
-                x[e] = upper ? p - x[e] : x[e] + p;
             }
         }
-        const float sc = a.scale_log2 * rsqrtf((float)D);
+        // the +-1 butterfly leaves a factor sqrt(D) that the scale takes out
+        const float sc = a.rotate ? a.scale_log2 * rsqrtf((float)D) : a.scale_log2;
         uint32_t hi[EPL / 2], lo[EPL / 2];
 #pragma unroll
         for (int e = 0; e < EPL; e += 2) split_h2(x[e] * sc, x[e + 1] * sc, hi[e / 2], lo[e / 2]);
@@ -632,7 +636,7 @@ cudaError_t launch_prefill(const void* q, const unsigned char* cache, int num_bl
                            const uint16_t* k_tables, const uint16_t* default_table,
                            const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,
                            const int32_t* q_start, int T, int max_q_len, float scale, float* out,
-                           int32_t* status, int head_dim, cudaStream_t stream) {
+                           int32_t* status, int head_dim, int rotate, cudaStream_t stream) {
     PrefillArgs a;
     a.q = static_cast<const uint16_t*>(q);
     a.cache = cache;
@@ -651,6 +655,7 @@ cudaError_t launch_prefill(const void* q, const unsigned char* cache, int num_bl
     a.scale_log2 = scale * 1.44269504088896340736f;
     a.out = out;
     a.status = status;
+    a.rotate = rotate;
     return head_dim == 128 ? launch_p<128>(a, max_q_len, stream) : launch_p<64>(a, max_q_len, stream);
 }
 

@@ -83,11 +83,20 @@ enum {
                                 allocation: nothing was computed; never expected */
 };
 
+/* Cache flags.  TQ_CACHE_UNROTATED: the keys are quantised without the
+ * Walsh-Hadamard rotation (y = k / ||k|| goes to the table directly).  The
+ * pages prefer the rotation because it spreads outlier channels evenly before
+ * the quantiser ("TurboQuant 在 AMD GPU 上把長上下文延遲壓下來", section 4); the
+ * unrotated cache is the baseline that shows what it buys.  Every call below
+ * honours the flag (the decode and prefill skip the query rotation), and a
+ * cache must be read with the flags it was written with. */
+enum { TQ_CACHE_UNROTATED = 1 };
+
 typedef struct {
     int32_t num_blocks;   /* physical 16-token blocks */
     int32_t num_kv_heads; /* H_kv */
     int32_t head_dim;     /* d: 64 or 128 */
-    int32_t reserved;     /* must be 0 */
+    int32_t flags;        /* 0 or TQ_CACHE_UNROTATED (other bits: TQ_ERR_INVALID_ARG) */
     void* data;           /* (device) [num_blocks][num_kv_heads][record], 16-byte aligned */
 } tq_cache_t;
 
@@ -226,7 +235,8 @@ TQ_API int tq_prefill_attention(const void* q, const tq_cache_t* cache, const ui
 /* Dequantise every valid token (checks only; the inverse of the section 2
  * encodings of "TurboQuant 在 AMD GPU 上把長上下文延遲壓下來"): K_hat and V_hat (device) fp32
  * [B][max_len][H_kv][d] in the original (unrotated) domain,
- * k_hat = fp16 norm * H * C[idx],  v_hat = code * scale + zero;
+ * k_hat = fp16 norm * H * C[idx] (fp16 norm * C[idx] for a TQ_CACHE_UNROTATED
+ * cache),  v_hat = code * scale + zero;
  * rows at or past seq_lens[b] are written as 0. */
 TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, const int32_t* block_tables,
                   int max_blocks, const int32_t* seq_lens, int B, int max_len, float* K_hat,

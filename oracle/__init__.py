@@ -75,7 +75,11 @@ def _declare(L):
     L.orc_pack_token.argtypes = [_P, _I, _I, _P, ctypes.c_uint16, _P, _P, _P]
     L.orc_unpack_token.argtypes = [_P, _I, _I, _P, _P, _P, _P, _P]
     L.orc_quantize_append.argtypes = [_P, _P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _I, _P, _P]
+    L.orc_quantize_append_ex.argtypes = [_P, _P, _I, _I, _I, _P, _I, _I, _P, _P, _P, _I, _P, _P, _I]
     L.orc_dequantize.argtypes = [_P, _I, _I, _I, _P, _P, _I, _P, _I, _I, _P, _P]
+    L.orc_dequantize_ex.argtypes = [_P, _I, _I, _I, _P, _P, _I, _P, _I, _I, _P, _P, _I]
+    L.orc_encode_k_unrotated.argtypes = [_P, _I, _P, _P, _P, _P]
+    L.orc_decode_k_unrotated.argtypes = [_P, ctypes.c_uint16, _I, _P, _P]
     L.orc_attention.argtypes = [_P, _I, _I, _I, _I, _P, _P, _I, _P, _D, _P]
     L.orc_prefill_attention.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _I, _P, _D, _P]
     L.orc_kmeans_table.argtypes = [_P, _I, _P, _I, _P]
@@ -161,6 +165,27 @@ def decode_k(idx: np.ndarray, norm16: int, table: np.ndarray) -> np.ndarray:
     return out
 
 
+def encode_k_unrotated(k_bits: np.ndarray, table: np.ndarray):
+    """The unrotated baseline: (idx, norm16 bits, y = k / n)."""
+    k = _c(k_bits, np.uint16)
+    d = k.shape[-1]
+    idx = np.zeros(d, np.uint8)
+    n16 = np.zeros(1, np.uint16)
+    y = np.zeros(d, np.float64)
+    _check(lib().orc_encode_k_unrotated(_ptr(k), d, _ptr(_h(table)), _ptr(idx), _ptr(n16), _ptr(y)),
+           "encode_k_unrotated")
+    return idx, int(n16[0]), y
+
+
+def decode_k_unrotated(idx: np.ndarray, norm16: int, table: np.ndarray) -> np.ndarray:
+    idx = _c(idx, np.uint8)
+    d = idx.shape[-1]
+    out = np.zeros(d, np.float64)
+    _check(lib().orc_decode_k_unrotated(_ptr(idx), int(norm16), d, _ptr(_h(table)), _ptr(out)),
+           "decode_k_unrotated")
+    return out
+
+
 def encode_v(v_bits: np.ndarray):
     v = _c(v_bits, np.uint16)
     d = v.shape[-1]
@@ -207,11 +232,12 @@ def unpack_token(record: np.ndarray, d: int, offset: int):
 
 
 # ---------------------------------------------------------------- paged cache
-def quantize_append(K_bits, V_bits, slots, cache, tables=None, block_table=None, want_aux=False):
+def quantize_append(K_bits, V_bits, slots, cache, tables=None, block_table=None, want_aux=False,
+                    rotate=True):
     """K_bits/V_bits: uint16 [T][Hkv][d]; cache: uint8 [num_blocks][Hkv][record] (updated in place).
 
-    Returns (rc, ky, vr): the rotated unit key coordinates and (v-z)/s, fp64 [T][Hkv][d]
-    when want_aux, else None.
+    Returns (rc, ky, vr): the (rotated, unless rotate=False) unit key coordinates and
+    (v-z)/s, fp64 [T][Hkv][d] when want_aux, else None.
     """
     K = _c(K_bits, np.uint16)
     V = _c(V_bits, np.uint16)
@@ -225,12 +251,13 @@ def quantize_append(K_bits, V_bits, slots, cache, tables=None, block_table=None,
     max_blocks = 0 if bt is None else bt.shape[1]
     ky = np.zeros((T, Hkv, d), np.float64) if want_aux else None
     vr = np.zeros((T, Hkv, d), np.float64) if want_aux else None
-    rc = lib().orc_quantize_append(_ptr(K), _ptr(V), T, Hkv, d, _ptr(bt), num_seqs, max_blocks,
-                                   _ptr(sl), _ptr(tb), _ptr(cache), num_blocks, _ptr(ky), _ptr(vr))
+    rc = lib().orc_quantize_append_ex(_ptr(K), _ptr(V), T, Hkv, d, _ptr(bt), num_seqs, max_blocks,
+                                      _ptr(sl), _ptr(tb), _ptr(cache), num_blocks, _ptr(ky), _ptr(vr),
+                                      1 if rotate else 0)
     return rc, ky, vr
 
 
-def dequantize(cache, Hkv, d, block_tables, seq_lens, max_len, tables=None):
+def dequantize(cache, Hkv, d, block_tables, seq_lens, max_len, tables=None, rotate=True):
     bt = _c(block_tables, np.int32)
     sl = _c(seq_lens, np.int32)
     B, max_blocks = bt.shape
@@ -239,8 +266,8 @@ def dequantize(cache, Hkv, d, block_tables, seq_lens, max_len, tables=None):
     Kh = np.full((B, max_len, Hkv, d), np.nan, np.float64)
     Vh = np.full((B, max_len, Hkv, d), np.nan, np.float64)
     tb = None if tables is None else _h(tables)
-    rc = lib().orc_dequantize(_ptr(cache), cache.shape[0], Hkv, d, _ptr(tb), _ptr(bt), max_blocks,
-                              _ptr(sl), B, max_len, _ptr(Kh), _ptr(Vh))
+    rc = lib().orc_dequantize_ex(_ptr(cache), cache.shape[0], Hkv, d, _ptr(tb), _ptr(bt), max_blocks,
+                                 _ptr(sl), B, max_len, _ptr(Kh), _ptr(Vh), 1 if rotate else 0)
     _check(rc, "dequantize")
     return Kh, Vh
 

@@ -295,6 +295,43 @@ int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const uint16_t *tab
     return 0;
 }
 
+/* The unrotated baseline ("TurboQuant 在 AMD GPU 上把長上下文延遲壓下來",
+ * section 4: the rotation is there to spread the energy of outlier channels
+ * evenly before the quantiser; without it the unit vector's own coordinates
+ * go to the table).  Encode: y_i = k_i / n, idx_i = nearest centroid; decode:
+ * k_hat = fp16(n) * C[idx]. */
+int orc_encode_k_unrotated(const uint16_t *k_bf16, int d, const uint16_t *table, uint8_t *idx,
+                           uint16_t *norm16, double *y_out)
+{
+    if (!is_pow2(d) || !k_bf16 || !table || !idx || !norm16)
+        return -1;
+    double ss = 0.0;
+    for (int i = 0; i < d; i++) {
+        double x = orc_bf16_to_double(k_bf16[i]);
+        ss += x * x;
+    }
+    double n = sqrt(ss);
+    *norm16 = orc_fp16_from_double(n, 0);
+    for (int i = 0; i < d; i++) {
+        double y = (n > 0.0) ? orc_bf16_to_double(k_bf16[i]) / n : 0.0;
+        idx[i] = (uint8_t)nearest_centroid(y, table);
+        if (y_out)
+            y_out[i] = y;
+    }
+    return 0;
+}
+
+int orc_decode_k_unrotated(const uint8_t *idx, uint16_t norm16, int d, const uint16_t *table,
+                           double *k_hat)
+{
+    if (!is_pow2(d) || !idx || !table || !k_hat)
+        return -1;
+    double n = orc_fp16_to_double(norm16);
+    for (int i = 0; i < d; i++)
+        k_hat[i] = n * orc_fp16_to_double(table[idx[i] & 15]);
+    return 0;
+}
+
 /* ------------------------------------------------------------------ */
 /* values                                                               */
 /* ------------------------------------------------------------------ */
@@ -462,6 +499,15 @@ int orc_quantize_append(const uint16_t *K, const uint16_t *V, int T, int Hkv, in
                         const int32_t *slots, const uint16_t *tables, uint8_t *cache,
                         int num_blocks, double *ky, double *vr)
 {
+    return orc_quantize_append_ex(K, V, T, Hkv, d, block_table, num_seqs, max_blocks, slots, tables,
+                                  cache, num_blocks, ky, vr, 1);
+}
+
+int orc_quantize_append_ex(const uint16_t *K, const uint16_t *V, int T, int Hkv, int d,
+                           const int32_t *block_table, int num_seqs, int max_blocks,
+                           const int32_t *slots, const uint16_t *tables, uint8_t *cache,
+                           int num_blocks, double *ky, double *vr, int rotate)
+{
     if (T < 0 || Hkv <= 0 || !is_pow2(d) || d % ORC_VGROUP || !slots || !cache)
         return -1;
     uint16_t deflt[16];
@@ -500,7 +546,10 @@ int orc_quantize_append(const uint16_t *K, const uint16_t *V, int T, int Hkv, in
             uint16_t kn;
             double *kyp = ky ? ky + ((size_t)t * Hkv + h) * d : NULL;
             double *vrp = vr ? vr + ((size_t)t * Hkv + h) * d : NULL;
-            orc_encode_k(k, d, head_table(tables, deflt, h), kidx, &kn, kyp);
+            if (rotate)
+                orc_encode_k(k, d, head_table(tables, deflt, h), kidx, &kn, kyp);
+            else
+                orc_encode_k_unrotated(k, d, head_table(tables, deflt, h), kidx, &kn, kyp);
             orc_encode_v(v, d, vq, vs, vz, vrp);
             uint8_t *record = cache + ((size_t)blk * Hkv + h) * rec;
             orc_pack_token(record, d, off, kidx, kn, vq, vs, vz);
@@ -516,6 +565,14 @@ int orc_quantize_append(const uint16_t *K, const uint16_t *V, int T, int Hkv, in
 int orc_dequantize(const uint8_t *cache, int num_blocks, int Hkv, int d, const uint16_t *tables,
                    const int32_t *block_tables, int max_blocks, const int32_t *seq_lens, int B,
                    int max_len, double *Khat, double *Vhat)
+{
+    return orc_dequantize_ex(cache, num_blocks, Hkv, d, tables, block_tables, max_blocks, seq_lens,
+                             B, max_len, Khat, Vhat, 1);
+}
+
+int orc_dequantize_ex(const uint8_t *cache, int num_blocks, int Hkv, int d, const uint16_t *tables,
+                      const int32_t *block_tables, int max_blocks, const int32_t *seq_lens, int B,
+                      int max_len, double *Khat, double *Vhat, int rotate)
 {
     if (!cache || !block_tables || !seq_lens || !Khat || !Vhat || !is_pow2(d) ||
         d % ORC_VGROUP)
@@ -548,7 +605,10 @@ int orc_dequantize(const uint8_t *cache, int num_blocks, int Hkv, int d, const u
                 uint16_t kn;
                 orc_unpack_token(record, d, t % ORC_BLOCK, kidx, &kn, vq, vs, vz);
                 size_t o = (((size_t)b * max_len + t) * Hkv + h) * d;
-                orc_decode_k(kidx, kn, d, head_table(tables, deflt, h), Khat + o);
+                if (rotate)
+                    orc_decode_k(kidx, kn, d, head_table(tables, deflt, h), Khat + o);
+                else
+                    orc_decode_k_unrotated(kidx, kn, d, head_table(tables, deflt, h), Khat + o);
                 orc_decode_v(vq, vs, vz, d, Vhat + o);
             }
         }

@@ -60,6 +60,13 @@ int orc_encode_k(const uint16_t *k_bf16, int d, const uint16_t *table, uint8_t *
 /* Key decode to the original domain: k_hat = fp16(n) * H * C[idx]. */
 int orc_decode_k(const uint8_t *idx, uint16_t norm16, int d, const uint16_t *table, double *k_hat);
 
+/* The same without the rotation (the baseline an unrotated cache holds):
+ * y_i = k_i / n, idx_i = argmin_c |y_i - C[c]|;  k_hat = fp16(n) * C[idx]. */
+int orc_encode_k_unrotated(const uint16_t *k_bf16, int d, const uint16_t *table, uint8_t *idx,
+                           uint16_t *norm16, double *y_out);
+int orc_decode_k_unrotated(const uint8_t *idx, uint16_t norm16, int d, const uint16_t *table,
+                           double *k_hat);
+
 /* Value encode per group of 32: z = fp16 down(min), s = fp16 up((max - z)/15),
  * q = clamp(round_half_even((v - z)/s), 0, 15) (q = 0 when s = 0).
  * r_out (may be NULL) receives (v - z)/s in fp64 (0 when s = 0). */
@@ -86,12 +93,21 @@ int orc_quantize_append(const uint16_t *K, const uint16_t *V, int T, int Hkv, in
                         const int32_t *block_table, int num_seqs, int max_blocks,
                         const int32_t *slots, const uint16_t *tables, uint8_t *cache,
                         int num_blocks, double *ky, double *vr);
+/* rotate = 0: keys by orc_encode_k_unrotated (an unrotated cache); 1: as above. */
+int orc_quantize_append_ex(const uint16_t *K, const uint16_t *V, int T, int Hkv, int d,
+                           const int32_t *block_table, int num_seqs, int max_blocks,
+                           const int32_t *slots, const uint16_t *tables, uint8_t *cache,
+                           int num_blocks, double *ky, double *vr, int rotate);
 
 /* Gather + dequantise every valid token of every sequence into
  * Khat, Vhat fp64 [B][max_len][Hkv][d] (original domain); rows past seq_len are 0. */
 int orc_dequantize(const uint8_t *cache, int num_blocks, int Hkv, int d, const uint16_t *tables,
                    const int32_t *block_tables, int max_blocks, const int32_t *seq_lens, int B,
                    int max_len, double *Khat, double *Vhat);
+/* rotate = 0: keys by orc_decode_k_unrotated. */
+int orc_dequantize_ex(const uint8_t *cache, int num_blocks, int Hkv, int d, const uint16_t *tables,
+                      const int32_t *block_tables, int max_blocks, const int32_t *seq_lens, int B,
+                      int max_len, double *Khat, double *Vhat, int rotate);
 
 /* Exact softmax attention in fp64 over dequantised K/V.
  * q bf16 [B][Hq][d]; query head h reads kv head h / (Hq/Hkv); out fp64 [B][Hq][d]. */

@@ -94,6 +94,16 @@ def test_argument_validation_without_launch(lib):
     assert rc == tq.TQ_ERR_INVALID_ARG
     rc = lib.tq_quantize_append(None, None, None, 0, 0, None, 0, ctypes.byref(c), None, None, None)
     assert rc == tq.TQ_OK  # T == 0 is a no-op
+    # cache flags: TQ_CACHE_UNROTATED is the only defined bit, checked by every call
+    for bad in (2, 4, 1 << 30):
+        c = tq._Cache(4, 2, 128, bad | tq.TQ_CACHE_UNROTATED, 0x1000)
+        rc = lib.tq_quantize_append(None, None, None, 0, 0, None, 0, ctypes.byref(c), None, None, None)
+        assert rc == tq.TQ_ERR_INVALID_ARG and b"flags" in lib.tq_last_error()
+        rc = lib.tq_dequantize(ctypes.byref(c), None, P(16), 1, P(16), 1, 16, P(16), P(16), None, None)
+        assert rc == tq.TQ_ERR_INVALID_ARG and b"flags" in lib.tq_last_error()
+    c = tq._Cache(4, 2, 128, tq.TQ_CACHE_UNROTATED, 0x1000)
+    rc = lib.tq_quantize_append(None, None, None, 0, 0, None, 0, ctypes.byref(c), None, None, None)
+    assert rc == tq.TQ_OK
     # decode: H_q not a multiple of H_kv, or a GQA group above 64, unsupported; workspace
     # too small; bad split count
     c = _cache_struct(heads=2)

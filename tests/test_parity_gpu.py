@@ -23,9 +23,9 @@ pytestmark = pytest.mark.gpu
 class GpuState:
     """A workload appended into a device cache through tq_quantize_append."""
 
-    def __init__(self, tq, w, tables=None):
+    def __init__(self, tq, w, tables=None, rotate=True):
         self.tq, self.w = tq, w
-        self.cache = tq.Cache(w.num_blocks, w.Hkv, w.d)
+        self.cache = tq.Cache(w.num_blocks, w.Hkv, w.d, rotate=rotate)
         self.bt = torch.from_numpy(w.block_tables).cuda()
         self.seq_lens = torch.from_numpy(w.seq_lens).cuda()
         self.tables_np = tables
@@ -57,7 +57,7 @@ class GpuState:
 class OracleSeq:
     """The oracle's encoding, dequantisation and attention for one (sequence, kv head)."""
 
-    def __init__(self, orc, w, b, h, table):
+    def __init__(self, orc, w, b, h, table, rotate=True):
         self.w, self.b, self.h = w, b, h
         L = int(w.seq_lens[b])
         K, V = w.kv(b)
@@ -68,11 +68,11 @@ class OracleSeq:
         assert self.table.dtype == np.float16
         self.cache = np.zeros((nblk, 1, orc.record_bytes(w.d)), np.uint8)
         rc, self.ky, self.vr = orc.quantize_append(Kb, Vb, np.arange(L, dtype=np.int32), self.cache,
-                                                   tables=self.table[None], want_aux=True)
+                                                   tables=self.table[None], want_aux=True, rotate=rotate)
         assert rc == 0
         bt = np.arange(nblk, dtype=np.int32)[None]
         self.Kh, self.Vh = orc.dequantize(self.cache, 1, w.d, bt, np.array([L], np.int32), L,
-                                          tables=self.table[None])
+                                          tables=self.table[None], rotate=rotate)
         self.norms = np.linalg.norm(K[:, h].double().numpy(), axis=-1)
         self.L = L
 
@@ -114,16 +114,16 @@ def table_for(w, tq, orc, calibrated=False):
     return np.stack(prod), np.stack(orct)
 
 
-def check_pairs(tq, orc, w, pairs, num_splits=0, calibrated=False, decode=True):
+def check_pairs(tq, orc, w, pairs, num_splits=0, calibrated=False, decode=True, rotate=True):
     prod_t, orc_t = table_for(w, tq, orc, calibrated)
     if calibrated:
         assert np.array_equal(prod_t, orc_t), "re-fitted tables differ between library and oracle"
-    g = GpuState(tq, w, prod_t)
+    g = GpuState(tq, w, prod_t, rotate=rotate)
     out = g.decode(num_splits=num_splits) if decode else None
     q_bits = bf16_bits(w.q())
     report = CodeReport()
     for b, h in pairs:
-        o = OracleSeq(orc, w, b, h, orc_t[h])
+        o = OracleSeq(orc, w, b, h, orc_t[h], rotate=rotate)
         compare_records(report, g.records(b, h), o, w.d)
         if decode:
             heads = slice(h * w.G, (h + 1) * w.G)

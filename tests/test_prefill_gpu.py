@@ -18,8 +18,8 @@ from workloads import bf16_bits
 pytestmark = pytest.mark.gpu
 
 
-def _gpu_cache(tq, w, tables=None):
-    cache = tq.Cache(w.num_blocks, w.Hkv, w.d)
+def _gpu_cache(tq, w, tables=None, rotate=True):
+    cache = tq.Cache(w.num_blocks, w.Hkv, w.d, rotate=rotate)
     bt = torch.from_numpy(w.block_tables).cuda()
     for K, V, slots in w.population():
         tq.quantize_append(K.cuda(), V.cuda(), slots.cuda(), cache, block_table=bt, k_tables=tables)
@@ -27,23 +27,24 @@ def _gpu_cache(tq, w, tables=None):
     return cache, bt
 
 
-def _oracle_prefill(orc, w, b, q_bits_b, qlen, table_rows):
+def _oracle_prefill(orc, w, b, q_bits_b, qlen, table_rows, rotate=True):
     """fp64 chunked-prefill attention of sequence b's last qlen tokens (oracle only)."""
     L = int(w.seq_lens[b])
     K, V = w.kv(b)
     nblk = (L + 15) // 16
     cache = np.zeros((nblk, w.Hkv, orc.record_bytes(w.d)), np.uint8)
     rc, _, _ = orc.quantize_append(bf16_bits(K), bf16_bits(V), np.arange(L, dtype=np.int32), cache,
-                                   tables=table_rows)
+                                   tables=table_rows, rotate=rotate)
     assert rc == 0
     bt = np.arange(nblk, dtype=np.int32)[None]
-    Kh, Vh = orc.dequantize(cache, w.Hkv, w.d, bt, np.array([L], np.int32), L, tables=table_rows)
+    Kh, Vh = orc.dequantize(cache, w.Hkv, w.d, bt, np.array([L], np.int32), L, tables=table_rows,
+                            rotate=rotate)
     return orc.prefill_attention(q_bits_b, np.array([0, qlen], np.int32), Kh, Vh,
                                  np.array([L], np.int32), w.scale)
 
 
-def _run_case(tq, orc, w, qlens, tables=None, oracle_tables=None, seed=5):
-    cache, bt = _gpu_cache(tq, w, tables)
+def _run_case(tq, orc, w, qlens, tables=None, oracle_tables=None, seed=5, rotate=True):
+    cache, bt = _gpu_cache(tq, w, tables, rotate)
     qlens = np.asarray(qlens, np.int32)
     q_start = np.concatenate([[0], np.cumsum(qlens)]).astype(np.int32)
     T = int(q_start[-1])
@@ -59,7 +60,7 @@ def _run_case(tq, orc, w, qlens, tables=None, oracle_tables=None, seed=5):
     q_bits = bf16_bits(q)
     for b in range(w.B):
         rows = slice(int(q_start[b]), int(q_start[b + 1]))
-        want = _oracle_prefill(orc, w, b, q_bits[rows], int(qlens[b]), oracle_tables)
+        want = _oracle_prefill(orc, w, b, q_bits[rows], int(qlens[b]), oracle_tables, rotate)
         check_attention(got[rows], want, f"{w.name} b={b} q_len={qlens[b]}")
     return got
 
@@ -114,3 +115,12 @@ def test_prefill_bad_length_sets_status_and_zeros(tq):
     torch.cuda.synchronize()
     assert int(st.item()) & tq.STATUS_BAD_LEN
     assert torch.all(out[8:] == 0) and torch.isfinite(out[:8]).all() and out[:8].abs().sum() > 0
+
+
+@pytest.mark.parametrize("name,over,qlens", [
+    ("tiny", dict(B=1, ctx=200), (130,)),                      # d 128, outlier channels
+    ("prefill_small_head", dict(B=2, ctx=300), (77, 150)),     # d 64, GQA 8
+])
+def test_prefill_on_unrotated_cache(tq, orc, name, over, qlens):
+    """TQ_CACHE_UNROTATED: the query is not rotated either; same oracle rule."""
+    _run_case(tq, orc, W.make(name, **over), qlens, rotate=False)

@@ -27,6 +27,9 @@ their 32-way concurrent, ~25K-token-prefix agent runs):
   prefill_small_head   16 seqs, 2048-token append chunks, 16 q / 2 kv heads
                        (GQA 8), d 64, N(0,1) with 2% of tokens x10, decode at
                        32768 tokens, seed 4
+  iid_normal           1 seq x 4096 tokens, 32 q / 8 kv heads, d 128, plain
+                       N(0,1) (keys uniform in direction: the reference case
+                       of the table-quality study), seed 5
 """
 from __future__ import annotations
 
@@ -53,7 +56,7 @@ class Workload:
     Hkv: int
     d: int
     seed: int
-    dist: str                      # "normal_outlier" | "student_t" | "normal_spike"
+    dist: str                      # "normal_outlier" | "student_t" | "normal_spike" | "normal"
     seq_lens: np.ndarray           # int32 [B]
     block_tables: np.ndarray       # int32 [B][max_blocks]
     num_blocks: int
@@ -246,6 +249,8 @@ def make(name: str, **over) -> Workload:
         B, Hq, Hkv, d, ctx, seed, dist = 32, 32, 8, 128, 0, 3, "student_t"
     elif name == "prefill_small_head":
         B, Hq, Hkv, d, ctx, seed, dist = 16, 16, 2, 64, 32768, 4, "normal_spike"
+    elif name == "iid_normal":
+        B, Hq, Hkv, d, ctx, seed, dist = 1, 32, 8, 128, 4096, 5, "normal"
     else:
         raise KeyError(name)
     B = over.pop("B", B)
