@@ -374,8 +374,8 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
             return graph_time(fn, reps)
         return graph_time(lambda: (flush.sum(), fn()), reps) - graph_time(lambda: flush.sum(), reps)
 
-    def build(w, tables=None):
-        cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev)
+    def build(w, tables=None, bf16=False):
+        cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev, bf16=bf16)
         bt = torch.from_numpy(w.block_tables).to(dev)
         for K, V, slots in w.population():
             tq.quantize_append(K.to(dev), V.to(dev), slots.to(dev), cache, block_table=bt,
@@ -439,6 +439,15 @@ def other_workloads(dev, peak, reps: int = 20) -> dict:
     kv = decode_kv_bytes(w)
     ms = decode(w, cache, bt, 0, cold=True)
     res["prefill_small_head_decode"] = {"ms": ms, "gbs": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / peak}
+    del cache
+
+    # the full-precision (bf16) cache that boundary layers keep, on the headline shape:
+    # 32 x 8192 tokens x 8 kv heads of bf16 keys and values (1.07 GB, more than L2)
+    w = W.make("qwen3_8b_layer")
+    cache, bt = build(w, bf16=True)
+    kv = int(w.seq_lens.sum()) * w.Hkv * 4 * w.d
+    ms = decode(w, cache, bt, 0)
+    res["bf16_decode"] = {"ms": ms, "kv_bytes": kv, "gbs": kv / ms / 1e6, "hbm_frac": kv / ms / 1e6 / peak}
     del cache
 
     # chunked-prefill attention (tcgen05): the second 2048-token chunk of every
@@ -842,6 +851,8 @@ def run_tq(args, rank, world, local):
     others = None
     if rank == 0 and world == 1 and not args.no_workloads:
         others = other_workloads(dev, peak)
+        # the same decode over the full-precision cache, against this one
+        others["bf16_decode"]["tq_speedup"] = others["bf16_decode"]["ms"] / dec_avg
 
     if rank == 0:
         line = {

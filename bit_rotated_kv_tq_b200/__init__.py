@@ -23,6 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libtq_b200.so")
 BLOCK = 16
 VALUE_GROUP = 32
 TQ_CACHE_UNROTATED = 1  # cache flag: keys quantised without the rotation
+TQ_CACHE_BF16 = 2       # cache flag: full-precision bf16 rows (layers kept unquantised)
 
 TQ_OK, TQ_ERR_INVALID_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_ALIGNMENT, TQ_ERR_CUDA, TQ_ERR_WORKSPACE = range(6)
 STATUS_BAD_SLOT, STATUS_BAD_BLOCK, STATUS_RANGE, STATUS_BAD_LEN, STATUS_TIMEOUT, STATUS_INTERNAL = \
@@ -58,6 +59,8 @@ def load(path: str | None = None):
     L.tq_record_bytes.argtypes = [_I]
     L.tq_cache_bytes.restype = _Z
     L.tq_cache_bytes.argtypes = [_I, _I, _I]
+    L.tq_cache_record_bytes.restype = _Z
+    L.tq_cache_record_bytes.argtypes = [_I, _I]
     L.tq_lloyd_max_table.argtypes = [_I, _P]
     L.tq_fit_k_table.argtypes = [_P, _I, _I, _P, _I, _P]
     L.tq_quantize_append.argtypes = [_P, _P, _P, _I, _I, _P, _I, ctypes.POINTER(_Cache), _P, _P, _P]
@@ -168,24 +171,27 @@ class Cache:
     """A paged TQ4/4 cache: uint8 [num_blocks][num_kv_heads][record] in device memory.
 
     rotate=False makes an unrotated cache (TQ_CACHE_UNROTATED: keys quantised without
-    the Walsh-Hadamard rotation, the baseline the rotation is measured against).
+    the Walsh-Hadamard rotation, the baseline the rotation is measured against);
+    bf16=True a full-precision cache (TQ_CACHE_BF16: bf16 rows, for the layers a
+    model keeps unquantised).
     """
 
     def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, device="cuda", data=None,
-                 rotate: bool = True):
+                 rotate: bool = True, bf16: bool = False):
+        flags = (0 if rotate else TQ_CACHE_UNROTATED) | (TQ_CACHE_BF16 if bf16 else 0)
         nbytes = int(load().tq_cache_bytes(num_blocks, num_kv_heads, head_dim))
-        if nbytes == 0:
-            raise TQError(TQ_ERR_UNSUPPORTED, f"cache shape ({num_blocks}, {num_kv_heads}, {head_dim})")
-        rec = record_bytes(head_dim)
+        rec = int(load().tq_cache_record_bytes(head_dim, flags))
+        if nbytes == 0 or rec == 0:
+            raise TQError(TQ_ERR_UNSUPPORTED,
+                          f"cache shape ({num_blocks}, {num_kv_heads}, {head_dim}), flags {flags}")
         if data is None:
             data = torch.zeros((num_blocks, num_kv_heads, rec), dtype=torch.uint8, device=device)
         if tuple(data.shape) != (num_blocks, num_kv_heads, rec) or data.dtype != torch.uint8:
             raise ValueError("cache data has the wrong shape or dtype")
         self.data = data
         self.num_blocks, self.num_kv_heads, self.head_dim = num_blocks, num_kv_heads, head_dim
-        self.rotate = bool(rotate)
-        self._c = _Cache(num_blocks, num_kv_heads, head_dim, 0 if rotate else TQ_CACHE_UNROTATED,
-                         data.data_ptr())
+        self.rotate, self.bf16, self.flags = bool(rotate), bool(bf16), flags
+        self._c = _Cache(num_blocks, num_kv_heads, head_dim, flags, data.data_ptr())
 
     @property
     def c(self):

@@ -111,7 +111,8 @@ bool check_cache(const tq_cache_t* c, int* err) {
         *err = fail(TQ_ERR_INVALID_ARG, "cache: null data or non-positive num_blocks/num_kv_heads");
         return false;
     }
-    if (c->flags & ~TQ_CACHE_UNROTATED) {
+    if ((c->flags & ~(TQ_CACHE_UNROTATED | TQ_CACHE_BF16)) ||
+        c->flags == (TQ_CACHE_UNROTATED | TQ_CACHE_BF16)) {
         *err = fail(TQ_ERR_INVALID_ARG, "cache: unknown flags 0x%x", (unsigned)c->flags);
         return false;
     }
@@ -167,6 +168,9 @@ int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tab
         (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
         return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: q/out/tables must be 4-byte aligned");
     const int d = cache->head_dim;
+    const bool bf16 = (cache->flags & TQ_CACHE_BF16) != 0;
+    if (bf16 && k_tables)
+        return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: a bf16 cache takes no key tables");
     a = DecodeArgs{};
     a.q = static_cast<const uint16_t*>(q);
     a.cache = static_cast<const unsigned char*>(cache->data);
@@ -185,6 +189,32 @@ int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tab
     a.num_splits = num_splits;
     a.max_seq_len = max_seq_len;
     a.status = status;
+    if (bf16) {
+        // items of up to 8 query heads; S ranges of blocks per item.  The kernel is
+        // bound by HBM, not by how evenly the SMs are loaded (an SM whose neighbours
+        // are done streams faster), so by default S is the fewest ranges that give
+        // every SM a CTA (one CTA keeps 96 KB of copies in flight), at most 16, at
+        // most the longest sequence's blocks, with partials inside the
+        // num_splits = 0 workspace
+        a.bf16 = 1;
+        a.bf_hgroups = (G + 7) / 8;
+        const long long items = (long long)B * Hkv * a.bf_hgroups;
+        int S = num_splits;
+        if (S == 0) {
+            const long long per = (long long)B * H_q * (4LL * d + 8);
+            long long cap = (long long)tq_decode_workspace_bytes(B, H_q, d, 0) / per;
+            cap = std::min(cap, 16LL);
+            cap = std::min(cap, (long long)std::max(1, (max_seq_len + kBlock - 1) / kBlock));
+            cap = std::max(cap, 1LL);
+            const long long sms = device_sms();
+            S = (int)std::min(cap, std::max(1LL, (sms + items - 1) / items));
+        }
+        if (items * S > 0x7fffffffLL)
+            return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * num_splits too large");
+        a.bf_splits = S;
+        need = S > 1 ? (size_t)B * H_q * S * ((size_t)d * sizeof(float) + sizeof(float2)) : 0;
+        return ok();
+    }
     if (!decode_plan(a, d, device_sms()))
         return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: B * H_kv * num_splits too large");
     need = decode_workspace_for(a, d);
@@ -195,6 +225,14 @@ int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tab
 // decode_workspace_for bytes, 16-byte aligned; unused when that is 0).
 int decode_launch(DecodeArgs& a, int head_dim, void* workspace, void* stream) {
     a.ws_o = static_cast<float*>(workspace);
+    if (a.bf16) {  // [B][H_q][S][d] partial outputs, then [B][H_q][S] (m, l)
+        a.ws_ml = workspace ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
+                                                        (size_t)a.B * a.Hq * a.bf_splits * head_dim)
+                            : nullptr;
+        cudaError_t e = launch_bf16_decode(a, head_dim, (cudaStream_t)stream);
+        if (e != cudaSuccess) return cuda_fail(e, "tq_decode_attention launch");
+        return ok();
+    }
     // [ranges][2][heads per item][d] partial outputs, then [ranges][2][heads per item] (m, l)
     a.ws_ml = workspace ? reinterpret_cast<float2*>(static_cast<float*>(workspace) +
                                                     (size_t)a.nranges * 2 * 4 * a.qpi * head_dim)
@@ -210,6 +248,13 @@ extern "C" {
 TQ_API size_t tq_record_bytes(int head_dim) {
     if (!supported_d(head_dim)) return 0;
     return head_dim == 128 ? (size_t)tq::Rec<128>::kBytes : (size_t)tq::Rec<64>::kBytes;
+}
+
+TQ_API size_t tq_cache_record_bytes(int head_dim, int flags) {
+    if (!supported_d(head_dim)) return 0;
+    if ((flags & ~(TQ_CACHE_UNROTATED | TQ_CACHE_BF16)) || flags == (TQ_CACHE_UNROTATED | TQ_CACHE_BF16))
+        return 0;
+    return (flags & TQ_CACHE_BF16) ? (size_t)64 * head_dim : tq_record_bytes(head_dim);
 }
 
 TQ_API size_t tq_cache_bytes(int num_blocks, int num_kv_heads, int head_dim) {
@@ -332,7 +377,13 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
     memcpy(a.default_table, default_table(cache->head_dim), sizeof a.default_table);
     a.status = status;
     a.rotate = (cache->flags & TQ_CACHE_UNROTATED) ? 0 : 1;
-    cudaError_t e = tq::launch_append(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
+    cudaError_t e;
+    if (cache->flags & TQ_CACHE_BF16) {
+        if (k_tables) return fail(TQ_ERR_INVALID_ARG, "tq_quantize_append: a bf16 cache takes no key tables");
+        e = tq::launch_bf16_append(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
+    } else {
+        e = tq::launch_append(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "tq_quantize_append launch");
     return ok();
 }
@@ -355,7 +406,12 @@ TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_sp
     const long long ranges =
         num_splits == 0 ? 2LL * device_sms() : (long long)B * H_q * num_splits + 1;
     const long long heads = num_splits == 0 && head_dim == 64 ? 8 : 4;
-    return (size_t)ranges * 2 * heads * ((size_t)head_dim * sizeof(float) + sizeof(float2));
+    const size_t per_head = (size_t)head_dim * sizeof(float) + sizeof(float2);
+    size_t n = (size_t)ranges * 2 * heads * per_head;
+    // the default plan of a bf16 cache: up to 8 ranges per query head, within the
+    // static entry's 8 MiB
+    if (num_splits == 0) n = std::max(n, std::min((size_t)8 * B * H_q * per_head, (size_t)8 << 20));
+    return n;
 }
 
 TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,
@@ -384,6 +440,8 @@ TQ_API int tq_prefill_attention(const void* q, const tq_cache_t* cache, const ui
                                 float* out, int32_t* status, void* stream) {
     int err;
     if (!check_cache(cache, &err)) return err;
+    if (cache->flags & TQ_CACHE_BF16)
+        return fail(TQ_ERR_UNSUPPORTED, "tq_prefill_attention: not available for a bf16 cache");
     if (B < 0 || H_q <= 0 || T < 0 || max_q_len < 0 || max_blocks <= 0)
         return fail(TQ_ERR_INVALID_ARG,
                     "tq_prefill_attention: need B, T, max_q_len >= 0, H_q > 0, max_blocks > 0");
@@ -438,7 +496,13 @@ TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, cons
     a.V_hat = V_hat;
     a.status = status;
     a.rotate = (cache->flags & TQ_CACHE_UNROTATED) ? 0 : 1;
-    cudaError_t e = tq::launch_dequant(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
+    cudaError_t e;
+    if (cache->flags & TQ_CACHE_BF16) {
+        if (k_tables) return fail(TQ_ERR_INVALID_ARG, "tq_dequantize: a bf16 cache takes no key tables");
+        e = tq::launch_bf16_dequant(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
+    } else {
+        e = tq::launch_dequant(a, cache->head_dim, device_sms(), (cudaStream_t)stream);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "tq_dequantize launch");
     return ok();
 }

@@ -100,6 +100,8 @@ struct DecodeArgs {
     int max_seq_len;
     int32_t* status;
     int rotate;                  // 0: TQ_CACHE_UNROTATED (the query is not rotated)
+    int bf16;                    // 1: a TQ_CACHE_BF16 cache (the bf16 kernels and plan)
+    int bf_splits, bf_hgroups;   // bf16 plan: ranges per item, items of <= 8 heads per kv head
     // set by decode_plan
     int qpi;              // groups of four query heads per item (1, or 2 at d = 64 with G > 4)
     int quads;            // items per kv head
@@ -143,6 +145,10 @@ bool decode_plan(DecodeArgs& a, int head_dim, int num_sms);  // ranges; false: t
 bool decode_needs_combine(const DecodeArgs& a);          // some item is cut by a range
 size_t decode_workspace_for(const DecodeArgs& a, int head_dim);  // partials, bytes
 cudaError_t launch_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);
+// the full-precision (TQ_CACHE_BF16) cache
+cudaError_t launch_bf16_append(const AppendArgs& a, int head_dim, int num_sms, cudaStream_t stream);
+cudaError_t launch_bf16_decode(const DecodeArgs& a, int head_dim, cudaStream_t stream);
+cudaError_t launch_bf16_dequant(const DequantArgs& a, int head_dim, int num_sms, cudaStream_t stream);
 cudaError_t launch_prefill(const void* q, const unsigned char* cache, int num_blocks, int Hkv, int Hq, int B,
                            const uint16_t* k_tables, const uint16_t* default_table,
                            const int32_t* block_tables, int max_blocks, const int32_t* seq_lens,

@@ -92,11 +92,26 @@ enum {
  * cache must be read with the flags it was written with. */
 enum { TQ_CACHE_UNROTATED = 1 };
 
+/* TQ_CACHE_BF16: a full-precision cache for the layers a model keeps unquantised.
+ * "TurboQuant 在 AMD GPU 上把長上下文延遲壓下來", section 3: for full-attention
+ * models, leaving the first and last layers unquantised recovers accuracy, since
+ * those boundary layers are the most sensitive to KV quantisation.  Its record
+ * of one (block, kv head) is the 16 tokens' bf16 key rows [16][d] followed by
+ * their bf16 value rows [16][d] (64 d bytes; within row r = token (keys) or
+ * 16 + token (values), the 16-byte chunk j is stored at position j ^ (r mod 8),
+ * so that one copy of a record lands in shared memory ready for conflict-free
+ * tensor-core loads).  tq_quantize_append stores the rows
+ * as they are (no key tables: k_tables must be NULL), and the decode calls and
+ * tq_dequantize read them (the decode's default split count is its own, within the
+ * num_splits = 0 workspace); tq_prefill_attention returns TQ_ERR_UNSUPPORTED for
+ * it.  Not combinable with TQ_CACHE_UNROTATED. */
+enum { TQ_CACHE_BF16 = 2 };
+
 typedef struct {
     int32_t num_blocks;   /* physical 16-token blocks */
     int32_t num_kv_heads; /* H_kv */
     int32_t head_dim;     /* d: 64 or 128 */
-    int32_t flags;        /* 0 or TQ_CACHE_UNROTATED (other bits: TQ_ERR_INVALID_ARG) */
+    int32_t flags;        /* 0, TQ_CACHE_UNROTATED or TQ_CACHE_BF16 (else TQ_ERR_INVALID_ARG) */
     void* data;           /* (device) [num_blocks][num_kv_heads][record], 16-byte aligned */
 } tq_cache_t;
 
@@ -104,6 +119,9 @@ typedef struct {
 TQ_API size_t tq_record_bytes(int head_dim);
 /* Bytes of a whole cache; 0 on an unsupported shape. */
 TQ_API size_t tq_cache_bytes(int num_blocks, int num_kv_heads, int head_dim);
+/* Bytes of one record of a cache with these flags (64 d for TQ_CACHE_BF16, else
+ * tq_record_bytes(d)); 0 on an unsupported head_dim or flag combination. */
+TQ_API size_t tq_cache_record_bytes(int head_dim, int flags);
 
 /* Key tables are 16 fp16 values (raw bit patterns), strictly ascending, so that
  * every centroid is an exact fp16 tensor-core operand.
@@ -147,7 +165,8 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
 /* Number of context splits tq_decode_attention uses when num_splits == 0. */
 TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len);
 /* Workspace bytes for tq_decode_attention with this many splits (fp32 partial
- * outputs and softmax statistics per (sequence, query head, split)). */
+ * outputs and softmax statistics per (sequence, query head, split)); with
+ * num_splits = 0, enough for the default plan of either kind of cache. */
 TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_splits);
 
 /* Decode attention over the compressed cache, one query per sequence -- the
