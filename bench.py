@@ -614,6 +614,28 @@ def prefill_decode_case(dev):
     print(json.dumps({"case": "prefill_decode", "ok": True}))
 
 
+def bf16_decode_case(dev):
+    """Decode over the full-precision (bf16) cache of 8 qwen3_8b_layer sequences
+    (8 x 8192 tokens, 8 kv heads, d 128: 268 MB of keys and values, more than L2),
+    3 warm-up calls then 1: the case the bf16 decode kernel is profiled on."""
+    import bit_rotated_kv_tq_b200 as tq
+
+    tq.load()
+    w = W.make("qwen3_8b_layer", B=8)
+    cache = tq.Cache(w.num_blocks, w.Hkv, w.d, device=dev, bf16=True)
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for K, V, slots in w.population():
+        tq.quantize_append(K.to(dev), V.to(dev), slots.to(dev), cache, block_table=bt, status=status)
+    lens = torch.from_numpy(w.seq_lens).to(dev)
+    q = w.q().to(dev)
+    for _ in range(4):
+        tq.decode_attention(q, cache, bt, lens, int(w.seq_lens.max()), w.scale, status=status)
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0
+    print(json.dumps({"case": "bf16_decode", "ok": True}))
+
+
 # ---------------------------------------------------------------- GPU arm
 def run_tq(args, rank, world, local):
     import bit_rotated_kv_tq_b200 as tq
@@ -890,7 +912,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["prefill_append", "prefill_decode", "prefill_attention"], default=None,
+    ap.add_argument("--case", choices=["prefill_append", "prefill_decode", "prefill_attention", "bf16_decode"],
+                    default=None,
                     help="run one small profiling case instead of the bench")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the long-context, agentic and prefill-chunk measurements")
@@ -911,6 +934,9 @@ def main():
         return
     if args.case == "prefill_attention":
         prefill_attention_case(torch.device("cuda", 0))
+        return
+    if args.case == "bf16_decode":
+        bf16_decode_case(torch.device("cuda", 0))
         return
     rank, world, local = dist_setup(args.gpus)
     try:
