@@ -478,13 +478,14 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
                 const float2 x = __ffma2_rn(Q[j], A2, M2);
                 const BinEntry e0 = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x.x) & 0x3f8u));
                 const BinEntry e1 = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x.y) & 0x3f8u));
-                // y - mid with one rounding: its sign is the decision
-                const float d0 = fmaf(Q[j].x, inv, -e0.mid);
-                const float d1 = fmaf(Q[j].y, inv, -e1.mid);
+                // mid - y with one rounding: its sign is the decision (y == mid gives
+                // +0 and the lower code, and is near anyway)
+                const float d0 = fmaf(-Q[j].x, inv, e0.mid);
+                const float d1 = fmaf(-Q[j].y, inv, e1.mid);
                 if (fminf(fabsf(d0), fabsf(d1)) < kKeyMargin) kpm |= 1u << j;
-                // k_hi - 1 where y <= mid (sign bit set; y == mid is near anyway)
-                const uint32_t c0 = (uint32_t)(e0.k_hi + (__float_as_int(d0) >> 31));
-                const uint32_t c1 = (uint32_t)(e1.k_hi + (__float_as_int(d1) >> 31));
+                // k_lo + 1 where y > mid (the sign bit of mid - y)
+                const uint32_t c0 = (uint32_t)e0.k_lo + (__float_as_uint(d0) >> 31);
+                const uint32_t c1 = (uint32_t)e1.k_lo + (__float_as_uint(d1) >> 31);
                 by[j] = c0 | (c1 << 4);
             }
 #pragma unroll
@@ -536,7 +537,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
                 // an all-zero key: y = 0 exactly, every element takes the code of 0
                 uint32_t c0 = 0;
                 const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(kBinMagic) & 0x3f8u));
-                if (!B.dense) c0 = (uint32_t)be.k_hi - (0.f > be.mid ? 0u : 1u);
+                if (!B.dense) c0 = (uint32_t)be.k_lo + (0.f > be.mid ? 1u : 0u);
                 else
                     for (int k = 0; k < 15; k++) c0 += 0.f > 0.5f * (B.c[k] + B.c[k + 1]) ? 1u : 0u;
 #pragma unroll
@@ -558,7 +559,7 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
                     if (!B.dense) {
                         const float x = fmaf((float)part * rden, kBinScale, kBinMagic);
                         const BinEntry be = *reinterpret_cast<const BinEntry*>(tab + (__float_as_uint(x) & 0x3f8u));
-                        idx = (uint32_t)be.k_hi - (part > (double)be.mid * denom ? 0u : 1u);
+                        idx = (uint32_t)be.k_lo + (part > (double)be.mid * denom ? 1u : 0u);
                     } else {
 #pragma unroll 1
                         for (int k = 0; k < 15; k++)

@@ -34,7 +34,7 @@ struct HeadBins {
 };
 struct __align__(8) BinEntry {
     float mid;  // the one midpoint inside the bin (with margins), or +inf
-    int k_hi;   // 1 + the number of midpoints strictly below the bin
+    int k_lo;   // the number of midpoints strictly below the bin (the code below its midpoint)
 };
 
 // One bin of a strictly ascending 16-entry table c: the midpoints below the
@@ -61,7 +61,7 @@ __host__ __device__ inline bool bin_entry(const float* c, int bin, BinEntry& e) 
         m_in = m;
     }
     e.mid = m_in;
-    e.k_hi = below + 1;
+    e.k_lo = below;
     return inside > 1;
 }
 
