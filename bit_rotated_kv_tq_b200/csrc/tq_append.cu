@@ -646,11 +646,16 @@ __global__ void __launch_bounds__(kAppWarps * 32, 1) append_kernel(AppendArgs a)
             *reinterpret_cast<uint4*>(rec + R::kKCodes + off * R::kCodeRow + sub * 16) =
                 make_uint4(kc[0], kc[1], kc[2], kc[3]);
             // code bytes 16 sub + r (m = 2 sub) and 16 sub + 8 + r (m = 2 sub + 1) of
-            // this token sit side by side in chunk r
-            unsigned char* vdst = rec + R::kVCodes + R::vcode_pos(off, 16 * sub);
+            // this token sit side by side in the chunk of r, its pair's chunks rotated
+            // by 2 (off / 2): chunks r and r + 1 (r even) stay adjacent
+            unsigned char* vdst = rec + R::kVCodes + R::vcode_pos(off, 16 * sub);  // chunk of r = 0
+            const int rot = (off >> 1) & 3;  // the rotation in chunk pairs
 #pragma unroll
-            for (int r = 0; r < 8; r++)
-                *reinterpret_cast<uint16_t*>(vdst + r * R::kPairChunk) = (uint16_t)sv[r];
+            for (int r = 0; r < 8; r += 2) {
+                unsigned char* cp = vdst + (((r >> 1) + rot) & 3) * (2 * R::kPairChunk) - 2 * rot * R::kPairChunk;
+                *reinterpret_cast<uint16_t*>(cp) = (uint16_t)sv[r];
+                *reinterpret_cast<uint16_t*>(cp + R::kPairChunk) = (uint16_t)sv[r + 1];
+            }
             if (sub == 0) *reinterpret_cast<uint16_t*>(rec + R::kKNorm + off * 2) = n16;
             const int gp = R::group_pos(off, sub);
             *reinterpret_cast<uint16_t*>(rec + R::kVScale + gp) = s16;

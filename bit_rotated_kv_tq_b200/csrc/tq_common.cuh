@@ -5,8 +5,11 @@
 //   [0, 8D)           key codes    [16][D/2] bytes, element 2j in the low nibble of byte j
 //   [8D, 8D+32)       key norms    [16] fp16
 //   [8D+32, 16D+32)   value codes  8D bytes, same nibble order, placed for the decode
-//                     fragments: byte j = 8m + r of token t sits at
-//                     (8 (t/2) + r) (D/8) + 4 (m/2) + 2 (t%2) + (m%2)
+//                     fragments: byte j = 8m + r of token t sits in chunk (D/8 bytes)
+//                     8 (t/2) + ((r + 2 (t/2)) mod 8), at byte 4 (m/2) + 2 (t%2) + (m%2)
+//                     of it (the rotation of a token pair's 8 chunks by 2 (t/2) puts
+//                     the chunks that one quarter warp of the decode reads in 8
+//                     different bank groups)
 //   [16D+32, 17D+32)  value scales fp16, the one of token t, group G at byte
 //                     2 (4 (c (D/32) + G) + u), c = (t%8)/2, u = 2 (t/8) + t%2
 //   [17D+32, 18D+32)  value zeros  fp16, same placement
@@ -39,8 +42,8 @@ struct Rec {
     static constexpr int kPairChunk = D / 8;  // value bytes of one (token pair, r) chunk
     // value byte j of token t, relative to kVCodes
     static __host__ __device__ constexpr int vcode_pos(int t, int j) {
-        return (8 * (t >> 1) + (j & 7)) * kPairChunk + 4 * ((j >> 3) >> 1) + 2 * (t & 1) +
-               ((j >> 3) & 1);
+        return (8 * (t >> 1) + (((j & 7) + 2 * (t >> 1)) & 7)) * kPairChunk + 4 * ((j >> 3) >> 1) +
+               2 * (t & 1) + ((j >> 3) & 1);
     }
     // scale (zero) of token t, group G, relative to kVScale (kVZero)
     static __host__ __device__ constexpr int group_pos(int t, int G) {

@@ -432,8 +432,10 @@ __device__ __forceinline__ void record_values(uint32_t rec, int g, int c, uint32
     // word G of a chunk holds m-tiles 2G (bytes 0, 2) and 2G + 1 (bytes 1, 3) of
     // tokens 2c, 2c+1 (va) and 2c+8, 2c+9 (vb)
     uint32_t va[KW], vb[KW];
-    ldw<KW>(rec + R::kVCodes + (c * 8 + g) * KB, va);
-    ldw<KW>(rec + R::kVCodes + ((c + 4) * 8 + g) * KB, vb);
+    // chunk r = g of token pairs c and c + 4, rotated by 2c (2 (c + 4) = 2c mod 8)
+    const int rr = (g + 2 * c) & 7;
+    ldw<KW>(rec + R::kVCodes + (c * 8 + rr) * KB, va);
+    ldw<KW>(rec + R::kVCodes + ((c + 4) * 8 + rr) * KB, vb);
 #pragma unroll
     for (int G_ = 0; G_ < NG; G_++) {
         const uint32_t A0 = va[G_], B0 = vb[G_], A1 = A0 >> 8, B1 = B0 >> 8;

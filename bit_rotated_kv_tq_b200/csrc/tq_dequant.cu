@@ -53,9 +53,9 @@ __global__ void __launch_bounds__(256) dequant_kernel(DequantArgs a) {
         uint32_t kw = 0, vw = 0;
         if (rec) {
             kw = *reinterpret_cast<const uint32_t*>(rec + R::kKCodes + off * R::kCodeRow + sub * 4);
-            const unsigned char* vsrc = rec + R::kVCodes + R::vcode_pos(off, 4 * sub);
 #pragma unroll
-            for (int i = 0; i < 4; i++) vw |= (uint32_t)vsrc[i * R::kPairChunk] << (8 * i);
+            for (int i = 0; i < 4; i++)
+                vw |= (uint32_t)rec[R::kVCodes + R::vcode_pos(off, 4 * sub + i)] << (8 * i);
             nrm = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec + R::kKNorm + off * 2));
             const int gp = R::group_pos(off, sub / 4);
             s = half_bits_to_float(*reinterpret_cast<const uint16_t*>(rec + R::kVScale + gp));

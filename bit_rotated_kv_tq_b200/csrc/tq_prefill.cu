@@ -407,7 +407,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
             float v[D / 8];
             if (valid) {
                 const uint32_t rec = st + (uint32_t)j * REC;
-                const uint32_t ch = rec + R::kVCodes + (uint32_t)((8 * (o >> 1) + r) * (D / 8));
+                const uint32_t ch =
+                    rec + R::kVCodes + (uint32_t)((8 * (o >> 1) + ((r + 2 * (o >> 1)) & 7)) * (D / 8));
                 float sc[D / 32], zr[D / 32];
 #pragma unroll
                 for (int g = 0; g < D / 32; g++) {

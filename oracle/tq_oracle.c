@@ -422,11 +422,13 @@ static size_t off_vcodes(int d) { return off_knorm(d) + ORC_BLOCK * 2; }
 static size_t off_vscale(int d) { return off_vcodes(d) + (size_t)ORC_BLOCK * d / 2; }
 static size_t off_vzero(int d) { return off_vscale(d) + (size_t)d; }
 
-/* offset of value code byte j of token t within the value-code area */
+/* offset of value code byte j of token t within the value-code area: chunk
+ * 8p + ((r + 2p) mod 8) of d/8 bytes (token pair p's chunks rotated by 2p),
+ * byte 4 (m/2) + 2e + (m mod 2) of it */
 static size_t vcode_pos(int d, int t, int j)
 {
     int p = t / 2, e = t % 2, m = j / 8, r = j % 8;
-    return (size_t)(8 * p + r) * (d / 8) + 4 * (m / 2) + 2 * e + (m % 2);
+    return (size_t)(8 * p + (r + 2 * p) % 8) * (d / 8) + 4 * (m / 2) + 2 * e + (m % 2);
 }
 
 /* offset of the scale (or zero) of token t, group G within its area */

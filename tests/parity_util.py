@@ -32,11 +32,11 @@ def layout(d):
 
 def value_code_positions(d):
     """[16][d/2] offsets of value byte j of token t in the value-code area:
-    (8 (t // 2) + j % 8) (d/8) + 4 ((j // 8) // 2) + 2 (t % 2) + (j // 8) % 2."""
+    (8 p + (j % 8 + 2 p) % 8) (d/8) + 4 ((j // 8) // 2) + 2 (t % 2) + (j // 8) % 2, p = t // 2."""
     t = np.arange(16)[:, None]
     j = np.arange(d // 2)[None, :]
-    m, r = j // 8, j % 8
-    return (8 * (t // 2) + r) * (d // 8) + 4 * (m // 2) + 2 * (t % 2) + m % 2
+    m, r, p = j // 8, j % 8, t // 2
+    return (8 * p + (r + 2 * p) % 8) * (d // 8) + 4 * (m // 2) + 2 * (t % 2) + m % 2
 
 
 def group_positions(d):

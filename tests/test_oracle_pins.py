@@ -382,15 +382,16 @@ def test_record_size_and_nibble_order(orc):
     assert np.all(row == int(g["key_e0_byte"][0], 16))
     assert int(rec[1024 + 10]) | (int(rec[1024 + 11]) << 8) == 0x3C00
     vc = rec[1056:1056 + 1024]
-    chunk19 = [int(x, 16) for x in g["value_ramp_chunk19_d128"]]
-    assert list(vc[19 * 16:20 * 16]) == chunk19
+    chunk23 = [int(x, 16) for x in g["value_ramp_chunk23_d128"]]
+    assert list(vc[23 * 16:24 * 16]) == chunk23
     odd_pos = [2, 3, 6, 7, 10, 11, 14, 15]
-    for r in range(8):  # chunk 16 + r: 0x11*r at m-even, 0x11*(r+8) at m-odd positions
-        ch = vc[(16 + r) * 16:(17 + r) * 16]
+    for r in range(8):  # chunk 16 + (r + 4) % 8: 0x11*r at m-even, 0x11*(r+8) at m-odd positions
+        c = 16 + (r + 4) % 8
+        ch = vc[c * 16:(c + 1) * 16]
         assert list(ch[odd_pos]) == [0x11 * r, 0x11 * (r + 8)] * 4
         assert not np.any(np.delete(ch, odd_pos))
     # reading the bytes back in natural order gives the worked example's code bytes
-    natural = [vc[(16 + j % 8) * 16 + 4 * (j // 16) + 2 + (j // 8) % 2] for j in range(64)]
+    natural = [vc[(16 + (j % 8 + 4) % 8) * 16 + 4 * (j // 16) + 2 + (j // 8) % 2] for j in range(64)]
     want = [int(x, 16) for x in g["value_ramp_bytes"]]
     assert natural[:16] == want and natural[16:32] == want
     offs = [int(x) for x in g["value_ramp_group_offsets_d128"]]
