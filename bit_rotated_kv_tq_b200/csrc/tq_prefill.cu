@@ -485,20 +485,38 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
 #pragma unroll
             for (int j = 0; j < 16; j++) x[c0 + j] = t16[j];
         }
-        float mx = -INFINITY;
         const bool whole = kStep * (s + 1) <= lim;  // the row sees every token of the step
+        if (__all_sync(kFull, whole)) {  // no mask: the norms by packed multiplies
 #pragma unroll
-        for (int c0 = 0; c0 < kStep; c0 += 4) {
-            const uint4 nw = ld_s128(sNorm + 4 * c0);
-            const float nn[4] = {__uint_as_float(nw.x), __uint_as_float(nw.y), __uint_as_float(nw.z),
-                                 __uint_as_float(nw.w)};
+            for (int c0 = 0; c0 < kStep; c0 += 4) {
+                const uint4 nw = ld_s128(sNorm + 4 * c0);
+                const float2 a = __fmul2_rn(make_float2(x[c0], x[c0 + 1]),
+                                            make_float2(__uint_as_float(nw.x), __uint_as_float(nw.y)));
+                const float2 b = __fmul2_rn(make_float2(x[c0 + 2], x[c0 + 3]),
+                                            make_float2(__uint_as_float(nw.z), __uint_as_float(nw.w)));
+                x[c0] = a.x;
+                x[c0 + 1] = a.y;
+                x[c0 + 2] = b.x;
+                x[c0 + 3] = b.y;
+            }
+        } else {
 #pragma unroll
-            for (int j = 0; j < 4; j++) {
-                const int t = kStep * s + c0 + j;
-                x[c0 + j] = whole || t < lim ? x[c0 + j] * nn[j] : -INFINITY;
-                mx = fmaxf(mx, x[c0 + j]);
+            for (int c0 = 0; c0 < kStep; c0 += 4) {
+                const uint4 nw = ld_s128(sNorm + 4 * c0);
+                const float nn[4] = {__uint_as_float(nw.x), __uint_as_float(nw.y), __uint_as_float(nw.z),
+                                     __uint_as_float(nw.w)};
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int t = kStep * s + c0 + j;
+                    x[c0 + j] = whole || t < lim ? x[c0 + j] * nn[j] : -INFINITY;
+                }
             }
         }
+        // the row maximum: four independent chains
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int j = 0; j < kStep; j++) m4[j & 3] = fmaxf(m4[j & 3], x[j]);
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         // the reference maximum moves only when the row maximum passes it by 2^8;
         // the accumulator row is rescaled then (tensor-memory loads and stores are
         // warp-wide: a lane whose row keeps its maximum scales by 1)
@@ -518,23 +536,36 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_kernel(PrefillArgs a) {
                 tmem_st16(tO + lane_off + (uint32_t)c0, t16);
             }
         }
-        // p = 2^(x - m) as fp16 high and low parts, 8 tokens per 16-byte row
+        // p = 2^(x - m) as fp16 high and low parts, 8 tokens per 16-byte row.  A row
+        // that has seen no token yet has every x at -inf and takes 0 as its maximum
+        // here: 2^-inf = 0 without a per-token test
         const uint32_t prow = sP + (uint32_t)((tid / 8) * 1024 + (tid % 8) * 16);
+        const float m_eff = m_run == -INFINITY ? 0.f : m_run;
+        const float2 nm2 = make_float2(-m_eff, -m_eff);
+        float2 l2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int t8 = 0; t8 < kStep / 8; t8++) {
             float p[8];
 #pragma unroll
-            for (int j = 0; j < 8; j++) {
-                const float xv = x[8 * t8 + j];
-                p[j] = xv == -INFINITY ? 0.f : exp2a(xv - m_run);
-                l_run += p[j];
+            for (int j = 0; j < 8; j += 2) {
+                const float2 d2 = __fadd2_rn(make_float2(x[8 * t8 + j], x[8 * t8 + j + 1]), nm2);
+                p[j] = exp2a(d2.x);
+                p[j + 1] = exp2a(d2.y);
+                l2 = __fadd2_rn(l2, make_float2(p[j], p[j + 1]));
             }
             uint32_t hi[4], lo[4];
 #pragma unroll
-            for (int e = 0; e < 4; e++) split_h2(p[2 * e], p[2 * e + 1], hi[e], lo[e]);
+            for (int e = 0; e < 4; e++) {
+                const __half2 h = __floats2half2_rn(p[2 * e], p[2 * e + 1]);
+                const float2 f = __half22float2(h);
+                const float2 r = __ffma2_rn(f, make_float2(-1.f, -1.f), make_float2(p[2 * e], p[2 * e + 1]));
+                hi[e] = *reinterpret_cast<const uint32_t*>(&h);
+                lo[e] = pack_h2(r.x, r.y);
+            }
             st_s128(prow + 128u * t8, make_uint4(hi[0], hi[1], hi[2], hi[3]));
             st_s128(prow + 16384u + 128u * t8, make_uint4(lo[0], lo[1], lo[2], lo[3]));
         }
+        l_run += l2.x + l2.y;
         async_proxy_fence();
         tc_before_sync();
         __syncthreads();
