@@ -195,3 +195,23 @@ def test_binding_checks_extents_before_anything_runs(lib):
     # the right extents on the host are refused for their placement
     with pytest.raises(ValueError, match="must be a CUDA tensor"):
         tq.decode_attention(bf(2, 8, 128), c, i32(2, 4), i32(2), 64, 0.1)
+
+
+def test_workspace_bounds_cover_the_bf16_plans(lib):
+    """A bf16 cache's decode keeps per (sequence, query head, range) an fp32 partial
+    output and its (max, sum): B H_q S (4 d + 8) bytes.  The workspace size the library
+    asks for must cover that for every explicit split count, and for its own default
+    (up to 8 ranges, within the 8 MiB of the static entry)."""
+    for B, Hq, d in [(1, 8, 64), (2, 32, 128), (32, 32, 128), (64, 64, 128), (16, 16, 64)]:
+        per = B * Hq * (4 * d + 8)
+        for S in (2, 3, 8, 64, 1024):
+            assert lib.tq_decode_workspace_bytes(B, Hq, d, S) >= per * S
+        assert lib.tq_decode_workspace_bytes(B, Hq, d, 0) >= min(8 * per, 8 << 20)
+        assert lib.tq_decode_workspace_bytes(B, Hq, d, 1) == 0
+    assert lib.tq_cache_record_bytes(128, tq.TQ_CACHE_BF16) == 8192
+    assert lib.tq_cache_record_bytes(64, tq.TQ_CACHE_BF16) == 4096
+    assert lib.tq_cache_record_bytes(128, 0) == lib.tq_record_bytes(128) == 2336
+    assert lib.tq_cache_record_bytes(128, tq.TQ_CACHE_UNROTATED) == 2336
+    assert lib.tq_cache_record_bytes(128, tq.TQ_CACHE_BF16 | tq.TQ_CACHE_UNROTATED) == 0
+    assert lib.tq_cache_record_bytes(96, 0) == 0
+
