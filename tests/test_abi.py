@@ -94,7 +94,8 @@ def test_argument_validation_without_launch(lib):
     assert rc == tq.TQ_ERR_INVALID_ARG
     rc = lib.tq_quantize_append(None, None, None, 0, 0, None, 0, ctypes.byref(c), None, None, None)
     assert rc == tq.TQ_OK  # T == 0 is a no-op
-    # cache flags: TQ_CACHE_UNROTATED is the only defined bit, checked by every call
+    # cache flags: TQ_CACHE_UNROTATED and TQ_CACHE_BF16 are the defined bits, never both;
+    # every call checks them
     for bad in (2, 4, 1 << 30):
         c = tq._Cache(4, 2, 128, bad | tq.TQ_CACHE_UNROTATED, 0x1000)
         rc = lib.tq_quantize_append(None, None, None, 0, 0, None, 0, ctypes.byref(c), None, None, None)
@@ -143,6 +144,37 @@ def test_argument_validation_without_launch(lib):
     # dequantize: misaligned output
     rc = lib.tq_dequantize(ctypes.byref(c), None, P(16), 4, P(16), 1, 8, P(20), P(16), None, None)
     assert rc == tq.TQ_ERR_ALIGNMENT
+
+
+def test_prefill_argument_validation_without_launch(lib):
+    """tq_prefill_attention rejects each bad argument on the host, before any launch."""
+    P = ctypes.c_void_p
+    c = _cache_struct(heads=2)
+    args = dict(q=P(16), k=None, bt=P(16), mb=4, sl=P(16), qs=P(16), B=1, Hq=4, T=8, mq=8, scale=0.1,
+                out=P(16))
+
+    def pre(cache=c, **kw):
+        a = {**args, **kw}
+        return lib.tq_prefill_attention(a["q"], ctypes.byref(cache), a["k"], a["bt"], a["mb"], a["sl"],
+                                        a["qs"], a["B"], a["Hq"], a["T"], a["mq"],
+                                        ctypes.c_float(a["scale"]), a["out"], None, None)
+
+    assert pre(cache=tq._Cache(4, 2, 128, tq.TQ_CACHE_BF16, 0x1000)) == tq.TQ_ERR_UNSUPPORTED
+    assert pre(cache=_cache_struct(d=96)) == tq.TQ_ERR_UNSUPPORTED
+    assert pre(cache=tq._Cache(4, 2, 128, tq.TQ_CACHE_BF16 | tq.TQ_CACHE_UNROTATED, 0x1000)) == tq.TQ_ERR_INVALID_ARG
+    for bad in (dict(B=-1), dict(Hq=0), dict(T=-1), dict(mq=-1), dict(mb=0), dict(q=None), dict(qs=None),
+                dict(out=None), dict(sl=None), dict(bt=None), dict(scale=float("inf"))):
+        assert pre(**bad) == tq.TQ_ERR_INVALID_ARG, bad
+    for empty in (dict(B=0), dict(T=0), dict(mq=0)):  # nothing to do: no launch, no pointer checks
+        assert pre(q=None, out=None, **empty) == tq.TQ_OK, empty
+    assert pre(B=65536) == tq.TQ_ERR_UNSUPPORTED
+    assert pre(Hq=5) == tq.TQ_ERR_UNSUPPORTED
+    assert pre(mq=1 << 30) == tq.TQ_ERR_UNSUPPORTED  # rows of (token, head) past 2^30
+    for mis in (dict(q=P(24)), dict(out=P(40)), dict(qs=P(18)), dict(sl=P(2)), dict(bt=P(6)),
+                dict(k=P(2))):
+        assert pre(**mis) == tq.TQ_ERR_ALIGNMENT, mis
+    # the unrotated cache is accepted by the same checks (the call stops at its empty batch)
+    assert pre(cache=tq._Cache(4, 2, 128, tq.TQ_CACHE_UNROTATED, 0x1000), B=0) == tq.TQ_OK
 
 
 def _host_cache(num_kv_heads=2, head_dim=128, num_blocks=1):
