@@ -481,6 +481,9 @@ TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, cons
         return fail(TQ_ERR_INVALID_ARG, "tq_dequantize: block_tables, seq_lens, K_hat, V_hat required");
     if (!aligned(K_hat, 16) || !aligned(V_hat, 16))
         return fail(TQ_ERR_ALIGNMENT, "tq_dequantize: K_hat and V_hat must be 16-byte aligned");
+    if (!aligned(block_tables, 4) || !aligned(seq_lens, 4) || (k_tables && !aligned(k_tables, 4)) ||
+        (status && !aligned(status, 4)))
+        return fail(TQ_ERR_ALIGNMENT, "tq_dequantize: int32 arrays and tables must be 4-byte aligned");
     tq::DequantArgs a;
     a.cache = static_cast<const unsigned char*>(cache->data);
     a.num_blocks = cache->num_blocks;

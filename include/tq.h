@@ -256,7 +256,9 @@ TQ_API int tq_prefill_attention(const void* q, const tq_cache_t* cache, const ui
  * [B][max_len][H_kv][d] in the original (unrotated) domain,
  * k_hat = fp16 norm * H * C[idx] (fp16 norm * C[idx] for a TQ_CACHE_UNROTATED
  * cache),  v_hat = code * scale + zero;
- * rows at or past seq_lens[b] are written as 0. */
+ * rows at or past seq_lens[b] are written as 0.  K_hat and V_hat must be
+ * 16-byte aligned, block_tables, seq_lens, k_tables and status 4-byte aligned
+ * (else TQ_ERR_ALIGNMENT, nothing enqueued). */
 TQ_API int tq_dequantize(const tq_cache_t* cache, const uint16_t* k_tables, const int32_t* block_tables,
                   int max_blocks, const int32_t* seq_lens, int B, int max_len, float* K_hat,
                   float* V_hat, int32_t* status, void* stream);

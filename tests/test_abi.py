@@ -141,9 +141,16 @@ def test_argument_validation_without_launch(lib):
     assert dec_static(Hq=4, L=65) == tq.TQ_ERR_INVALID_ARG
     assert dec_static(Hq=4, q=None) == tq.TQ_ERR_INVALID_ARG
     assert dec_static(Hq=4, B=0) == tq.TQ_OK
-    # dequantize: misaligned output
-    rc = lib.tq_dequantize(ctypes.byref(c), None, P(16), 4, P(16), 1, 8, P(20), P(16), None, None)
-    assert rc == tq.TQ_ERR_ALIGNMENT
+    # dequantize: bad sizes, missing pointers, misaligned output or int32 arrays
+    def deq(k=None, bt=P(16), mb=4, sl=P(16), B=1, L=8, K=P(16), V=P(16), st=None):
+        return lib.tq_dequantize(ctypes.byref(c), k, bt, mb, sl, B, L, K, V, st, None)
+
+    for bad in (dict(B=-1), dict(L=-1), dict(mb=0), dict(bt=None), dict(sl=None), dict(K=None),
+                dict(V=None)):
+        assert deq(**bad) == tq.TQ_ERR_INVALID_ARG, bad
+    assert deq(B=0, K=None, V=None) == tq.TQ_OK and deq(L=0, K=None, V=None) == tq.TQ_OK
+    for mis in (dict(K=P(20)), dict(V=P(24)), dict(bt=P(18)), dict(sl=P(6)), dict(k=P(2)), dict(st=P(1))):
+        assert deq(**mis) == tq.TQ_ERR_ALIGNMENT, mis
 
 
 def test_prefill_argument_validation_without_launch(lib):
