@@ -164,9 +164,11 @@ int decode_prepare(const void* q, const tq_cache_t* cache, const uint16_t* k_tab
     if (G > 64)
         return fail(TQ_ERR_UNSUPPORTED, "tq_decode_attention: GQA group %d (supported 1..64)", G);
     if (!isfinite(scale)) return fail(TQ_ERR_INVALID_ARG, "tq_decode_attention: scale not finite");
-    if (!aligned(q, 4) || !aligned(out, 4) || !aligned(block_tables, 4) || !aligned(seq_lens, 4) ||
+    // the split kernel stores its outputs as pairs of floats
+    if (!aligned(out, 8)) return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: out must be 8-byte aligned");
+    if (!aligned(q, 4) || !aligned(block_tables, 4) || !aligned(seq_lens, 4) ||
         (k_tables && !aligned(k_tables, 4)) || (status && !aligned(status, 4)))
-        return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: q/out/tables must be 4-byte aligned");
+        return fail(TQ_ERR_ALIGNMENT, "tq_decode_attention: q and the tables must be 4-byte aligned");
     const int d = cache->head_dim;
     const bool bf16 = (cache->flags & TQ_CACHE_BF16) != 0;
     if (bf16 && k_tables)

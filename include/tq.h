@@ -184,8 +184,11 @@ TQ_API size_t tq_decode_workspace_bytes(int B, int H_q, int head_dim, int num_sp
  *   seq_lens     (device) int32 [B], each in [0, max_blocks*16]
  *   max_seq_len  (host)   upper bound of seq_lens (sizes the split grid); a
  *                         longer seq_len sets TQ_STATUS_BAD_LEN and is cut
- *   out          (device) fp32 [B][H_q][d]; a sequence of length 0 gets 0
+ *   out          (device) fp32 [B][H_q][d], 8-byte aligned; a sequence of length 0
+ *                gets 0
  *   workspace    (device) >= tq_decode_workspace_bytes(...), 16-byte aligned
+ * q, block_tables, seq_lens, k_tables and status must be 4-byte aligned (a
+ * pointer that misses its alignment: TQ_ERR_ALIGNMENT, nothing enqueued).
  *   num_splits   0 = tq_decode_default_splits(...), else 1..1024
  * Splits of one sequence are merged by a log-sum-exp combine kernel. */
 TQ_API int tq_decode_attention(const void* q, const tq_cache_t* cache, const uint16_t* k_tables,

@@ -124,6 +124,10 @@ def test_argument_validation_without_launch(lib):
     assert dec(Hq=4, L=65) == tq.TQ_ERR_INVALID_ARG  # max_seq_len beyond max_blocks * 16
     assert dec(Hq=4, scale=float("nan")) == tq.TQ_ERR_INVALID_ARG
     assert dec(Hq=4, B=0) == tq.TQ_OK
+    # out takes 8-byte pair stores; q and the int32 arrays need 4 bytes
+    for mis in (dict(out=P(20)), dict(out=P(18)), dict(q=P(18)), dict(bt=P(2)), dict(sl=P(6)), dict(k=P(2))):
+        assert dec(Hq=4, **mis) == tq.TQ_ERR_ALIGNMENT, mis
+    assert dec(Hq=4, B=0, out=P(20)) == tq.TQ_OK  # an empty batch checks no pointer
     # explicit splits: at most B * H_q * S + 1 ranges, two partial slots of four heads each
     assert lib.tq_decode_workspace_bytes(2, 8, 128, 4) == (2 * 8 * 4 + 1) * 2 * 4 * (128 * 4 + 8)
     assert lib.tq_decode_workspace_bytes(2, 8, 64, 3) == (2 * 8 * 3 + 1) * 2 * 4 * (64 * 4 + 8)
@@ -141,6 +145,7 @@ def test_argument_validation_without_launch(lib):
     assert dec_static(Hq=4, L=65) == tq.TQ_ERR_INVALID_ARG
     assert dec_static(Hq=4, q=None) == tq.TQ_ERR_INVALID_ARG
     assert dec_static(Hq=4, B=0) == tq.TQ_OK
+    assert dec_static(Hq=4, out=P(20)) == tq.TQ_ERR_ALIGNMENT
     # dequantize: bad sizes, missing pointers, misaligned output or int32 arrays
     def deq(k=None, bt=P(16), mb=4, sl=P(16), B=1, L=8, K=P(16), V=P(16), st=None):
         return lib.tq_dequantize(ctypes.byref(c), k, bt, mb, sl, B, L, K, V, st, None)
