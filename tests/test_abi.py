@@ -232,6 +232,16 @@ def test_binding_checks_extents_before_anything_runs(lib):
         (lambda: tq.decode_attention_static(bf(2, 8, 128), c, i32(2, 4), i32(1), 64, 0.1),
          "seq_lens has shape"),
         (lambda: tq.dequantize(c, i32(2, 4), i32(3), 64), "seq_lens has shape"),
+        (lambda: tq.prefill_attention(bf(8, 256), c, i32(2, 4), i32(2), i32(3), 4, 0.1), "q has shape"),
+        (lambda: tq.prefill_attention(bf(8, 4, 64), c, i32(2, 4), i32(2), i32(3), 4, 0.1), "q has shape"),
+        (lambda: tq.prefill_attention(bf(8, 4, 128), c, i32(3, 4), i32(2), i32(3), 4, 0.1),
+         "block_tables has shape"),
+        (lambda: tq.prefill_attention(bf(8, 4, 128), c, i32(2, 4), i32(2), i32(2), 4, 0.1),
+         "q_start has shape"),
+        (lambda: tq.prefill_attention(bf(8, 4, 128), c, i32(2, 4), i32(2), i32(3), 4, 0.1,
+                                      out=torch.zeros((8, 4, 64))), "out has shape"),
+        (lambda: tq.prefill_attention(bf(8, 4, 128), c, i32(2, 4), i32(2), i32(3), 4, 0.1, status=i32(0)),
+         "status must hold"),
     ]
     for call, msg in cases:
         with pytest.raises(ValueError, match=msg):
