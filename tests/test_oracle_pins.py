@@ -560,6 +560,22 @@ def test_attention_invariant_to_token_order(orc):
 
 
 # ---------------------------------------------------------------- calibration
+@pytest.mark.parametrize("d", [64, 128])
+def test_rotated_unit_samples_are_hadamard_of_unit_keys(orc, d):
+    """The calibration samples are the rotated unit keys y = H k / ||k|| (H = scipy's
+    Sylvester matrix / sqrt(d)), row for row; a zero key gives zeros."""
+    kb = bf16_bits_of(RNG.standard_t(4, (12, d)) * RNG.lognormal(0, 1, d))
+    kb[5] = 0
+    k = torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16).double().numpy()
+    Hs = scipy.linalg.hadamard(d) / math.sqrt(d)
+    n = np.linalg.norm(k, axis=1, keepdims=True)
+    want = np.where(n > 0, (k / np.where(n > 0, n, 1)) @ Hs.T, 0.0)
+    got = orc.rotated_unit_samples(kb)
+    assert got.shape == (12, d)
+    assert np.allclose(got, want, rtol=0, atol=1e-14)
+    assert np.all(got[5] == 0)
+
+
 def test_kmeans_table_lowers_mse_on_its_samples(orc):
     d = 128
     init = orc.default_table(d)
