@@ -16,7 +16,6 @@ import torch
 import workloads as W
 from test_parity_gpu import GpuState, OracleSeq, check_pairs
 from test_quality_oracle import calibrated_tables, oracle_study
-from workloads import bf16_bits
 
 pytestmark = pytest.mark.gpu
 
