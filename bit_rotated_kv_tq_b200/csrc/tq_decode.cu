@@ -12,9 +12,9 @@
 // then staged and unpacked once for both.  The virtual record space items x
 // nmax (nmax = blocks of the longest sequence) is cut into ranges: evenly over
 // every half of a full grid, or into ceil(nmax / S) records per range with S
-// splits.  The grid is persistent: one CTA of 16 warps per SM, made of two
-// independent halves of 8 warps, half h taking ranges h, h + H, ...  Within a
-// range's part of an item (a segment) the 8 warps take its 16-token blocks
+// splits.  The grid is persistent: one CTA of 12 warps per SM, made of two
+// independent halves of 6 warps, half h taking ranges h, h + H, ...  Within a
+// range's part of an item (a segment) the 6 warps take its 16-token blocks
 // round-robin.  Each warp streams its records through a private ring of
 // shared-memory stages with bulk asynchronous copies (cp.async.bulk +
 // mbarrier); the ring runs across segment boundaries, so the next segment's
