@@ -69,6 +69,16 @@ def test_fit_k_table_equals_oracle(lib, orc):
         bits = keys.view(torch.int16).numpy().view(np.uint16)
         want, it2 = orc.kmeans_table(orc.rotated_unit_samples(bits), init, 100)
         assert np.array_equal(got, want) and it == it2
+    # degenerate calibration sets: no vector keeps the initial table; zero keys put every
+    # sample at 0, which moves the level that takes 0 (the lower of the two middle ones)
+    init = orc.default_table(128)
+    got, it = tq.fit_k_table(torch.zeros((0, 128), dtype=torch.bfloat16), init, 10)
+    assert it == 0 and np.array_equal(got.view(np.uint16), init.view(np.uint16))
+    zeros = torch.zeros((3, 128), dtype=torch.bfloat16)
+    got, it = tq.fit_k_table(zeros, init, 10)
+    want, it2 = orc.kmeans_table(orc.rotated_unit_samples(np.zeros((3, 128), np.uint16)), init, 10)
+    assert np.array_equal(got, want) and it == it2
+    assert float(got[7]) == 0.0 and np.array_equal(np.delete(got, 7), np.delete(init, 7))
 
 
 def _cache_struct(num_blocks=4, heads=2, d=128, data=0x1000):
