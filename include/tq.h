@@ -162,7 +162,11 @@ TQ_API int tq_quantize_append(const void* K, const void* V, const int32_t* block
                        const tq_cache_t* cache, const uint16_t* k_tables, int32_t* status,
                        void* stream);
 
-/* Number of context splits tq_decode_attention uses when num_splits == 0. */
+/* Number of context splits tq_decode_attention uses when num_splits == 0.  It
+ * returns 0: the default plan has no fixed split count, it cuts the space of
+ * (sequence, kv head, block) records evenly over the whole GPU, so an item is
+ * split only where a cut falls inside it.  The arguments are kept for callers
+ * that size their own plans from them. */
 TQ_API int tq_decode_default_splits(int B, int H_kv, int max_seq_len);
 /* Workspace bytes for tq_decode_attention with this many splits (fp32 partial
  * outputs and softmax statistics per (sequence, query head, split)); with
