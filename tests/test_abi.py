@@ -142,6 +142,7 @@ def test_argument_validation_without_launch(lib):
     assert lib.tq_decode_workspace_bytes(2, 8, 128, 4) == (2 * 8 * 4 + 1) * 2 * 4 * (128 * 4 + 8)
     assert lib.tq_decode_workspace_bytes(2, 8, 64, 3) == (2 * 8 * 3 + 1) * 2 * 4 * (64 * 4 + 8)
     assert lib.tq_decode_workspace_bytes(2, 8, 128, 1) == 0
+    assert lib.tq_decode_default_splits(32, 8, 8192) == 0  # the even cut, no fixed count
     # the fixed-scratch entry runs the same checks first, with the same codes
     def dec_static(**kw):
         a = {**args, **kw}
